@@ -1,0 +1,203 @@
+/*
+ * eta.h - C ABI of the B200 (sm_100a) library for the decode step of
+ * Elastic Threshold Attention (ETA).
+ *
+ * Source of the operations: "Elastic Threshold Attention: Learned Contextual
+ * Sparsity for Long-Context Decoding"
+ *   - query-conditioned threshold tau = w_tau . q + b_tau, or frozen per-head
+ *     constants c (section 1; section 4.7; Appendix D.1, D.2)
+ *   - effective threshold tau~ = tau - a and the tempered logit
+ *     S~ = S * sigmoid(beta (S - tau~)), S = q k / sqrt(d) (Appendix G.1)
+ *   - per-block metadata mu_B (fp16), sigma_B (fp16), M_B (fp32) per KV head
+ *     (Appendix F.1; section 3.2)
+ *   - O(1) block screen, GQA union loading with per-head masking (section 3.1,
+ *     section 4.3 "Dual Bound", Appendix F.1)
+ *   - split-KV chunks merged by an associative online-softmax reduction,
+ *     top-1 rescue, predicated tail block (section 3.2; Appendix F.3, F.4)
+ *   - always-loaded window: lwb = 2 blocks plus the tail block (section 4.8)
+ *
+ * Conventions shared by every entry point:
+ *   - Every pointer inside a descriptor is DEVICE memory of the current CUDA
+ *     device, borrowed (never freed or retained by the library), and 16-byte
+ *     aligned unless said otherwise.  Descriptors themselves are host memory
+ *     read during the call only.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  Calls are
+ *     asynchronous and stream-ordered; none synchronises the host except
+ *     eta_read_device_status.
+ *   - The library never allocates or frees device memory.  Scratch memory is
+ *     the caller's `workspace`, sized by eta_decode_workspace_size.
+ *   - Arguments are validated on the host before any launch; a failed
+ *     validation returns an error code and launches nothing.  Values that
+ *     live in device memory (seq_lens, first_token) are checked by the
+ *     kernels: an out-of-range value is clamped and recorded in the device
+ *     status word, read back with eta_read_device_status.
+ *   - Layouts (row-major, contiguous):
+ *       K, V cache   [batch, n_kv_heads, max_ctx, head_dim]   kv_dtype
+ *       q, out       [batch, n_q_heads, head_dim]             kv_dtype
+ *       mu, sigma    [batch, n_kv_heads, nb_max, head_dim]     fp16
+ *       max_norm     [batch, n_kv_heads, nb_max]               fp32
+ *     with nb_max = ceil(max_ctx / block_size).  Query head h reads KV head
+ *     h / (n_q_heads / n_kv_heads).
+ *   - Supported: head_dim in {64, 128}; block_size in {16, 32, 64, 128};
+ *     group size n_q_heads / n_kv_heads in {1, 2, 4, 8}.
+ */
+#ifndef ETA_H
+#define ETA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ETA_OK = 0,
+  ETA_ERR_INVALID_ARG = 1,     /* bad pointer, size, alignment or value     */
+  ETA_ERR_UNSUPPORTED = 2,     /* valid but not implemented (e.g. d = 96)   */
+  ETA_ERR_WORKSPACE = 3,       /* workspace NULL or smaller than required   */
+  ETA_ERR_CUDA = 4,            /* a CUDA runtime call failed                */
+  ETA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out        */
+  ETA_ERR_DEVICE_RANGE = 6     /* a device-resident length was out of range */
+} eta_status;
+
+typedef enum { ETA_F32 = 0, ETA_BF16 = 1 } eta_dtype;
+typedef enum { ETA_TAU_LEARNED = 0, ETA_TAU_CALIBRATED = 1 } eta_tau_mode;
+
+/* Attention-kernel choice (eta_decode_params.attend_impl). */
+typedef enum {
+  ETA_ATTEND_AUTO = 0,   /* tensor-core kernel where supported, else CUDA-core */
+  ETA_ATTEND_SIMT = 1,   /* CUDA-core FMA kernel (all supported shapes)       */
+  ETA_ATTEND_TC = 2      /* tcgen05 tensor-core kernel (bf16, d = 128,
+                            block_size in {64, 128}, group size >= 2)          */
+} eta_attend_impl;
+
+/* The KV cache of one attention layer. */
+typedef struct {
+  int batch;          /* >= 1                                                */
+  int n_q_heads;      /* multiple of n_kv_heads                              */
+  int n_kv_heads;     /* >= 1                                                */
+  int head_dim;       /* 64 or 128                                           */
+  int block_size;     /* tokens per KV block b                               */
+  int max_ctx;        /* token capacity per (sequence, KV head), >= 1        */
+  eta_dtype kv_dtype; /* dtype of K, V, q and out                            */
+  const void* k_cache;
+  const void* v_cache;
+  const int* seq_lens; /* [batch] device, 0 <= seq_lens[i] <= max_ctx         */
+} eta_cache_desc;
+
+/* Per-block, per-KV-head metadata (Appendix F.1): centroid mu_B, coordinate
+ * standard deviation sigma_B (both fp16), maximum norm M_B (fp32) of the
+ * block's keys around the stored fp16 centroid, rounded up so that the
+ * geometric bound <q, mu_B> + ||q|| M_B never under-estimates a key's logit. */
+typedef struct {
+  void* mu;        /* fp16 [batch, n_kv_heads, nb_max, head_dim]             */
+  void* sigma;     /* fp16 [batch, n_kv_heads, nb_max, head_dim]             */
+  float* max_norm; /* fp32 [batch, n_kv_heads, nb_max] (4-byte aligned)      */
+} eta_summary_desc;
+
+/*
+ * eta_block_summary_update - refresh the metadata of the blocks touched by a
+ * KV append ("metadata ... refreshed on KV append"; Appendix F.1).
+ *
+ * For every sequence i, recomputes the blocks j with
+ *   first_token[i] / block_size <= j < ceil(seq_lens[i] / block_size),
+ * at most `max_blocks` of them per sequence (pass 1 for a one-token append,
+ * nb_max to rebuild everything).  A partial tail block is summarised over its
+ * present tokens only.  Other blocks are left untouched.
+ *   first_token : [batch] device int, lowest position written since the last
+ *                 update (4-byte aligned).
+ * Errors: ETA_ERR_INVALID_ARG for NULL/misaligned pointers or bad sizes,
+ * ETA_ERR_UNSUPPORTED for an unsupported head_dim/block_size,
+ * ETA_ERR_CUDA if the launch fails.
+ */
+eta_status eta_block_summary_update(const eta_cache_desc* cache,
+                                    const eta_summary_desc* summary,
+                                    const int* first_token, int max_blocks,
+                                    void* stream);
+
+/* All inputs and outputs of one decode step. */
+typedef struct {
+  eta_cache_desc cache;
+  eta_summary_desc summary;          /* must be current for seq_lens         */
+  const void* q;                     /* [batch, n_q_heads, head_dim]         */
+  eta_tau_mode tau_mode;
+  const float* w_tau;                /* [n_q_heads, head_dim] (learned)      */
+  const float* b_tau;                /* [n_q_heads]           (learned)      */
+  const float* c_tau;                /* [n_q_heads]           (calibrated)   */
+  float scale;                       /* logit scale, usually 1/sqrt(d), > 0  */
+  float beta;                        /* gate sharpness, > 0 (5 = terminal)   */
+  float offset_a;                    /* tau~ = tau - a                       */
+  float z;                           /* probabilistic half's z (> 0);
+                                        INFINITY = strict geometric screen   */
+  int n_local_blocks;                /* lwb >= 0: the tail block and the lwb
+                                        blocks before it are always loaded;
+                                        -1: none is, every block is screened  */
+  int screen_enabled;                /* 0: every block is loaded (dense path) */
+  int attend_impl;                   /* eta_attend_impl                      */
+  void* out;                         /* [batch, n_q_heads, head_dim] written */
+  float* lse;                        /* [batch, n_q_heads] or NULL: log-sum-
+                                        exp of the tempered logits (-inf for
+                                        an empty sequence)                   */
+  /* Optional selection outputs (NULL to skip; all int32/uint32, 4-aligned): */
+  int* admitted_count;               /* [batch, n_q_heads] blocks per head   */
+  int* union_count;                  /* [batch, n_kv_heads] union blocks     */
+  int* union_list;                   /* [batch, n_kv_heads, nb_max]: union
+                                        block ids ascending, then -1 fill    */
+  unsigned* union_mask;              /* [batch, n_kv_heads, nb_max]: bit j set
+                                        if query head g*G + j admitted block
+                                        union_list[...]; 0 fill              */
+  void* workspace;                   /* device scratch, 256-byte aligned     */
+  size_t workspace_bytes;
+  void* timing_events[4];            /* optional cudaEvent_t (NULL = none):
+                                        recorded before the screen, before
+                                        the attention kernel, before the
+                                        merge and after the last kernel      */
+} eta_decode_params;
+
+/*
+ * eta_decode_workspace_size - bytes of workspace eta_decode needs for these
+ * shapes (host-only, launches nothing).  Depends on the cache shape, the
+ * attention-kernel choice and the current device's SM count.
+ * Errors: ETA_ERR_INVALID_ARG / ETA_ERR_UNSUPPORTED as eta_decode.
+ */
+eta_status eta_decode_workspace_size(const eta_decode_params* p, size_t* bytes);
+
+/*
+ * eta_decode - one ETA decode step for every (sequence, query head):
+ *   1. tau~ per head (projection or constant, minus a);
+ *   2. every screenable block scored against tau~; admitted set per head =
+ *      screened blocks with Score >= tau~ plus the always-loaded window; a
+ *      head left with no block admits its highest-scoring block (top-1
+ *      rescue, lowest index on ties); the GQA union of a KV head's admitted
+ *      sets is the load set;
+ *   3. only the union's K/V blocks are read; each query head attends over the
+ *      tokens (< seq_len) of its own admitted blocks with
+ *      S~ = S sigmoid(beta (S - tau~)), weights exp(S~);
+ *   4. split partials merged: out = sum e^{S~} v / sum e^{S~}, lse.
+ * Outputs are written in kv_dtype (round-to-nearest-even for bf16).
+ * Errors: ETA_ERR_INVALID_ARG, ETA_ERR_UNSUPPORTED, ETA_ERR_WORKSPACE,
+ * ETA_ERR_CUDA (launch failure).  Device-side problems (a bounded wait that
+ * ran out, a seq_len outside [0, max_ctx]) are reported by
+ * eta_read_device_status.
+ */
+eta_status eta_decode(const eta_decode_params* p, void* stream);
+
+/*
+ * eta_read_device_status - synchronise `stream`, read and clear the device
+ * status word kept in `workspace`.  Returns ETA_OK, ETA_ERR_DEVICE_TIMEOUT
+ * or ETA_ERR_DEVICE_RANGE (or ETA_ERR_CUDA if the copy fails).
+ */
+eta_status eta_read_device_status(void* workspace, void* stream);
+
+/* Static description of a status code. */
+const char* eta_status_string(eta_status s);
+
+/* Library build description (kernels compiled, architecture). */
+const char* eta_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ETA_H */

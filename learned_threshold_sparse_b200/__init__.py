@@ -1,0 +1,260 @@
+"""Python binding of the ETA decode library (libeta.so, sm_100a).
+
+Argument marshalling only: every step of the decode path runs in the CUDA
+kernels behind the C ABI declared in ``include/eta.h``.  PyTorch provides the
+device memory and the stream.  The functions mirror the C entry points:
+
+    eta_block_summary_update(...)   refresh per-block metadata after an append
+    eta_decode_workspace_size(...)  bytes of scratch for a decode call
+    eta_decode(...)                 one decode step (screen, attend, merge)
+    eta_read_device_status(...)     read and clear the device status word
+    eta_status_string(code), eta_build_info()
+
+There is no fallback: if libeta.so is missing or fails to load, importing
+this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Dict, Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libeta.so")
+
+ETA_OK = 0
+ETA_ERR_INVALID_ARG = 1
+ETA_ERR_UNSUPPORTED = 2
+ETA_ERR_WORKSPACE = 3
+ETA_ERR_CUDA = 4
+ETA_ERR_DEVICE_TIMEOUT = 5
+ETA_ERR_DEVICE_RANGE = 6
+
+ETA_F32 = 0
+ETA_BF16 = 1
+ETA_TAU_LEARNED = 0
+ETA_TAU_CALIBRATED = 1
+ETA_ATTEND_AUTO = 0
+ETA_ATTEND_SIMT = 1
+ETA_ATTEND_TC = 2
+
+
+class EtaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {eta_status_string(code)} (status {code})")
+        self.code = code
+
+
+class eta_cache_desc(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int), ("block_size", ctypes.c_int), ("max_ctx", ctypes.c_int),
+        ("kv_dtype", ctypes.c_int), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p),
+    ]
+
+
+class eta_summary_desc(ctypes.Structure):
+    _fields_ = [("mu", ctypes.c_void_p), ("sigma", ctypes.c_void_p), ("max_norm", ctypes.c_void_p)]
+
+
+class eta_decode_params(ctypes.Structure):
+    _fields_ = [
+        ("cache", eta_cache_desc), ("summary", eta_summary_desc), ("q", ctypes.c_void_p),
+        ("tau_mode", ctypes.c_int), ("w_tau", ctypes.c_void_p), ("b_tau", ctypes.c_void_p),
+        ("c_tau", ctypes.c_void_p), ("scale", ctypes.c_float), ("beta", ctypes.c_float),
+        ("offset_a", ctypes.c_float), ("z", ctypes.c_float), ("n_local_blocks", ctypes.c_int),
+        ("screen_enabled", ctypes.c_int), ("attend_impl", ctypes.c_int), ("out", ctypes.c_void_p),
+        ("lse", ctypes.c_void_p), ("admitted_count", ctypes.c_void_p), ("union_count", ctypes.c_void_p),
+        ("union_list", ctypes.c_void_p), ("union_mask", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
+        ("workspace_bytes", ctypes.c_size_t), ("timing_events", ctypes.c_void_p * 4),
+    ]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run learned_threshold_sparse_b200.build.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER
+    lib.eta_block_summary_update.argtypes = [P(eta_cache_desc), P(eta_summary_desc), ctypes.c_void_p,
+                                             ctypes.c_int, ctypes.c_void_p]
+    lib.eta_block_summary_update.restype = ctypes.c_int
+    lib.eta_decode_workspace_size.argtypes = [P(eta_decode_params), P(ctypes.c_size_t)]
+    lib.eta_decode_workspace_size.restype = ctypes.c_int
+    lib.eta_decode.argtypes = [P(eta_decode_params), ctypes.c_void_p]
+    lib.eta_decode.restype = ctypes.c_int
+    lib.eta_read_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    lib.eta_read_device_status.restype = ctypes.c_int
+    lib.eta_status_string.argtypes = [ctypes.c_int]
+    lib.eta_status_string.restype = ctypes.c_char_p
+    lib.eta_build_info.argtypes = []
+    lib.eta_build_info.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+SYMBOLS = ("eta_block_summary_update", "eta_decode_workspace_size", "eta_decode",
+           "eta_read_device_status", "eta_status_string", "eta_build_info")
+
+
+def library():
+    return _lib
+
+
+def eta_status_string(code: int) -> str:
+    return _lib.eta_status_string(int(code)).decode()
+
+
+def eta_build_info() -> str:
+    return _lib.eta_build_info().decode()
+
+
+# ------------------------------------------------------------ marshalling
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream: Optional[torch.cuda.Stream]):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _kv_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return ETA_F32
+    if t.dtype == torch.bfloat16:
+        return ETA_BF16
+    raise TypeError(f"unsupported K/V dtype {t.dtype}")
+
+
+def cache_desc(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, n_q_heads: int,
+               block_size: int) -> eta_cache_desc:
+    B, Hkv, Tmax, d = k.shape
+    return eta_cache_desc(B, n_q_heads, Hkv, d, block_size, Tmax, _kv_dtype(k), k.data_ptr(), v.data_ptr(),
+                          seq_lens.data_ptr())
+
+
+def alloc_summary(batch: int, n_kv_heads: int, max_ctx: int, head_dim: int, block_size: int,
+                  device="cuda") -> Dict[str, torch.Tensor]:
+    nb = (max_ctx + block_size - 1) // block_size
+    return {
+        "mu": torch.zeros((batch, n_kv_heads, nb, head_dim), dtype=torch.float16, device=device),
+        "sigma": torch.zeros((batch, n_kv_heads, nb, head_dim), dtype=torch.float16, device=device),
+        "max_norm": torch.zeros((batch, n_kv_heads, nb), dtype=torch.float32, device=device),
+    }
+
+
+def eta_block_summary_update(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor,
+                             summary: Dict[str, torch.Tensor], block_size: int,
+                             first_token: torch.Tensor, max_blocks: int, n_q_heads: Optional[int] = None,
+                             stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Recompute the metadata of the blocks at or after first_token[i] (at most
+    max_blocks per sequence)."""
+    cache = cache_desc(k, v, seq_lens, n_q_heads or k.shape[1], block_size)
+    summ = eta_summary_desc(summary["mu"].data_ptr(), summary["sigma"].data_ptr(),
+                            summary["max_norm"].data_ptr())
+    rc = _lib.eta_block_summary_update(ctypes.byref(cache), ctypes.byref(summ),
+                                       ctypes.c_void_p(first_token.data_ptr()), int(max_blocks),
+                                       _stream_handle(stream))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_block_summary_update")
+
+
+def make_params(q, k, v, seq_lens, summary, block_size, tau_mode, w_tau=None, b_tau=None,
+                c_tau=None, scale=None, beta=5.0, offset_a=0.0, z=2.0, n_local_blocks=2,
+                screen_enabled=True, attend_impl=ETA_ATTEND_AUTO, out=None, lse=None,
+                admitted_count=None, union_count=None, union_list=None, union_mask=None,
+                workspace=None, events=None) -> eta_decode_params:
+    B, Hq, d = q.shape
+    p = eta_decode_params()
+    p.cache = cache_desc(k, v, seq_lens, Hq, block_size)
+    if summary is not None:
+        p.summary = eta_summary_desc(summary["mu"].data_ptr(), summary["sigma"].data_ptr(),
+                                     summary["max_norm"].data_ptr())
+    p.q = q.data_ptr()
+    p.tau_mode = ETA_TAU_LEARNED if tau_mode in ("learned", ETA_TAU_LEARNED) else ETA_TAU_CALIBRATED
+    p.w_tau = None if w_tau is None else w_tau.data_ptr()
+    p.b_tau = None if b_tau is None else b_tau.data_ptr()
+    p.c_tau = None if c_tau is None else c_tau.data_ptr()
+    p.scale = float(1.0 / math.sqrt(d) if scale is None else scale)
+    p.beta = float(beta)
+    p.offset_a = float(offset_a)
+    p.z = float(z)
+    p.n_local_blocks = int(n_local_blocks)
+    p.screen_enabled = 1 if screen_enabled else 0
+    p.attend_impl = int(attend_impl)
+    p.out = None if out is None else out.data_ptr()
+    p.lse = None if lse is None else lse.data_ptr()
+    p.admitted_count = None if admitted_count is None else admitted_count.data_ptr()
+    p.union_count = None if union_count is None else union_count.data_ptr()
+    p.union_list = None if union_list is None else union_list.data_ptr()
+    p.union_mask = None if union_mask is None else union_mask.data_ptr()
+    if workspace is not None:
+        p.workspace = workspace.data_ptr()
+        p.workspace_bytes = workspace.numel() * workspace.element_size()
+    if events is not None:
+        for j, e in enumerate(events):
+            p.timing_events[j] = None if e is None else e.cuda_event
+    return p
+
+
+def eta_decode_workspace_size(params: eta_decode_params) -> int:
+    n = ctypes.c_size_t(0)
+    rc = _lib.eta_decode_workspace_size(ctypes.byref(params), ctypes.byref(n))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_decode_workspace_size")
+    return int(n.value)
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """Zero-filled workspace (the leading status word must start at zero)."""
+    return torch.zeros(((nbytes + 255) // 256) * 256, dtype=torch.uint8, device=device)
+
+
+def eta_decode(params: eta_decode_params, stream: Optional[torch.cuda.Stream] = None) -> None:
+    rc = _lib.eta_decode(ctypes.byref(params), _stream_handle(stream))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_decode")
+
+
+def eta_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
+    return int(_lib.eta_read_device_status(ctypes.c_void_p(workspace.data_ptr()), _stream_handle(stream)))
+
+
+def decode(q, k, v, seq_lens, summary, block_size, tau_mode, *, w_tau=None, b_tau=None, c_tau=None,
+           scale=None, beta=5.0, offset_a=0.0, z=2.0, n_local_blocks=2, screen_enabled=True,
+           attend_impl=ETA_ATTEND_AUTO, selection=False, workspace=None, out=None, lse=None,
+           events=None, stream=None) -> Dict[str, torch.Tensor]:
+    """Allocate outputs (and the workspace if not given) with torch and run one
+    decode step.  Returns {"out", "lse", "workspace"} plus, with selection=True,
+    {"admitted_count", "union_count", "union_list", "union_mask"}."""
+    B, Hq, d = q.shape
+    Hkv, Tmax = k.shape[1], k.shape[2]
+    nb = (Tmax + block_size - 1) // block_size
+    dev = q.device
+    res = {"out": out if out is not None else torch.empty_like(q),
+           "lse": lse if lse is not None else torch.empty((B, Hq), dtype=torch.float32, device=dev)}
+    if selection:
+        res["admitted_count"] = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+        res["union_count"] = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
+        res["union_list"] = torch.empty((B, Hkv, nb), dtype=torch.int32, device=dev)
+        res["union_mask"] = torch.empty((B, Hkv, nb), dtype=torch.int32, device=dev)
+    kw = dict(w_tau=w_tau, b_tau=b_tau, c_tau=c_tau, scale=scale, beta=beta, offset_a=offset_a, z=z,
+              n_local_blocks=n_local_blocks, screen_enabled=screen_enabled, attend_impl=attend_impl,
+              out=res["out"], lse=res["lse"], admitted_count=res.get("admitted_count"),
+              union_count=res.get("union_count"), union_list=res.get("union_list"),
+              union_mask=res.get("union_mask"), events=events)
+    params = make_params(q, k, v, seq_lens, summary, block_size, tau_mode, **kw)
+    if workspace is None:
+        workspace = alloc_workspace(eta_decode_workspace_size(params), dev)
+    params.workspace = workspace.data_ptr()
+    params.workspace_bytes = workspace.numel()
+    eta_decode(params, stream)
+    res["workspace"] = workspace
+    return res

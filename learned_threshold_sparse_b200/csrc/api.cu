@@ -1,0 +1,307 @@
+// C ABI of the ETA decode library: host-side validation, workspace layout and
+// the stream-ordered launch sequence
+//   screen (+ rescue) -> attention over the admitted union -> merge (+ export).
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "eta_internal.h"
+
+namespace eta {
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+eta_status check_cache(const eta_cache_desc* c) {
+  if (!c) return ETA_ERR_INVALID_ARG;
+  if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 || c->max_ctx < 1 || c->block_size < 1)
+    return ETA_ERR_INVALID_ARG;
+  if (c->n_q_heads % c->n_kv_heads != 0) return ETA_ERR_INVALID_ARG;
+  if (c->kv_dtype != ETA_F32 && c->kv_dtype != ETA_BF16) return ETA_ERR_INVALID_ARG;
+  if (c->batch > 65535 || c->n_kv_heads > 65535 || c->n_q_heads > 65535) return ETA_ERR_UNSUPPORTED;
+  const int G = c->n_q_heads / c->n_kv_heads;
+  if (c->head_dim != 64 && c->head_dim != 128) return ETA_ERR_UNSUPPORTED;
+  if (c->block_size != 16 && c->block_size != 32 && c->block_size != 64 && c->block_size != 128)
+    return ETA_ERR_UNSUPPORTED;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return ETA_ERR_UNSUPPORTED;
+  const long long nbmax = (static_cast<long long>(c->max_ctx) + c->block_size - 1) / c->block_size;
+  if (nbmax > kMaxBlocksPerSeq) return ETA_ERR_UNSUPPORTED;
+  if (!c->k_cache || !c->v_cache || !c->seq_lens) return ETA_ERR_INVALID_ARG;
+  if (!aligned(c->k_cache, 16) || !aligned(c->v_cache, 16) || !aligned(c->seq_lens, 4))
+    return ETA_ERR_INVALID_ARG;
+  return ETA_OK;
+}
+
+eta_status check_summary(const eta_summary_desc* s) {
+  if (!s || !s->mu || !s->sigma || !s->max_norm) return ETA_ERR_INVALID_ARG;
+  if (!aligned(s->mu, 16) || !aligned(s->sigma, 16) || !aligned(s->max_norm, 4)) return ETA_ERR_INVALID_ARG;
+  return ETA_OK;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+eta_status make_shape(const eta_decode_params* p, Shape* out) {
+  const eta_cache_desc& c = p->cache;
+  Shape s;
+  s.B = c.batch;
+  s.Hq = c.n_q_heads;
+  s.Hkv = c.n_kv_heads;
+  s.G = c.n_q_heads / c.n_kv_heads;
+  s.d = c.head_dim;
+  s.b = c.block_size;
+  s.max_ctx = c.max_ctx;
+  s.nbmax = (c.max_ctx + c.block_size - 1) / c.block_size;
+  s.elt = c.kv_dtype == ETA_F32 ? 4 : 2;
+  s.nseg = s.B * s.Hkv;
+  // Screen CTAs cover `chunk` blocks; keep the number of (segment, chunk)
+  // pairs <= 4096 so the attention kernel's prefix table fits in shared memory.
+  int chunk = 32;
+  while (static_cast<long long>(s.nseg) * ((s.nbmax + chunk - 1) / chunk) > 4096 && chunk < 1024) chunk *= 2;
+  s.chunk = chunk;
+  s.nchunks = (s.nbmax + chunk - 1) / chunk;
+  if (static_cast<long long>(s.nseg) * s.nchunks > 16384) return ETA_ERR_UNSUPPORTED;
+  s.list_stride = s.nchunks * chunk;
+  s.rescue = (p->n_local_blocks < 0 && p->screen_enabled) ? 1 : 0;
+  const bool tc_ok = attend_tc_supported(s);
+  if (p->attend_impl == ETA_ATTEND_TC && !tc_ok) return ETA_ERR_UNSUPPORTED;
+  s.attend_kind = (p->attend_impl == ETA_ATTEND_SIMT || !tc_ok) ? ETA_ATTEND_SIMT : ETA_ATTEND_TC;
+  const int sms = sm_count();
+  if (sms <= 0) return ETA_ERR_CUDA;
+  if (s.attend_kind == ETA_ATTEND_SIMT) {
+    if (attend_simt_smem(s) == 0) return ETA_ERR_UNSUPPORTED;
+    s.attend_ctas = sms * attend_simt_ctas_per_sm(s);
+  } else {
+    if (attend_tc_smem(s) == 0) return ETA_ERR_UNSUPPORTED;
+    s.attend_ctas = sms;
+  }
+  *out = s;
+  return ETA_OK;
+}
+
+eta_status check_params(const eta_decode_params* p) {
+  if (!p) return ETA_ERR_INVALID_ARG;
+  eta_status st = check_cache(&p->cache);
+  if (st != ETA_OK) return st;
+  if (p->screen_enabled) {
+    st = check_summary(&p->summary);
+    if (st != ETA_OK) return st;
+  }
+  if (!p->q || !aligned(p->q, 16) || !p->out || !aligned(p->out, 16)) return ETA_ERR_INVALID_ARG;
+  if (p->tau_mode == ETA_TAU_LEARNED) {
+    if (!p->w_tau || !p->b_tau || !aligned(p->w_tau, 4) || !aligned(p->b_tau, 4)) return ETA_ERR_INVALID_ARG;
+  } else if (p->tau_mode == ETA_TAU_CALIBRATED) {
+    if (!p->c_tau || !aligned(p->c_tau, 4)) return ETA_ERR_INVALID_ARG;
+  } else {
+    return ETA_ERR_INVALID_ARG;
+  }
+  if (!(p->scale > 0.f) || !isfinite(p->scale)) return ETA_ERR_INVALID_ARG;
+  if (!(p->beta > 0.f) || !isfinite(p->beta)) return ETA_ERR_INVALID_ARG;
+  if (!isfinite(p->offset_a)) return ETA_ERR_INVALID_ARG;
+  if (!(p->z > 0.f)) return ETA_ERR_INVALID_ARG;  // +inf allowed, NaN rejected
+  if (p->n_local_blocks < -1) return ETA_ERR_INVALID_ARG;
+  if (p->attend_impl < ETA_ATTEND_AUTO || p->attend_impl > ETA_ATTEND_TC) return ETA_ERR_INVALID_ARG;
+  if (p->lse && !aligned(p->lse, 4)) return ETA_ERR_INVALID_ARG;
+  if ((p->admitted_count && !aligned(p->admitted_count, 4)) || (p->union_count && !aligned(p->union_count, 4)) ||
+      (p->union_list && !aligned(p->union_list, 4)) || (p->union_mask && !aligned(p->union_mask, 4)))
+    return ETA_ERR_INVALID_ARG;
+  return ETA_OK;
+}
+
+}  // namespace
+
+Workspace workspace_layout(const Shape& s) {
+  Workspace w;
+  size_t off = 0;
+  w.status = off;
+  off = align256(off + 16);
+  w.tau = off;
+  off = align256(off + static_cast<size_t>(s.B) * s.Hq * sizeof(float));
+  w.chunk_count = off;
+  off = align256(off + static_cast<size_t>(s.nseg) * s.nchunks * sizeof(int));
+  w.chunk_list = off;
+  off = align256(off + static_cast<size_t>(s.nseg) * s.list_stride * sizeof(int) + 4 * sizeof(int));
+  w.head_count = off;
+  off = align256(off + static_cast<size_t>(s.B) * s.Hq * sizeof(int));
+  w.head_best = off;
+  off = align256(off + static_cast<size_t>(s.B) * s.Hq * sizeof(unsigned long long));
+  w.seg_start = off;
+  off = align256(off + static_cast<size_t>(s.nseg + 1) * sizeof(int));
+  w.partials = off;
+  off = align256(off + static_cast<size_t>(s.nseg + s.attend_ctas) * s.G * (s.d + 2) * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+}  // namespace eta
+
+using namespace eta;
+
+extern "C" {
+
+const char* eta_status_string(eta_status s) {
+  switch (s) {
+    case ETA_OK: return "ok";
+    case ETA_ERR_INVALID_ARG: return "invalid argument";
+    case ETA_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case ETA_ERR_WORKSPACE: return "workspace missing or too small";
+    case ETA_ERR_CUDA: return "CUDA runtime error";
+    case ETA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
+    case ETA_ERR_DEVICE_RANGE: return "a device-resident length was out of range (clamped)";
+  }
+  return "unknown status";
+}
+
+const char* eta_build_info(void) {
+  return "eta decode library: sm_100a; kernels: block_summary, screen, rescue, attend_simt, attend_tc, "
+         "combine, export";
+}
+
+eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summary_desc* summary,
+                                    const int* first_token, int max_blocks, void* stream) {
+  eta_status st = check_cache(cache);
+  if (st != ETA_OK) return st;
+  st = check_summary(summary);
+  if (st != ETA_OK) return st;
+  if (!first_token || !aligned(first_token, 4)) return ETA_ERR_INVALID_ARG;
+  const int nbmax = (cache->max_ctx + cache->block_size - 1) / cache->block_size;
+  if (max_blocks < 1 || max_blocks > nbmax) return ETA_ERR_INVALID_ARG;
+  SummaryArgs a;
+  a.k = cache->k_cache;
+  a.seq_lens = cache->seq_lens;
+  a.first_token = first_token;
+  a.mu = static_cast<uint16_t*>(summary->mu);
+  a.sigma = static_cast<uint16_t*>(summary->sigma);
+  a.max_norm = summary->max_norm;
+  a.B = cache->batch;
+  a.Hkv = cache->n_kv_heads;
+  a.d = cache->head_dim;
+  a.b = cache->block_size;
+  a.max_ctx = cache->max_ctx;
+  a.nbmax = nbmax;
+  a.elt = cache->kv_dtype == ETA_F32 ? 4 : 2;
+  a.max_blocks = max_blocks;
+  return launch_summary(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+eta_status eta_decode_workspace_size(const eta_decode_params* p, size_t* bytes) {
+  if (!bytes) return ETA_ERR_INVALID_ARG;
+  eta_status st = check_params(p);
+  if (st != ETA_OK) return st;
+  Shape s;
+  st = make_shape(p, &s);
+  if (st != ETA_OK) return st;
+  *bytes = workspace_layout(s).total;
+  return ETA_OK;
+}
+
+eta_status eta_decode(const eta_decode_params* p, void* stream) {
+  eta_status st = check_params(p);
+  if (st != ETA_OK) return st;
+  Shape s;
+  st = make_shape(p, &s);
+  if (st != ETA_OK) return st;
+  const Workspace w = workspace_layout(s);
+  if (!p->workspace || !aligned(p->workspace, 256)) return ETA_ERR_WORKSPACE;
+  if (p->workspace_bytes < w.total) return ETA_ERR_WORKSPACE;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(p->workspace);
+  auto ev = [&](int k) {
+    if (p->timing_events[k]) cudaEventRecord(static_cast<cudaEvent_t>(p->timing_events[k]), cs);
+  };
+
+  ScreenArgs sa;
+  sa.q = p->q;
+  sa.w_tau = p->w_tau;
+  sa.b_tau = p->b_tau;
+  sa.c_tau = p->c_tau;
+  sa.mu = static_cast<const uint16_t*>(p->summary.mu);
+  sa.sigma = static_cast<const uint16_t*>(p->summary.sigma);
+  sa.max_norm = p->summary.max_norm;
+  sa.seq_lens = p->cache.seq_lens;
+  sa.tau_mode = p->tau_mode;
+  sa.lwb = p->n_local_blocks;
+  sa.screen_enabled = p->screen_enabled ? 1 : 0;
+  sa.scale = p->scale;
+  sa.offset_a = p->offset_a;
+  sa.z = p->z;
+  sa.s = s;
+  sa.status = reinterpret_cast<unsigned*>(ws + w.status);
+  sa.tau = reinterpret_cast<float*>(ws + w.tau);
+  sa.chunk_count = reinterpret_cast<int*>(ws + w.chunk_count);
+  sa.chunk_list = reinterpret_cast<int*>(ws + w.chunk_list);
+  sa.head_count = reinterpret_cast<int*>(ws + w.head_count);
+  sa.head_best = reinterpret_cast<unsigned long long*>(ws + w.head_best);
+
+  ev(0);
+  if (s.rescue) {
+    if (cudaMemsetAsync(ws + w.head_count, 0, w.seg_start - w.head_count, cs) != cudaSuccess) return ETA_ERR_CUDA;
+  }
+  if (launch_screen(sa, cs) != cudaSuccess) return ETA_ERR_CUDA;
+  if (s.rescue && launch_rescue(sa, cs) != cudaSuccess) return ETA_ERR_CUDA;
+
+  AttendArgs aa;
+  aa.k = p->cache.k_cache;
+  aa.v = p->cache.v_cache;
+  aa.q = p->q;
+  aa.seq_lens = p->cache.seq_lens;
+  aa.tau = sa.tau;
+  aa.chunk_count = sa.chunk_count;
+  aa.chunk_list = sa.chunk_list;
+  aa.scale = p->scale;
+  aa.beta = p->beta;
+  aa.s = s;
+  aa.status = sa.status;
+  aa.seg_start = reinterpret_cast<int*>(ws + w.seg_start);
+  aa.partials = reinterpret_cast<float*>(ws + w.partials);
+  ev(1);
+  const cudaError_t ea = s.attend_kind == ETA_ATTEND_TC ? launch_attend_tc(aa, cs) : launch_attend_simt(aa, cs);
+  if (ea != cudaSuccess) return ETA_ERR_CUDA;
+
+  CombineArgs ca;
+  ca.seg_start = aa.seg_start;
+  ca.partials = aa.partials;
+  ca.s = s;
+  ca.out = p->out;
+  ca.lse = p->lse;
+  ev(2);
+  if (launch_combine(ca, cs) != cudaSuccess) return ETA_ERR_CUDA;
+
+  if (p->admitted_count || p->union_count || p->union_list || p->union_mask) {
+    ExportArgs xa;
+    xa.chunk_count = sa.chunk_count;
+    xa.chunk_list = sa.chunk_list;
+    xa.seq_lens = p->cache.seq_lens;
+    xa.s = s;
+    xa.admitted_count = p->admitted_count;
+    xa.union_count = p->union_count;
+    xa.union_list = p->union_list;
+    xa.union_mask = p->union_mask;
+    if (launch_export(xa, cs) != cudaSuccess) return ETA_ERR_CUDA;
+  }
+  ev(3);
+  return ETA_OK;
+}
+
+eta_status eta_read_device_status(void* workspace, void* stream) {
+  if (!workspace || !aligned(workspace, 256)) return ETA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, cs) != cudaSuccess) return ETA_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return ETA_ERR_CUDA;
+  const unsigned zero = 0;
+  if (cudaMemcpyAsync(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice, cs) != cudaSuccess) return ETA_ERR_CUDA;
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return ETA_ERR_CUDA;
+  if (word & kStatusTimeout) return ETA_ERR_DEVICE_TIMEOUT;
+  if (word & kStatusRange) return ETA_ERR_DEVICE_RANGE;
+  return ETA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,484 @@
+// Split-KV attention over the admitted (GQA-union) blocks, CUDA-core version.
+//
+// Source: Elastic Threshold Attention,
+//   Appendix F.1 step 2   a listed block is fetched once for the G query heads
+//                         of its KV head; each head accumulates only the
+//                         blocks it admitted (head-mask bit),
+//   Appendix G.1          S = q k / sqrt(d), S~ = S sigmoid(beta (S - tau~)),
+//                         weights exp(S~) (online softmax in base 2),
+//   Appendix F.2          fp32 accumulation and softmax state,
+//   section 3.2, F.3      split-KV partials (acc, m, l) merged later,
+//   Appendix F.4          tail block: rows >= seq_len are masked.
+//
+// Persistent grid, one CTA per SM.  The global list of admitted units
+// (segment, block, head mask), ordered by (sequence, KV head, block), is cut
+// into equal contiguous ranges, one per CTA, so every CTA streams the same
+// number of K/V blocks whatever the per-sequence densities.  Warp 8 is the
+// producer: it walks the CTA's range and issues 1-D bulk copies (TMA) of the
+// contiguous K and V tiles of each unit into a ring of shared-memory stages
+// guarded by mbarriers.  Warps 0-7 consume: each keeps its own online-softmax
+// state for the G heads; at a segment boundary the eight states are merged
+// and written as one partial per (segment, CTA).
+#include <math.h>
+
+#include "eta_device.cuh"
+
+namespace eta {
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxStages = 8;
+
+struct UnitInfo {
+  int seg, blk, mask, nrows;
+};
+
+template <int ELT, int D, int G>
+struct Cfg {
+  static constexpr int LPR = D * ELT / 16;  // lanes per K/V row (8, 16, 32)
+  static constexpr int RPW = 32 / LPR;      // rows per warp per step
+  static constexpr int EPL = 16 / ELT;      // elements per lane
+  static constexpr int ROWS = kConsumerWarps * RPW;  // rows per step
+  static constexpr int MAX_STEPS = (128 + ROWS - 1) / ROWS;
+  static constexpr int REP = LPR / G;       // lanes holding the same head
+  static_assert(G <= LPR, "group size larger than lanes per row");
+};
+
+struct Smem {
+  size_t kv, bars, info, scratch, prefix, flags, total;
+};
+
+__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline Smem smem_layout(int stages, int b, int d, int elt, int G, int nprefix) {
+  Smem L;
+  L.kv = 0;
+  size_t off = static_cast<size_t>(stages) * 2 * b * d * elt;
+  L.bars = off = align_up(off, 16);
+  off += (2 * stages + 1) * sizeof(uint64_t);
+  L.info = off = align_up(off, 16);
+  off += stages * sizeof(UnitInfo);
+  L.scratch = off = align_up(off, 16);
+  off += static_cast<size_t>(kConsumerWarps) * G * (d + 2) * sizeof(float);
+  L.prefix = off = align_up(off, 16);
+  off += static_cast<size_t>(nprefix + 1) * sizeof(int);
+  L.flags = off = align_up(off, 16);
+  off += 16 + kMaxStages * sizeof(int);
+  L.total = align_up(off, 128);
+  return L;
+}
+
+// Reduce G values across the LPR lanes of one row, halving the values held
+// per stage; afterwards lane sub holds head sub / (LPR / G).
+template <int G, int LPR>
+__device__ __forceinline__ float row_transpose_reduce(float (&v)[G], int sub) {
+  int n = G;
+#pragma unroll
+  for (int o = LPR / 2; o >= 1; o >>= 1) {
+    if (n > 1) {
+      const bool upper = (sub & o) != 0;
+      const int half = n >> 1;
+#pragma unroll
+      for (int j = 0; j < (G > 1 ? G / 2 : 1); ++j) {
+        if (j < half) {
+          const float send = upper ? v[j] : v[j + half];
+          const float keep = upper ? v[j + half] : v[j];
+          v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      n = half;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    }
+  }
+  return v[0];
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned* status,
+                                              volatile int* abort_flag) {
+  if (dev::mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!dev::mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > dev::kWaitCycles) {
+      atomicOr(status, kStatusTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+template <int ELT, int D, int G>
+__global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, int stages) {
+  using C = Cfg<ELT, D, G>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const Shape& s = a.s;
+  const int nprefix = s.nseg * s.nchunks;
+  const Smem L = smem_layout(stages, s.b, D, ELT, G, nprefix);
+  uint8_t* kv = smem + L.kv;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty = full + stages;
+  uint64_t* flush_bar = empty + stages;  // consumer-warp rendezvous (count 8)
+  UnitInfo* info = reinterpret_cast<UnitInfo*>(smem + L.info);
+  float* scratch = reinterpret_cast<float*>(smem + L.scratch);
+  int* prefix = reinterpret_cast<int*>(smem + L.prefix);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L.flags);
+  int* issued_parity = reinterpret_cast<int*>(smem + L.flags + 16);  // per stage, -1 = never
+  const size_t tile_bytes = static_cast<size_t>(s.b) * D * ELT;
+
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  if (t == 0) {
+    for (int k = 0; k < stages; ++k) {
+      dev::mbar_init(&full[k], 1);
+      dev::mbar_init(&empty[k], kConsumerWarps);
+      issued_parity[k] = -1;
+    }
+    dev::mbar_init(flush_bar, kConsumerWarps);
+    *abort_flag = 0;
+    dev::fence_barrier_init();
+  }
+
+  // Everything below reads what the screen wrote.
+  dev::pdl_wait();
+  dev::pdl_trigger();
+
+  // Exclusive prefix of the per-chunk entry counts, in (segment, chunk) order.
+  {
+    const int per = (nprefix + kThreads - 1) / kThreads;
+    const int lo = min(nprefix, t * per), hi = min(nprefix, lo + per);
+    int sum = 0;
+    for (int x = lo; x < hi; ++x) sum += a.chunk_count[x];
+    // block-wide exclusive scan of the per-thread sums
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    __shared__ int s_warp[kConsumerWarps + 1];
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int woff = 0;
+    for (int k = 0; k < warp; ++k) woff += s_warp[k];
+    int run = woff + incl - sum;
+    for (int x = lo; x < hi; ++x) {
+      const int cnt = a.chunk_count[x];
+      prefix[x] = run;
+      run += cnt;
+    }
+    if (t == kThreads - 1) prefix[nprefix] = woff + incl;
+  }
+  __syncthreads();
+
+  const long long U = prefix[nprefix];
+  const long long N = gridDim.x;
+  const long long u0 = U * blockIdx.x / N;
+  const long long u1 = U * (blockIdx.x + 1) / N;
+  const int nunits = static_cast<int>(u1 - u0);
+  if (blockIdx.x == 0) {
+    for (int sg = t; sg <= s.nseg; sg += kThreads) a.seg_start[sg] = prefix[sg * s.nchunks];
+  }
+  if (nunits == 0) return;
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    // chunk x holding unit u0: last x with prefix[x] <= u0
+    int lo = 0, hi = nprefix;  // invariant prefix[lo] <= u0 < prefix[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (prefix[mid] <= u0) lo = mid; else hi = mid;
+    }
+    int x = lo;
+    int idx = static_cast<int>(u0 - prefix[x]);
+    int remaining = nunits;
+    int stage = 0;
+    uint32_t phase = 0;
+    int cur_seg = -1, T = 0;
+    const uint8_t* kbase = nullptr;
+    const uint8_t* vbase = nullptr;
+    bool ok = true;
+    while (remaining > 0 && ok) {
+      const int cnt = prefix[x + 1] - prefix[x];
+      const int take = min(cnt - idx, remaining);
+      if (take <= 0) { ++x; idx = 0; continue; }
+      const int seg = x / s.nchunks;
+      const int cin = x - seg * s.nchunks;
+      if (seg != cur_seg) {
+        cur_seg = seg;
+        const int i = seg / s.Hkv;
+        int tt = a.seq_lens[i];
+        T = tt < 0 ? 0 : (tt > s.max_ctx ? s.max_ctx : tt);
+        const size_t row0 = static_cast<size_t>(seg) * s.max_ctx;
+        kbase = static_cast<const uint8_t*>(a.k) + row0 * D * ELT;
+        vbase = static_cast<const uint8_t*>(a.v) + row0 * D * ELT;
+      }
+      const int* list = a.chunk_list + static_cast<size_t>(seg) * s.list_stride +
+                        static_cast<size_t>(cin) * s.chunk + idx;
+      for (int j0 = 0; j0 < take && ok; j0 += 32) {
+        const int nn = min(32, take - j0);
+        const int e = lane < nn ? list[j0 + lane] : 0;
+        for (int jj = 0; jj < nn; ++jj) {
+          const int ent = __shfl_sync(0xffffffffu, e, jj);
+          if (lane == 0) {
+            if (!wait_or_abort(&empty[stage], phase ^ 1u, a.status, abort_flag)) {
+              ok = false;
+            } else {
+              const int blk = ent & kMaxBlocksPerSeq;
+              const int nrows = min(s.b, T - blk * s.b);
+              info[stage] = UnitInfo{seg, blk, static_cast<int>(static_cast<unsigned>(ent) >> kEntryBlockBits), nrows};
+              const uint32_t bytes = static_cast<uint32_t>(nrows) * D * ELT;
+              dev::mbar_arrive_expect_tx(&full[stage], 2u * bytes);
+              const size_t off = static_cast<size_t>(blk) * s.b * D * ELT;
+              dev::bulk_g2s(kv + static_cast<size_t>(stage) * 2 * tile_bytes, kbase + off, bytes, &full[stage]);
+              dev::bulk_g2s(kv + static_cast<size_t>(stage) * 2 * tile_bytes + tile_bytes, vbase + off, bytes,
+                            &full[stage]);
+              issued_parity[stage] = static_cast<int>(phase);
+            }
+          }
+          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+          if (!ok) break;
+          if (++stage == stages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      remaining -= take;
+      idx = 0;
+      ++x;
+    }
+    if (!ok && lane == 0) {
+      // Let the copies already issued land before the CTA exits.
+      for (int k = 0; k < stages; ++k) {
+        if (issued_parity[k] < 0) continue;
+        const long long t0 = clock64();
+        while (!dev::mbar_try_wait(&full[k], static_cast<uint32_t>(issued_parity[k])) &&
+               clock64() - t0 < dev::kWaitCycles) {
+        }
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers
+  const int rg = lane / C::LPR;        // row within the warp's step
+  const int sub = lane - rg * C::LPR;  // 16-byte column slot of the row
+  const int hh = sub / C::REP;         // head this lane reduces to
+  const float scale = a.scale, beta = a.beta;
+
+  float q[G][C::EPL], acc[G][C::EPL];
+  float m_run = -INFINITY, l_run = 0.f, tau_h = 0.f;
+  int cur_seg = -1;
+  int stage = 0;
+  uint32_t phase = 0;
+
+  // Rendezvous of the 8 consumer warps on flush_bar: the first wait of a flush
+  // completes an even phase, the second an odd one.  Bounded: on a timeout
+  // the flush is abandoned and the kernel winds down.
+  auto rendezvous = [&](uint32_t parity) -> bool {
+    __syncwarp();
+    if (lane == 0) dev::mbar_arrive(flush_bar);
+    return wait_or_abort(flush_bar, parity, a.status, abort_flag);
+  };
+
+  auto flush = [&](int seg) -> bool {
+    // rows of the warp -> one state per warp
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+#pragma unroll
+      for (int e = 0; e < C::EPL; ++e)
+#pragma unroll
+        for (int o = C::LPR; o < 32; o <<= 1) acc[h][e] += __shfl_xor_sync(0xffffffffu, acc[h][e], o);
+#pragma unroll
+    for (int o = C::LPR; o < 32; o <<= 1) l_run += __shfl_xor_sync(0xffffffffu, l_run, o);
+    float* my = scratch + static_cast<size_t>(warp) * G * (D + 2);
+    if (rg == 0) {
+#pragma unroll
+      for (int h = 0; h < G; ++h)
+#pragma unroll
+        for (int e = 0; e < C::EPL; ++e) my[h * (D + 2) + sub * C::EPL + e] = acc[h][e];
+      if (sub % C::REP == 0) {
+        my[hh * (D + 2) + D] = m_run;
+        my[hh * (D + 2) + D + 1] = l_run;
+      }
+    }
+    if (!rendezvous(0u)) return false;
+    float* part = a.partials + static_cast<size_t>(seg + blockIdx.x) * G * (D + 2);
+    for (int x = t; x < G * D; x += kConsumerWarps * 32) {
+      const int h = x / D, e = x - h * D;
+      float mstar = -INFINITY;
+      for (int w = 0; w < kConsumerWarps; ++w) mstar = fmaxf(mstar, scratch[(w * G + h) * (D + 2) + D]);
+      float sum = 0.f, lsum = 0.f;
+      if (mstar != -INFINITY) {
+        for (int w = 0; w < kConsumerWarps; ++w) {
+          const float* ws = scratch + (w * G + h) * (D + 2);
+          const float f = ws[D] == -INFINITY ? 0.f : dev::fast_exp2(ws[D] - mstar);
+          sum = fmaf(f, ws[e], sum);
+          lsum = fmaf(f, ws[D + 1], lsum);
+        }
+      }
+      part[h * (D + 2) + e] = sum;
+      if (e == 0) {
+        part[h * (D + 2) + D] = mstar;
+        part[h * (D + 2) + D + 1] = lsum;
+      }
+    }
+    return rendezvous(1u);
+  };
+
+  for (int u = 0; u < nunits; ++u) {
+    if (!wait_or_abort(&full[stage], phase, a.status, abort_flag)) break;
+    const UnitInfo in = info[stage];
+    if (in.seg != cur_seg) {
+      if (cur_seg >= 0 && !flush(cur_seg)) break;
+      cur_seg = in.seg;
+      const int i = in.seg / s.Hkv, g = in.seg - i * s.Hkv;
+      const size_t qrow = static_cast<size_t>(i) * s.Hq + g * G;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        float tmp[C::EPL];
+        dev::Row16<ELT>::load(static_cast<const uint8_t*>(a.q) + ((qrow + h) * D + sub * C::EPL) * ELT, tmp);
+#pragma unroll
+        for (int e = 0; e < C::EPL; ++e) {
+          q[h][e] = tmp[e];
+          acc[h][e] = 0.f;
+        }
+      }
+      tau_h = a.tau[qrow + hh];
+      m_run = -INFINITY;
+      l_run = 0.f;
+    }
+    const uint8_t* Kt = kv + static_cast<size_t>(stage) * 2 * tile_bytes;
+    const uint8_t* Vt = Kt + tile_bytes;
+    const int nrows = in.nrows;
+    const bool head_on = (in.mask >> hh) & 1;
+    const int nsteps = (nrows + C::ROWS - 1) / C::ROWS;
+
+    float st[C::MAX_STEPS];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < C::MAX_STEPS; ++k) {
+      st[k] = -INFINITY;
+      if (k < nsteps) {
+        const int r = k * C::ROWS + warp * C::RPW + rg;
+        const bool valid = r < nrows;
+        float kx[C::EPL];
+        dev::Row16<ELT>::load(Kt + (static_cast<size_t>(valid ? r : 0) * D + sub * C::EPL) * ELT, kx);
+        float part[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          float acc_d = 0.f;
+#pragma unroll
+          for (int e = 0; e < C::EPL; ++e) acc_d = fmaf(q[h][e], kx[e], acc_d);
+          part[h] = acc_d;
+        }
+        const float dot = row_transpose_reduce<G, C::LPR>(part, sub);
+        const float S = dot * scale;
+        const float St = S * dev::logistic(beta * (S - tau_h));
+        st[k] = (valid && head_on) ? St * kLog2e : -INFINITY;
+        mx = fmaxf(mx, st[k]);
+      }
+    }
+#pragma unroll
+    for (int o = C::LPR; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float m_new = fmaxf(m_run, mx);
+    const float alpha = (m_new == -INFINITY || m_run == -INFINITY) ? (m_run == -INFINITY ? 0.f : 1.f)
+                                                                  : dev::fast_exp2(m_run - m_new);
+    float p[C::MAX_STEPS];
+    float psum = 0.f;
+#pragma unroll
+    for (int k = 0; k < C::MAX_STEPS; ++k) {
+      p[k] = (st[k] == -INFINITY) ? 0.f : dev::fast_exp2(st[k] - m_new);
+      psum += p[k];
+    }
+    l_run = l_run * alpha + psum;
+    m_run = m_new;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float ah = __shfl_sync(0xffffffffu, alpha, h * C::REP);
+#pragma unroll
+      for (int e = 0; e < C::EPL; ++e) acc[h][e] *= ah;
+    }
+#pragma unroll
+    for (int k = 0; k < C::MAX_STEPS; ++k) {
+      if (k < nsteps) {
+        const int r = k * C::ROWS + warp * C::RPW + rg;
+        const bool valid = r < nrows;
+        float vx[C::EPL];
+        dev::Row16<ELT>::load(Vt + (static_cast<size_t>(valid ? r : 0) * D + sub * C::EPL) * ELT, vx);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          const float ph = __shfl_sync(0xffffffffu, p[k], rg * C::LPR + h * C::REP);
+          if (valid) {
+#pragma unroll
+            for (int e = 0; e < C::EPL; ++e) acc[h][e] = fmaf(ph, vx[e], acc[h][e]);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) dev::mbar_arrive(&empty[stage]);
+    if (++stage == stages) { stage = 0; phase ^= 1u; }
+  }
+  if (cur_seg >= 0 && !*abort_flag) flush(cur_seg);
+}
+
+template <int ELT, int D, int G>
+cudaError_t launch_typed(const AttendArgs& a, cudaStream_t st, int stages, size_t smem) {
+  auto kern = attend_simt_kernel<ELT, D, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.s.attend_ctas);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a, stages);
+}
+
+template <int ELT, int D>
+cudaError_t launch_g(const AttendArgs& a, cudaStream_t st, int stages, size_t smem) {
+  switch (a.s.G) {
+    case 1: return launch_typed<ELT, D, 1>(a, st, stages, smem);
+    case 2: return launch_typed<ELT, D, 2>(a, st, stages, smem);
+    case 4: return launch_typed<ELT, D, 4>(a, st, stages, smem);
+    case 8: return launch_typed<ELT, D, 8>(a, st, stages, smem);
+  }
+  return cudaErrorInvalidValue;
+}
+
+constexpr size_t kSmemBudget = 227 * 1024;
+
+int pick_stages(const Shape& s) {
+  for (int st = kMaxStages; st >= 2; --st) {
+    if (smem_layout(st, s.b, s.d, s.elt, s.G, s.nseg * s.nchunks).total <= kSmemBudget) return st;
+  }
+  return 0;
+}
+
+}  // namespace
+
+size_t attend_simt_smem(const Shape& s) {
+  const int st = pick_stages(s);
+  if (st == 0) return 0;
+  return smem_layout(st, s.b, s.d, s.elt, s.G, s.nseg * s.nchunks).total;
+}
+
+int attend_simt_ctas_per_sm(const Shape&) { return 1; }
+
+cudaError_t launch_attend_simt(const AttendArgs& a, cudaStream_t st) {
+  const int stages = pick_stages(a.s);
+  if (stages == 0) return cudaErrorInvalidConfiguration;
+  const size_t smem = smem_layout(stages, a.s.b, a.s.d, a.s.elt, a.s.G, a.s.nseg * a.s.nchunks).total;
+  if (a.s.elt == 2) {
+    return a.s.d == 64 ? launch_g<2, 64>(a, st, stages, smem) : launch_g<2, 128>(a, st, stages, smem);
+  }
+  return a.s.d == 64 ? launch_g<4, 64>(a, st, stages, smem) : launch_g<4, 128>(a, st, stages, smem);
+}
+
+}  // namespace eta

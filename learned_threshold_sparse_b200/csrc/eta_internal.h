@@ -1,0 +1,121 @@
+// Internal declarations shared by the launchers and the C ABI of the ETA
+// decode library.  Not installed; the public interface is include/eta.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "eta.h"
+
+namespace eta {
+
+// Device status word bits (first word of the workspace).
+constexpr unsigned kStatusTimeout = 1u;  // a bounded wait ran out
+constexpr unsigned kStatusRange = 2u;    // a device-resident length was clamped
+
+// List entries written by the screen: block id in the low 24 bits, the
+// admitting heads of the group in the high 8 bits.
+constexpr int kEntryBlockBits = 24;
+constexpr int kMaxBlocksPerSeq = (1 << kEntryBlockBits) - 1;
+
+// Shape of one decode launch, derived on the host from eta_decode_params.
+struct Shape {
+  int B, Hq, Hkv, G, d, b, max_ctx, nbmax;
+  int elt;           // bytes per K/V element
+  int nseg;          // B * Hkv  (one segment = one (sequence, KV head))
+  int chunk;         // blocks screened per screen CTA (multiple of 32)
+  int nchunks;       // chunks per segment
+  int list_stride;   // list entries per segment = nchunks * chunk
+  int attend_ctas;   // persistent attention CTAs
+  int attend_kind;   // ETA_ATTEND_SIMT or ETA_ATTEND_TC
+  int rescue;        // 1 when n_local_blocks < 0 (top-1 rescue may fire)
+};
+
+// Byte offsets of the workspace regions (all 256-byte aligned).
+struct Workspace {
+  size_t status, tau, chunk_count, chunk_list, head_count, head_best, seg_start,
+      partials, total;
+};
+
+Workspace workspace_layout(const Shape& s);
+
+// Arguments of the screen kernel.
+struct ScreenArgs {
+  const void* q;
+  const float* w_tau;
+  const float* b_tau;
+  const float* c_tau;
+  const uint16_t* mu;     // fp16 bits
+  const uint16_t* sigma;  // fp16 bits
+  const float* max_norm;
+  const int* seq_lens;
+  int tau_mode, lwb, screen_enabled;
+  float scale, offset_a, z;
+  Shape s;
+  unsigned* status;
+  float* tau;              // [B, Hq] tau~
+  int* chunk_count;        // [nseg, nchunks]
+  int* chunk_list;         // [nseg, list_stride]
+  int* head_count;         // [B, Hq]   (rescue mode)
+  unsigned long long* head_best;  // [B, Hq] (rescue mode)
+};
+
+struct AttendArgs {
+  const void* k;
+  const void* v;
+  const void* q;
+  const int* seq_lens;
+  const float* tau;
+  const int* chunk_count;
+  const int* chunk_list;
+  float scale, beta;
+  Shape s;
+  unsigned* status;
+  int* seg_start;          // [nseg + 1] unit offsets (written by CTA 0)
+  float* partials;         // [nseg + attend_ctas][G][d + 2]
+};
+
+struct CombineArgs {
+  const int* seg_start;
+  const float* partials;
+  Shape s;
+  void* out;
+  float* lse;
+};
+
+struct ExportArgs {
+  const int* chunk_count;
+  const int* chunk_list;
+  const int* seq_lens;
+  Shape s;
+  int* admitted_count;
+  int* union_count;
+  int* union_list;
+  unsigned* union_mask;
+};
+
+struct SummaryArgs {
+  const void* k;
+  const int* seq_lens;
+  const int* first_token;
+  uint16_t* mu;
+  uint16_t* sigma;
+  float* max_norm;
+  int B, Hkv, d, b, max_ctx, nbmax, elt, max_blocks;
+};
+
+// Launchers (each returns the launch's cudaError_t).
+cudaError_t launch_summary(const SummaryArgs& a, cudaStream_t st);
+cudaError_t launch_screen(const ScreenArgs& a, cudaStream_t st);
+cudaError_t launch_rescue(const ScreenArgs& a, cudaStream_t st);
+cudaError_t launch_attend_simt(const AttendArgs& a, cudaStream_t st);
+size_t attend_simt_smem(const Shape& s);
+int attend_simt_ctas_per_sm(const Shape& s);
+cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st);
+size_t attend_tc_smem(const Shape& s);
+bool attend_tc_supported(const Shape& s);
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
+cudaError_t launch_export(const ExportArgs& a, cudaStream_t st);
+
+}  // namespace eta

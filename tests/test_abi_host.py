@@ -1,0 +1,141 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/eta.h declares, and rejects bad arguments before
+launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import learned_threshold_sparse_b200 as eta
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "eta.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(eta_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared_symbols()
+    assert "eta_decode" in names and "eta_block_summary_update" in names
+    lib = eta.library()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(eta.SYMBOLS) | {n for n in names if hasattr(eta, n)}
+    for n in names:
+        assert hasattr(eta, n), f"binding lacks {n}"
+
+
+def test_status_strings():
+    for code in range(7):
+        assert eta.eta_status_string(code)
+    assert "sm_100a" in eta.eta_build_info()
+
+
+def _params(**over):
+    fake = 1 << 20  # aligned, never dereferenced on the host
+    p = eta.eta_decode_params()
+    p.cache = eta.eta_cache_desc(1, 16, 4, 128, 64, 4096, eta.ETA_BF16, fake, fake, fake)
+    p.summary = eta.eta_summary_desc(fake, fake, fake)
+    p.q = fake
+    p.tau_mode = eta.ETA_TAU_CALIBRATED
+    p.c_tau = fake
+    p.scale = 0.088
+    p.beta = 5.0
+    p.z = 2.0
+    p.n_local_blocks = 2
+    p.screen_enabled = 1
+    p.out = fake
+    for k, v in over.items():
+        if "." in k:
+            a, b = k.split(".")
+            setattr(getattr(p, a), b, v)
+        else:
+            setattr(p, k, v)
+    return p
+
+
+@pytest.mark.parametrize("over,code", [
+    ({"cache.head_dim": 96}, eta.ETA_ERR_UNSUPPORTED),
+    ({"cache.block_size": 48}, eta.ETA_ERR_UNSUPPORTED),
+    ({"cache.n_q_heads": 12, "cache.n_kv_heads": 8}, eta.ETA_ERR_INVALID_ARG),
+    ({"cache.n_q_heads": 48, "cache.n_kv_heads": 4}, eta.ETA_ERR_UNSUPPORTED),
+    ({"cache.batch": 0}, eta.ETA_ERR_INVALID_ARG),
+    ({"cache.max_ctx": 0}, eta.ETA_ERR_INVALID_ARG),
+    ({"cache.kv_dtype": 7}, eta.ETA_ERR_INVALID_ARG),
+    ({"cache.k_cache": None}, eta.ETA_ERR_INVALID_ARG),
+    ({"cache.v_cache": (1 << 20) + 8}, eta.ETA_ERR_INVALID_ARG),
+    ({"q": None}, eta.ETA_ERR_INVALID_ARG),
+    ({"out": (1 << 20) + 4}, eta.ETA_ERR_INVALID_ARG),
+    ({"summary.mu": None}, eta.ETA_ERR_INVALID_ARG),
+    ({"tau_mode": eta.ETA_TAU_LEARNED}, eta.ETA_ERR_INVALID_ARG),
+    ({"c_tau": None}, eta.ETA_ERR_INVALID_ARG),
+    ({"scale": 0.0}, eta.ETA_ERR_INVALID_ARG),
+    ({"scale": float("nan")}, eta.ETA_ERR_INVALID_ARG),
+    ({"beta": -1.0}, eta.ETA_ERR_INVALID_ARG),
+    ({"z": 0.0}, eta.ETA_ERR_INVALID_ARG),
+    ({"z": float("nan")}, eta.ETA_ERR_INVALID_ARG),
+    ({"offset_a": float("inf")}, eta.ETA_ERR_INVALID_ARG),
+    ({"n_local_blocks": -2}, eta.ETA_ERR_INVALID_ARG),
+    ({"attend_impl": 9}, eta.ETA_ERR_INVALID_ARG),
+    ({"lse": (1 << 20) + 2}, eta.ETA_ERR_INVALID_ARG),
+])
+def test_invalid_arguments_rejected_before_launch(over, code):
+    p = _params(**over)
+    assert eta.library().eta_decode(ctypes.byref(p), None) == code
+    n = ctypes.c_size_t(0)
+    assert eta.library().eta_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == code
+
+
+def test_null_params():
+    assert eta.library().eta_decode(None, None) == eta.ETA_ERR_INVALID_ARG
+    assert eta.library().eta_decode_workspace_size(None, None) == eta.ETA_ERR_INVALID_ARG
+    assert eta.library().eta_read_device_status(None, None) == eta.ETA_ERR_INVALID_ARG
+
+
+def test_summary_update_validation():
+    fake = 1 << 20
+    c = eta.eta_cache_desc(1, 4, 4, 64, 64, 4096, eta.ETA_F32, fake, fake, fake)
+    s = eta.eta_summary_desc(fake, fake, fake)
+    lib = eta.library()
+    assert lib.eta_block_summary_update(ctypes.byref(c), ctypes.byref(s), None, 1, None) == eta.ETA_ERR_INVALID_ARG
+    assert lib.eta_block_summary_update(ctypes.byref(c), ctypes.byref(s), fake, 0, None) == eta.ETA_ERR_INVALID_ARG
+    assert lib.eta_block_summary_update(ctypes.byref(c), ctypes.byref(s), fake, 65, None) == eta.ETA_ERR_INVALID_ARG
+    s2 = eta.eta_summary_desc(fake + 2, fake, fake)
+    assert lib.eta_block_summary_update(ctypes.byref(c), ctypes.byref(s2), fake, 1, None) == eta.ETA_ERR_INVALID_ARG
+    c2 = eta.eta_cache_desc(1, 4, 4, 80, 64, 4096, eta.ETA_F32, fake, fake, fake)
+    assert lib.eta_block_summary_update(ctypes.byref(c2), ctypes.byref(s), fake, 1, None) == eta.ETA_ERR_UNSUPPORTED
+
+
+def test_struct_layout_matches_header(tmp_path):
+    # Compile a C probe of include/eta.h and compare every field offset and
+    # struct size with the ctypes mirror used by the binding.
+    fields = {
+        "eta_cache_desc": eta.eta_cache_desc,
+        "eta_summary_desc": eta.eta_summary_desc,
+        "eta_decode_params": eta.eta_decode_params,
+    }
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "eta.h"', "int main(void) {"]
+    for sname, cls in fields.items():
+        lines.append(f'printf("{sname} size %zu\\n", sizeof({sname}));')
+        for fname, _ in cls._fields_:
+            lines.append(f'printf("{sname} {fname} %zu\\n", offsetof({sname}, {fname}));')
+    lines.append("return 0; }")
+    src = tmp_path / "probe.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "probe"
+    import subprocess
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {}
+    for ln in out:
+        if ln.strip():
+            a, b, c = ln.split()
+            got[(a, b)] = int(c)
+    for sname, cls in fields.items():
+        assert got[(sname, "size")] == ctypes.sizeof(cls), sname
+        for fname, _ in cls._fields_:
+            assert got[(sname, fname)] == getattr(cls, fname).offset, (sname, fname)
