@@ -214,6 +214,9 @@ def run_eta(args):
     out = torch.empty_like(q)
     lse = torch.empty((wl.batch, wl.n_q_heads), dtype=torch.float32, device=dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in ev:  # materialise the cudaEvent_t handles the library records into
+        e.record()
+    torch.cuda.synchronize()
     params = eta.make_params(q, k, v, seq, summ, wl.block_size, wl.tau_mode, w_tau=w_tau, b_tau=b_tau,
                              c_tau=c_tau, scale=wl.scale, beta=wl.beta, offset_a=wl.offset_a, z=wl.z,
                              n_local_blocks=wl.n_local_blocks, screen_enabled=not args.dense,

@@ -200,6 +200,8 @@ def make_params(q, k, v, seq_lens, summary, block_size, tau_mode, w_tau=None, b_
         p.workspace_bytes = workspace.numel() * workspace.element_size()
     if events is not None:
         for j, e in enumerate(events):
+            if e is not None and not e.cuda_event:
+                e.record()  # torch creates the underlying cudaEvent_t lazily
             p.timing_events[j] = None if e is None else e.cuda_event
     return p
 

@@ -135,7 +135,7 @@ Workspace workspace_layout(const Shape& s) {
   w.seg_start = off;
   off = align256(off + static_cast<size_t>(s.nseg + 1) * sizeof(int));
   w.partials = off;
-  off = align256(off + static_cast<size_t>(s.nseg + s.attend_ctas) * s.G * (s.d + 2) * sizeof(float));
+  off = align256(off + static_cast<size_t>(s.nseg + s.attend_ctas) * s.G * partial_stride(s.d) * sizeof(float));
   w.total = off;
   return w;
 }

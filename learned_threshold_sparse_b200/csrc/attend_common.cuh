@@ -1,0 +1,120 @@
+// Work split shared by the attention kernels.
+//
+// The screen writes, per (segment = (sequence, KV head), chunk), the admitted
+// blocks of the chunk in ascending order plus their count.  Read in
+// (segment, chunk) order these lists form one global sequence of "units"
+// (segment, block, head mask).  Every persistent attention CTA takes an equal
+// contiguous range [U c / N, U (c + 1) / N) of it, so the K/V bytes a CTA
+// streams do not depend on how the densities vary across sequences and heads.
+#pragma once
+
+#include "eta_device.cuh"
+
+namespace eta {
+namespace dev {
+
+struct UnitInfo {
+  int seg, blk, mask, nrows;
+};
+
+// Exclusive prefix of the chunk counts into prefix[0..n] (prefix[n] = total),
+// computed by all `nthreads` threads of the CTA.  Ends with __syncthreads().
+template <int NTHREADS>
+__device__ __forceinline__ void chunk_prefix(const int* __restrict__ counts, int n, int* prefix) {
+  __shared__ int s_warp[NTHREADS / 32];
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int per = (n + NTHREADS - 1) / NTHREADS;
+  const int lo = min(n, t * per), hi = min(n, lo + per);
+  int sum = 0;
+  for (int x = lo; x < hi; ++x) sum += counts[x];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  int woff = 0;
+  for (int k = 0; k < warp; ++k) woff += s_warp[k];
+  int run = woff + incl - sum;
+  for (int x = lo; x < hi; ++x) {
+    const int c = counts[x];
+    prefix[x] = run;
+    run += c;
+  }
+  if (t == NTHREADS - 1) prefix[n] = woff + incl;
+  __syncthreads();
+}
+
+// Walk the units [u0, u0 + nunits) with one warp.  `issue(info)` runs on lane
+// 0 for every unit, in order, and returns false to stop (abort).  Returns
+// false if the walk was stopped or the counts were inconsistent.
+template <class Issue>
+__device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefix, int nprefix, long long u0,
+                                           int nunits, Issue&& issue) {
+  const Shape& s = a.s;
+  const int lane = threadIdx.x & 31;
+  int lo = 0, hi = nprefix;  // invariant prefix[lo] <= u0 < prefix[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid] <= u0) lo = mid; else hi = mid;
+  }
+  int x = lo;
+  int idx = static_cast<int>(u0 - prefix[x]);
+  int remaining = nunits;
+  int cur_seg = -1, T = 0;
+  while (remaining > 0) {
+    if (x >= nprefix) return false;
+    const int cnt = prefix[x + 1] - prefix[x];
+    const int take = min(cnt - idx, remaining);
+    if (take <= 0) { ++x; idx = 0; continue; }
+    const int seg = x / s.nchunks;
+    const int cin = x - seg * s.nchunks;
+    if (seg != cur_seg) {
+      cur_seg = seg;
+      const int tt = a.seq_lens[seg / s.Hkv];
+      T = tt < 0 ? 0 : (tt > s.max_ctx ? s.max_ctx : tt);
+    }
+    const int* list = a.chunk_list + static_cast<size_t>(seg) * s.list_stride + static_cast<size_t>(cin) * s.chunk + idx;
+    for (int j0 = 0; j0 < take; j0 += 32) {
+      const int nn = min(32, take - j0);
+      const int e = lane < nn ? list[j0 + lane] : 0;
+      for (int jj = 0; jj < nn; ++jj) {
+        const int ent = __shfl_sync(0xffffffffu, e, jj);
+        int ok = 1;
+        if (lane == 0) {
+          const int blk = ent & kMaxBlocksPerSeq;
+          const UnitInfo in{seg, blk, static_cast<int>(static_cast<unsigned>(ent) >> kEntryBlockBits),
+                            min(s.b, T - blk * s.b)};
+          ok = issue(in) ? 1 : 0;
+        }
+        if (__shfl_sync(0xffffffffu, ok, 0) == 0) return false;
+      }
+    }
+    remaining -= take;
+    idx = 0;
+    ++x;
+  }
+  return true;
+}
+
+// Bounded wait that also gives up as soon as another role raised the CTA's
+// abort flag; a timeout raises it.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned* status,
+                                              volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      atomicOr(status, kStatusTimeout);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+  return true;
+}
+
+}  // namespace dev
+}  // namespace eta

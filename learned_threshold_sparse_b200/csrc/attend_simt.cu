@@ -21,7 +21,7 @@
 // and written as one partial per (segment, CTA).
 #include <math.h>
 
-#include "eta_device.cuh"
+#include "attend_common.cuh"
 
 namespace eta {
 namespace {
@@ -31,9 +31,8 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxStages = 8;
 
-struct UnitInfo {
-  int seg, blk, mask, nrows;
-};
+using dev::UnitInfo;
+using dev::wait_or_abort;
 
 template <int ELT, int D, int G>
 struct Cfg {
@@ -96,21 +95,6 @@ __device__ __forceinline__ float row_transpose_reduce(float (&v)[G], int sub) {
   return v[0];
 }
 
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned* status,
-                                              volatile int* abort_flag) {
-  if (dev::mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!dev::mbar_try_wait(bar, parity)) {
-    if (*abort_flag) return false;
-    if (clock64() - t0 > dev::kWaitCycles) {
-      atomicOr(status, kStatusTimeout);
-      *abort_flag = 1;
-      return false;
-    }
-  }
-  return true;
-}
-
 template <int ELT, int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, int stages) {
   using C = Cfg<ELT, D, G>;
@@ -146,32 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
   dev::pdl_trigger();
 
   // Exclusive prefix of the per-chunk entry counts, in (segment, chunk) order.
-  {
-    const int per = (nprefix + kThreads - 1) / kThreads;
-    const int lo = min(nprefix, t * per), hi = min(nprefix, lo + per);
-    int sum = 0;
-    for (int x = lo; x < hi; ++x) sum += a.chunk_count[x];
-    // block-wide exclusive scan of the per-thread sums
-    int incl = sum;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    __shared__ int s_warp[kConsumerWarps + 1];
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    int woff = 0;
-    for (int k = 0; k < warp; ++k) woff += s_warp[k];
-    int run = woff + incl - sum;
-    for (int x = lo; x < hi; ++x) {
-      const int cnt = a.chunk_count[x];
-      prefix[x] = run;
-      run += cnt;
-    }
-    if (t == kThreads - 1) prefix[nprefix] = woff + incl;
-  }
-  __syncthreads();
+  dev::chunk_prefix<kThreads>(a.chunk_count, nprefix, prefix);
 
   const long long U = prefix[nprefix];
   const long long N = gridDim.x;
@@ -185,68 +144,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
-    // chunk x holding unit u0: last x with prefix[x] <= u0
-    int lo = 0, hi = nprefix;  // invariant prefix[lo] <= u0 < prefix[hi]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (prefix[mid] <= u0) lo = mid; else hi = mid;
-    }
-    int x = lo;
-    int idx = static_cast<int>(u0 - prefix[x]);
-    int remaining = nunits;
     int stage = 0;
     uint32_t phase = 0;
-    int cur_seg = -1, T = 0;
-    const uint8_t* kbase = nullptr;
-    const uint8_t* vbase = nullptr;
-    bool ok = true;
-    while (remaining > 0 && ok) {
-      const int cnt = prefix[x + 1] - prefix[x];
-      const int take = min(cnt - idx, remaining);
-      if (take <= 0) { ++x; idx = 0; continue; }
-      const int seg = x / s.nchunks;
-      const int cin = x - seg * s.nchunks;
-      if (seg != cur_seg) {
-        cur_seg = seg;
-        const int i = seg / s.Hkv;
-        int tt = a.seq_lens[i];
-        T = tt < 0 ? 0 : (tt > s.max_ctx ? s.max_ctx : tt);
-        const size_t row0 = static_cast<size_t>(seg) * s.max_ctx;
-        kbase = static_cast<const uint8_t*>(a.k) + row0 * D * ELT;
-        vbase = static_cast<const uint8_t*>(a.v) + row0 * D * ELT;
-      }
-      const int* list = a.chunk_list + static_cast<size_t>(seg) * s.list_stride +
-                        static_cast<size_t>(cin) * s.chunk + idx;
-      for (int j0 = 0; j0 < take && ok; j0 += 32) {
-        const int nn = min(32, take - j0);
-        const int e = lane < nn ? list[j0 + lane] : 0;
-        for (int jj = 0; jj < nn; ++jj) {
-          const int ent = __shfl_sync(0xffffffffu, e, jj);
-          if (lane == 0) {
-            if (!wait_or_abort(&empty[stage], phase ^ 1u, a.status, abort_flag)) {
-              ok = false;
-            } else {
-              const int blk = ent & kMaxBlocksPerSeq;
-              const int nrows = min(s.b, T - blk * s.b);
-              info[stage] = UnitInfo{seg, blk, static_cast<int>(static_cast<unsigned>(ent) >> kEntryBlockBits), nrows};
-              const uint32_t bytes = static_cast<uint32_t>(nrows) * D * ELT;
-              dev::mbar_arrive_expect_tx(&full[stage], 2u * bytes);
-              const size_t off = static_cast<size_t>(blk) * s.b * D * ELT;
-              dev::bulk_g2s(kv + static_cast<size_t>(stage) * 2 * tile_bytes, kbase + off, bytes, &full[stage]);
-              dev::bulk_g2s(kv + static_cast<size_t>(stage) * 2 * tile_bytes + tile_bytes, vbase + off, bytes,
-                            &full[stage]);
-              issued_parity[stage] = static_cast<int>(phase);
-            }
-          }
-          ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-          if (!ok) break;
-          if (++stage == stages) { stage = 0; phase ^= 1u; }
-        }
-      }
-      remaining -= take;
-      idx = 0;
-      ++x;
-    }
+    const bool ok = dev::walk_units(a, prefix, nprefix, u0, nunits, [&](const UnitInfo& in) -> bool {
+      if (!wait_or_abort(&empty[stage], phase ^ 1u, a.status, abort_flag)) return false;
+      info[stage] = in;
+      const uint32_t bytes = static_cast<uint32_t>(in.nrows) * D * ELT;
+      dev::mbar_arrive_expect_tx(&full[stage], 2u * bytes);
+      const size_t off = (static_cast<size_t>(in.seg) * s.max_ctx + static_cast<size_t>(in.blk) * s.b) * D * ELT;
+      uint8_t* dst = kv + static_cast<size_t>(stage) * 2 * tile_bytes;
+      dev::bulk_g2s(dst, static_cast<const uint8_t*>(a.k) + off, bytes, &full[stage]);
+      dev::bulk_g2s(dst + tile_bytes, static_cast<const uint8_t*>(a.v) + off, bytes, &full[stage]);
+      issued_parity[stage] = static_cast<int>(phase);
+      if (++stage == stages) { stage = 0; phase ^= 1u; }
+      return true;
+    });
+    if (!ok && lane == 0) *abort_flag = 1;
     if (!ok && lane == 0) {
       // Let the copies already issued land before the CTA exits.
       for (int k = 0; k < stages; ++k) {
@@ -303,7 +216,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
       }
     }
     if (!rendezvous(0u)) return false;
-    float* part = a.partials + static_cast<size_t>(seg + blockIdx.x) * G * (D + 2);
+    float* part = a.partials + static_cast<size_t>(seg + blockIdx.x) * G * partial_stride(D);
     for (int x = t; x < G * D; x += kConsumerWarps * 32) {
       const int h = x / D, e = x - h * D;
       float mstar = -INFINITY;
@@ -317,10 +230,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
           lsum = fmaf(f, ws[D + 1], lsum);
         }
       }
-      part[h * (D + 2) + e] = sum;
+      part[h * partial_stride(D) + e] = sum;
       if (e == 0) {
-        part[h * (D + 2) + D] = mstar;
-        part[h * (D + 2) + D + 1] = lsum;
+        part[h * partial_stride(D) + D] = mstar;
+        part[h * partial_stride(D) + D + 1] = lsum;
       }
     }
     return rendezvous(1u);
@@ -452,7 +365,7 @@ cudaError_t launch_g(const AttendArgs& a, cudaStream_t st, int stages, size_t sm
   return cudaErrorInvalidValue;
 }
 
-constexpr size_t kSmemBudget = 227 * 1024;
+constexpr size_t kSmemBudget = 224 * 1024;  // leaves room for static shared memory
 
 int pick_stages(const Shape& s) {
   for (int st = kMaxStages; st >= 2; --st) {

@@ -165,9 +165,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-// logistic(x) = 1 / (1 + 2^(-x log2 e)); exact limits 0 and 1 for |x| large.
+__device__ __forceinline__ float fast_rcp(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// logistic(x) = 1 / (1 + 2^(-x log2 e)); limits 0 (for 2^(...) = +inf) and 1.
 __device__ __forceinline__ float logistic(float x) {
-  return 1.0f / (1.0f + fast_exp2(-x * 1.4426950408889634f));
+  return fast_rcp(1.0f + fast_exp2(-x * 1.4426950408889634f));
 }
 
 }  // namespace dev

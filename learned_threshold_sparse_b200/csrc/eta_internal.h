@@ -10,6 +10,10 @@
 
 namespace eta {
 
+// Floats per (partial slot, head): d accumulator entries, m, l, 2 pad so
+// every row starts 16-byte aligned.
+__host__ __device__ constexpr int partial_stride(int d) { return d + 4; }
+
 // Device status word bits (first word of the workspace).
 constexpr unsigned kStatusTimeout = 1u;  // a bounded wait ran out
 constexpr unsigned kStatusRange = 2u;    // a device-resident length was clamped
@@ -73,7 +77,7 @@ struct AttendArgs {
   Shape s;
   unsigned* status;
   int* seg_start;          // [nseg + 1] unit offsets (written by CTA 0)
-  float* partials;         // [nseg + attend_ctas][G][d + 2]
+  float* partials;         // [nseg + attend_ctas][G][partial_stride(d)]
 };
 
 struct CombineArgs {

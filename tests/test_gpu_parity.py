@@ -63,7 +63,7 @@ def test_block_summary_parity(case):
 
 def test_summary_append_touches_only_tail_block():
     wl = workloads.custom(seed=3, batch=2, n_q_heads=4, n_kv_heads=2, head_dim=128, block_size=64,
-                          seq_lens=[700, 640], dtype=BF16)
+                          seq_lens=[700, 640], dtype=BF16, max_ctx=800)
     t = upload(wl)
     summ = gpu_summary(wl, t)
     before = {k: v.clone() for k, v in summ.items()}
@@ -119,6 +119,29 @@ def test_decode_parity_small(c):
     compare(wl, g, r)
     dens = g["union_count"].sum() / max(1, sum(wl.n_blocks(i) for i in range(wl.batch)) * wl.n_kv_heads)
     assert 0.0 < dens <= 1.0
+
+
+TC_CASES = [c for c in SMALL if c["dtype"] == BF16 and c["d"] == 128 and c["b"] in (64, 128)
+            and c["Hq"] // c["Hkv"] in (2, 4, 8)]
+
+
+@pytest.mark.parametrize("impl", [eta.ETA_ATTEND_SIMT, eta.ETA_ATTEND_TC], ids=["simt", "tc"])
+@pytest.mark.parametrize("c", TC_CASES, ids=[c["id"] for c in TC_CASES])
+def test_decode_parity_each_attention_kernel(c, impl):
+    wl = _small(c)
+    g = gpu_decode(wl, attend_impl=impl)
+    r = oracle_decode(wl)
+    compare(wl, g, r)
+
+
+def test_tc_kernel_rejects_unsupported_shape():
+    wl = _small(SMALL[0])  # fp32, d 64, no GQA
+    t = upload(wl)
+    summ = gpu_summary(wl, t)
+    with pytest.raises(eta.EtaError) as e:
+        eta.decode(t["q"], t["k"], t["v"], t["seq"], summ, wl.block_size, "learned", w_tau=t["w_tau"],
+                   b_tau=t["b_tau"], attend_impl=eta.ETA_ATTEND_TC)
+    assert e.value.code == eta.ETA_ERR_UNSUPPORTED
 
 
 VARIANTS = [

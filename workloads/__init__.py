@@ -17,6 +17,7 @@ input data: they are stored in ``tests/golden/thresholds.json`` and written by
 """
 from __future__ import annotations
 
+import concurrent.futures as cf
 import dataclasses
 import json
 import math
@@ -105,6 +106,28 @@ def _normal(rng: np.random.Generator, shape, std: float = 1.0) -> np.ndarray:
     return x
 
 
+_CHUNK = 1 << 22
+
+
+def _normal_big(key, shape, std: float = 1.0) -> np.ndarray:
+    """N(0, std^2) float32 array filled in parallel: element block j (of 2^22
+    elements, row-major) comes from its own PCG64 stream seeded with key + [j],
+    so the values do not depend on the thread count."""
+    n = int(np.prod(shape))
+    out = np.empty(n, np.float32)
+
+    def fill(j):
+        lo, hi = j * _CHUNK, min(n, (j + 1) * _CHUNK)
+        out[lo:hi] = np.random.default_rng(list(key) + [j]).standard_normal(size=hi - lo, dtype=np.float32)
+
+    nblk = (n + _CHUNK - 1) // _CHUNK
+    with cf.ThreadPoolExecutor(max_workers=min(8, max(1, os.cpu_count() or 1))) as ex:
+        list(ex.map(fill, range(nblk)))
+    if std != 1.0:
+        out *= np.float32(std)
+    return out.reshape(shape)
+
+
 def _to_kv(x: np.ndarray, dtype: str) -> torch.Tensor:
     t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
     return t if dtype == F32 else t.to(torch.bfloat16)
@@ -183,8 +206,8 @@ def single(seed: int = 0, T: int = 32768) -> Workload:
     B, Hq, Hkv, d, b = 1, 16, 4, 128, 64
     G = Hq // Hkv
     q = _group_queries(rng, B, Hq, Hkv, d, 0.5)
-    k = _normal(rng, (B, Hkv, T, d))
-    v = _normal(rng, (B, Hkv, T, d))
+    k = _normal_big([2, seed, 0], (B, Hkv, T, d))
+    v = _normal_big([2, seed, 1], (B, Hkv, T, d))
     nb = (T + b - 1) // b
     n_plant = max(1, round(0.05 * nb))
     planted = {}
@@ -206,13 +229,14 @@ def single(seed: int = 0, T: int = 32768) -> Workload:
     return _attach_thresholds(wl)
 
 
-def _cluster_keys(rng, T: int, d: int, b: int, n_centres: int = 64, spread: float = 0.3) -> np.ndarray:
+def _cluster_keys(rng, T: int, d: int, b: int, n_centres: int = 64, spread: float = 0.3,
+                  noise_key=None) -> np.ndarray:
     centres = _normal(rng, (n_centres, d))
     nb = (T + b - 1) // b
     pick = rng.integers(0, n_centres, size=nb)
     per_token = np.repeat(pick, b)[:T]
     keys = centres[per_token]
-    keys += _normal(rng, (T, d), spread)
+    keys += _normal(rng, (T, d), spread) if noise_key is None else _normal_big(noise_key, (T, d), spread)
     return keys
 
 
@@ -224,8 +248,8 @@ def long(seed: int = 0, T: int = 131072) -> Workload:
     rng = np.random.default_rng([3, seed])
     B, Hq, Hkv, d, b = 1, 16, 4, 128, 64
     q = _group_queries(rng, B, Hq, Hkv, d, 0.5)
-    k = np.stack([_cluster_keys(rng, T, d, b) for _ in range(Hkv)])[None]
-    v = _normal(rng, (B, Hkv, T, d))
+    k = np.stack([_cluster_keys(rng, T, d, b, noise_key=[3, seed, 0, g]) for g in range(Hkv)])[None]
+    v = _normal_big([3, seed, 1], (B, Hkv, T, d))
     wl = Workload(name="c3_long", seed=seed, batch=B, n_q_heads=Hq, n_kv_heads=Hkv,
                   head_dim=d, block_size=b, max_ctx=T, seq_lens=[T], dtype=BF16,
                   tau_mode=TAU_CALIBRATED, q=_to_kv(q, BF16), k=_to_kv(k, BF16),
@@ -242,8 +266,8 @@ def max_context(seed: int = 0, T: int = 524288) -> Workload:
     B, Hq, Hkv, d, b = 1, 16, 4, 128, 128
     G = Hq // Hkv
     q = _group_queries(rng, B, Hq, Hkv, d, 0.5)
-    k = _normal(rng, (B, Hkv, T, d))
-    v = _normal(rng, (B, Hkv, T, d))
+    k = _normal_big([4, seed, 0], (B, Hkv, T, d))
+    v = _normal_big([4, seed, 1], (B, Hkv, T, d))
     nb = (T + b - 1) // b
     planted = {}
     for g in range(Hkv):
@@ -275,8 +299,8 @@ def batched(seed: int = 0, batch: int = 8, t_lo: int = 16384, t_hi: int = 131072
     v = torch.zeros((B, Hkv, Tmax, d), dtype=torch.bfloat16)
     for i, T in enumerate(lens):
         for g in range(Hkv):
-            k[i, g, :T] = _to_kv(_cluster_keys(rng, T, d, b), BF16)
-            v[i, g, :T] = _to_kv(_normal(rng, (T, d)), BF16)
+            k[i, g, :T] = _to_kv(_cluster_keys(rng, T, d, b, noise_key=[5, seed, 0, i, g]), BF16)
+            v[i, g, :T] = _to_kv(_normal_big([5, seed, 1, i, g], (T, d)), BF16)
     c_tau = rng.uniform(0.5, 2.0, size=Hq).astype(np.float32)
     return Workload(name="c5_batched", seed=seed, batch=B, n_q_heads=Hq, n_kv_heads=Hkv,
                     head_dim=d, block_size=b, max_ctx=Tmax, seq_lens=lens, dtype=BF16,
