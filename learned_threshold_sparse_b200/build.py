@@ -1,6 +1,6 @@
 """Build libeta.so (the ETA decode library) in-tree with nvcc for sm_100a.
 
-    python -m learned_threshold_sparse_b200.build        # or build() from Python
+    python learned_threshold_sparse_b200/build.py     # or build() from Python
 
 Each CUDA source is compiled in parallel to an object under _build/, then
 linked into learned_threshold_sparse_b200/libeta.so (CUDA runtime linked

@@ -16,7 +16,8 @@ namespace {
 // One CTA (4 warps) per (query head, sequence).  The attention CTAs that
 // touched segment `seg` are those owning its first and last unit; CTA c owns
 // units [U c / N, U (c + 1) / N), so unit u belongs to CTA ((u + 1) N - 1) / U.
-// Their partials sit at slots seg + c.  Warps stride over the partials (loads
+// Their partials sit at slots seg + c (CTAs in between that own no unit at all
+// wrote none).  Warps stride over the partials (loads
 // independent, so they overlap), lanes over the coordinates.
 constexpr int kCombineThreads = 128;
 
@@ -44,8 +45,11 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
   const int PS = partial_stride(D);
   const size_t stride = static_cast<size_t>(s.G) * PS;
   const float* base = a.partials + (static_cast<size_t>(seg) * s.G + j) * PS;
+  // CTAs with an empty range (fewer units than CTAs) wrote no partial.
+  auto owns_units = [&](int c) { return U * c / N != U * (c + 1) / N; };
   float mloc = -INFINITY;
-  for (int c = c0 + t; c <= c1; c += kCombineThreads) mloc = fmaxf(mloc, base[c * stride + D]);
+  for (int c = c0 + t; c <= c1; c += kCombineThreads)
+    if (owns_units(c)) mloc = fmaxf(mloc, base[c * stride + D]);
   mloc = dev::warp_max(mloc);
   if (lane == 0) s_red[w] = mloc;
   __syncthreads();
@@ -57,6 +61,7 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
   if (mstar != -INFINITY) {
 #pragma unroll 4
     for (int c = c0 + w; c <= c1; c += kCombineThreads / 32) {
+      if (!owns_units(c)) continue;
       const float* p = base + c * stride;
       const float m = p[D];
       const float f = (m == -INFINITY) ? 0.f : dev::fast_exp2(m - mstar);

@@ -224,6 +224,30 @@ def test_simt_and_auto_agree():
     assert np.abs(a["out"] - b["out"]).max() <= 2e-2
 
 
+def test_workspace_reuse_across_shapes():
+    # A workspace keeps the previous call's bytes; nothing stale may leak into
+    # the next call (tiny problems leave most attention CTAs without units).
+    a = workloads.custom(seed=41, batch=3, n_q_heads=16, n_kv_heads=4, head_dim=128, block_size=64,
+                         seq_lens=[3000, 130, 1777], dtype=BF16, tau_mode="calibrated", key_kind="cluster",
+                         tau_bias=1.0)
+    b = workloads.custom(seed=42, batch=2, n_q_heads=8, n_kv_heads=2, head_dim=64, block_size=32,
+                         seq_lens=[900, 47], dtype=F32, tau_bias=1e6).with_params(n_local_blocks=-1)
+    ws = eta.alloc_workspace(64 << 20)
+    ws.fill_(0x7f)  # non-zero garbage everywhere except the status word
+    ws[:16].zero_()
+    for wl in (a, b, a, b):
+        t = upload(wl)
+        summ = gpu_summary(wl, t)
+        res = eta.decode(t["q"], t["k"], t["v"], t["seq"], summ, wl.block_size, wl.tau_mode, w_tau=t["w_tau"],
+                         b_tau=t["b_tau"], c_tau=t["c_tau"], n_local_blocks=wl.n_local_blocks, selection=True,
+                         workspace=ws)
+        torch.cuda.synchronize()
+        g = {k: v.float().cpu().numpy() if k == "out" else v.cpu().numpy()
+             for k, v in res.items() if k != "workspace"}
+        g["status"] = eta.eta_read_device_status(ws)
+        compare(wl, g, oracle_decode(wl))
+
+
 def test_repeat_calls_are_deterministic():
     wl = _small(SMALL[4])
     t = upload(wl)
