@@ -183,6 +183,36 @@ eta_status eta_decode_workspace_size(const eta_decode_params* p, size_t* bytes);
  */
 eta_status eta_decode(const eta_decode_params* p, void* stream);
 
+/* Size of the fixed device scratch used by eta_decode_noalloc (8 MiB). */
+#define ETA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
+/*
+ * eta_decode_noalloc - eta_decode for callers that cannot allocate device
+ * memory.  No counterpart in the paper: this is a deployment variant.
+ *
+ * eta_decode needs a workspace from the caller.  Some callers cannot provide
+ * one: a plugin running inside a host program that owns every device
+ * allocation, or a code path where a cudaMalloc would synchronise the whole
+ * device.  This entry point takes the same parameters, ignores
+ * p->workspace and p->workspace_bytes, and uses a fixed array of
+ * ETA_NOALLOC_SCRATCH_BYTES that the library declares in device memory
+ * (every GPU that loads the library holds it until the process exits).  It
+ * calls no cudaMalloc, cudaFree or allocating library routine.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current) and caches it; make that first call before any
+ *     stream capture.
+ *   - Every call shares the one array, which keeps the last call's contents.
+ *     Calls that overlap on the GPU (different streams, or different host
+ *     threads without ordering) race on it and give wrong results.
+ *   - The device status word lives in that array: it is cleared at the start
+ *     of every call and cannot be read back (eta_read_device_status needs a
+ *     caller workspace).
+ * Errors: as eta_decode, plus ETA_ERR_WORKSPACE when
+ * eta_decode_workspace_size(p) exceeds ETA_NOALLOC_SCRATCH_BYTES, and
+ * ETA_ERR_CUDA if the array's address cannot be obtained.
+ */
+eta_status eta_decode_noalloc(const eta_decode_params* p, void* stream);
+
 /*
  * eta_read_device_status - synchronise `stream`, read and clear the device
  * status word kept in `workspace`.  Returns ETA_OK, ETA_ERR_DEVICE_TIMEOUT

@@ -86,6 +86,8 @@ def _load():
     lib.eta_decode_workspace_size.restype = ctypes.c_int
     lib.eta_decode.argtypes = [P(eta_decode_params), ctypes.c_void_p]
     lib.eta_decode.restype = ctypes.c_int
+    lib.eta_decode_noalloc.argtypes = [P(eta_decode_params), ctypes.c_void_p]
+    lib.eta_decode_noalloc.restype = ctypes.c_int
     lib.eta_read_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.eta_read_device_status.restype = ctypes.c_int
     lib.eta_status_string.argtypes = [ctypes.c_int]
@@ -97,8 +99,10 @@ def _load():
 
 _lib = _load()
 
-SYMBOLS = ("eta_block_summary_update", "eta_decode_workspace_size", "eta_decode",
+SYMBOLS = ("eta_block_summary_update", "eta_decode_workspace_size", "eta_decode", "eta_decode_noalloc",
            "eta_read_device_status", "eta_status_string", "eta_build_info")
+
+NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
 
 
 def library():
@@ -223,6 +227,15 @@ def eta_decode(params: eta_decode_params, stream: Optional[torch.cuda.Stream] = 
     rc = _lib.eta_decode(ctypes.byref(params), _stream_handle(stream))
     if rc != ETA_OK:
         raise EtaError(rc, "eta_decode")
+
+
+def eta_decode_noalloc(params: eta_decode_params, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """eta_decode without a caller workspace, for callers that cannot allocate
+    device memory: the library's fixed device scratch is used instead (see
+    include/eta.h).  Calls sharing that scratch must not overlap on the GPU."""
+    rc = _lib.eta_decode_noalloc(ctypes.byref(params), _stream_handle(stream))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_decode_noalloc")
 
 
 def eta_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:
