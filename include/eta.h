@@ -152,7 +152,9 @@ typedef struct {
   void* timing_events[4];            /* optional cudaEvent_t (NULL = none):
                                         recorded before the screen, before
                                         the attention kernel, before the
-                                        merge and after the last kernel      */
+                                        merge and after the last kernel
+                                        (events between the kernels keep
+                                        them from overlapping their launch) */
 } eta_decode_params;
 
 /*

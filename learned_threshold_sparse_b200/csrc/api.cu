@@ -1,6 +1,7 @@
 // C ABI of the ETA decode library: host-side validation, workspace layout and
 // the stream-ordered launch sequence
-//   screen (+ rescue) -> attention over the admitted union -> merge (+ export).
+//   screen (+ rescue) -> attention over the admitted union -> merge of the
+//   split partials of segments shared by several attention CTAs (+ export).
 #include <math.h>
 #include <stdio.h>
 #include <string.h>
@@ -61,10 +62,13 @@ eta_status make_shape(const eta_decode_params* p, Shape* out) {
   s.nbmax = (c.max_ctx + c.block_size - 1) / c.block_size;
   s.elt = c.kv_dtype == ETA_F32 ? 4 : 2;
   s.nseg = s.B * s.Hkv;
-  // Screen CTAs cover `chunk` blocks; keep the number of (segment, chunk)
-  // pairs <= 4096 so the attention kernel's prefix table fits in shared memory.
+  // Screen CTAs cover `chunk` blocks: about two screen CTAs per SM (one
+  // resident wave), and at most 4096 (segment, chunk) pairs so the attention
+  // kernel's prefix table fits in shared memory.
+  const int sms_for_chunk = sm_count() > 0 ? sm_count() : 148;
   int chunk = 32;
-  while (static_cast<long long>(s.nseg) * ((s.nbmax + chunk - 1) / chunk) > 4096 && chunk < 1024) chunk *= 2;
+  auto pairs = [&](int ch) { return static_cast<long long>(s.nseg) * ((s.nbmax + ch - 1) / ch); };
+  while (chunk < 1024 && (pairs(chunk) > 2LL * sms_for_chunk || pairs(chunk) > 4096)) chunk *= 2;
   s.chunk = chunk;
   s.nchunks = (s.nbmax + chunk - 1) / chunk;
   if (static_cast<long long>(s.nseg) * s.nchunks > 16384) return ETA_ERR_UNSUPPORTED;
@@ -160,8 +164,8 @@ const char* eta_status_string(eta_status s) {
 }
 
 const char* eta_build_info(void) {
-  return "eta decode library: sm_100a; kernels: block_summary, screen, rescue, attend_simt, attend_tc, "
-         "combine, export";
+  return "eta decode library: sm_100a; kernels: block_summary, screen, rescue, attend_simt, attend_tc, merge, "
+         "export";
 }
 
 eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summary_desc* summary,
@@ -237,6 +241,8 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
   sa.tau = reinterpret_cast<float*>(ws + w.tau);
   sa.chunk_count = reinterpret_cast<int*>(ws + w.chunk_count);
   sa.chunk_list = reinterpret_cast<int*>(ws + w.chunk_list);
+  sa.out = p->out;
+  sa.lse = p->lse;
   sa.head_count = reinterpret_cast<int*>(ws + w.head_count);
   sa.head_best = reinterpret_cast<unsigned long long*>(ws + w.head_best);
 
@@ -261,18 +267,20 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
   aa.status = sa.status;
   aa.seg_start = reinterpret_cast<int*>(ws + w.seg_start);
   aa.partials = reinterpret_cast<float*>(ws + w.partials);
+  aa.out = p->out;
+  aa.lse = p->lse;
   ev(1);
   const cudaError_t ea = s.attend_kind == ETA_ATTEND_TC ? launch_attend_tc(aa, cs) : launch_attend_simt(aa, cs);
   if (ea != cudaSuccess) return ETA_ERR_CUDA;
 
-  CombineArgs ca;
-  ca.seg_start = aa.seg_start;
-  ca.partials = aa.partials;
-  ca.s = s;
-  ca.out = p->out;
-  ca.lse = p->lse;
   ev(2);
-  if (launch_combine(ca, cs) != cudaSuccess) return ETA_ERR_CUDA;
+  MergeArgs ma;
+  ma.seg_start = aa.seg_start;
+  ma.partials = aa.partials;
+  ma.s = s;
+  ma.out = p->out;
+  ma.lse = p->lse;
+  if (launch_merge(ma, cs) != cudaSuccess) return ETA_ERR_CUDA;
 
   if (p->admitted_count || p->union_count || p->union_list || p->union_mask) {
     ExportArgs xa;

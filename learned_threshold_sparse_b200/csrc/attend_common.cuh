@@ -99,6 +99,51 @@ __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefi
   return true;
 }
 
+// The attention CTAs covering segment seg: CTA c owns units
+// [U c / N, U (c + 1) / N), so unit u belongs to CTA ((u + 1) N - 1) / U.
+// Returns how many of the CTAs in [c0, c1] own at least one unit (with fewer
+// units than CTAs some ranges are empty; those CTAs write no partial).
+struct SegCtas {
+  int c0, c1, n;
+  bool all;  // U >= N: every CTA owns a unit
+  // With U < N both U and N are small, so 32-bit arithmetic is exact.
+  __device__ __forceinline__ bool owns(int c, long long U, long long N) const {
+    if (all) return true;
+    const unsigned u = static_cast<unsigned>(U), nn = static_cast<unsigned>(N), cc = static_cast<unsigned>(c);
+    return u * cc / nn != u * (cc + 1u) / nn;
+  }
+};
+
+__device__ __forceinline__ SegCtas seg_ctas(long long us, long long ue, long long U, long long N) {
+  SegCtas r{0, -1, 0, U >= N};
+  if (ue <= us) return r;
+  r.c0 = static_cast<int>(((us + 1) * N - 1) / U);
+  r.c1 = static_cast<int>((ue * N - 1) / U);
+  if (r.all) {
+    r.n = r.c1 - r.c0 + 1;
+  } else {
+    for (int c = r.c0; c <= r.c1; ++c) r.n += r.owns(c, U, N) ? 1 : 0;
+  }
+  return r;
+}
+
+// Output element idx (kv dtype: fp32, or bf16 rounded to nearest even).
+__device__ __forceinline__ void store_out_slot(void* out, int elt, size_t idx, float o) {
+  if (elt == 4) {
+    static_cast<float*>(out)[idx] = o;
+  } else {
+    static_cast<uint16_t*>(out)[idx] = f32_to_bf16_rn(o);
+  }
+}
+
+__device__ __forceinline__ void store_out(const AttendArgs& a, size_t idx, float o) {
+  store_out_slot(a.out, a.s.elt, idx, o);
+}
+
+__device__ __forceinline__ float lse_of(float m2, float l) {
+  return l > 0.f ? (m2 + log2f(l)) * 0.6931471805599453f : -INFINITY;
+}
+
 // Bounded wait that also gives up as soon as another role raised the CTA's
 // abort flag; a timeout raises it.
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, unsigned* status,

@@ -185,17 +185,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
   int stage = 0;
   uint32_t phase = 0;
 
-  // Rendezvous of the 8 consumer warps on flush_bar: the first wait of a flush
-  // completes an even phase, the second an odd one.  Bounded: on a timeout
-  // the flush is abandoned and the kernel winds down.
-  auto rendezvous = [&](uint32_t parity) -> bool {
+  // Rendezvous of the 8 consumer warps on flush_bar (bounded: on a timeout
+  // the flush is abandoned and the kernel winds down).  Consecutive
+  // rendezvous complete consecutive phases.
+  uint32_t rv_phase = 0;
+  auto rendezvous = [&]() -> bool {
     __syncwarp();
     if (lane == 0) dev::mbar_arrive(flush_bar);
-    return wait_or_abort(flush_bar, parity, a.status, abort_flag);
+    const bool r = wait_or_abort(flush_bar, rv_phase, a.status, abort_flag);
+    rv_phase ^= 1u;
+    return r;
   };
 
+  // Segment done in this CTA: the eight warp states are merged; the result is
+  // written straight to the output when no other CTA touches the segment,
+  // else kept as this CTA's partial for the merge kernel.
   auto flush = [&](int seg) -> bool {
-    // rows of the warp -> one state per warp
 #pragma unroll
     for (int h = 0; h < G; ++h)
 #pragma unroll
@@ -215,7 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
         my[hh * (D + 2) + D + 1] = l_run;
       }
     }
-    if (!rendezvous(0u)) return false;
+    if (!rendezvous()) return false;
+    const dev::SegCtas sc = dev::seg_ctas(prefix[seg * s.nchunks], prefix[(seg + 1) * s.nchunks], U, N);
+    const int si = seg / s.Hkv, sg = seg - si * s.Hkv;
     float* part = a.partials + static_cast<size_t>(seg + blockIdx.x) * G * partial_stride(D);
     for (int x = t; x < G * D; x += kConsumerWarps * 32) {
       const int h = x / D, e = x - h * D;
@@ -230,13 +237,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
           lsum = fmaf(f, ws[D + 1], lsum);
         }
       }
-      part[h * partial_stride(D) + e] = sum;
-      if (e == 0) {
-        part[h * partial_stride(D) + D] = mstar;
-        part[h * partial_stride(D) + D + 1] = lsum;
+      if (sc.n == 1) {
+        const size_t orow = static_cast<size_t>(si) * s.Hq + sg * G + h;
+        dev::store_out(a, orow * D + e, lsum > 0.f ? sum / lsum : 0.f);
+        if (e == 0 && a.lse) a.lse[orow] = dev::lse_of(mstar, lsum);
+      } else {
+        part[h * partial_stride(D) + e] = sum;
+        if (e == 0) {
+          part[h * partial_stride(D) + D] = mstar;
+          part[h * partial_stride(D) + D + 1] = lsum;
+        }
       }
     }
-    return rendezvous(1u);
+    return rendezvous();  // the warp states may be overwritten after this
   };
 
   for (int u = 0; u < nunits; ++u) {

@@ -78,7 +78,7 @@ __host__ __device__ inline Layout tc_layout(int nstages, int br, int nprefix) {
   L.prefix = off = align_to(off, 16);
   off += static_cast<size_t>(nprefix + 1) * sizeof(int);
   L.misc = off = align_to(off, 16);
-  off += 16 + kMaxStages * sizeof(int);
+  off += 16 + kMaxStages * sizeof(int) + 16;
   L.total = align_to(off, 128) + 1024;  // + slack to align the dynamic base to 1024
   return L;
 }
@@ -191,7 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* prefix = reinterpret_cast<int*>(base + L.prefix);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L.misc + 4);
-  int* issued_parity = reinterpret_cast<int*>(base + L.misc + 16);
+  int* issued_parity = reinterpret_cast<int*>(base + L.misc + 32);
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   if (t == 0) {
@@ -368,6 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int h = 0; h < G; ++h) acc[h] = fmaf(acc[h], alpha_prev[h], o[h]);
       return true;
     };
+    // Segment done in this CTA: written straight to the output when no other
+    // CTA touches it, else kept as this CTA's partial for the merge kernel.
     auto flush = [&](int seg) -> bool {
       float* sums = red + 2 * 4 * 8;
 #pragma unroll
@@ -376,16 +378,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) sums[q4 * 8 + h] = lw;
       }
       if (!rendezvous()) return false;
-      float* part = a.partials + static_cast<size_t>(seg + blockIdx.x) * G * partial_stride(D);
+      const dev::SegCtas sc = dev::seg_ctas(prefix[seg * s.nchunks], prefix[(seg + 1) * s.nchunks], U, N);
+      if (sc.n == 1) {
+        const int i = seg / s.Hkv, g = seg - i * s.Hkv;
 #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        part[h * partial_stride(D) + dcol] = acc[h];
-        if (dcol == h) {
-          part[h * partial_stride(D) + D] = m_run[h];
-          part[h * partial_stride(D) + D + 1] = sums[h] + sums[8 + h] + sums[16 + h] + sums[24 + h];
+        for (int h = 0; h < G; ++h) {
+          const float l = sums[h] + sums[8 + h] + sums[16 + h] + sums[24 + h];
+          const size_t orow = static_cast<size_t>(i) * s.Hq + g * G + h;
+          dev::store_out(a, orow * D + dcol, l > 0.f ? acc[h] / l : 0.f);
+          if (dcol == h && a.lse) a.lse[orow] = dev::lse_of(m_run[h], l);
+        }
+      } else {
+        float* part = a.partials + static_cast<size_t>(seg + blockIdx.x) * G * partial_stride(D);
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+          part[h * partial_stride(D) + dcol] = acc[h];
+          if (dcol == h) {
+            part[h * partial_stride(D) + D] = m_run[h];
+            part[h * partial_stride(D) + D + 1] = sums[h] + sums[8 + h] + sums[16 + h] + sums[24 + h];
+          }
         }
       }
-      return rendezvous();
+      return true;
     };
 
     int pending = -1;  // unit whose O^T is not folded in yet
@@ -464,9 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int h = 0; h < G; ++h) alpha_prev[h] = alpha[h];
       pending = j;
     }
-    if (ok && pending >= 0) {
-      if (correction(pending)) flush(cur_seg);
-    }
+    if (ok && pending >= 0) ok = correction(pending) && flush(cur_seg);
   }
   tc_fence_before();
   __syncthreads();

@@ -61,6 +61,8 @@ struct ScreenArgs {
   float* tau;              // [B, Hq] tau~
   int* chunk_count;        // [nseg, nchunks]
   int* chunk_list;         // [nseg, list_stride]
+  void* out;               // written here only for empty sequences
+  float* lse;
   int* head_count;         // [B, Hq]   (rescue mode)
   unsigned long long* head_best;  // [B, Hq] (rescue mode)
 };
@@ -78,10 +80,12 @@ struct AttendArgs {
   unsigned* status;
   int* seg_start;          // [nseg + 1] unit offsets (written by CTA 0)
   float* partials;         // [nseg + attend_ctas][G][partial_stride(d)]
+  void* out;               // [B, Hq, d] kv dtype: segments owned by one CTA
+  float* lse;              // [B, Hq] or null
 };
 
-struct CombineArgs {
-  const int* seg_start;
+struct MergeArgs {
+  const int* seg_start;    // [nseg + 1] unit offsets written by the attention kernel
   const float* partials;
   Shape s;
   void* out;
@@ -119,7 +123,7 @@ int attend_simt_ctas_per_sm(const Shape& s);
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st);
 size_t attend_tc_smem(const Shape& s);
 bool attend_tc_supported(const Shape& s);
-cudaError_t launch_combine(const CombineArgs& a, cudaStream_t st);
+cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_export(const ExportArgs& a, cudaStream_t st);
 
 }  // namespace eta

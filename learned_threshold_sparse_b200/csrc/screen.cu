@@ -16,8 +16,11 @@
 // the geometric half alone when z = +inf.
 //
 // Grid (nchunks, Hkv, B): each CTA screens `chunk` consecutive blocks of one
-// (sequence, KV head) -- one warp per block, lanes split the head dimension --
-// and writes the admitted blocks of its chunk, ascending, as list entries
+// (sequence, KV head).  The metadata rows are staged in shared memory with
+// 1-D bulk copies (rounds of 64 blocks; the first round overlaps the threshold
+// computation); lanes split the head dimension, and the 2G partial sums of
+// 32 / (2G) blocks are reduced together by one transposing butterfly.  The
+// admitted blocks of the chunk are written, ascending, as list entries
 // (block id | head mask << 24) plus the chunk's entry count.
 #include <math.h>
 
@@ -57,25 +60,61 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[N], int lane) {
   return v[0];
 }
 
+constexpr int kRound = 64;  // blocks of metadata staged in shared memory per round
+
+template <int D>
+constexpr size_t screen_smem_bytes() {
+  return 2ull * 2 * kRound * D * sizeof(uint16_t);  // two buffers of mu and sigma rows
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
-  constexpr int CPL = D / 32;  // coordinates per lane
+  constexpr int CPL = D / 32;        // coordinates per lane
+  constexpr int NV = 2 * G;          // values per block: <q_h, mu>, sum q_h^2 sigma^2
+  constexpr int NB = 32 / NV;        // blocks reduced together (32 values per lane)
   const Shape& s = a.s;
   const int c = blockIdx.x, g = blockIdx.y, i = blockIdx.z;
   const int seg = i * s.Hkv + g;
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
 
+  extern __shared__ __align__(128) uint8_t dsm[];
+  uint16_t* stage = reinterpret_cast<uint16_t*>(dsm);  // [2 buffers][mu, sigma][kRound][D]
   __shared__ float s_q[G][D];
   __shared__ float s_tau[G];
   __shared__ float s_qn[G];
+  __shared__ float s_mn[kMaxChunk];
   __shared__ uint8_t s_mask[kMaxChunk];
   __shared__ int s_wsum[kWarps];
   __shared__ int s_cnt[G];
   __shared__ unsigned long long s_best[G];
+  __shared__ __align__(8) uint64_t s_bar[2];
 
   // The attention kernel may be scheduled now; it waits for this grid's
   // completion before reading anything written here.
   dev::pdl_trigger();
+
+  const int blk0 = c * s.chunk;
+  const int avail = min(s.chunk, s.nbmax - blk0);  // rows of this chunk inside the arrays
+  const size_t mbase = (static_cast<size_t>(seg) * s.nbmax) * D;
+  const size_t nbase = static_cast<size_t>(seg) * s.nbmax;
+  auto issue_round = [&](int r0, int rows) {
+    const int buf = (r0 / kRound) & 1;
+    uint16_t* mu_b = stage + static_cast<size_t>(buf) * 2 * kRound * D;
+    const uint32_t bytes = static_cast<uint32_t>(rows) * D * 2;
+    dev::mbar_arrive_expect_tx(&s_bar[buf], 2 * bytes);
+    dev::bulk_g2s(mu_b, a.mu + mbase + static_cast<size_t>(blk0 + r0) * D, bytes, &s_bar[buf]);
+    dev::bulk_g2s(mu_b + kRound * D, a.sigma + mbase + static_cast<size_t>(blk0 + r0) * D, bytes, &s_bar[buf]);
+  };
+  // Stage the first round of metadata before the sequence length is known
+  // (rows past it are in bounds and simply not used), together with the
+  // block norms, while the threshold is computed.
+  if (t == 0) {
+    dev::mbar_init(&s_bar[0], 1);
+    dev::mbar_init(&s_bar[1], 1);
+    dev::fence_barrier_init();
+    issue_round(0, min(kRound, avail));
+  }
+  for (int x = t; x < avail; x += kThreads) s_mn[x] = a.max_norm[nbase + blk0 + x];
 
   int T = a.seq_lens[i];
   if (T < 0 || T > s.max_ctx) {
@@ -83,8 +122,10 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
     T = T < 0 ? 0 : s.max_ctx;
   }
   const int nb = (T + s.b - 1) / s.b;
-  const int blk0 = c * s.chunk;
   const int nloc = max(0, min(s.chunk, nb - blk0));
+  const int first_forced = (!a.screen_enabled) ? 0 : (a.lwb >= 0 ? max(0, nb - 1 - a.lwb) : nb);
+  const int nscreen = max(0, min(nloc, first_forced - blk0));  // leading blocks of the chunk that are screened
+  if (t == 0 && nscreen > kRound) issue_round(kRound, min(kRound, nscreen - kRound));
 
   for (int x = t; x < G * D; x += kThreads) {
     const int h = x / D, e = x - h * D;
@@ -93,6 +134,14 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
   if (t < G) {
     s_cnt[t] = 0;
     s_best[t] = 0ull;
+  }
+  if (c == 0 && nb == 0) {
+    // an empty sequence has no unit to attend: its outputs are 0, lse -inf
+    for (int x = t; x < G * D; x += kThreads) {
+      const size_t o = (static_cast<size_t>(i) * s.Hq + g * G) * D + x;
+      if (s.elt == 4) static_cast<float*>(a.out)[o] = 0.f; else static_cast<uint16_t*>(a.out)[o] = 0;
+    }
+    if (t < G && a.lse) a.lse[static_cast<size_t>(i) * s.Hq + g * G + t] = -INFINITY;
   }
   __syncthreads();
   if (w < G) {
@@ -112,11 +161,8 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
       if (c == 0) a.tau[static_cast<size_t>(i) * s.Hq + hq] = tau;
     }
   }
+  for (int lb = nscreen + t; lb < nloc; lb += kThreads) s_mask[lb] = static_cast<uint8_t>((1u << G) - 1u);
   __syncthreads();
-  if (nloc == 0) {
-    if (t == 0) a.chunk_count[static_cast<size_t>(seg) * s.nchunks + c] = 0;
-    return;
-  }
 
   float qr[G][CPL], q2[G][CPL];
 #pragma unroll
@@ -128,58 +174,34 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
     }
   const float scale = a.scale, z = a.z;
   const bool strict = isinf(z);
-  const int first_forced = (!a.screen_enabled) ? 0 : (a.lwb >= 0 ? max(0, nb - 1 - a.lwb) : nb);
-  const size_t mbase = (static_cast<size_t>(seg) * s.nbmax) * D;
-  const size_t nbase = static_cast<size_t>(seg) * s.nbmax;
-  constexpr unsigned kAll = (1u << G) - 1u;
+  // after the reduction lane l holds value l % NV of block l / NV of the group
+  const int vb = lane / NV, vq = lane % NV;
+  const float my_tau = s_tau[vq % G], my_qn = s_qn[vq % G];
 
-  for (int lb0 = w; lb0 < nloc; lb0 += 4 * kWarps) {
-    // four blocks per warp in flight
-    uint32_t mu_raw[4][CPL / 2], sg_raw[4][CPL / 2];
-    float mn[4];
+  bool staged_ok = true;
+  for (int r0 = 0; r0 < nscreen && staged_ok; r0 += kRound) {
+    const int r = min(kRound, nscreen - r0);
+    const int buf = (r0 / kRound) & 1;
+    const uint16_t* mu_s = stage + static_cast<size_t>(buf) * 2 * kRound * D;
+    const uint16_t* sg_s = mu_s + kRound * D;
+    if (!dev::mbar_wait(&s_bar[buf], (r0 / (2 * kRound)) & 1, a.status)) { staged_ok = false; break; }
+    for (int gb = w * NB; gb < r; gb += kWarps * NB) {
+      float v[32];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int lb = lb0 + u * kWarps;
-      const int blk = blk0 + lb;
-      if (lb < nloc && blk < first_forced) {
-        const uint32_t* pm = reinterpret_cast<const uint32_t*>(a.mu + mbase + static_cast<size_t>(blk) * D + lane * CPL);
-        const uint32_t* ps = reinterpret_cast<const uint32_t*>(a.sigma + mbase + static_cast<size_t>(blk) * D + lane * CPL);
-        if constexpr (CPL == 4) {
-          const uint2 x = *reinterpret_cast<const uint2*>(pm);
-          const uint2 y = *reinterpret_cast<const uint2*>(ps);
-          mu_raw[u][0] = x.x; mu_raw[u][1] = x.y;
-          sg_raw[u][0] = y.x; sg_raw[u][1] = y.y;
-        } else {
-          mu_raw[u][0] = pm[0];
-          sg_raw[u][0] = ps[0];
-        }
-        mn[u] = a.max_norm[nbase + blk];
-      } else {
-#pragma unroll
-        for (int k = 0; k < CPL / 2; ++k) mu_raw[u][k] = sg_raw[u][k] = 0u;
-        mn[u] = 0.f;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int lb = lb0 + u * kWarps;
-      if (lb >= nloc) break;
-      const int blk = blk0 + lb;
-      unsigned m;
-      if (blk >= first_forced) {
-        m = kAll;
-      } else {
+      for (int u = 0; u < NB; ++u) {
+        const int lb = min(gb + u, r - 1);  // a short last group repeats a valid row
         float mu[CPL], s2[CPL];
 #pragma unroll
         for (int k = 0; k < CPL / 2; ++k) {
-          mu[2 * k] = dev::fp16_to_f32(static_cast<uint16_t>(mu_raw[u][k] & 0xffffu));
-          mu[2 * k + 1] = dev::fp16_to_f32(static_cast<uint16_t>(mu_raw[u][k] >> 16));
-          const float a0 = dev::fp16_to_f32(static_cast<uint16_t>(sg_raw[u][k] & 0xffffu));
-          const float a1 = dev::fp16_to_f32(static_cast<uint16_t>(sg_raw[u][k] >> 16));
+          const uint32_t m2 = *reinterpret_cast<const uint32_t*>(mu_s + lb * D + lane * CPL + 2 * k);
+          const uint32_t g2 = *reinterpret_cast<const uint32_t*>(sg_s + lb * D + lane * CPL + 2 * k);
+          mu[2 * k] = dev::fp16_to_f32(static_cast<uint16_t>(m2 & 0xffffu));
+          mu[2 * k + 1] = dev::fp16_to_f32(static_cast<uint16_t>(m2 >> 16));
+          const float a0 = dev::fp16_to_f32(static_cast<uint16_t>(g2 & 0xffffu));
+          const float a1 = dev::fp16_to_f32(static_cast<uint16_t>(g2 >> 16));
           s2[2 * k] = a0 * a0;
           s2[2 * k + 1] = a1 * a1;
         }
-        float v[2 * G];
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float dot = 0.f, sq = 0.f;
@@ -188,34 +210,48 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
             dot = fmaf(qr[h][k], mu[k], dot);
             sq = fmaf(q2[h][k], s2[k], sq);
           }
-          v[h] = dot;
-          v[G + h] = sq;
-        }
-        const float red = transpose_reduce32<2 * G>(v, lane);
-        // lanes [0, 16) hold <q_h, mu> for h = lane / (16 / G); lanes
-        // [16, 32) hold the matching sum of q^2 sigma^2.
-        const float sq = __shfl_xor_sync(0xffffffffu, red, 16);
-        const int hh = (lane & 15) / (16 / G);
-        const float geo = s_qn[hh] * mn[u];
-        const float spread = strict ? geo : fminf(geo, z * sqrtf(sq));
-        const float score = scale * (red + spread);
-        const bool pass = (lane < 16) && (lane % (16 / G) == 0) && (score >= s_tau[hh]);
-        const unsigned bal = __ballot_sync(0xffffffffu, pass);
-        m = 0u;
-#pragma unroll
-        for (int h = 0; h < G; ++h) m |= ((bal >> (h * (16 / G))) & 1u) << h;
-        if (s.rescue && lane < 16 && (lane % (16 / G) == 0)) {
-          const unsigned long long key =
-              (static_cast<unsigned long long>(dev::float_order_key(score)) << 32) |
-              static_cast<unsigned long long>(0xffffffffu - static_cast<unsigned>(blk));
-          atomicMax(&s_best[hh], key);
-          if (pass) atomicAdd(&s_cnt[hh], 1);
+          v[u * NV + h] = dot;
+          v[u * NV + G + h] = sq;
         }
       }
-      if (lane == 0) s_mask[lb] = static_cast<uint8_t>(m);
+      const float red = transpose_reduce32<32>(v, lane);
+      const float sq = __shfl_down_sync(0xffffffffu, red, G);  // sum q^2 sigma^2 of the same (block, head)
+      const int lb = gb + vb;
+      const bool head_lane = vq < G && lb < r;
+      float score = 0.f;
+      bool pass = false;
+      if (head_lane) {
+        const float geo = my_qn * s_mn[r0 + lb];
+        const float spread = strict ? geo : fminf(geo, z * sqrtf(sq));
+        score = scale * (red + spread);
+        pass = score >= my_tau;
+      }
+      const unsigned bal = __ballot_sync(0xffffffffu, pass);
+      if (vq == 0 && lb < r) s_mask[r0 + lb] = static_cast<uint8_t>((bal >> (vb * NV)) & ((1u << G) - 1u));
+      if (s.rescue && head_lane) {
+        const int blk = blk0 + r0 + lb;
+        const unsigned long long key =
+            (static_cast<unsigned long long>(dev::float_order_key(score)) << 32) |
+            static_cast<unsigned long long>(0xffffffffu - static_cast<unsigned>(blk));
+        atomicMax(&s_best[vq], key);
+        if (pass) atomicAdd(&s_cnt[vq], 1);
+      }
     }
+    __syncthreads();  // this buffer's rows are consumed
+    if (t == 0 && r0 + 2 * kRound < nscreen) issue_round(r0 + 2 * kRound, min(kRound, nscreen - r0 - 2 * kRound));
   }
+  if (!staged_ok) {
+    // a staging wait ran out (recorded in the status word): admit the rest
+    for (int lb = t; lb < nscreen; lb += kThreads) s_mask[lb] = static_cast<uint8_t>((1u << G) - 1u);
+  }
+  // The speculative first copy lands before exit even when nothing here
+  // was screened.
+  if (t == 0 && nscreen == 0) dev::mbar_wait(&s_bar[0], 0, a.status);
   __syncthreads();
+  if (nloc == 0) {
+    if (t == 0) a.chunk_count[static_cast<size_t>(seg) * s.nchunks + c] = 0;
+    return;
+  }
 
   // Ascending compaction of the chunk's admitted blocks.
   int base = 0;
@@ -276,17 +312,25 @@ __global__ void rescue_kernel(ScreenArgs a) {
   }
 }
 
+template <int D, int G>
+cudaError_t launch_screen_typed(const ScreenArgs& a, cudaStream_t st) {
+  constexpr size_t smem = screen_smem_bytes<D>();
+  auto kern = screen_kernel<D, G>;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(a.s.nchunks, a.s.Hkv, a.s.B), kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_screen_d(const ScreenArgs& a, cudaStream_t st) {
-  dim3 grid(a.s.nchunks, a.s.Hkv, a.s.B);
   switch (a.s.G) {
-    case 1: screen_kernel<D, 1><<<grid, kThreads, 0, st>>>(a); break;
-    case 2: screen_kernel<D, 2><<<grid, kThreads, 0, st>>>(a); break;
-    case 4: screen_kernel<D, 4><<<grid, kThreads, 0, st>>>(a); break;
-    case 8: screen_kernel<D, 8><<<grid, kThreads, 0, st>>>(a); break;
-    default: return cudaErrorInvalidValue;
+    case 1: return launch_screen_typed<D, 1>(a, st);
+    case 2: return launch_screen_typed<D, 2>(a, st);
+    case 4: return launch_screen_typed<D, 4>(a, st);
+    case 8: return launch_screen_typed<D, 8>(a, st);
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
