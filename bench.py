@@ -145,27 +145,30 @@ class ClockSampler:
                 "samples": len(sms)}
 
 
+ATTEND_SOURCES = ("attend_tc.cu", "attend_common.cuh", "eta_device.cuh", "eta_internal.h")
+
+
+def attend_source_sha1():
+    """Hash of the sources the attention kernel is compiled from."""
+    h = hashlib.sha1()
+    for name in ATTEND_SOURCES:
+        with open(os.path.join(ROOT, "learned_threshold_sparse_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def _traffic(workload):
     """dram bytes per attention launch from the committed ncu summary, or None
-    when the attention kernel's source changed since that capture."""
+    when the attention kernel's sources changed since that capture."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         table = json.load(f)
     ent = table.get(workload)
-    if not ent or ent.get("source_sha1") != _attend_source_sha1(ent.get("kernel_source")):
+    if not ent or ent.get("source_sha1") != attend_source_sha1():
         return None
     return ent.get("dram_bytes_per_launch")
-
-
-def _attend_source_sha1(name):
-    if not name:
-        return None
-    p = os.path.join(ROOT, "learned_threshold_sparse_b200", "csrc", name)
-    if not os.path.exists(p):
-        return None
-    return hashlib.sha1(open(p, "rb").read()).hexdigest()
 
 
 # ------------------------------------------------------------------ eta arm
