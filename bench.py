@@ -4,8 +4,9 @@
 
 One step = one eta_decode call (threshold + block screen, attention over the
 admitted GQA-union blocks, split merge) over the whole batch of the workload,
-inputs resident in HBM, L2 flushed (256 MiB write) before every step outside
-the step's events.  Prints ONE JSON line (rank 0).
+inputs resident in HBM, L2 flushed before every step outside the step's
+events by reading a 256 MiB buffer (the evicted lines are clean, so the step
+does not pay for writing back a flush buffer).  Prints ONE JSON line (rank 0).
 
 value  = effective HBM bandwidth of the step: algorithmic bytes (K+V of the
          union-admitted blocks at their real lengths + all block metadata + q,
@@ -228,7 +229,15 @@ def run_eta(args):
     params.workspace = ws.data_ptr()
     params.workspace_bytes = ws.numel()
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush_buf = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    class _Flush:
+        @staticmethod
+        def fill_(_):
+            torch.sum(flush_buf, dim=0, out=flush_sink)
+
+    flush = _Flush()
 
     def one_step():
         eta.eta_decode(params, stream)
@@ -368,7 +377,7 @@ def run_eta(args):
                 "head_density": round(head_density, 4),
                 "bytes_per_step": nbytes,
                 "kv_union_bytes_per_step": kv_union,
-                "l2": "flushed before every step (256 MiB write, outside the step events)",
+                "l2": "flushed before every step by reading a 256 MiB buffer (outside the step events)",
                 "parallelism": f"replicas x{world} (each rank decodes its own batch)",
             },
             "kernels_ms": {"screen": round(statistics.mean(screen_ms), 6), "attend": round(att_ms, 6),
