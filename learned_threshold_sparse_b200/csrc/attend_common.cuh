@@ -99,6 +99,25 @@ __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefi
   return true;
 }
 
+// Tiles of up to `bpt` consecutive units of one segment that the unit range
+// [u0, u1) splits into (a tile never crosses a segment boundary).
+__device__ __forceinline__ int count_tiles(const int* prefix, const Shape& s, long long u0, long long u1, int bpt) {
+  if (u1 <= u0) return 0;
+  int lo = 0, hi = s.nseg;  // last segment whose first unit is <= u0
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (prefix[mid * s.nchunks] <= u0) lo = mid; else hi = mid;
+  }
+  int tiles = 0;
+  for (int seg = lo; seg < s.nseg; ++seg) {
+    const long long a = max(u0, static_cast<long long>(prefix[seg * s.nchunks]));
+    const long long b = min(u1, static_cast<long long>(prefix[(seg + 1) * s.nchunks]));
+    if (a >= u1) break;
+    if (b > a) tiles += static_cast<int>((b - a + bpt - 1) / bpt);
+  }
+  return tiles;
+}
+
 // The attention CTAs covering segment seg: CTA c owns units
 // [U c / N, U (c + 1) / N), so unit u belongs to CTA ((u + 1) N - 1) / U.
 // Returns how many of the CTAs in [c0, c1] own at least one unit (with fewer

@@ -12,10 +12,11 @@
 //   section 3.2, F.3      split-KV partials (acc, m, l) merged later,
 //   Appendix F.4          tail block: rows >= seq_len are masked.
 //
-// Per unit (one admitted b-token block of one (sequence, KV head)):
-//   S^T [b x 16]   = K [b x 128] . Q^T [128 x 16]     (M = b, N = 16 query rows:
-//                                                      the G heads, rest unused)
-//   O^T [128 x 16] = V^T [128 x b] . P^T [b x 16]     (M = d, N = 16)
+// Per tile (128 key rows: one admitted 128-token block, or two consecutive
+// admitted 64-token blocks of the same (sequence, KV head)):
+//   S^T [128 x 16] = K [128 x 128] . Q^T [128 x 16]   (M = 128 rows, N = 16 query
+//                                                      rows: the G heads, rest unused)
+//   O^T [128 x 16] = V^T [128 x 128] . P^T [128 x 16] (M = d, N = 16)
 // K, V and the group's 16 query rows arrive by TMA (128-byte swizzle) into a
 // ring of shared-memory stages; one thread issues the MMAs; four warps read S
 // from tensor memory (thread = token), apply the tempering and the online
@@ -45,12 +46,19 @@ constexpr int kTmemCols = 64;       // S buffers at columns 0, 16; O buffers at 
 constexpr int kMaxStages = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <int BR>
+constexpr int TR = 128;  // key rows per tile
+
 struct Tile {
-  static constexpr int PANEL = BR * 128;  // one 64-column (128-byte) panel of a BR-row tile
+  static constexpr int PANEL = TR * 128;  // one 64-column (128-byte) panel of a 128-row tile
   static constexpr int K0 = 0, K1 = PANEL, V0 = 2 * PANEL, V1 = 3 * PANEL, Q0 = 4 * PANEL, Q1 = 4 * PANEL + 2048;
   static constexpr int STAGE = 4 * PANEL + 4096;
-  static constexpr int P_BYTES = NQ * BR * 2;
+  static constexpr int P_BYTES = NQ * TR * 2;
+};
+
+// What the producer tells the consumers about a tile: its segment and, per
+// block of the tile, the admitting heads and the rows present (0 = absent).
+struct TileInfo {
+  int seg, mask0, mask1, nrows0, nrows1;
 };
 
 struct Layout {
@@ -60,10 +68,10 @@ struct Layout {
 __host__ __device__ inline size_t align_to(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Offsets relative to a 1024-byte aligned base.
-__host__ __device__ inline Layout tc_layout(int nstages, int br, int nprefix) {
+__host__ __device__ inline Layout tc_layout(int nstages, int nprefix) {
   Layout L;
-  const size_t stage = static_cast<size_t>(4 * br * 128 + 4096);
-  const size_t pbytes = static_cast<size_t>(NQ * br * 2);
+  const size_t stage = static_cast<size_t>(Tile::STAGE);
+  const size_t pbytes = static_cast<size_t>(Tile::P_BYTES);
   size_t off = 0;
   L.stages = off;
   off += nstages * stage;
@@ -72,7 +80,7 @@ __host__ __device__ inline Layout tc_layout(int nstages, int br, int nprefix) {
   L.bars = off = align_to(off, 16);
   off += (2 * kMaxStages + 12) * sizeof(uint64_t);
   L.info = off = align_to(off, 16);
-  off += kMaxStages * sizeof(UnitInfo);
+  off += kMaxStages * sizeof(TileInfo);
   L.red = off = align_to(off, 16);
   off += 2 * 4 * 8 * sizeof(float) + 4 * 8 * sizeof(float);
   L.prefix = off = align_to(off, 16);
@@ -166,14 +174,15 @@ template <int BR, int G>
 __global__ void __launch_bounds__(kThreads, 1)
     attend_tc_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                      const __grid_constant__ CUtensorMap tq, AttendArgs a, int nstages) {
-  using TL = Tile<BR>;
+  using TL = Tile;
+  constexpr int BPT = TR / BR;  // blocks per tile
   extern __shared__ uint8_t smem_raw[];
   const Shape& s = a.s;
   const int nprefix = s.nseg * s.nchunks;
   const uint32_t raw = dev::smem_u32(smem_raw);
   const uint32_t base_u32 = (raw + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - raw);
-  const Layout L = tc_layout(nstages, BR, nprefix);
+  const Layout L = tc_layout(nstages, nprefix);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L.bars);
   Bars B;
@@ -186,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.o_free = B.o_full + 2;
   B.rv = B.o_free + 2;
   B.done = B.rv + 1;
-  UnitInfo* info = reinterpret_cast<UnitInfo*>(base + L.info);
+  TileInfo* info = reinterpret_cast<TileInfo*>(base + L.info);
   float* red = reinterpret_cast<float*>(base + L.red);  // [2][4][8] tile maxima, then [4][8] flush sums
   int* prefix = reinterpret_cast<int*>(base + L.prefix);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L.misc);
@@ -239,28 +248,50 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (blockIdx.x == 0)
     for (int sg = t; sg <= s.nseg; sg += kThreads) a.seg_start[sg] = prefix[sg * s.nchunks];
 
+  const int ntiles = dev::count_tiles(prefix, s, u0, u1, BPT);
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // Consecutive units of one segment are packed BPT to a tile; block i of a
+    // tile fills rows [i BR, (i + 1) BR) of every 128-row panel.
     if (nunits > 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const bool ok = dev::walk_units(a, prefix, nprefix, u0, nunits, [&](const UnitInfo& in) -> bool {
+      TileInfo pend{-1, 0, 0, 0, 0};
+      int pblk[2] = {0, 0};
+      int npend = 0;
+      auto emit = [&]() -> bool {
         if (!wait_or_abort(&B.kv_empty[stage], phase ^ 1u, a.status, abort_flag)) return false;
-        info[stage] = in;
+        info[stage] = pend;
         const uint32_t st = base_u32 + static_cast<uint32_t>(L.stages + stage * TL::STAGE);
-        dev::mbar_arrive_expect_tx(&B.kv_full[stage], TL::STAGE);
-        const int krow = in.seg * s.max_ctx + in.blk * BR;
-        const int qrow = in.seg * s.G;
-        tma_load_2d(st + TL::K0, &tk, 0, krow, &B.kv_full[stage]);
-        tma_load_2d(st + TL::K1, &tk, 64, krow, &B.kv_full[stage]);
-        tma_load_2d(st + TL::V0, &tv, 0, krow, &B.kv_full[stage]);
-        tma_load_2d(st + TL::V1, &tv, 64, krow, &B.kv_full[stage]);
+        dev::mbar_arrive_expect_tx(&B.kv_full[stage], static_cast<uint32_t>(npend * 4 * BR * 128 + 4096));
+        for (int i = 0; i < npend; ++i) {
+          const int krow = pend.seg * s.max_ctx + pblk[i] * BR;
+          const uint32_t ro = static_cast<uint32_t>(i * BR * 128);
+          tma_load_2d(st + TL::K0 + ro, &tk, 0, krow, &B.kv_full[stage]);
+          tma_load_2d(st + TL::K1 + ro, &tk, 64, krow, &B.kv_full[stage]);
+          tma_load_2d(st + TL::V0 + ro, &tv, 0, krow, &B.kv_full[stage]);
+          tma_load_2d(st + TL::V1 + ro, &tv, 64, krow, &B.kv_full[stage]);
+        }
+        const int qrow = pend.seg * s.G;
         tma_load_2d(st + TL::Q0, &tq, 0, qrow, &B.kv_full[stage]);
         tma_load_2d(st + TL::Q1, &tq, 64, qrow, &B.kv_full[stage]);
         issued_parity[stage] = static_cast<int>(phase);
         if (++stage == nstages) { stage = 0; phase ^= 1u; }
+        npend = 0;
+        return true;
+      };
+      bool ok = dev::walk_units(a, prefix, nprefix, u0, nunits, [&](const UnitInfo& in) -> bool {
+        if (npend > 0 && (in.seg != pend.seg || npend == BPT) && !emit()) return false;
+        if (npend == 0) pend = TileInfo{in.seg, 0, 0, 0, 0};
+        pblk[npend] = in.blk;
+        if (npend == 0) { pend.mask0 = in.mask; pend.nrows0 = in.nrows; }
+        else { pend.mask1 = in.mask; pend.nrows1 = in.nrows; }
+        ++npend;
         return true;
       });
+      if (ok && lane == 0 && npend > 0) ok = emit();
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
       if (!ok && lane == 0) {
         *abort_flag = 1;
         for (int k = 0; k < nstages; ++k) {  // let issued copies land
@@ -274,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc_qk = idesc_bf16(BR, NQ, 0);
+    constexpr uint32_t idesc_qk = idesc_bf16(TR, NQ, 0);
     constexpr uint32_t idesc_pv = idesc_bf16(D, NQ, 1);
     bool ok = true;
     auto issue_pv = [&](int i) -> bool {
@@ -287,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vbase = base_u32 + static_cast<uint32_t>(L.stages + st_i * TL::STAGE) + TL::V0;
         const uint32_t pbase = base_u32 + static_cast<uint32_t>(L.pbuf + pb * TL::P_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BR / 16; ++kk) {
+        for (int kk = 0; kk < TR / 16; ++kk) {
           const uint64_t ad = sw128_desc(vbase + kk * 2048, TL::PANEL, 1024);
           const uint64_t bd = sw128_desc(pbase + (kk >> 2) * 2048 + (kk & 3) * 32, 16, 1024);
           mma_bf16(tmem + 32 + pb * 16, ad, bd, idesc_pv, kk > 0 ? 1u : 0u);
@@ -298,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       return true;
     };
-    for (int j = 0; j < nunits && ok; ++j) {
+    for (int j = 0; j < ntiles && ok; ++j) {
       const int st_j = j % nstages;
       const int sb = j & 1;
       if (!wait_or_abort(&B.kv_full[st_j], (j / nstages) & 1, a.status, abort_flag)) { ok = false; break; }
@@ -319,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
     }
-    if (ok && nunits > 0) issue_pv(nunits - 1);
+    if (ok && ntiles > 0) issue_pv(ntiles - 1);
     // every MMA issued so far has completed once `done` flips
     if (lane == 0) mma_commit(B.done);
     __syncwarp();
@@ -332,7 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax / correction
     const int q4 = warp & 3;  // TMEM lane quarter this warp may access
     const uint32_t tlane = static_cast<uint32_t>(32 * q4) << 16;
-    const int row = (BR == 128) ? 32 * q4 + lane : (lane < 16 ? 16 * q4 + lane : -1);
+    const int row = 32 * q4 + lane;  // key row of the tile this thread owns in S^T
+    const int rblk = row / BR, rrow = row - rblk * BR;
     const int dcol = 32 * q4 + lane;  // output coordinate of this thread in O^T
     const float scale = a.scale, beta = a.beta;
     float m_run[G], l_thr[G], acc[G], alpha_prev[G], tau_h[G];
@@ -403,10 +435,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     int pending = -1;  // unit whose O^T is not folded in yet
-    for (int j = 0; j < nunits && ok; ++j) {
+    for (int j = 0; j < ntiles && ok; ++j) {
       const int st_j = j % nstages;
       if (!wait_or_abort(&B.kv_full[st_j], (j / nstages) & 1, a.status, abort_flag)) { ok = false; break; }
-      const UnitInfo in = info[st_j];
+      const TileInfo in = info[st_j];
       if (in.seg != cur_seg) {
         if (pending >= 0) {
           if (!correction(pending) || !flush(cur_seg)) { ok = false; break; }
@@ -430,14 +462,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) dev::mbar_arrive(&B.s_free[sb]);
 
-      const bool valid = row >= 0 && row < in.nrows;
+      const int rmask = rblk == 0 ? in.mask0 : in.mask1;
+      const bool valid = rrow < (rblk == 0 ? in.nrows0 : in.nrows1);
       float x[G];
       float* wmax = red + (j & 1) * 32;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
         const float S = sv[h] * scale;
         const float St = S * dev::logistic(beta * (S - tau_h[h]));
-        x[h] = (valid && ((in.mask >> h) & 1)) ? St * kLog2e : -INFINITY;
+        x[h] = (valid && ((rmask >> h) & 1)) ? St * kLog2e : -INFINITY;
         const float mw = dev::warp_max(x[h]);
         if (lane == 0) wmax[q4 * 8 + h] = mw;
       }
@@ -452,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha[h] = (m_run[h] == -INFINITY) ? 0.f : dev::fast_exp2(m_run[h] - m_new);
         const float p = (x[h] == -INFINITY) ? 0.f : dev::fast_exp2(x[h] - m_new);
         const uint16_t pbits = dev::f32_to_bf16_rn(p);
-        if (row >= 0) {
+        {
           const int kp = row >> 6, tc = row & 63;
           const int off = kp * 2048 + h * 128 + (((tc >> 3) ^ (h & 7)) << 4) + (tc & 7) * 2;
           *reinterpret_cast<uint16_t*>(pbuf + off) = pbits;
@@ -460,14 +493,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_thr[h] = fmaf(l_thr[h], alpha[h], __uint_as_float(static_cast<uint32_t>(pbits) << 16));
         m_run[h] = m_new;
       }
-      if (in.nrows < BR) {
-        // tail block: rows past the sequence end are zeroed so that stale or
-        // non-finite bytes there cannot reach the accumulator (0 * inf)
+      if (in.nrows0 < BR || (BPT == 2 && in.nrows1 < BR)) {
+        // rows of a tile that hold no key (past a sequence end, or an absent
+        // second block) are zeroed in V so that stale or non-finite bytes
+        // there cannot reach the accumulator (0 * inf)
         uint8_t* vb = base + L.stages + st_j * TL::STAGE + TL::V0;
-        const int nz = (BR - in.nrows) * 8;  // 16-byte chunks per panel
-        for (int c = t - 64; c < 2 * nz; c += 128) {
-          const int pnl = c / nz, r = c - pnl * nz;
-          *reinterpret_cast<uint4*>(vb + pnl * TL::PANEL + in.nrows * 128 + r * 16) = make_uint4(0u, 0u, 0u, 0u);
+        for (int bi = 0; bi < BPT; ++bi) {
+          const int nr = bi == 0 ? in.nrows0 : in.nrows1;
+          const int nz = (BR - nr) * 8;  // 16-byte chunks per panel
+          for (int c = t - 64; c < 2 * nz; c += 128) {
+            const int pnl = c / nz, r = c - pnl * nz;
+            *reinterpret_cast<uint4*>(vb + pnl * TL::PANEL + (bi * BR + nr) * 128 + r * 16) =
+                make_uint4(0u, 0u, 0u, 0u);
+          }
         }
       }
       fence_proxy_async();
@@ -516,7 +554,7 @@ constexpr size_t kSmemBudget = 224 * 1024;
 
 int pick_stages(const Shape& s) {
   for (int st = kMaxStages; st >= 2; --st)
-    if (tc_layout(st, s.b, s.nseg * s.nchunks).total <= kSmemBudget) return st;
+    if (tc_layout(st, s.nseg * s.nchunks).total <= kSmemBudget) return st;
   return 0;
 }
 
@@ -559,13 +597,13 @@ bool attend_tc_supported(const Shape& s) {
 
 size_t attend_tc_smem(const Shape& s) {
   const int st = pick_stages(s);
-  return st ? tc_layout(st, s.b, s.nseg * s.nchunks).total : 0;
+  return st ? tc_layout(st, s.nseg * s.nchunks).total : 0;
 }
 
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st) {
   const int stages = pick_stages(a.s);
   if (stages == 0) return cudaErrorInvalidConfiguration;
-  const size_t smem = tc_layout(stages, a.s.b, a.s.nseg * a.s.nchunks).total;
+  const size_t smem = tc_layout(stages, a.s.nseg * a.s.nchunks).total;
   CUtensorMap tk, tv, tq;
   const uint64_t rows = static_cast<uint64_t>(a.s.nseg) * a.s.max_ctx;
   if (!make_map(&tk, a.k, rows, a.s.b) || !make_map(&tv, a.v, rows, a.s.b) ||
