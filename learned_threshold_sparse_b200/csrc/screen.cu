@@ -62,9 +62,11 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[N], int lane) {
 
 constexpr int kRound = 64;  // blocks of metadata staged in shared memory per round
 
+// Staging buffers of mu and sigma rows: the second one is used only when a
+// chunk needs more than one round.
 template <int D>
-constexpr size_t screen_smem_bytes() {
-  return 2ull * 2 * kRound * D * sizeof(uint16_t);  // two buffers of mu and sigma rows
+constexpr size_t screen_smem_bytes(int chunk) {
+  return (chunk > kRound ? 2ull : 1ull) * 2 * kRound * D * sizeof(uint16_t);
 }
 
 template <int D, int G>
@@ -314,9 +316,10 @@ __global__ void rescue_kernel(ScreenArgs a) {
 
 template <int D, int G>
 cudaError_t launch_screen_typed(const ScreenArgs& a, cudaStream_t st) {
-  constexpr size_t smem = screen_smem_bytes<D>();
+  const size_t smem = screen_smem_bytes<D>(a.s.chunk);
   auto kern = screen_kernel<D, G>;
-  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  const cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(screen_smem_bytes<D>(2 * kRound)));
   if (e != cudaSuccess) return e;
   kern<<<dim3(a.s.nchunks, a.s.Hkv, a.s.B), kThreads, smem, st>>>(a);
   return cudaGetLastError();
