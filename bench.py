@@ -70,6 +70,22 @@ def _workload_desc(wl):
             f"ctx {min(wl.seq_lens)}-{max(wl.seq_lens)}, block {wl.block_size}, {wl.dtype}, {wl.tau_mode} tau")
 
 
+def max_over_ranks(x: float, device) -> float:
+    """Largest x over the ranks of the default process group (x itself when
+    not distributed): the job's step time is the slowest rank's."""
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(world: int, bytes_per_rank_step: int, ms: float) -> float:
+    """Aggregate effective bandwidth of all ranks (weak scaling: every rank
+    moves the same bytes per step) for a max-over-ranks step time in ms."""
+    return world * bytes_per_rank_step / (ms * 1e-3) / 1e9
+
+
 def union_bytes(wl, union_list, union_count):
     """K+V bytes of the union-admitted blocks, tails at their real length."""
     tot = 0
@@ -289,12 +305,8 @@ def run_eta(args):
     clk = clocks.stop()
     assert eta.eta_read_device_status(ws) == eta.ETA_OK
 
-    ms = statistics.mean(step_ms)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-    value = world * nbytes / (ms * 1e-3) / 1e9
+    ms = max_over_ranks(statistics.mean(step_ms), dev)
+    value = whole_job_gbs(world, nbytes, ms)
 
     # ---- end to end through the public API, host buffers
     q_h = wl.q.pin_memory()
@@ -337,11 +349,7 @@ def run_eta(args):
         e1.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
     assert torch.equal(out_h, out.cpu())
-    e2e = statistics.mean(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e = float(t.item())
+    e2e = max_over_ranks(statistics.mean(e2e_ms), dev)
     h2d = (q_h.numel() + knew.numel() + vnew.numel()) * wl.elt_bytes
     d2h = out_h.numel() * wl.elt_bytes
 
@@ -388,7 +396,7 @@ def run_eta(args):
                          "frac": round(achieved / peak, 4), "traffic": traffic,
                          "algorithmic_bytes_per_launch": kv_union},
             "step_frac_of_peak": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4),
-            "e2e": {"value": round(world * nbytes / (e2e * 1e-3) / 1e9, 2), "unit": UNIT,
+            "e2e": {"value": round(whole_job_gbs(world, nbytes, e2e), 2), "unit": UNIT,
                     "ms_per_step": round(e2e, 6), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": 3 * args.steps,
             "clocks": clk,
