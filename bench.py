@@ -13,8 +13,9 @@ value  = effective HBM bandwidth of the step: algorithmic bytes (K+V of the
          threshold parameters and outputs) / device step time, summed over
          ranks (each rank decodes its own copy of the batch: weak scaling).
 e2e    = the same bytes / end-to-end step time through the public API: the
-         new token's q, k, v copied from pinned host memory, the tail block's
-         metadata refreshed, the decode, the output copied back to pinned host.
+         new token's q, k, v copied in one transfer from pinned host memory,
+         eta_append_kv (K/V rows written, their block's metadata refreshed),
+         eta_decode, the output copied back to pinned host memory.
 roofline = the attention kernel: union K+V bytes per launch / its mean
          launch time (CUDA events on the launch stream, second run of K
          steps) vs the measured HBM copy bandwidth.
@@ -308,18 +309,23 @@ def run_eta(args):
     ms = max_over_ranks(statistics.mean(step_ms), dev)
     value = whole_job_gbs(world, nbytes, ms)
 
-    # ---- end to end through the public API, host buffers
-    q_h = wl.q.pin_memory()
-    knew = torch.stack([wl.k[i, :, wl.seq_lens[i] - 1] for i in range(wl.batch)]).contiguous().pin_memory()
-    vnew = torch.stack([wl.v[i, :, wl.seq_lens[i] - 1] for i in range(wl.batch)]).contiguous().pin_memory()
+    # ---- end to end through the public API, host buffers: the step's new
+    # query, key and value rows go up in one copy from pinned memory, the
+    # append writes the K/V rows and refreshes their block, the decode runs,
+    # the output comes back to pinned memory.
+    B_, Hq_, Hkv_, d_ = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    nq, nkv = B_ * Hq_ * d_, B_ * Hkv_ * d_
+    knew = torch.stack([wl.k[i, :, wl.seq_lens[i] - 1] for i in range(B_)])
+    vnew = torch.stack([wl.v[i, :, wl.seq_lens[i] - 1] for i in range(B_)])
+    packed_h = torch.cat([wl.q.reshape(-1), knew.reshape(-1), vnew.reshape(-1)]).pin_memory()
+    packed_d = torch.empty(packed_h.shape, dtype=packed_h.dtype, device=dev)
+    q_in = packed_d[:nq].view(B_, Hq_, d_)
+    k_in = packed_d[nq:nq + nkv].view(B_, Hkv_, d_)
+    v_in = packed_d[nq + nkv:].view(B_, Hkv_, d_)
     out_h = torch.empty_like(wl.q).pin_memory()
     last = torch.tensor([T - 1 for T in wl.seq_lens], dtype=torch.int32, device=dev)
-    idx_b = torch.arange(wl.batch, device=dev)
-    pos = last.long()
-    knew_d = torch.empty(knew.shape, dtype=knew.dtype, device=dev)
-    vnew_d = torch.empty(vnew.shape, dtype=vnew.dtype, device=dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    params_e2e = eta.make_params(q, k, v, seq, summ, wl.block_size, wl.tau_mode, w_tau=w_tau, b_tau=b_tau,
+    params_e2e = eta.make_params(q_in, k, v, seq, summ, wl.block_size, wl.tau_mode, w_tau=w_tau, b_tau=b_tau,
                                  c_tau=c_tau, scale=wl.scale, beta=wl.beta, offset_a=wl.offset_a, z=wl.z,
                                  n_local_blocks=wl.n_local_blocks, screen_enabled=not args.dense,
                                  attend_impl=args.attend_impl, out=out, lse=lse)
@@ -327,12 +333,8 @@ def run_eta(args):
     params_e2e.workspace_bytes = ws.numel()
 
     def e2e_step():
-        q.copy_(q_h, non_blocking=True)
-        knew_d.copy_(knew, non_blocking=True)
-        vnew_d.copy_(vnew, non_blocking=True)
-        k[idx_b, :, pos] = knew_d
-        v[idx_b, :, pos] = vnew_d
-        eta.eta_block_summary_update(k, v, seq, summ, wl.block_size, last, 1, wl.n_q_heads, stream)
+        packed_d.copy_(packed_h, non_blocking=True)
+        eta.eta_append_kv(k, v, seq, summ, wl.block_size, k_in, v_in, last, wl.n_q_heads, stream)
         eta.eta_decode(params_e2e, stream)
         out_h.copy_(out, non_blocking=True)
 
@@ -350,7 +352,7 @@ def run_eta(args):
         e2e_ms.append(e0.elapsed_time(e1))
     assert torch.equal(out_h, out.cpu())
     e2e = max_over_ranks(statistics.mean(e2e_ms), dev)
-    h2d = (q_h.numel() + knew.numel() + vnew.numel()) * wl.elt_bytes
+    h2d = packed_h.numel() * wl.elt_bytes
     d2h = out_h.numel() * wl.elt_bytes
 
     peak, peak_kind = _peaks()

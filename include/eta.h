@@ -116,6 +116,24 @@ eta_status eta_block_summary_update(const eta_cache_desc* cache,
                                     const int* first_token, int max_blocks,
                                     void* stream);
 
+/*
+ * eta_append_kv - the KV append of one decode step, fused with the metadata
+ * refresh it requires ("refreshed on KV append"; Appendix F.1): for every
+ * sequence i and KV head g, writes k_new[i, g, :] and v_new[i, g, :] into
+ * row pos[i] of the caches and recomputes the summary of the block holding
+ * that row over its present tokens [j b, seq_lens[i]) (seq_lens must already
+ * count the new token).  One launch.
+ *   k_new, v_new : [batch, n_kv_heads, head_dim] device, kv_dtype, 16-byte aligned
+ *   pos          : [batch] device int, 4-byte aligned; a position outside
+ *                  [0, max_ctx) writes nothing for that sequence
+ * The cache descriptor's k_cache / v_cache are written (they must be
+ * writable device memory).
+ * Errors: ETA_ERR_INVALID_ARG, ETA_ERR_UNSUPPORTED, ETA_ERR_CUDA.
+ */
+eta_status eta_append_kv(const eta_cache_desc* cache, const eta_summary_desc* summary,
+                         const void* k_new, const void* v_new, const int* pos,
+                         void* stream);
+
 /* All inputs and outputs of one decode step. */
 typedef struct {
   eta_cache_desc cache;

@@ -5,6 +5,7 @@ kernels behind the C ABI declared in ``include/eta.h``.  PyTorch provides the
 device memory and the stream.  The functions mirror the C entry points:
 
     eta_block_summary_update(...)   refresh per-block metadata after an append
+    eta_append_kv(...)              write a new token's K/V and refresh its block
     eta_decode_workspace_size(...)  bytes of scratch for a decode call
     eta_decode(...)                 one decode step (screen, attend, merge)
     eta_read_device_status(...)     read and clear the device status word
@@ -82,6 +83,9 @@ def _load():
     lib.eta_block_summary_update.argtypes = [P(eta_cache_desc), P(eta_summary_desc), ctypes.c_void_p,
                                              ctypes.c_int, ctypes.c_void_p]
     lib.eta_block_summary_update.restype = ctypes.c_int
+    lib.eta_append_kv.argtypes = [P(eta_cache_desc), P(eta_summary_desc), ctypes.c_void_p, ctypes.c_void_p,
+                                  ctypes.c_void_p, ctypes.c_void_p]
+    lib.eta_append_kv.restype = ctypes.c_int
     lib.eta_decode_workspace_size.argtypes = [P(eta_decode_params), P(ctypes.c_size_t)]
     lib.eta_decode_workspace_size.restype = ctypes.c_int
     lib.eta_decode.argtypes = [P(eta_decode_params), ctypes.c_void_p]
@@ -99,7 +103,7 @@ def _load():
 
 _lib = _load()
 
-SYMBOLS = ("eta_block_summary_update", "eta_decode_workspace_size", "eta_decode", "eta_decode_noalloc",
+SYMBOLS = ("eta_block_summary_update", "eta_append_kv", "eta_decode_workspace_size", "eta_decode", "eta_decode_noalloc",
            "eta_read_device_status", "eta_status_string", "eta_build_info")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
@@ -168,6 +172,20 @@ def eta_block_summary_update(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.T
                                        _stream_handle(stream))
     if rc != ETA_OK:
         raise EtaError(rc, "eta_block_summary_update")
+
+
+def eta_append_kv(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, summary: Dict[str, torch.Tensor],
+                  block_size: int, k_new: torch.Tensor, v_new: torch.Tensor, pos: torch.Tensor,
+                  n_q_heads: Optional[int] = None, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Write k_new / v_new [B, Hkv, d] at row pos[i] of each sequence and refresh
+    the summary of the block holding it (seq_lens must already count it)."""
+    cache = cache_desc(k, v, seq_lens, n_q_heads or k.shape[1], block_size)
+    summ = eta_summary_desc(summary["mu"].data_ptr(), summary["sigma"].data_ptr(),
+                            summary["max_norm"].data_ptr())
+    rc = _lib.eta_append_kv(ctypes.byref(cache), ctypes.byref(summ), ctypes.c_void_p(k_new.data_ptr()),
+                            ctypes.c_void_p(v_new.data_ptr()), ctypes.c_void_p(pos.data_ptr()), _stream_handle(stream))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_append_kv")
 
 
 def make_params(q, k, v, seq_lens, summary, block_size, tau_mode, w_tau=None, b_tau=None,

@@ -195,6 +195,37 @@ eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summa
   return launch_summary(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
 }
 
+eta_status eta_append_kv(const eta_cache_desc* cache, const eta_summary_desc* summary, const void* k_new,
+                         const void* v_new, const int* pos, void* stream) {
+  eta_status st = check_cache(cache);
+  if (st != ETA_OK) return st;
+  st = check_summary(summary);
+  if (st != ETA_OK) return st;
+  if (!k_new || !v_new || !pos || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(pos, 4))
+    return ETA_ERR_INVALID_ARG;
+  SummaryArgs a;
+  a.k = cache->k_cache;
+  a.seq_lens = cache->seq_lens;
+  a.first_token = nullptr;
+  a.mu = static_cast<uint16_t*>(summary->mu);
+  a.sigma = static_cast<uint16_t*>(summary->sigma);
+  a.max_norm = summary->max_norm;
+  a.B = cache->batch;
+  a.Hkv = cache->n_kv_heads;
+  a.d = cache->head_dim;
+  a.b = cache->block_size;
+  a.max_ctx = cache->max_ctx;
+  a.nbmax = (cache->max_ctx + cache->block_size - 1) / cache->block_size;
+  a.elt = cache->kv_dtype == ETA_F32 ? 4 : 2;
+  a.max_blocks = 1;
+  // The cache descriptor's pointers are const for the decode; the append
+  // writes through them by contract of this entry point.
+  return launch_append(a, k_new, v_new, pos, const_cast<void*>(cache->k_cache), const_cast<void*>(cache->v_cache),
+                       static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? ETA_OK
+             : ETA_ERR_CUDA;
+}
+
 eta_status eta_decode_workspace_size(const eta_decode_params* p, size_t* bytes) {
   if (!bytes) return ETA_ERR_INVALID_ARG;
   eta_status st = check_params(p);

@@ -115,6 +115,8 @@ struct SummaryArgs {
 
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_summary(const SummaryArgs& a, cudaStream_t st);
+cudaError_t launch_append(const SummaryArgs& a, const void* k_new, const void* v_new, const int* pos,
+                          void* k_cache, void* v_cache, cudaStream_t st);
 cudaError_t launch_screen(const ScreenArgs& a, cudaStream_t st);
 cudaError_t launch_rescue(const ScreenArgs& a, cudaStream_t st);
 cudaError_t launch_attend_simt(const AttendArgs& a, cudaStream_t st);

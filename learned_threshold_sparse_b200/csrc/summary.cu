@@ -3,6 +3,10 @@
 // the block's keys around the stored centroid in fp32, rounded up.
 // Source: Elastic Threshold Attention, Appendix F.1 (compact metadata layout)
 // and section 3.2; recomputed for the blocks an append touched.
+//
+// Two kernels: summary_kernel refreshes a range of blocks per sequence;
+// append_kernel writes one new token per (sequence, KV head) into the cache
+// and refreshes the block that holds it, in one launch.
 #include "eta_device.cuh"
 
 namespace eta {
@@ -10,35 +14,36 @@ namespace {
 
 constexpr int kThreads = 128;
 
-// One CTA per touched block.  Pass 1: mean per coordinate; pass 2: population
-// variance around the fp32 mean; pass 3: max over rows of ||k - mu_hat||^2.
-// All accumulation in fp32 (Appendix F.2 promotes squares and dot products to
-// fp32).
-__global__ void __launch_bounds__(kThreads) summary_kernel(SummaryArgs a) {
-  const int i = blockIdx.z, g = blockIdx.y;
-  int T = a.seq_lens[i];
-  T = T < 0 ? 0 : (T > a.max_ctx ? a.max_ctx : T);
-  const int nb = (T + a.b - 1) / a.b;
-  int ft = a.first_token[i];
-  ft = ft < 0 ? 0 : ft;
-  const int j = ft / a.b + static_cast<int>(blockIdx.x);
-  if (j >= nb) return;
-  const int r0 = j * a.b;
-  const int n = min(a.b, T - r0);
-  const size_t row0 = (static_cast<size_t>(i) * a.Hkv + g) * a.max_ctx + r0;
-  const int d = a.d;
-  const int t = threadIdx.x;
+__host__ __device__ inline size_t block_stage_bytes(int b, int d, int elt) {
+  return static_cast<size_t>(b) * d * elt;
+}
 
+// Summary of block j of (sequence i, KV head g) over its n present rows,
+// staged once in shared memory (raw K bytes).  Pass 1: mean per coordinate;
+// pass 2: population variance around the fp32 mean; pass 3: max over rows of
+// ||k - mu_hat||^2 with mu_hat the stored fp16 centroid.  All accumulation in
+// fp32 (Appendix F.2 promotes squares and dot products to fp32).
+__device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n, uint8_t* stage) {
+  const int d = a.d, t = threadIdx.x;
+  const size_t row0 = (static_cast<size_t>(i) * a.Hkv + g) * a.max_ctx + static_cast<size_t>(j) * a.b;
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.k) + row0 * d * a.elt);
+  const int nvec = n * d * a.elt / 16;
+  for (int x = t; x < nvec; x += kThreads) reinterpret_cast<uint4*>(stage)[x] = src[x];
   __shared__ float s_mu[128];
   __shared__ float s_wmax[kThreads / 32];
-
+  __syncthreads();
+  auto at = [&](int r, int e) -> float {
+    const size_t idx = static_cast<size_t>(r) * d + e;
+    if (a.elt == 4) return reinterpret_cast<const float*>(stage)[idx];
+    return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(stage)[idx]) << 16);
+  };
   if (t < d) {
     float sum = 0.f;
-    for (int r = 0; r < n; ++r) sum += dev::load_elt(a.k, (row0 + r) * d + t, a.elt);
+    for (int r = 0; r < n; ++r) sum += at(r, t);
     const float mean = sum / static_cast<float>(n);
     float ss = 0.f;
     for (int r = 0; r < n; ++r) {
-      const float x = dev::load_elt(a.k, (row0 + r) * d + t, a.elt) - mean;
+      const float x = at(r, t) - mean;
       ss = fmaf(x, x, ss);
     }
     const float sd = sqrtf(ss / static_cast<float>(n));
@@ -49,18 +54,16 @@ __global__ void __launch_bounds__(kThreads) summary_kernel(SummaryArgs a) {
     s_mu[t] = dev::fp16_to_f32(mu_h);
   }
   __syncthreads();
-
   // M_B: warp w takes rows w, w+4, ...; lanes split the coordinates.
   const int w = t >> 5, lane = t & 31;
   float best = 0.f;
   for (int r = w; r < n; r += kThreads / 32) {
     float ss = 0.f;
     for (int e = lane; e < d; e += 32) {
-      const float x = dev::load_elt(a.k, (row0 + r) * d + e, a.elt) - s_mu[e];
+      const float x = at(r, e) - s_mu[e];
       ss = fmaf(x, x, ss);
     }
-    ss = dev::warp_sum(ss);
-    best = fmaxf(best, ss);
+    best = fmaxf(best, dev::warp_sum(ss));
   }
   if (lane == 0) s_wmax[w] = best;
   __syncthreads();
@@ -74,11 +77,70 @@ __global__ void __launch_bounds__(kThreads) summary_kernel(SummaryArgs a) {
   }
 }
 
+__device__ __forceinline__ int clamp_len(int T, int max_ctx) { return T < 0 ? 0 : (T > max_ctx ? max_ctx : T); }
+
+// One CTA per touched block.
+__global__ void __launch_bounds__(kThreads) summary_kernel(SummaryArgs a) {
+  extern __shared__ __align__(16) uint8_t stage[];
+  const int i = blockIdx.z, g = blockIdx.y;
+  const int T = clamp_len(a.seq_lens[i], a.max_ctx);
+  const int nb = (T + a.b - 1) / a.b;
+  int ft = a.first_token[i];
+  ft = ft < 0 ? 0 : ft;
+  const int j = ft / a.b + static_cast<int>(blockIdx.x);
+  if (j >= nb) return;
+  summarize_block(a, i, g, j, min(a.b, T - j * a.b), stage);
+}
+
+// One CTA per (KV head, sequence): write the new token's K and V rows at
+// position pos[i], then refresh the block holding it over the rows present
+// (seq_lens[i] already counts the new token).  A position outside
+// [0, max_ctx) writes nothing.
+__global__ void __launch_bounds__(kThreads) append_kernel(SummaryArgs a, const void* k_new, const void* v_new,
+                                                          const int* pos, void* k_cache, void* v_cache) {
+  extern __shared__ __align__(16) uint8_t stage[];
+  const int g = blockIdx.x, i = blockIdx.y;
+  const int p = pos[i];
+  if (p < 0 || p >= a.max_ctx) return;
+  const int d = a.d, t = threadIdx.x;
+  const size_t src = (static_cast<size_t>(i) * a.Hkv + g) * d;
+  const size_t dst = ((static_cast<size_t>(i) * a.Hkv + g) * a.max_ctx + p) * d;
+  const int nvec = d * a.elt / 16;
+  for (int x = t; x < nvec; x += kThreads) {
+    reinterpret_cast<uint4*>(static_cast<uint8_t*>(k_cache) + dst * a.elt)[x] =
+        reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_new) + src * a.elt)[x];
+    reinterpret_cast<uint4*>(static_cast<uint8_t*>(v_cache) + dst * a.elt)[x] =
+        reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_new) + src * a.elt)[x];
+  }
+  __syncthreads();  // the new row is read back by the block summary below
+  const int T = clamp_len(a.seq_lens[i], a.max_ctx);
+  const int j = p / a.b;
+  if (j * a.b >= T) return;
+  summarize_block(a, i, g, j, min(a.b, T - j * a.b), stage);
+}
+
+template <class K>
+cudaError_t set_smem(K kern, size_t smem) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+}
+
 }  // namespace
 
 cudaError_t launch_summary(const SummaryArgs& a, cudaStream_t st) {
+  const size_t smem = block_stage_bytes(a.b, a.d, a.elt);
+  cudaError_t e = set_smem(summary_kernel, smem);
+  if (e != cudaSuccess) return e;
   dim3 grid(a.max_blocks, a.Hkv, a.B);
-  summary_kernel<<<grid, kThreads, 0, st>>>(a);
+  summary_kernel<<<grid, kThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append(const SummaryArgs& a, const void* k_new, const void* v_new, const int* pos,
+                          void* k_cache, void* v_cache, cudaStream_t st) {
+  const size_t smem = block_stage_bytes(a.b, a.d, a.elt);
+  cudaError_t e = set_smem(append_kernel, smem);
+  if (e != cudaSuccess) return e;
+  append_kernel<<<dim3(a.Hkv, a.B), kThreads, smem, st>>>(a, k_new, v_new, pos, k_cache, v_cache);
   return cudaGetLastError();
 }
 

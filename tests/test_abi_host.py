@@ -139,3 +139,15 @@ def test_struct_layout_matches_header(tmp_path):
         assert got[(sname, "size")] == ctypes.sizeof(cls), sname
         for fname, _ in cls._fields_:
             assert got[(sname, fname)] == getattr(cls, fname).offset, (sname, fname)
+
+
+def test_append_kv_validation():
+    fake = 1 << 20
+    c = eta.eta_cache_desc(1, 4, 4, 64, 64, 4096, eta.ETA_BF16, fake, fake, fake)
+    s = eta.eta_summary_desc(fake, fake, fake)
+    lib = eta.library()
+    assert lib.eta_append_kv(ctypes.byref(c), ctypes.byref(s), None, fake, fake, None) == eta.ETA_ERR_INVALID_ARG
+    assert lib.eta_append_kv(ctypes.byref(c), ctypes.byref(s), fake, fake + 8, fake, None) == eta.ETA_ERR_INVALID_ARG
+    assert lib.eta_append_kv(ctypes.byref(c), ctypes.byref(s), fake, fake, fake + 2, None) == eta.ETA_ERR_INVALID_ARG
+    c2 = eta.eta_cache_desc(1, 4, 4, 96, 64, 4096, eta.ETA_BF16, fake, fake, fake)
+    assert lib.eta_append_kv(ctypes.byref(c2), ctypes.byref(s), fake, fake, fake, None) == eta.ETA_ERR_UNSUPPORTED

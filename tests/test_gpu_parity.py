@@ -87,6 +87,38 @@ def test_summary_append_touches_only_tail_block():
     assert torch.equal(summ["max_norm"][1, :, :10], before["max_norm"][1, :, :10])
 
 
+@pytest.mark.parametrize("dtype,d,b", [(BF16, 128, 64), (F32, 64, 128), (BF16, 64, 32)])
+def test_append_kv_writes_rows_and_refreshes_block(dtype, d, b):
+    wl = workloads.custom(seed=13, batch=3, n_q_heads=4, n_kv_heads=2, head_dim=d, block_size=b,
+                          seq_lens=[700, 640, 300], dtype=dtype, max_ctx=800)
+    t = upload(wl)
+    summ = gpu_summary(wl, t)
+    before = {k: v.clone() for k, v in summ.items()}
+    gen = torch.Generator().manual_seed(7)
+    knew = torch.randn(3, 2, d, generator=gen).to(wl.torch_dtype)
+    vnew = torch.randn(3, 2, d, generator=gen).to(wl.torch_dtype)
+    pos = [700, 640, 800]  # the third position is outside the cache: nothing written
+    new_lens = [701, 641, 300]
+    t["seq"] = torch.tensor(new_lens, dtype=torch.int32, device="cuda")
+    eta.eta_append_kv(t["k"], t["v"], t["seq"], summ, b, knew.cuda(), vnew.cuda(),
+                      torch.tensor(pos, dtype=torch.int32, device="cuda"), 4)
+    torch.cuda.synchronize()
+    k_ref, v_ref = wl.k.clone(), wl.v.clone()
+    for i in range(2):
+        k_ref[i, :, pos[i]] = knew[i]
+        v_ref[i, :, pos[i]] = vnew[i]
+    assert torch.equal(t["k"].cpu(), k_ref) and torch.equal(t["v"].cpu(), v_ref)
+    ref = oracle.summarize(k_ref, new_lens, b)
+    for i in range(2):
+        j = pos[i] // b
+        got = summ["mu"][i, :, j].cpu().numpy().astype(np.float32)
+        r = ref["mu"][i, :, j].astype(np.float32)
+        assert np.all(np.abs(got - r) <= _fp16_ulp(r))
+        np.testing.assert_allclose(summ["max_norm"][i, :, j].cpu().numpy(), ref["max_norm"][i, :, j], rtol=2e-5)
+        assert torch.equal(summ["mu"][i, :, :j], before["mu"][i, :, :j])
+    assert torch.equal(summ["mu"][2], before["mu"][2]) and torch.equal(summ["max_norm"][2], before["max_norm"][2])
+
+
 # ------------------------------------------------------------ decode, small
 
 SMALL = [
