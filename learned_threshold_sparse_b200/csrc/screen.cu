@@ -118,6 +118,20 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
   }
   for (int x = t; x < avail; x += kThreads) s_mn[x] = a.max_norm[nbase + blk0 + x];
 
+  // Threshold inputs of this warp's head, loaded now so that they share the
+  // first round trip with the metadata copies and the query rows.
+  float w_reg[D / 32], q_reg[D / 32];
+  float b_or_c = 0.f;
+  if (w < G) {
+    const int hq = g * G + w;
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) {
+      const int e = lane + 32 * k;
+      q_reg[k] = dev::load_elt(a.q, (static_cast<size_t>(i) * s.Hq + hq) * D + e, s.elt);
+      w_reg[k] = a.tau_mode == ETA_TAU_LEARNED ? a.w_tau[static_cast<size_t>(hq) * D + e] : 0.f;
+    }
+    b_or_c = a.tau_mode == ETA_TAU_LEARNED ? a.b_tau[hq] : a.c_tau[hq];
+  }
   int T = a.seq_lens[i];
   if (T < 0 || T > s.max_ctx) {
     if (t == 0 && c == 0 && g == 0) atomicOr(a.status, kStatusRange);
@@ -145,18 +159,17 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
     }
     if (t < G && a.lse) a.lse[static_cast<size_t>(i) * s.Hq + g * G + t] = -INFINITY;
   }
-  __syncthreads();
   if (w < G) {
     const int hq = g * G + w;
     float tw = 0.f, qq = 0.f;
-    for (int e = lane; e < D; e += 32) {
-      const float qe = s_q[w][e];
-      qq = fmaf(qe, qe, qq);
-      if (a.tau_mode == ETA_TAU_LEARNED) tw = fmaf(a.w_tau[static_cast<size_t>(hq) * D + e], qe, tw);
+#pragma unroll
+    for (int k = 0; k < D / 32; ++k) {
+      qq = fmaf(q_reg[k], q_reg[k], qq);
+      tw = fmaf(w_reg[k], q_reg[k], tw);
     }
     tw = dev::warp_sum(tw);
     qq = dev::warp_sum(qq);
-    const float tau = (a.tau_mode == ETA_TAU_LEARNED ? tw + a.b_tau[hq] : a.c_tau[hq]) - a.offset_a;
+    const float tau = (a.tau_mode == ETA_TAU_LEARNED ? tw + b_or_c : b_or_c) - a.offset_a;
     if (lane == 0) {
       s_tau[w] = tau;
       s_qn[w] = sqrtf(qq);
