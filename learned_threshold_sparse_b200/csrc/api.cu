@@ -42,13 +42,6 @@ eta_status check_summary(const eta_summary_desc* s) {
   return ETA_OK;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-  return n;
-}
-
 eta_status make_shape(const eta_decode_params* p, Shape* out) {
   const eta_cache_desc& c = p->cache;
   Shape s;
@@ -65,7 +58,9 @@ eta_status make_shape(const eta_decode_params* p, Shape* out) {
   // Screen CTAs cover `chunk` blocks: about two screen CTAs per SM (one
   // resident wave), and at most 4096 (segment, chunk) pairs so the attention
   // kernel's prefix table fits in shared memory.
-  const int sms_for_chunk = sm_count() > 0 ? sm_count() : 148;
+  const int sms = device_sms();
+  if (sms <= 0) return ETA_ERR_CUDA;
+  const int sms_for_chunk = sms;
   int chunk = 32;
   auto pairs = [&](int ch) { return static_cast<long long>(s.nseg) * ((s.nbmax + ch - 1) / ch); };
   while (chunk < 1024 && (pairs(chunk) > 2LL * sms_for_chunk || pairs(chunk) > 4096)) chunk *= 2;
@@ -77,8 +72,6 @@ eta_status make_shape(const eta_decode_params* p, Shape* out) {
   const bool tc_ok = attend_tc_supported(s);
   if (p->attend_impl == ETA_ATTEND_TC && !tc_ok) return ETA_ERR_UNSUPPORTED;
   s.attend_kind = (p->attend_impl == ETA_ATTEND_SIMT || !tc_ok) ? ETA_ATTEND_SIMT : ETA_ATTEND_TC;
-  const int sms = sm_count();
-  if (sms <= 0) return ETA_ERR_CUDA;
   if (s.attend_kind == ETA_ATTEND_SIMT) {
     if (attend_simt_smem(s) == 0) return ETA_ERR_UNSUPPORTED;
     s.attend_ctas = sms * attend_simt_ctas_per_sm(s);
@@ -120,6 +113,41 @@ eta_status check_params(const eta_decode_params* p) {
 }
 
 }  // namespace
+
+int device_sms() {
+  static std::atomic<int> cache[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  if (slot) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (slot) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+cudaError_t ensure_smem(const void* kern, size_t bytes, SmemLimit& lim, bool* skipped) {
+  *skipped = false;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const int want = static_cast<int>(bytes);
+  const bool slot = dev >= 0 && dev < kMaxDevices;
+  if (slot && lim.bytes[dev].load(std::memory_order_relaxed) >= want) {
+    *skipped = true;
+    return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, want);
+  if (e == cudaSuccess && slot) {
+    int cur = lim.bytes[dev].load(std::memory_order_relaxed);
+    while (cur < want && !lim.bytes[dev].compare_exchange_weak(cur, want, std::memory_order_relaxed)) {
+    }
+  }
+  return e;
+}
 
 Workspace workspace_layout(const Shape& s) {
   Workspace w;

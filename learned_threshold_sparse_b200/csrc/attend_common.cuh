@@ -18,15 +18,19 @@ struct UnitInfo {
 };
 
 // Exclusive prefix of the chunk counts into prefix[0..n] (prefix[n] = total),
-// computed by all `nthreads` threads of the CTA.  Ends with __syncthreads().
+// computed by all `nthreads` threads of the CTA: one coalesced pass copies the
+// counts into shared memory, then every thread scans a contiguous slice in
+// place.  Ends with __syncthreads().
 template <int NTHREADS>
 __device__ __forceinline__ void chunk_prefix(const int* __restrict__ counts, int n, int* prefix) {
   __shared__ int s_warp[NTHREADS / 32];
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  for (int x = t; x < n; x += NTHREADS) prefix[x] = counts[x];
+  __syncthreads();
   const int per = (n + NTHREADS - 1) / NTHREADS;
   const int lo = min(n, t * per), hi = min(n, lo + per);
   int sum = 0;
-  for (int x = lo; x < hi; ++x) sum += counts[x];
+  for (int x = lo; x < hi; ++x) sum += prefix[x];
   int incl = sum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -39,7 +43,7 @@ __device__ __forceinline__ void chunk_prefix(const int* __restrict__ counts, int
   for (int k = 0; k < warp; ++k) woff += s_warp[k];
   int run = woff + incl - sum;
   for (int x = lo; x < hi; ++x) {
-    const int c = counts[x];
+    const int c = prefix[x];
     prefix[x] = run;
     run += c;
   }
@@ -47,12 +51,33 @@ __device__ __forceinline__ void chunk_prefix(const int* __restrict__ counts, int
   __syncthreads();
 }
 
+// Split of the U units over N CTAs: CTA c owns [start(c), start(c + 1)) with
+// start(c) = floor(U c / N).  The host keeps U below 2^24 (segments x chunks
+// and the chunk size are both bounded) and N is a few hundred at most, so
+// with U = q N + r every product below fits in 32 bits.
+struct UnitSplit {
+  unsigned U, N, q, r;
+  __device__ __forceinline__ UnitSplit(unsigned u, unsigned n) : U(u), N(n), q(u / n), r(u % n) {}
+  __device__ __forceinline__ unsigned start(unsigned c) const { return q * c + (r * c) / N; }
+  __device__ __forceinline__ bool owns_any(unsigned c) const { return start(c) != start(c + 1); }
+  // The CTA whose range holds unit u < U: a floating-point estimate of
+  // u N / U, corrected to the exact range boundaries.
+  __device__ __forceinline__ unsigned owner(unsigned u) const {
+    unsigned c = static_cast<unsigned>((static_cast<float>(u) + 0.5f) * static_cast<float>(N) / static_cast<float>(U));
+    if (c > N - 1) c = N - 1;
+    while (c + 1 < N && start(c + 1) <= u) ++c;
+    while (c > 0 && start(c) > u) --c;
+    return c;
+  }
+};
+
 // Walk the units [u0, u0 + nunits) with one warp.  `issue(info)` runs on lane
 // 0 for every unit, in order, and returns false to stop (abort).  Returns
-// false if the walk was stopped or the counts were inconsistent.
+// false if the walk was stopped or the counts were inconsistent.  seq_T, when
+// not null, holds the clamped sequence lengths in shared memory.
 template <class Issue>
-__device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefix, int nprefix, long long u0,
-                                           int nunits, Issue&& issue) {
+__device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefix, int nprefix, int u0, int nunits,
+                                           const int* seq_T, Issue&& issue) {
   const Shape& s = a.s;
   const int lane = threadIdx.x & 31;
   int lo = 0, hi = nprefix;  // invariant prefix[lo] <= u0 < prefix[hi]
@@ -61,7 +86,7 @@ __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefi
     if (prefix[mid] <= u0) lo = mid; else hi = mid;
   }
   int x = lo;
-  int idx = static_cast<int>(u0 - prefix[x]);
+  int idx = u0 - prefix[x];
   int remaining = nunits;
   int cur_seg = -1, T = 0;
   while (remaining > 0) {
@@ -73,8 +98,12 @@ __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefi
     const int cin = x - seg * s.nchunks;
     if (seg != cur_seg) {
       cur_seg = seg;
-      const int tt = a.seq_lens[seg / s.Hkv];
-      T = tt < 0 ? 0 : (tt > s.max_ctx ? s.max_ctx : tt);
+      if (seq_T) {
+        T = seq_T[seg / s.Hkv];
+      } else {
+        const int tt = a.seq_lens[seg / s.Hkv];
+        T = tt < 0 ? 0 : (tt > s.max_ctx ? s.max_ctx : tt);
+      }
     }
     const int* list = a.chunk_list + static_cast<size_t>(seg) * s.list_stride + static_cast<size_t>(cin) * s.chunk + idx;
     for (int j0 = 0; j0 < take; j0 += 32) {
@@ -99,9 +128,10 @@ __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefi
   return true;
 }
 
-// Tiles of up to `bpt` consecutive units of one segment that the unit range
+// Tiles of up to BPT consecutive units of one segment that the unit range
 // [u0, u1) splits into (a tile never crosses a segment boundary).
-__device__ __forceinline__ int count_tiles(const int* prefix, const Shape& s, long long u0, long long u1, int bpt) {
+template <int BPT>
+__device__ __forceinline__ int count_tiles(const int* prefix, const Shape& s, int u0, int u1) {
   if (u1 <= u0) return 0;
   int lo = 0, hi = s.nseg;  // last segment whose first unit is <= u0
   while (hi - lo > 1) {
@@ -110,40 +140,12 @@ __device__ __forceinline__ int count_tiles(const int* prefix, const Shape& s, lo
   }
   int tiles = 0;
   for (int seg = lo; seg < s.nseg; ++seg) {
-    const long long a = max(u0, static_cast<long long>(prefix[seg * s.nchunks]));
-    const long long b = min(u1, static_cast<long long>(prefix[(seg + 1) * s.nchunks]));
+    const int a = max(u0, prefix[seg * s.nchunks]);
+    const int b = min(u1, prefix[(seg + 1) * s.nchunks]);
     if (a >= u1) break;
-    if (b > a) tiles += static_cast<int>((b - a + bpt - 1) / bpt);
+    if (b > a) tiles += (b - a + BPT - 1) / BPT;
   }
   return tiles;
-}
-
-// The attention CTAs covering segment seg: CTA c owns units
-// [U c / N, U (c + 1) / N), so unit u belongs to CTA ((u + 1) N - 1) / U.
-// Returns how many of the CTAs in [c0, c1] own at least one unit (with fewer
-// units than CTAs some ranges are empty; those CTAs write no partial).
-struct SegCtas {
-  int c0, c1, n;
-  bool all;  // U >= N: every CTA owns a unit
-  // With U < N both U and N are small, so 32-bit arithmetic is exact.
-  __device__ __forceinline__ bool owns(int c, long long U, long long N) const {
-    if (all) return true;
-    const unsigned u = static_cast<unsigned>(U), nn = static_cast<unsigned>(N), cc = static_cast<unsigned>(c);
-    return u * cc / nn != u * (cc + 1u) / nn;
-  }
-};
-
-__device__ __forceinline__ SegCtas seg_ctas(long long us, long long ue, long long U, long long N) {
-  SegCtas r{0, -1, 0, U >= N};
-  if (ue <= us) return r;
-  r.c0 = static_cast<int>(((us + 1) * N - 1) / U);
-  r.c1 = static_cast<int>((ue * N - 1) / U);
-  if (r.all) {
-    r.n = r.c1 - r.c0 + 1;
-  } else {
-    for (int c = r.c0; c <= r.c1; ++c) r.n += r.owns(c, U, N) ? 1 : 0;
-  }
-  return r;
 }
 
 // Output element idx (kv dtype: fp32, or bf16 rounded to nearest even).

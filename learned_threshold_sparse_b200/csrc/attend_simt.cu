@@ -132,11 +132,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
   // Exclusive prefix of the per-chunk entry counts, in (segment, chunk) order.
   dev::chunk_prefix<kThreads>(a.chunk_count, nprefix, prefix);
 
-  const long long U = prefix[nprefix];
-  const long long N = gridDim.x;
-  const long long u0 = U * blockIdx.x / N;
-  const long long u1 = U * (blockIdx.x + 1) / N;
-  const int nunits = static_cast<int>(u1 - u0);
+  const dev::UnitSplit split(static_cast<unsigned>(prefix[nprefix]), gridDim.x);
+  const int u0 = static_cast<int>(split.start(blockIdx.x));
+  const int u1 = static_cast<int>(split.start(blockIdx.x + 1));
+  const int nunits = u1 - u0;
   if (blockIdx.x == 0) {
     for (int sg = t; sg <= s.nseg; sg += kThreads) a.seg_start[sg] = prefix[sg * s.nchunks];
   }
@@ -146,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
     // ------------------------------------------------------------ producer
     int stage = 0;
     uint32_t phase = 0;
-    const bool ok = dev::walk_units(a, prefix, nprefix, u0, nunits, [&](const UnitInfo& in) -> bool {
+    const bool ok = dev::walk_units(a, prefix, nprefix, u0, nunits, nullptr, [&](const UnitInfo& in) -> bool {
       if (!wait_or_abort(&empty[stage], phase ^ 1u, a.status, abort_flag)) return false;
       info[stage] = in;
       const uint32_t bytes = static_cast<uint32_t>(in.nrows) * D * ELT;
@@ -221,7 +220,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
       }
     }
     if (!rendezvous()) return false;
-    const dev::SegCtas sc = dev::seg_ctas(prefix[seg * s.nchunks], prefix[(seg + 1) * s.nchunks], U, N);
+    // no other CTA touches the segment when all its units are in this range
+    const bool sole = prefix[seg * s.nchunks] >= u0 && prefix[(seg + 1) * s.nchunks] <= u1;
     const int si = seg / s.Hkv, sg = seg - si * s.Hkv;
     float* part = a.partials + static_cast<size_t>(seg + blockIdx.x) * G * partial_stride(D);
     for (int x = t; x < G * D; x += kConsumerWarps * 32) {
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
           lsum = fmaf(f, ws[D + 1], lsum);
         }
       }
-      if (sc.n == 1) {
+      if (sole) {
         const size_t orow = static_cast<size_t>(si) * s.Hq + sg * G + h;
         dev::store_out(a, orow * D + e, lsum > 0.f ? sum / lsum : 0.f);
         if (e == 0 && a.lse) a.lse[orow] = dev::lse_of(mstar, lsum);
@@ -352,8 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
 template <int ELT, int D, int G>
 cudaError_t launch_typed(const AttendArgs& a, cudaStream_t st, int stages, size_t smem) {
   auto kern = attend_simt_kernel<ELT, D, G>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  static SmemLimit lim;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.s.attend_ctas);
   cfg.blockDim = dim3(kThreads);
@@ -364,7 +363,8 @@ cudaError_t launch_typed(const AttendArgs& a, cudaStream_t st, int stages, size_
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, a, stages);
+  return launch_with_smem(reinterpret_cast<const void*>(kern), smem, lim,
+                          [&] { return cudaLaunchKernelEx(&cfg, kern, a, stages); });
 }
 
 template <int ELT, int D>

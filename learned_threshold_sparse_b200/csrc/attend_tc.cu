@@ -47,6 +47,7 @@ constexpr int kMaxStages = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int TR = 128;  // key rows per tile
+constexpr int kSmemSeqs = 256;  // sequence lengths staged in shared memory up to this batch
 
 struct Tile {
   static constexpr int PANEL = TR * 128;  // one 64-column (128-byte) panel of a 128-row tile
@@ -62,13 +63,15 @@ struct TileInfo {
 };
 
 struct Layout {
-  size_t stages, pbuf, bars, info, red, prefix, misc, total;
+  size_t stages, pbuf, bars, info, red, prefix, seqs, misc, total;
 };
 
 __host__ __device__ inline size_t align_to(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Offsets relative to a 1024-byte aligned base.
-__host__ __device__ inline Layout tc_layout(int nstages, int nprefix) {
+__host__ __device__ inline int smem_seqs(int B) { return B <= kSmemSeqs ? B : 0; }
+
+__host__ __device__ inline Layout tc_layout(int nstages, int nprefix, int nseqs) {
   Layout L;
   const size_t stage = static_cast<size_t>(Tile::STAGE);
   const size_t pbytes = static_cast<size_t>(Tile::P_BYTES);
@@ -85,6 +88,8 @@ __host__ __device__ inline Layout tc_layout(int nstages, int nprefix) {
   off += 2 * 4 * 8 * sizeof(float) + 4 * 8 * sizeof(float);
   L.prefix = off = align_to(off, 16);
   off += static_cast<size_t>(nprefix + 1) * sizeof(int);
+  L.seqs = off = align_to(off, 16);
+  off += static_cast<size_t>(nseqs) * sizeof(int);
   L.misc = off = align_to(off, 16);
   off += 16 + kMaxStages * sizeof(int) + 16;
   L.total = align_to(off, 128) + 1024;  // + slack to align the dynamic base to 1024
@@ -182,7 +187,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t raw = dev::smem_u32(smem_raw);
   const uint32_t base_u32 = (raw + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - raw);
-  const Layout L = tc_layout(nstages, nprefix);
+  const int nseqs = smem_seqs(s.B);
+  const Layout L = tc_layout(nstages, nprefix, nseqs);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L.bars);
   Bars B;
@@ -198,6 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   TileInfo* info = reinterpret_cast<TileInfo*>(base + L.info);
   float* red = reinterpret_cast<float*>(base + L.red);  // [2][4][8] tile maxima, then [4][8] flush sums
   int* prefix = reinterpret_cast<int*>(base + L.prefix);
+  int* seq_T = reinterpret_cast<int*>(base + L.seqs);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L.misc + 4);
   int* issued_parity = reinterpret_cast<int*>(base + L.misc + 32);
@@ -231,6 +238,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tv)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tq)) : "memory");
   }
+  // Inputs the screen does not write are read while it still runs.
+  for (int x = t; x < nseqs; x += kThreads) {
+    const int tt = a.seq_lens[x];
+    seq_T[x] = tt < 0 ? 0 : (tt > s.max_ctx ? s.max_ctx : tt);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -240,15 +252,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   dev::pdl_trigger();
   dev::chunk_prefix<kThreads>(a.chunk_count, nprefix, prefix);
 
-  const long long U = prefix[nprefix];
-  const long long N = gridDim.x;
-  const long long u0 = U * blockIdx.x / N;
-  const long long u1 = U * (blockIdx.x + 1) / N;
-  const int nunits = static_cast<int>(u1 - u0);
+  const dev::UnitSplit split(static_cast<unsigned>(prefix[nprefix]), gridDim.x);
+  const int u0 = static_cast<int>(split.start(blockIdx.x));
+  const int u1 = static_cast<int>(split.start(blockIdx.x + 1));
+  const int nunits = u1 - u0;
   if (blockIdx.x == 0)
     for (int sg = t; sg <= s.nseg; sg += kThreads) a.seg_start[sg] = prefix[sg * s.nchunks];
 
-  const int ntiles = dev::count_tiles(prefix, s, u0, u1, BPT);
+  const int ntiles = dev::count_tiles<BPT>(prefix, s, u0, u1);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -281,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         npend = 0;
         return true;
       };
-      bool ok = dev::walk_units(a, prefix, nprefix, u0, nunits, [&](const UnitInfo& in) -> bool {
+      bool ok = dev::walk_units(a, prefix, nprefix, u0, nunits, nseqs ? seq_T : nullptr,
+                                [&](const UnitInfo& in) -> bool {
         if (npend > 0 && (in.seg != pend.seg || npend == BPT) && !emit()) return false;
         if (npend == 0) pend = TileInfo{in.seg, 0, 0, 0, 0};
         pblk[npend] = in.blk;
@@ -410,8 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) sums[q4 * 8 + h] = lw;
       }
       if (!rendezvous()) return false;
-      const dev::SegCtas sc = dev::seg_ctas(prefix[seg * s.nchunks], prefix[(seg + 1) * s.nchunks], U, N);
-      if (sc.n == 1) {
+      // no other CTA touches the segment when all its units are in this range
+      if (prefix[seg * s.nchunks] >= u0 && prefix[(seg + 1) * s.nchunks] <= u1) {
         const int i = seg / s.Hkv, g = seg - i * s.Hkv;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -538,7 +550,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
+bool encode_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
@@ -550,11 +562,35 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows)
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The maps of the last few (pointer, rows, box) triples, per host thread: a
+// decode loop over a fixed cache re-encodes nothing.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
+  struct Entry {
+    const void* ptr;
+    uint64_t rows;
+    uint32_t box;
+    CUtensorMap map;
+  };
+  constexpr int kEntries = 8;
+  thread_local Entry cache[kEntries] = {};
+  thread_local int next = 0;
+  for (int i = 0; i < kEntries; ++i) {
+    if (cache[i].ptr == ptr && cache[i].rows == rows && cache[i].box == box_rows && ptr) {
+      *m = cache[i].map;
+      return true;
+    }
+  }
+  if (!encode_map(m, ptr, rows, box_rows)) return false;
+  cache[next] = Entry{ptr, rows, box_rows, *m};
+  next = (next + 1) % kEntries;
+  return true;
+}
+
 constexpr size_t kSmemBudget = 224 * 1024;
 
 int pick_stages(const Shape& s) {
   for (int st = kMaxStages; st >= 2; --st)
-    if (tc_layout(st, s.nseg * s.nchunks).total <= kSmemBudget) return st;
+    if (tc_layout(st, s.nseg * s.nchunks, smem_seqs(s.B)).total <= kSmemBudget) return st;
   return 0;
 }
 
@@ -562,8 +598,7 @@ template <int BR, int G>
 cudaError_t launch_typed(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq, const AttendArgs& a,
                          cudaStream_t st, int stages, size_t smem) {
   auto kern = attend_tc_kernel<BR, G>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
+  static SmemLimit lim;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(a.s.attend_ctas);
   cfg.blockDim = dim3(kThreads);
@@ -574,7 +609,8 @@ cudaError_t launch_typed(const CUtensorMap& tk, const CUtensorMap& tv, const CUt
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, a, stages);
+  return launch_with_smem(reinterpret_cast<const void*>(kern), smem, lim,
+                          [&] { return cudaLaunchKernelEx(&cfg, kern, tk, tv, tq, a, stages); });
 }
 
 template <int BR>
@@ -597,13 +633,13 @@ bool attend_tc_supported(const Shape& s) {
 
 size_t attend_tc_smem(const Shape& s) {
   const int st = pick_stages(s);
-  return st ? tc_layout(st, s.nseg * s.nchunks).total : 0;
+  return st ? tc_layout(st, s.nseg * s.nchunks, smem_seqs(s.B)).total : 0;
 }
 
 cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st) {
   const int stages = pick_stages(a.s);
   if (stages == 0) return cudaErrorInvalidConfiguration;
-  const size_t smem = tc_layout(stages, a.s.nseg * a.s.nchunks).total;
+  const size_t smem = tc_layout(stages, a.s.nseg * a.s.nchunks, smem_seqs(a.s.B)).total;
   CUtensorMap tk, tv, tq;
   const uint64_t rows = static_cast<uint64_t>(a.s.nseg) * a.s.max_ctx;
   if (!make_map(&tk, a.k, rows, a.s.b) || !make_map(&tv, a.v, rows, a.s.b) ||

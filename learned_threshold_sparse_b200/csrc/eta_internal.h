@@ -6,6 +6,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "eta.h"
 
 namespace eta {
@@ -112,6 +114,47 @@ struct SummaryArgs {
   float* max_norm;
   int B, Hkv, d, b, max_ctx, nbmax, elt, max_blocks;
 };
+
+// ---------------------------------------------------------------- host helpers
+// Driver attribute queries and settings cost on the order of a microsecond
+// each; a decode issues several launches, so their per-device results are
+// cached here (api.cu).
+
+constexpr int kMaxDevices = 64;
+
+// Largest dynamic shared memory already allowed for one kernel, per device.
+struct SmemLimit {
+  std::atomic<int> bytes[kMaxDevices];
+  void forget(int dev) {
+    if (dev >= 0 && dev < kMaxDevices) bytes[dev].store(0, std::memory_order_relaxed);
+  }
+};
+
+// Raises `kern`'s dynamic shared memory limit on the current device to at
+// least `bytes` unless the cache says it already is; *skipped reports that.
+cudaError_t ensure_smem(const void* kern, size_t bytes, SmemLimit& lim, bool* skipped);
+
+// ensure_smem + launch().  If the launch fails after the attribute call was
+// skipped (the setting can be lost, e.g. by a device reset), the attribute is
+// set again and the launch retried once.
+template <class Launch>
+cudaError_t launch_with_smem(const void* kern, size_t bytes, SmemLimit& lim, Launch&& launch) {
+  bool skipped = false;
+  cudaError_t e = ensure_smem(kern, bytes, lim, &skipped);
+  if (e != cudaSuccess) return e;
+  e = launch();
+  if (e != cudaSuccess && skipped) {
+    (void)cudaGetLastError();
+    int dev = -1;
+    if (cudaGetDevice(&dev) == cudaSuccess) lim.forget(dev);
+    e = ensure_smem(kern, bytes, lim, &skipped);
+    if (e == cudaSuccess) e = launch();
+  }
+  return e;
+}
+
+// Streaming multiprocessors of the current device (0 on error), cached.
+int device_sms();
 
 // Launchers (each returns the launch's cudaError_t).
 cudaError_t launch_summary(const SummaryArgs& a, cudaStream_t st);

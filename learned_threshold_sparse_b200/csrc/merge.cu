@@ -29,16 +29,17 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(MergeArgs a) {
   const int seg = blockIdx.x / s.G, h = blockIdx.x - seg * s.G;
   const int slice = blockIdx.y;
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-  const long long U = a.seg_start[s.nseg];
-  const long long N = s.attend_ctas;
-  const dev::SegCtas sc = dev::seg_ctas(a.seg_start[seg], a.seg_start[seg + 1], U, N);
-  if (sc.n <= 1) return;  // written by its only attention CTA (or empty)
+  const int us = a.seg_start[seg], ue = a.seg_start[seg + 1];
+  if (ue <= us) return;  // empty segment
+  const dev::UnitSplit split(static_cast<unsigned>(a.seg_start[s.nseg]), static_cast<unsigned>(s.attend_ctas));
+  const int c0 = static_cast<int>(split.owner(us)), c1 = static_cast<int>(split.owner(ue - 1));
+  if (c0 == c1) return;  // written by its only attention CTA
 
   const int PS = partial_stride(s.d);
   const size_t cstride = static_cast<size_t>(s.G) * PS;
   const float* col = a.partials + static_cast<size_t>(seg) * cstride + static_cast<size_t>(h) * PS;
   const int e = slice * 32 + lane;
-  const int span = sc.c1 - sc.c0 + 1;
+  const int span = c1 - c0 + 1;
 
   float mx = -INFINITY, ls = 0.f, acc = 0.f;
   for (int k0 = w; k0 < span; k0 += kMergeWarps * kBatch) {
@@ -46,7 +47,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(MergeArgs a) {
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int k = min(k0 + u * kMergeWarps, span - 1);
-      const float* p = col + static_cast<size_t>(sc.c0 + k) * cstride;
+      const float* p = col + static_cast<size_t>(c0 + k) * cstride;
       m[u] = __ldcg(p + s.d);
       l[u] = __ldcg(p + s.d + 1);
       x[u] = __ldcg(p + e);
@@ -55,7 +56,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(MergeArgs a) {
     for (int u = 0; u < kBatch; ++u) {
       const int k = k0 + u * kMergeWarps;
       // an unused slot may hold any bits: skip it rather than weight it by 0
-      if (k >= span || !sc.owns(sc.c0 + k, U, N) || m[u] == -INFINITY) continue;
+      if (k >= span || !split.owns_any(c0 + k) || m[u] == -INFINITY) continue;
       if (m[u] > mx) {
         const float f = (mx == -INFINITY) ? 0.f : dev::fast_exp2(mx - m[u]);
         ls = fmaf(ls, f, l[u]);

@@ -331,11 +331,11 @@ template <int D, int G>
 cudaError_t launch_screen_typed(const ScreenArgs& a, cudaStream_t st) {
   const size_t smem = screen_smem_bytes<D>(a.s.chunk);
   auto kern = screen_kernel<D, G>;
-  const cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(screen_smem_bytes<D>(2 * kRound)));
-  if (e != cudaSuccess) return e;
-  kern<<<dim3(a.s.nchunks, a.s.Hkv, a.s.B), kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  static SmemLimit lim;
+  return launch_with_smem(reinterpret_cast<const void*>(kern), screen_smem_bytes<D>(2 * kRound), lim, [&] {
+    kern<<<dim3(a.s.nchunks, a.s.Hkv, a.s.B), kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+  });
 }
 
 template <int D>

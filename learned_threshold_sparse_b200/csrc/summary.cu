@@ -119,29 +119,25 @@ __global__ void __launch_bounds__(kThreads) append_kernel(SummaryArgs a, const v
   summarize_block(a, i, g, j, min(a.b, T - j * a.b), stage);
 }
 
-template <class K>
-cudaError_t set_smem(K kern, size_t smem) {
-  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-}
-
 }  // namespace
 
 cudaError_t launch_summary(const SummaryArgs& a, cudaStream_t st) {
   const size_t smem = block_stage_bytes(a.b, a.d, a.elt);
-  cudaError_t e = set_smem(summary_kernel, smem);
-  if (e != cudaSuccess) return e;
-  dim3 grid(a.max_blocks, a.Hkv, a.B);
-  summary_kernel<<<grid, kThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  static SmemLimit lim;
+  return launch_with_smem(reinterpret_cast<const void*>(summary_kernel), smem, lim, [&] {
+    summary_kernel<<<dim3(a.max_blocks, a.Hkv, a.B), kThreads, smem, st>>>(a);
+    return cudaGetLastError();
+  });
 }
 
 cudaError_t launch_append(const SummaryArgs& a, const void* k_new, const void* v_new, const int* pos,
                           void* k_cache, void* v_cache, cudaStream_t st) {
   const size_t smem = block_stage_bytes(a.b, a.d, a.elt);
-  cudaError_t e = set_smem(append_kernel, smem);
-  if (e != cudaSuccess) return e;
-  append_kernel<<<dim3(a.Hkv, a.B), kThreads, smem, st>>>(a, k_new, v_new, pos, k_cache, v_cache);
-  return cudaGetLastError();
+  static SmemLimit lim;
+  return launch_with_smem(reinterpret_cast<const void*>(append_kernel), smem, lim, [&] {
+    append_kernel<<<dim3(a.Hkv, a.B), kThreads, smem, st>>>(a, k_new, v_new, pos, k_cache, v_cache);
+    return cudaGetLastError();
+  });
 }
 
 }  // namespace eta
