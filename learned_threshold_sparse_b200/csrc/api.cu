@@ -164,8 +164,6 @@ Workspace workspace_layout(const Shape& s) {
   off = align256(off + static_cast<size_t>(s.B) * s.Hq * sizeof(int));
   w.head_best = off;
   off = align256(off + static_cast<size_t>(s.B) * s.Hq * sizeof(unsigned long long));
-  w.seg_start = off;
-  off = align256(off + static_cast<size_t>(s.nseg + 1) * sizeof(int));
   w.partials = off;
   off = align256(off + static_cast<size_t>(s.nseg + s.attend_ctas) * s.G * partial_stride(s.d) * sizeof(float));
   w.total = off;
@@ -307,7 +305,7 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
 
   ev(0);
   if (s.rescue) {
-    if (cudaMemsetAsync(ws + w.head_count, 0, w.seg_start - w.head_count, cs) != cudaSuccess) return ETA_ERR_CUDA;
+    if (cudaMemsetAsync(ws + w.head_count, 0, w.partials - w.head_count, cs) != cudaSuccess) return ETA_ERR_CUDA;
   }
   if (launch_screen(sa, cs) != cudaSuccess) return ETA_ERR_CUDA;
   if (s.rescue && launch_rescue(sa, cs) != cudaSuccess) return ETA_ERR_CUDA;
@@ -324,7 +322,6 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
   aa.beta = p->beta;
   aa.s = s;
   aa.status = sa.status;
-  aa.seg_start = reinterpret_cast<int*>(ws + w.seg_start);
   aa.partials = reinterpret_cast<float*>(ws + w.partials);
   aa.out = p->out;
   aa.lse = p->lse;
@@ -334,7 +331,7 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
 
   ev(2);
   MergeArgs ma;
-  ma.seg_start = aa.seg_start;
+  ma.chunk_count = sa.chunk_count;
   ma.partials = aa.partials;
   ma.s = s;
   ma.out = p->out;

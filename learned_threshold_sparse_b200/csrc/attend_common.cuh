@@ -51,6 +51,34 @@ __device__ __forceinline__ void chunk_prefix(const int* __restrict__ counts, int
   __syncthreads();
 }
 
+// The same prefix computed by one warp alone (no CTA-wide barrier), for
+// tables small enough that a lane's slice stays short.  Ends with __syncwarp().
+constexpr int kWarpPrefixMax = 2048;
+
+__device__ __forceinline__ void warp_prefix(const int* __restrict__ counts, int n, int* prefix) {
+  const int lane = threadIdx.x & 31;
+  for (int x = lane; x < n; x += 32) prefix[x] = counts[x];
+  __syncwarp();
+  const int per = (n + 31) / 32;
+  const int lo = min(n, lane * per), hi = min(n, lo + per);
+  int sum = 0;
+  for (int x = lo; x < hi; ++x) sum += prefix[x];
+  int incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  int run = incl - sum;
+  for (int x = lo; x < hi; ++x) {
+    const int c = prefix[x];
+    prefix[x] = run;
+    run += c;
+  }
+  if (lane == 31) prefix[n] = incl;
+  __syncwarp();
+}
+
 // Split of the U units over N CTAs: CTA c owns [start(c), start(c + 1)) with
 // start(c) = floor(U c / N).  The host keeps U below 2^24 (segments x chunks
 // and the chunk size are both bounded) and N is a few hundred at most, so

@@ -136,9 +136,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
   const int u0 = static_cast<int>(split.start(blockIdx.x));
   const int u1 = static_cast<int>(split.start(blockIdx.x + 1));
   const int nunits = u1 - u0;
-  if (blockIdx.x == 0) {
-    for (int sg = t; sg <= s.nseg; sg += kThreads) a.seg_start[sg] = prefix[sg * s.nchunks];
-  }
   if (nunits == 0) return;
 
   if (warp == kConsumerWarps) {

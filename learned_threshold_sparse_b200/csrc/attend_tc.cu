@@ -47,7 +47,8 @@ constexpr int kMaxStages = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
 constexpr int TR = 128;  // key rows per tile
-constexpr int kSmemSeqs = 256;  // sequence lengths staged in shared memory up to this batch
+constexpr int kSmemSeqs = 256;
+constexpr int kPrefixBar = 1;   // named barrier: producer publishes the prefix table  // sequence lengths staged in shared memory up to this batch
 
 struct Tile {
   static constexpr int PANEL = TR * 128;  // one 64-column (128-byte) panel of a 128-row tile
@@ -250,16 +251,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   dev::pdl_wait();  // screen results visible from here on
   dev::pdl_trigger();
-  dev::chunk_prefix<kThreads>(a.chunk_count, nprefix, prefix);
+  // The producer scans the chunk counts itself and publishes the table on a
+  // named barrier, so its first copies do not wait on CTA-wide barriers; the
+  // other warps pick the table up there (large tables: all warps scan).
+  const bool warp_scan = nprefix <= dev::kWarpPrefixMax;
+  if (warp_scan) {
+    if (warp == 0) {
+      dev::warp_prefix(a.chunk_count, nprefix, prefix);
+      __threadfence_block();
+      dev::named_bar_arrive(kPrefixBar, kThreads);
+    } else {
+      dev::named_bar_sync(kPrefixBar, kThreads);
+    }
+  } else {
+    dev::chunk_prefix<kThreads>(a.chunk_count, nprefix, prefix);
+  }
 
   const dev::UnitSplit split(static_cast<unsigned>(prefix[nprefix]), gridDim.x);
   const int u0 = static_cast<int>(split.start(blockIdx.x));
   const int u1 = static_cast<int>(split.start(blockIdx.x + 1));
   const int nunits = u1 - u0;
-  if (blockIdx.x == 0)
-    for (int sg = t; sg <= s.nseg; sg += kThreads) a.seg_start[sg] = prefix[sg * s.nchunks];
 
-  const int ntiles = dev::count_tiles<BPT>(prefix, s, u0, u1);
+  const int ntiles = warp == 0 ? 0 : dev::count_tiles<BPT>(prefix, s, u0, u1);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -294,13 +307,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       };
       bool ok = dev::walk_units(a, prefix, nprefix, u0, nunits, nseqs ? seq_T : nullptr,
                                 [&](const UnitInfo& in) -> bool {
-        if (npend > 0 && (in.seg != pend.seg || npend == BPT) && !emit()) return false;
+        if (npend > 0 && in.seg != pend.seg && !emit()) return false;
         if (npend == 0) pend = TileInfo{in.seg, 0, 0, 0, 0};
         pblk[npend] = in.blk;
         if (npend == 0) { pend.mask0 = in.mask; pend.nrows0 = in.nrows; }
         else { pend.mask1 = in.mask; pend.nrows1 = in.nrows; }
         ++npend;
-        return true;
+        return npend < BPT || emit();  // a full tile goes out at once
       });
       if (ok && lane == 0 && npend > 0) ok = emit();
       ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;

@@ -40,8 +40,7 @@ struct Shape {
 
 // Byte offsets of the workspace regions (all 256-byte aligned).
 struct Workspace {
-  size_t status, tau, chunk_count, chunk_list, head_count, head_best, seg_start,
-      partials, total;
+  size_t status, tau, chunk_count, chunk_list, head_count, head_best, partials, total;
 };
 
 Workspace workspace_layout(const Shape& s);
@@ -80,14 +79,13 @@ struct AttendArgs {
   float scale, beta;
   Shape s;
   unsigned* status;
-  int* seg_start;          // [nseg + 1] unit offsets (written by CTA 0)
   float* partials;         // [nseg + attend_ctas][G][partial_stride(d)]
   void* out;               // [B, Hq, d] kv dtype: segments owned by one CTA
   float* lse;              // [B, Hq] or null
 };
 
 struct MergeArgs {
-  const int* seg_start;    // [nseg + 1] unit offsets written by the attention kernel
+  const int* chunk_count;  // [nseg, nchunks] admitted entries per chunk (screen output)
   const float* partials;
   Shape s;
   void* out;

@@ -24,16 +24,45 @@ constexpr int kMergeWarps = 8;
 constexpr int kBatch = 8;  // partials in flight per lane
 
 __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(MergeArgs a) {
-  dev::pdl_wait();
   const Shape& s = a.s;
   const int seg = blockIdx.x / s.G, h = blockIdx.x - seg * s.G;
   const int slice = blockIdx.y;
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
-  const int us = a.seg_start[seg], ue = a.seg_start[seg + 1];
+
+  // The segment's unit range [us, ue) and the total U, from the screen's chunk
+  // counts.  The screen (and rescue) grids completed before the attention
+  // kernel passed its own dependency wait, and this grid is launched only
+  // after every attention CTA passed it, so the counts are final here; they
+  // are read from L2 before this grid's own wait, overlapping the attention.
+  __shared__ int s_rng[3];
+  if (w == 0) {
+    const int n = s.nseg * s.nchunks, lo = seg * s.nchunks, hi = lo + s.nchunks;
+    int before = 0, inside = 0, total = 0;
+    for (int x = lane; x < n; x += 32) {
+      const int c = __ldcg(a.chunk_count + x);
+      total += c;
+      before += x < lo ? c : 0;
+      inside += (x >= lo && x < hi) ? c : 0;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      total += __shfl_xor_sync(0xffffffffu, total, o);
+      before += __shfl_xor_sync(0xffffffffu, before, o);
+      inside += __shfl_xor_sync(0xffffffffu, inside, o);
+    }
+    if (lane == 0) {
+      s_rng[0] = before;
+      s_rng[1] = before + inside;
+      s_rng[2] = total;
+    }
+  }
+  __syncthreads();
+  const int us = s_rng[0], ue = s_rng[1];
   if (ue <= us) return;  // empty segment
-  const dev::UnitSplit split(static_cast<unsigned>(a.seg_start[s.nseg]), static_cast<unsigned>(s.attend_ctas));
+  const dev::UnitSplit split(static_cast<unsigned>(s_rng[2]), static_cast<unsigned>(s.attend_ctas));
   const int c0 = static_cast<int>(split.owner(us)), c1 = static_cast<int>(split.owner(ue - 1));
   if (c0 == c1) return;  // written by its only attention CTA
+  dev::pdl_wait();  // the partials are complete from here on
 
   const int PS = partial_stride(s.d);
   const size_t cstride = static_cast<size_t>(s.G) * PS;
