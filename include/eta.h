@@ -234,6 +234,66 @@ eta_status eta_decode(const eta_decode_params* p, void* stream);
 eta_status eta_decode_noalloc(const eta_decode_params* p, void* stream);
 
 /*
+ * ------------------------------------------------------------------------
+ * Causal forward pass over whole sequences (prefill / training forward).
+ *
+ * Source: Elastic Threshold Attention, section 2.3 (fused training kernel:
+ * no T x T matrix in HBM), Appendix E.1 (query tiles with their own
+ * thresholds, causal inner loop over key tiles), Appendix E.3 (inclusion
+ * probability sigma_ij = sigmoid(beta (S_ij - tau~_i)), multiplicative mask
+ * S~ = S sigma, row sum R_i = sum_j sigma_ij), Appendix E.4 (O, the
+ * log-sum-exp and the row vector kept for the backward pass).
+ *
+ * For every sequence b, query head h (KV head h / G, G = n_q_heads /
+ * n_kv_heads) and query row i < seq_len:
+ *   tau~_i  = w_tau[h] . q_i + b_tau[h] - a  (learned) or c_tau[h] - a,
+ *   S_ij    = scale q_i . k_j  for the keys j <= i,
+ *   out_i   = sum_j e^{S~_ij} v_j / sum_j e^{S~_ij},
+ *   lse_i   = ln sum_j e^{S~_ij},   gate_sum_i = sum_j sigma_ij.
+ * Layouts (row-major): q, out [batch, n_q_heads, seq_len, head_dim];
+ * k, v [batch, n_kv_heads, kv_stride, head_dim] (a KV cache with
+ * max_ctx = kv_stride; rows >= seq_len of a head are never used);
+ * lse, gate_sum [batch, n_q_heads, seq_len] fp32.
+ * Supported: bf16, head_dim = 128, any group size, 1 <= seq_len <= kv_stride,
+ * batch * n_q_heads * seq_len and batch * n_kv_heads * kv_stride < 2^31.
+ * ------------------------------------------------------------------------
+ */
+typedef struct {
+  int batch, n_q_heads, n_kv_heads, head_dim;
+  int seq_len;                       /* tokens per sequence (queries = keys) */
+  int kv_stride;                     /* rows per KV head in k and v, >= seq_len */
+  eta_dtype dtype;                   /* ETA_BF16                              */
+  const void* q;                     /* [batch, n_q_heads, seq_len, d]        */
+  const void* k;                     /* [batch, n_kv_heads, kv_stride, d]     */
+  const void* v;                     /* same layout as k                      */
+  eta_tau_mode tau_mode;
+  const float* w_tau;                /* [n_q_heads, d] (learned), 16-aligned  */
+  const float* b_tau;                /* [n_q_heads]    (learned)              */
+  const float* c_tau;                /* [n_q_heads]    (calibrated)           */
+  float scale;                       /* > 0, usually 1/sqrt(d)                */
+  float beta;                        /* >= 0 (0: sigma = 1/2 everywhere)      */
+  float offset_a;                    /* tau~ = tau - a                        */
+  void* out;                         /* [batch, n_q_heads, seq_len, d] bf16   */
+  float* lse;                        /* or NULL                               */
+  float* gate_sum;                   /* or NULL                               */
+  void* workspace;                   /* >= ETA_PREFILL_WORKSPACE_BYTES, 256-
+                                        aligned: holds the device status word
+                                        read by eta_read_device_status        */
+  size_t workspace_bytes;
+} eta_prefill_params;
+
+#define ETA_PREFILL_WORKSPACE_BYTES ((size_t)256)
+
+/*
+ * eta_prefill - the causal forward pass above, one launch.
+ * Errors: ETA_ERR_INVALID_ARG (NULL or misaligned pointer, bad size or
+ * value), ETA_ERR_UNSUPPORTED (dtype, head_dim, sizes past the limits),
+ * ETA_ERR_WORKSPACE, ETA_ERR_CUDA (launch failure).  A bounded device-side
+ * wait that ran out is reported by eta_read_device_status.
+ */
+eta_status eta_prefill(const eta_prefill_params* p, void* stream);
+
+/*
  * eta_read_device_status - synchronise `stream`, read and clear the device
  * status word kept in `workspace`.  Returns ETA_OK, ETA_ERR_DEVICE_TIMEOUT
  * or ETA_ERR_DEVICE_RANGE (or ETA_ERR_CUDA if the copy fails).

@@ -9,6 +9,7 @@ device memory and the stream.  The functions mirror the C entry points:
     eta_decode_workspace_size(...)  bytes of scratch for a decode call
     eta_decode(...)                 one decode step (screen, attend, merge)
     eta_read_device_status(...)     read and clear the device status word
+    eta_prefill(...) / prefill(...) causal forward pass over whole sequences
     eta_status_string(code), eta_build_info()
 
 There is no fallback: if libeta.so is missing or fails to load, importing
@@ -75,6 +76,21 @@ class eta_decode_params(ctypes.Structure):
     ]
 
 
+class eta_prefill_params(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int), ("seq_len", ctypes.c_int), ("kv_stride", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+        ("tau_mode", ctypes.c_int), ("w_tau", ctypes.c_void_p), ("b_tau", ctypes.c_void_p),
+        ("c_tau", ctypes.c_void_p), ("scale", ctypes.c_float), ("beta", ctypes.c_float),
+        ("offset_a", ctypes.c_float), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p),
+        ("gate_sum", ctypes.c_void_p), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
+PREFILL_WORKSPACE_BYTES = 256  # ETA_PREFILL_WORKSPACE_BYTES in include/eta.h
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is not built; run learned_threshold_sparse_b200.build.build()")
@@ -94,6 +110,8 @@ def _load():
     lib.eta_decode_noalloc.restype = ctypes.c_int
     lib.eta_read_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.eta_read_device_status.restype = ctypes.c_int
+    lib.eta_prefill.argtypes = [P(eta_prefill_params), ctypes.c_void_p]
+    lib.eta_prefill.restype = ctypes.c_int
     lib.eta_status_string.argtypes = [ctypes.c_int]
     lib.eta_status_string.restype = ctypes.c_char_p
     lib.eta_build_info.argtypes = []
@@ -104,7 +122,7 @@ def _load():
 _lib = _load()
 
 SYMBOLS = ("eta_block_summary_update", "eta_append_kv", "eta_decode_workspace_size", "eta_decode", "eta_decode_noalloc",
-           "eta_read_device_status", "eta_status_string", "eta_build_info")
+           "eta_read_device_status", "eta_prefill", "eta_status_string", "eta_build_info")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
 
@@ -291,3 +309,55 @@ def decode(q, k, v, seq_lens, summary, block_size, tau_mode, *, w_tau=None, b_ta
     eta_decode(params, stream)
     res["workspace"] = workspace
     return res
+
+
+# ------------------------------------------------------------ causal forward
+
+def make_prefill_params(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, seq_len: int, tau_mode: str, *,
+                        w_tau=None, b_tau=None, c_tau=None, scale: Optional[float] = None, beta: float = 5.0,
+                        offset_a: float = 0.0, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                        gate_sum: Optional[torch.Tensor] = None,
+                        workspace: Optional[torch.Tensor] = None) -> eta_prefill_params:
+    """q [B, Hq, T, d], k and v [B, Hkv, kv_stride, d] (kv_stride >= T), all
+    bf16 on the device; out like q."""
+    B, Hq, T, d = q.shape
+    p = eta_prefill_params()
+    p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim = B, Hq, k.shape[1], d
+    p.seq_len, p.kv_stride = int(seq_len), k.shape[2]
+    p.dtype = _kv_dtype(q)
+    p.q, p.k, p.v = q.data_ptr(), k.data_ptr(), v.data_ptr()
+    p.tau_mode = ETA_TAU_LEARNED if tau_mode == "learned" else ETA_TAU_CALIBRATED
+    p.w_tau = None if w_tau is None else w_tau.data_ptr()
+    p.b_tau = None if b_tau is None else b_tau.data_ptr()
+    p.c_tau = None if c_tau is None else c_tau.data_ptr()
+    p.scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    p.beta = float(beta)
+    p.offset_a = float(offset_a)
+    p.out = out.data_ptr()
+    p.lse = None if lse is None else lse.data_ptr()
+    p.gate_sum = None if gate_sum is None else gate_sum.data_ptr()
+    if workspace is not None:
+        p.workspace = workspace.data_ptr()
+        p.workspace_bytes = workspace.numel()
+    return p
+
+
+def eta_prefill(params: eta_prefill_params, stream: Optional[torch.cuda.Stream] = None) -> None:
+    rc = _lib.eta_prefill(ctypes.byref(params), _stream_handle(stream))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_prefill")
+
+
+def prefill(q, k, v, seq_len: int, tau_mode: str, *, w_tau=None, b_tau=None, c_tau=None, scale=None, beta=5.0,
+            offset_a=0.0, stream=None) -> Dict[str, torch.Tensor]:
+    """Allocate the outputs and a workspace, run eta_prefill; returns out, lse,
+    gate_sum and the workspace (for eta_read_device_status)."""
+    out = torch.empty_like(q)
+    B, Hq, T, _ = q.shape
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=q.device)
+    gate = torch.empty_like(lse)
+    ws = alloc_workspace(PREFILL_WORKSPACE_BYTES, q.device)
+    p = make_prefill_params(q, k, v, seq_len, tau_mode, w_tau=w_tau, b_tau=b_tau, c_tau=c_tau, scale=scale,
+                            beta=beta, offset_a=offset_a, out=out, lse=lse, gate_sum=gate, workspace=ws)
+    eta_prefill(p, stream)
+    return {"out": out, "lse": lse, "gate_sum": gate, "workspace": ws}

@@ -191,7 +191,7 @@ const char* eta_status_string(eta_status s) {
 
 const char* eta_build_info(void) {
   return "eta decode library: sm_100a; kernels: block_summary, screen, rescue, attend_simt, attend_tc, merge, "
-         "export";
+         "export, prefill_tc";
 }
 
 eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summary_desc* summary,
@@ -352,6 +352,57 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
   }
   ev(3);
   return ETA_OK;
+}
+
+eta_status eta_prefill(const eta_prefill_params* p, void* stream) {
+  if (!p) return ETA_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->n_q_heads < 1 || p->n_kv_heads < 1 || p->seq_len < 1 || p->kv_stride < p->seq_len)
+    return ETA_ERR_INVALID_ARG;
+  if (p->n_q_heads % p->n_kv_heads != 0) return ETA_ERR_INVALID_ARG;
+  if (p->dtype != ETA_BF16 && p->dtype != ETA_F32) return ETA_ERR_INVALID_ARG;
+  if (p->dtype != ETA_BF16 || p->head_dim != 128) return ETA_ERR_UNSUPPORTED;
+  if (p->batch > 65535 || p->n_q_heads > 65535) return ETA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p->batch) * p->n_q_heads * p->seq_len >= (1ll << 31) ||
+      static_cast<long long>(p->batch) * p->n_kv_heads * p->kv_stride >= (1ll << 31))
+    return ETA_ERR_UNSUPPORTED;
+  if (!p->q || !p->k || !p->v || !p->out) return ETA_ERR_INVALID_ARG;
+  if (!aligned(p->q, 16) || !aligned(p->k, 16) || !aligned(p->v, 16) || !aligned(p->out, 16))
+    return ETA_ERR_INVALID_ARG;
+  if (p->tau_mode == ETA_TAU_LEARNED) {
+    if (!p->w_tau || !p->b_tau || !aligned(p->w_tau, 16) || !aligned(p->b_tau, 4)) return ETA_ERR_INVALID_ARG;
+  } else if (p->tau_mode == ETA_TAU_CALIBRATED) {
+    if (!p->c_tau || !aligned(p->c_tau, 4)) return ETA_ERR_INVALID_ARG;
+  } else {
+    return ETA_ERR_INVALID_ARG;
+  }
+  if (!(p->scale > 0.f) || !isfinite(p->scale)) return ETA_ERR_INVALID_ARG;
+  if (!(p->beta >= 0.f) || !isfinite(p->beta)) return ETA_ERR_INVALID_ARG;
+  if (!isfinite(p->offset_a)) return ETA_ERR_INVALID_ARG;
+  if ((p->lse && !aligned(p->lse, 4)) || (p->gate_sum && !aligned(p->gate_sum, 4))) return ETA_ERR_INVALID_ARG;
+  if (!p->workspace || !aligned(p->workspace, 256) || p->workspace_bytes < ETA_PREFILL_WORKSPACE_BYTES)
+    return ETA_ERR_WORKSPACE;
+  PrefillArgs a;
+  a.q = p->q;
+  a.k = p->k;
+  a.v = p->v;
+  a.w_tau = p->w_tau;
+  a.b_tau = p->b_tau;
+  a.c_tau = p->c_tau;
+  a.out = p->out;
+  a.lse = p->lse;
+  a.gate_sum = p->gate_sum;
+  a.status = static_cast<unsigned*>(p->workspace);
+  a.B = p->batch;
+  a.Hq = p->n_q_heads;
+  a.Hkv = p->n_kv_heads;
+  a.G = p->n_q_heads / p->n_kv_heads;
+  a.T = p->seq_len;
+  a.kv_stride = p->kv_stride;
+  a.tau_mode = p->tau_mode;
+  a.scale = p->scale;
+  a.beta = p->beta;
+  a.offset_a = p->offset_a;
+  return launch_prefill_tc(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
 }
 
 eta_status eta_read_device_status(void* workspace, void* stream) {

@@ -210,5 +210,12 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, un
   return true;
 }
 
+// wait_or_abort by a whole warp with one answer for all lanes: warp-wide
+// instructions (tensor-memory loads and stores) may follow it.
+__device__ __forceinline__ bool warp_wait_or_abort(uint64_t* bar, uint32_t parity, unsigned* status,
+                                                   volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, wait_or_abort(bar, parity, status, abort_flag) ? 1 : 0) != 0;
+}
+
 }  // namespace dev
 }  // namespace eta

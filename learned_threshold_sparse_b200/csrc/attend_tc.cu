@@ -31,12 +31,14 @@
 #include <math.h>
 
 #include "attend_common.cuh"
+#include "tc_common.cuh"
 
 namespace eta {
 namespace {
 
 using dev::UnitInfo;
 using dev::wait_or_abort;
+using namespace tc;
 
 constexpr int D = 128;
 constexpr int NQ = 16;              // N of both MMAs
@@ -95,72 +97,6 @@ __host__ __device__ inline Layout tc_layout(int nstages, int nprefix, int nseqs)
   off += 16 + kMaxStages * sizeof(int) + 16;
   L.total = align_to(off, 128) + 1024;  // + slack to align the dynamic base to 1024
   return L;
-}
-
-// ------------------------------------------------------------ PTX wrappers
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(dev::smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
-  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dev::smem_u32(slot)),
-               "r"(ncols)
-               : "memory");
-  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
-  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                         uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   dev::smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
-  uint32_t r[8];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-      : "r"(taddr)
-      : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int k = 0; k < 8; ++k) v[k] = __uint_as_float(r[k]);
-}
-
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start,
-// leading and stride byte offsets >> 4, version 1 at bit 46, layout 2 at 61).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
-         (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
-}
-
-// Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(a_mn_major) << 15) |
-         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // Barrier indices inside the barrier block.
@@ -414,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     auto correction = [&](int i) -> bool {
       const int ob = i & 1;
-      if (!wait_or_abort(&B.o_full[ob], (i >> 1) & 1, a.status, abort_flag)) return false;
+      if (!dev::warp_wait_or_abort(&B.o_full[ob], (i >> 1) & 1, a.status, abort_flag)) return false;
       tc_fence_after();
       float o[8];
       tmem_ld8(tmem + tlane + 32 + ob * 16, o);
@@ -479,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       const int sb = j & 1;
-      if (!wait_or_abort(&B.s_full[sb], (j >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+      if (!dev::warp_wait_or_abort(&B.s_full[sb], (j >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float sv[8];
       tmem_ld8(tmem + tlane + sb * 16, sv);
@@ -550,54 +486,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------ host side
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-bool encode_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(D * 2)};
-  cuuint32_t box[2] = {64u, box_rows};
-  cuuint32_t estr[2] = {1u, 1u};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// The maps of the last few (pointer, rows, box) triples, per host thread: a
-// decode loop over a fixed cache re-encodes nothing.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
-  struct Entry {
-    const void* ptr;
-    uint64_t rows;
-    uint32_t box;
-    CUtensorMap map;
-  };
-  constexpr int kEntries = 8;
-  thread_local Entry cache[kEntries] = {};
-  thread_local int next = 0;
-  for (int i = 0; i < kEntries; ++i) {
-    if (cache[i].ptr == ptr && cache[i].rows == rows && cache[i].box == box_rows && ptr) {
-      *m = cache[i].map;
-      return true;
-    }
-  }
-  if (!encode_map(m, ptr, rows, box_rows)) return false;
-  cache[next] = Entry{ptr, rows, box_rows, *m};
-  next = (next + 1) % kEntries;
-  return true;
-}
 
 constexpr size_t kSmemBudget = 224 * 1024;
 

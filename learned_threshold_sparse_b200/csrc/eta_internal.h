@@ -103,6 +103,23 @@ struct ExportArgs {
   unsigned* union_mask;
 };
 
+// Arguments of the causal forward (prefill) kernel; q, k, v also feed the
+// host-side tensor maps.
+struct PrefillArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const float* w_tau;
+  const float* b_tau;
+  const float* c_tau;
+  void* out;
+  float* lse;
+  float* gate_sum;
+  unsigned* status;
+  int B, Hq, Hkv, G, T, kv_stride, tau_mode;
+  float scale, beta, offset_a;
+};
+
 struct SummaryArgs {
   const void* k;
   const int* seq_lens;
@@ -168,5 +185,6 @@ size_t attend_tc_smem(const Shape& s);
 bool attend_tc_supported(const Shape& s);
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_export(const ExportArgs& a, cudaStream_t st);
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st);
 
 }  // namespace eta

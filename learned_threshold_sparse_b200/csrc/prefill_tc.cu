@@ -1,0 +1,409 @@
+// Causal ETA forward pass over whole sequences (prefill / training forward)
+// on the 5th-generation tensor cores, bf16 Q/K/V, d = 128.
+//
+// Source: Elastic Threshold Attention,
+//   section 2.3          fused kernel: no T x T matrix in HBM,
+//   Appendix E.1         query tiles with their own thresholds; the inner
+//                        loop runs causally over key tiles,
+//   Appendix E.3         sigma_ij = sigmoid(beta (S_ij - tau~_i)),
+//                        S~ = S sigma (multiplicative mask), R_i = sum_j sigma_ij,
+//   Appendix E.4         O, the log-sum-exp L and the row vector kept for the
+//                        backward pass,
+//   Appendix G.1         tau~ = tau - a, tau = w_tau . q + b_tau or a constant.
+//
+// One CTA per (128 query rows, query head, sequence); heavy (late) query tiles
+// are scheduled first.  Per key tile j of 128 keys:
+//   S [128 q x 128 k]  = Q . K_j^T        (M = 128, N = 128, both K-major)
+//   O [128 q x 128 d] += P_j . V_j        (A = P K-major, B = V MN-major)
+// S is double-buffered in tensor memory (columns 0-127, 128-255), O lives at
+// columns 256-383.  Roles: warp 0 issues the tensor copies (Q once, then K/V
+// tiles into a 2-stage ring), warp 1 owns tensor memory and issues the MMAs,
+// warps 2-5 (thread = query row = tensor-memory lane) read S, apply the gate
+// and the online softmax, write P (bf16, 128-byte swizzle) for the second
+// MMA and keep the running max lazily: O is rescaled in tensor memory only
+// when the row max grows by more than 2^8, so the exponentials stay <= 2^8.
+#include <math.h>
+
+#include "attend_common.cuh"
+#include "tc_common.cuh"
+
+namespace eta {
+namespace {
+
+using namespace tc;
+using dev::wait_or_abort;
+
+constexpr int D = 128;
+constexpr int BM = 128;  // query rows per CTA
+constexpr int BN = 128;  // keys per tile
+constexpr int kWarps = 6;
+constexpr int kThreads = kWarps * 32;
+constexpr int kStages = 2;
+constexpr uint32_t kTmemCols = 512;  // S0 0..127, S1 128..255, O 256..383
+constexpr uint32_t kOCol = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLazy = 8.0f;  // rescale O only when the max grows by more than this (base 2)
+
+constexpr uint32_t PANEL = BM * 128;           // one 64-column panel of 128 rows (16 KB)
+constexpr uint32_t TILE = 2 * PANEL;           // 128 rows x 128 bf16 (32 KB)
+constexpr uint32_t OFF_Q = 0;
+constexpr uint32_t OFF_STAGE = TILE;           // stage s: K at OFF_STAGE + 2 s TILE, V after it
+constexpr uint32_t OFF_P = OFF_STAGE + kStages * 2 * TILE;
+constexpr uint32_t OFF_BARS = OFF_P + TILE;
+constexpr uint32_t kSmemBytes = OFF_BARS + 256 + 1024;  // barriers, flags, alignment slack
+
+
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// sigmoid(x) = (1 + tanh(x / 2)) / 2: one special-function op.
+__device__ __forceinline__ float gate(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  return static_cast<uint32_t>(dev::f32_to_bf16_rn(lo)) | (static_cast<uint32_t>(dev::f32_to_bf16_rn(hi)) << 16);
+}
+
+__device__ __forceinline__ float bf16_lo_f(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16_hi_f(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
+struct Bars {
+  uint64_t* q_full;    // producer -> MMA (tx bytes)
+  uint64_t* kv_full;   // [2] producer -> MMA (tx bytes)
+  uint64_t* kv_empty;  // [2] MMA commit -> producer
+  uint64_t* s_full;    // [2] MMA commit -> softmax
+  uint64_t* s_free;    // [2] softmax (4 warps) -> MMA
+  uint64_t* p_full;    // softmax (4 warps) -> MMA
+  uint64_t* o_done;    // MMA commit after every P V -> softmax
+  uint64_t* done;      // final commit of the MMA warp
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                      const __grid_constant__ CUtensorMap tv, PrefillArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = dev::smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_u32 - raw);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(base + OFF_BARS);
+  Bars Bs;
+  Bs.q_full = bar;
+  Bs.kv_full = bar + 1;
+  Bs.kv_empty = bar + 3;
+  Bs.s_full = bar + 5;
+  Bs.s_free = bar + 7;
+  Bs.p_full = bar + 9;
+  Bs.o_done = bar + 10;
+  Bs.done = bar + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_BARS + 128);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + OFF_BARS + 132);
+  int* issued = reinterpret_cast<int*>(base + OFF_BARS + 136);  // [2] parity of the last copy per stage, -1 none
+
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int nqt = (a.T + BM - 1) / BM;
+  const int qt = nqt - 1 - static_cast<int>(blockIdx.x);  // heavy tiles first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int g = h / a.G;
+  const int q0 = qt * BM;
+  const int nt = qt + 1;  // key tiles 0..qt (causal)
+
+  if (t == 0) {
+    dev::mbar_init(Bs.q_full, 1);
+    for (int k = 0; k < kStages; ++k) {
+      dev::mbar_init(&Bs.kv_full[k], 1);
+      dev::mbar_init(&Bs.kv_empty[k], 1);
+      dev::mbar_init(&Bs.s_full[k], 1);
+      dev::mbar_init(&Bs.s_free[k], 4);
+      issued[k] = -1;
+    }
+    dev::mbar_init(Bs.p_full, 4);
+    dev::mbar_init(Bs.o_done, 1);
+    dev::mbar_init(Bs.done, 1);
+    *abort_flag = 0;
+    dev::fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tq)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tk)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tv)) : "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      dev::mbar_arrive_expect_tx(Bs.q_full, TILE);
+      const int qrow = (b * a.Hq + h) * a.T + q0;
+      tma_load_2d(base_u32 + OFF_Q, &tq, 0, qrow, Bs.q_full);
+      tma_load_2d(base_u32 + OFF_Q + PANEL, &tq, 64, qrow, Bs.q_full);
+      const int krow0 = (b * a.Hkv + g) * a.kv_stride;
+      for (int j = 0; j < nt; ++j) {
+        const int st = j & 1;
+        if (!wait_or_abort(&Bs.kv_empty[st], ((j >> 1) & 1) ^ 1, a.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const uint32_t ks = base_u32 + OFF_STAGE + static_cast<uint32_t>(st) * 2 * TILE, vs = ks + TILE;
+        dev::mbar_arrive_expect_tx(&Bs.kv_full[st], 2 * TILE);
+        const int krow = krow0 + j * BN;
+        tma_load_2d(ks, &tk, 0, krow, &Bs.kv_full[st]);
+        tma_load_2d(ks + PANEL, &tk, 64, krow, &Bs.kv_full[st]);
+        tma_load_2d(vs, &tv, 0, krow, &Bs.kv_full[st]);
+        tma_load_2d(vs + PANEL, &tv, 64, krow, &Bs.kv_full[st]);
+        issued[st] = (j >> 1) & 1;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        // let the copies already issued land before the CTA winds down
+        const long long t0 = clock64();
+        while (!dev::mbar_try_wait(Bs.q_full, 0) && clock64() - t0 < dev::kWaitCycles) {
+        }
+        for (int k = 0; k < kStages; ++k) {
+          if (issued[k] < 0) continue;
+          const long long t1 = clock64();
+          while (!dev::mbar_try_wait(&Bs.kv_full[k], static_cast<uint32_t>(issued[k])) &&
+                 clock64() - t1 < dev::kWaitCycles) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0, 0);
+    constexpr uint32_t idesc_pv = idesc_bf16(BM, D, 0, 1);
+    bool ok = wait_or_abort(Bs.q_full, 0, a.status, abort_flag);
+    auto issue_pv = [&](int i) -> bool {
+      if (!wait_or_abort(Bs.p_full, static_cast<uint32_t>(i & 1), a.status, abort_flag)) return false;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t vs = base_u32 + OFF_STAGE + static_cast<uint32_t>(i & 1) * 2 * TILE + TILE;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t ad = sw128_desc(base_u32 + OFF_P + (kk >> 2) * PANEL + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = sw128_desc(vs + kk * 2048, PANEL, 1024);
+          mma_bf16(tmem + kOCol, ad, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(Bs.o_done);
+        mma_commit(&Bs.kv_empty[i & 1]);
+      }
+      __syncwarp();
+      return true;
+    };
+    for (int j = 0; j < nt && ok; ++j) {
+      const int st = j & 1;
+      if (!wait_or_abort(&Bs.kv_full[st], (j >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+      if (!wait_or_abort(&Bs.s_free[st], ((j >> 1) & 1) ^ 1, a.status, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t ks = base_u32 + OFF_STAGE + static_cast<uint32_t>(st) * 2 * TILE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * PANEL + (kk & 3) * 32;
+          const uint64_t ad = sw128_desc(base_u32 + OFF_Q + off, 16, 1024);
+          const uint64_t bd = sw128_desc(ks + off, 16, 1024);
+          mma_bf16(tmem + static_cast<uint32_t>(st) * BN, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&Bs.s_full[st]);
+      }
+      __syncwarp();
+      if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
+    }
+    if (ok) issue_pv(nt - 1);
+    // every MMA issued so far has completed once `done` flips
+    if (lane == 0) mma_commit(Bs.done);
+    __syncwarp();
+    {
+      const long long t0 = clock64();
+      while (!dev::mbar_try_wait(Bs.done, 0) && clock64() - t0 < dev::kWaitCycles) {
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int qq = warp & 3;  // tensor-memory lane quarter of this warp
+    const uint32_t lane_base = static_cast<uint32_t>(32 * qq) << 16;
+    const int r = 32 * qq + lane;  // query row of the tile
+    const int i = q0 + r;
+    const bool row_ok = i < a.T;
+    const size_t row = static_cast<size_t>(b * a.Hq + h) * a.T + i;
+    float tau = 0.f;
+    if (row_ok) {
+      if (a.tau_mode == ETA_TAU_LEARNED) {
+        const uint4* qp = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.q) + row * D);
+        const float4* wp = reinterpret_cast<const float4*>(a.w_tau + static_cast<size_t>(h) * D);
+        float acc = 0.f;
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 u = qp[c];
+          const float4 w0 = wp[2 * c], w1 = wp[2 * c + 1];
+          acc = fmaf(bf16_lo_f(u.x), w0.x, acc);
+          acc = fmaf(bf16_hi_f(u.x), w0.y, acc);
+          acc = fmaf(bf16_lo_f(u.y), w0.z, acc);
+          acc = fmaf(bf16_hi_f(u.y), w0.w, acc);
+          acc = fmaf(bf16_lo_f(u.z), w1.x, acc);
+          acc = fmaf(bf16_hi_f(u.z), w1.y, acc);
+          acc = fmaf(bf16_lo_f(u.w), w1.z, acc);
+          acc = fmaf(bf16_hi_f(u.w), w1.w, acc);
+        }
+        tau = acc + a.b_tau[h] - a.offset_a;
+      } else {
+        tau = a.c_tau[h] - a.offset_a;
+      }
+    }
+    const float scale = a.scale, beta = a.beta;
+    float m_run = -INFINITY, l_run = 0.f, rsum = 0.f;
+    bool ok = true;
+    uint8_t* prow = base + OFF_P + r * 128;
+    for (int j = 0; j < nt && ok; ++j) {
+      const int sb = j & 1;
+      if (!dev::warp_wait_or_abort(&Bs.s_full[sb], (j >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t s[4][32];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) tmem_ld32_nowait(tmem + lane_base + static_cast<uint32_t>(sb) * BN + 32 * k, s[k]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(&Bs.s_free[sb]);
+
+      // keys j BN + c with c <= lim are seen by this row (causal; rows past
+      // the sequence see none)
+      const int lim = row_ok ? min(BN - 1, i - j * BN) : -1;
+      float mt = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float S = __uint_as_float(s[k][c]) * scale;
+          const float sg = gate(beta * (S - tau));
+          const float x = S * sg * kLog2e;
+          const bool on = 32 * k + c <= lim;
+          rsum += on ? sg : 0.f;
+          mt = fmaxf(mt, on ? x : -INFINITY);
+          s[k][c] = __float_as_uint(on ? x : -INFINITY);
+        }
+      }
+      // P V of the previous tile done: the P buffer is free and O is stable
+      if (j > 0 && !dev::warp_wait_or_abort(Bs.o_done, static_cast<uint32_t>((j - 1) & 1), a.status, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // A row whose max grew past the margin moves its reference to the new
+      // max; if it had weights already, its O row is rescaled.  Tensor-memory
+      // loads and stores are warp-wide instructions, so the whole warp runs
+      // them when any of its rows needs it (alpha = 1 for the others).
+      const bool grow = mt > m_run + kLazy;
+      const bool rescale = grow && m_run != -INFINITY;
+      if (__any_sync(0xffffffffu, rescale)) {
+        const float alpha = rescale ? dev::fast_exp2(m_run - mt) : 1.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t o[32];
+          tmem_ld32_nowait(tmem + lane_base + kOCol + 32 * k, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(tmem + lane_base + kOCol + 32 * k, o);
+        }
+        tmem_wait_st();
+        l_run *= alpha;
+      }
+      if (grow) m_run = mt;
+      // P_j = 2^(x - m_run), bf16, 128-byte swizzle: 16-byte chunk q of row r
+      // sits at chunk q ^ (r & 7) of the row's 128 bytes in its panel
+      float lsum = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t w[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = __uint_as_float(s[k][8 * c8 + 2 * e]);
+            const float x1 = __uint_as_float(s[k][8 * c8 + 2 * e + 1]);
+            const float p0 = x0 == -INFINITY ? 0.f : dev::fast_exp2(x0 - m_run);
+            const float p1 = x1 == -INFINITY ? 0.f : dev::fast_exp2(x1 - m_run);
+            w[e] = pack_bf16(p0, p1);
+            lsum += bf16_lo_f(w[e]) + bf16_hi_f(w[e]);
+          }
+          const int col = 32 * k + 8 * c8;
+          const int panel = col >> 6, chunk = (col & 63) >> 3;
+          *reinterpret_cast<uint4*>(prow + panel * PANEL + ((chunk ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+      l_run += lsum;
+      // V rows of this tile past the sequence end hold no key: zeroed so that
+      // stale or non-finite bytes there cannot reach O (0 * inf)
+      const int kvalid = a.T - j * BN;
+      if (kvalid < BN) {
+        uint8_t* vt = base + OFF_STAGE + sb * 2 * TILE + TILE;
+        const int nz = (BN - kvalid) * 8;  // 16-byte chunks per panel
+        for (int c = t - 64; c < 2 * nz; c += 128) {
+          const int pnl = c / nz, rem = c - pnl * nz;
+          *reinterpret_cast<uint4*>(vt + pnl * PANEL + (kvalid + (rem >> 3)) * 128 + (rem & 7) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+      fence_proxy_async();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(Bs.p_full);
+    }
+    if (ok) ok = dev::warp_wait_or_abort(Bs.o_done, static_cast<uint32_t>((nt - 1) & 1), a.status, abort_flag);
+    tc_fence_after();
+    if (ok) {
+      const float inv = (row_ok && l_run > 0.f) ? 1.f / l_run : 0.f;
+      uint4* orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + row * D);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t o[32];
+        tmem_ld32_nowait(tmem + lane_base + kOCol + 32 * k, o);
+        tmem_wait_ld();
+        if (row_ok) {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w[e] = pack_bf16(__uint_as_float(o[8 * c8 + 2 * e]) * inv, __uint_as_float(o[8 * c8 + 2 * e + 1]) * inv);
+            orow[4 * k + c8] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      if (row_ok) {
+        if (a.lse) a.lse[row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
+        if (a.gate_sum) a.gate_sum[row] = rsum;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  const uint64_t qrows = static_cast<uint64_t>(a.B) * a.Hq * a.T;
+  const uint64_t kvrows = static_cast<uint64_t>(a.B) * a.Hkv * a.kv_stride;
+  if (!make_map(&tq, a.q, qrows, BM) || !make_map(&tk, a.k, kvrows, BN) || !make_map(&tv, a.v, kvrows, BN))
+    return cudaErrorInvalidValue;
+  static SmemLimit lim;
+  const dim3 grid((a.T + BM - 1) / BM, a.Hq, a.B);
+  return launch_with_smem(reinterpret_cast<const void*>(prefill_tc_kernel), kSmemBytes, lim, [&] {
+    prefill_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
+    return cudaGetLastError();
+  });
+}
+
+}  // namespace eta

@@ -117,6 +117,7 @@ def test_struct_layout_matches_header(tmp_path):
         "eta_cache_desc": eta.eta_cache_desc,
         "eta_summary_desc": eta.eta_summary_desc,
         "eta_decode_params": eta.eta_decode_params,
+        "eta_prefill_params": eta.eta_prefill_params,
     }
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "eta.h"', "int main(void) {"]
     for sname, cls in fields.items():
@@ -151,3 +152,38 @@ def test_append_kv_validation():
     assert lib.eta_append_kv(ctypes.byref(c), ctypes.byref(s), fake, fake, fake + 2, None) == eta.ETA_ERR_INVALID_ARG
     c2 = eta.eta_cache_desc(1, 4, 4, 96, 64, 4096, eta.ETA_BF16, fake, fake, fake)
     assert lib.eta_append_kv(ctypes.byref(c2), ctypes.byref(s), fake, fake, fake, None) == eta.ETA_ERR_UNSUPPORTED
+
+
+def _prefill_ok():
+    fake = 1 << 20  # never dereferenced: every case below fails validation before a launch
+    p = eta.eta_prefill_params()
+    p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim, p.seq_len, p.kv_stride = 1, 8, 2, 128, 1000, 1024
+    p.dtype = eta.ETA_BF16
+    p.q = p.k = p.v = p.out = fake
+    p.tau_mode = eta.ETA_TAU_LEARNED
+    p.w_tau = p.b_tau = fake
+    p.scale, p.beta, p.offset_a = 0.088, 5.0, 0.0
+    p.workspace, p.workspace_bytes = fake, eta.PREFILL_WORKSPACE_BYTES
+    return p
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("seq_len", 0, 1), ("kv_stride", 999, 1), ("n_kv_heads", 3, 1), ("head_dim", 64, 2), ("dtype", 0, 2),
+    ("q", 0, 1), ("k", (1 << 20) + 8, 1), ("w_tau", (1 << 20) + 4, 1), ("scale", 0.0, 1),
+    ("beta", -1.0, 1), ("beta", float("nan"), 1), ("tau_mode", 7, 1), ("workspace_bytes", 16, 3),
+    ("workspace", 0, 3), ("lse", (1 << 20) + 2, 1),
+])
+def test_prefill_validation(field, value, code):
+    p = _prefill_ok()
+    setattr(p, field, value)
+    assert eta.library().eta_prefill(ctypes.byref(p), None) == code
+
+
+def test_prefill_size_limits():
+    p = _prefill_ok()
+    p.batch, p.n_q_heads, p.n_kv_heads, p.seq_len, p.kv_stride = 64, 64, 64, 1 << 20, 1 << 20
+    assert eta.library().eta_prefill(ctypes.byref(p), None) == eta.ETA_ERR_UNSUPPORTED
+    p = _prefill_ok()
+    p.tau_mode = eta.ETA_TAU_CALIBRATED
+    p.c_tau = None
+    assert eta.library().eta_prefill(ctypes.byref(p), None) == eta.ETA_ERR_INVALID_ARG

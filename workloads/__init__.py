@@ -345,6 +345,63 @@ def custom(seed: int, batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int
                     w_tau=w_tau, b_tau=b_tau, c_tau=c_tau, scale=1.0 / math.sqrt(d))
 
 
+@dataclasses.dataclass
+class PrefillInputs:
+    """Inputs of one causal forward pass over whole sequences: ``q``
+    ``[B, Hq, T, d]``, ``k``/``v`` ``[B, Hkv, kv_stride, d]`` (bf16, host) and
+    fp32 threshold parameters as in ``Workload``."""
+
+    seed: int
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    seq_len: int
+    kv_stride: int
+    tau_mode: str
+    q: torch.Tensor
+    k: torch.Tensor
+    v: torch.Tensor
+    w_tau: Optional[np.ndarray]
+    b_tau: Optional[np.ndarray]
+    c_tau: Optional[np.ndarray]
+    scale: float
+    beta: float = 5.0
+    offset_a: float = 0.0
+
+
+def prefill_case(seed: int, batch: int, n_q_heads: int, n_kv_heads: int, seq_len: int,
+                 kv_stride: Optional[int] = None, head_dim: int = 128, tau_mode: str = TAU_LEARNED,
+                 tau_bias: float = 0.5, tau_std: float = 1.0, key_ramp: float = 0.0,
+                 tail_fill: float = 0.0, beta: float = 5.0, offset_a: float = 0.0) -> PrefillInputs:
+    """Seeded prefill inputs.  q, k, v ~ N(0, 1); with ``key_ramp`` > 0 key j
+    is scaled by 1 + key_ramp j / T, so the logits grow along the sequence.
+    Rows of k and v at positions >= seq_len (up to ``kv_stride``) hold
+    ``tail_fill`` (NaN allowed).  Learned mode: W_tau ~ N(0, tau_std^2 / d),
+    b_tau = tau_bias; calibrated: c_tau = tau_bias + U[-0.2, 0.2] per head."""
+    rng = np.random.default_rng([7, seed])
+    B, Hq, Hkv, T, d = batch, n_q_heads, n_kv_heads, seq_len, head_dim
+    S = kv_stride if kv_stride is not None else T
+    q = rng.standard_normal((B, Hq, T, d), dtype=np.float32)
+    k = np.full((B, Hkv, S, d), tail_fill, np.float32)
+    v = np.full((B, Hkv, S, d), tail_fill, np.float32)
+    k[:, :, :T] = rng.standard_normal((B, Hkv, T, d), dtype=np.float32)
+    v[:, :, :T] = rng.standard_normal((B, Hkv, T, d), dtype=np.float32)
+    if key_ramp:
+        k[:, :, :T] *= (1.0 + key_ramp * np.arange(T, dtype=np.float32) / T)[None, None, :, None]
+    if tau_mode == TAU_LEARNED:
+        w_tau = _normal(rng, (Hq, d), tau_std / math.sqrt(d))
+        b_tau = np.full((Hq,), tau_bias, np.float32)
+        c_tau = None
+    else:
+        w_tau = b_tau = None
+        c_tau = (tau_bias + rng.uniform(-0.2, 0.2, size=Hq)).astype(np.float32)
+    return PrefillInputs(seed=seed, batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=d, seq_len=T, kv_stride=S,
+                         tau_mode=tau_mode, q=_to_kv(q, BF16), k=_to_kv(k, BF16), v=_to_kv(v, BF16),
+                         w_tau=w_tau, b_tau=b_tau, c_tau=c_tau, scale=1.0 / math.sqrt(d), beta=beta,
+                         offset_a=offset_a)
+
+
 def _attach_thresholds(wl: Workload) -> Workload:
     entry = _load_thresholds(wl.name, wl.seed)
     if entry is None:
