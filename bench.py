@@ -163,7 +163,7 @@ class ClockSampler:
                 "samples": len(sms)}
 
 
-ATTEND_SOURCES = ("attend_tc.cu", "attend_common.cuh", "eta_device.cuh", "eta_internal.h")
+ATTEND_SOURCES = ("attend_tc.cu", "attend_common.cuh", "tc_common.cuh", "eta_device.cuh", "eta_internal.h")
 
 
 def attend_source_sha1():
@@ -489,6 +489,77 @@ def run_reference(args):
     }
 
 
+def run_prefill(args):
+    """Causal forward pass (eta_prefill) over a whole sequence: tensor flops of
+    the two contractions over the causal triangle per second, against the
+    measured dense bf16 peak.  Not the decode metric; printed on its own line."""
+    import learned_threshold_sparse_b200 as eta
+
+    B, Hq, Hkv, T = (int(x) for x in args.prefill_shape.split(","))
+    d = 128
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    case = workloads.prefill_case(args.seed, batch=B, n_q_heads=Hq, n_kv_heads=Hkv, seq_len=T, head_dim=d)
+    q, k, v = case.q.to(dev), case.k.to(dev), case.v.to(dev)
+    w = torch.from_numpy(case.w_tau).to(dev)
+    bt = torch.from_numpy(case.b_tau).to(dev)
+    out = torch.empty_like(q)
+    lse = torch.empty((B, Hq, T), dtype=torch.float32, device=dev)
+    gate = torch.empty_like(lse)
+    ws = eta.alloc_workspace(eta.PREFILL_WORKSPACE_BYTES, dev)
+    params = eta.make_prefill_params(q, k, v, T, case.tau_mode, w_tau=w, b_tau=bt, scale=case.scale,
+                                     beta=case.beta, offset_a=case.offset_a, out=out, lse=lse, gate_sum=gate,
+                                     workspace=ws)
+    stream = torch.cuda.current_stream(dev)
+    flush_buf = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        eta.eta_prefill(params, stream)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.3)
+    ms = []
+    for _ in range(args.steps):
+        torch.sum(flush_buf, dim=0, out=flush_sink)
+        e0.record(stream)
+        eta.eta_prefill(params, stream)
+        e1.record(stream)
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    clk = clocks.stop()
+    assert eta.eta_read_device_status(ws) == eta.ETA_OK
+    flops = 4.0 * d * (T * (T + 1) / 2) * B * Hq
+    t = statistics.mean(ms)
+    tflops = flops / (t * 1e-3) / 1e12
+    peak_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peak, kind = 1590.0, "fallback"
+    if os.path.exists(peak_path):
+        with open(peak_path) as f:
+            peak, kind = float(json.load(f)["bf16_tflops"]), "measured"
+    return {
+        "metric": "ETA causal forward (prefill) tensor TFLOP/s",
+        "value": round(tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(t, 4),
+        "higher_is_better": True,
+        "dtype": "bf16",
+        "accum": "f32",
+        "data": "synthetic",
+        "config": {"workload": f"prefill: batch {B}, {Hq} query / {Hkv} KV heads, seq {T}, d {d}, bf16, learned tau",
+                   "flops_per_step": flops,
+                   "l2": "flushed before every step by reading a 256 MiB buffer (outside the events)"},
+        "roofline": {"kernel": "prefill_tc", "bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
+                     "peak_kind": kind + " dense bf16 (burst)", "unit": "TFLOP/s", "frac": round(tflops / peak, 4)},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -500,10 +571,15 @@ def main():
     ap.add_argument("--attend-impl", type=int, default=0, choices=[0, 1, 2])
     ap.add_argument("--dense", action="store_true", help="screen off: every block loaded")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill", action="store_true", help="time the causal forward pass instead of the decode step")
+    ap.add_argument("--prefill-shape", default="1,32,8,8192", help="batch,n_q_heads,n_kv_heads,seq_len")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    line = run_reference(args) if args.impl == "reference" else run_eta(args)
+    if args.prefill:
+        line = run_prefill(args)
+    else:
+        line = run_reference(args) if args.impl == "reference" else run_eta(args)
     if line is not None:
         print(json.dumps(line), flush=True)
 
