@@ -13,15 +13,20 @@
 //
 // One CTA per (128 query rows, query head, sequence); heavy (late) query tiles
 // are scheduled first.  Per key tile j of 128 keys:
-//   S [128 q x 128 k]  = Q . K_j^T        (M = 128, N = 128, both K-major)
-//   O [128 q x 128 d] += P_j . V_j        (A = P K-major, B = V MN-major)
-// S is double-buffered in tensor memory (columns 0-127, 128-255), O lives at
-// columns 256-383.  Roles: warp 0 issues the tensor copies (Q once, then K/V
-// tiles into a 2-stage ring), warp 1 owns tensor memory and issues the MMAs,
-// warps 2-5 (thread = query row = tensor-memory lane) read S, apply the gate
-// and the online softmax, write P (bf16, 128-byte swizzle) for the second
-// MMA and keep the running max lazily: O is rescaled in tensor memory only
-// when the row max grows by more than 2^8, so the exponentials stay <= 2^8.
+//   S [128 q x 128 k]  = Q . K_j^T   (M = 128, N = 128; Q, K from shared memory)
+//   O [128 q x 128 d] += P_j . V_j   (A = P from tensor memory, B = V MN-major)
+// Tensor memory: S double-buffered in columns 0-127 / 128-255, O in 256-383.
+// P_j (bf16, two per column) overwrites the S_j columns it was computed from,
+// so tile j + 2's S (issued after P_j . V_j by the same thread, and the MMAs
+// run in issue order) never races it.
+//
+// Roles: warp 0 issues the tensor copies (Q once, K/V tiles into a 2-stage
+// ring); warp 1 owns tensor memory and issues the MMAs; warps 2-9 run the
+// softmax, two warps per query-row quarter (tensor-memory lane quarter),
+// each on 64 of the 128 key columns: gate, causal mask, tile max (exchanged
+// between the two halves of a row through shared memory), exp2 and P.  The
+// running max moves lazily: O is rescaled in tensor memory only when a row's
+// max grows by more than 2^8, so the weights stay <= 2^8.
 #include <math.h>
 
 #include "attend_common.cuh"
@@ -32,12 +37,15 @@ namespace {
 
 using namespace tc;
 using dev::wait_or_abort;
+using dev::warp_wait_or_abort;
 
 constexpr int D = 128;
 constexpr int BM = 128;  // query rows per CTA
 constexpr int BN = 128;  // keys per tile
-constexpr int kWarps = 6;
+constexpr int kSoftWarps = 8;
+constexpr int kWarps = 2 + kSoftWarps;
 constexpr int kThreads = kWarps * 32;
+constexpr int kSoftThreads = kSoftWarps * 32;
 constexpr int kStages = 2;
 constexpr uint32_t kTmemCols = 512;  // S0 0..127, S1 128..255, O 256..383
 constexpr uint32_t kOCol = 256;
@@ -45,14 +53,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLazy = 8.0f;  // rescale O only when the max grows by more than this (base 2)
 
-constexpr uint32_t PANEL = BM * 128;           // one 64-column panel of 128 rows (16 KB)
-constexpr uint32_t TILE = 2 * PANEL;           // 128 rows x 128 bf16 (32 KB)
+constexpr uint32_t PANEL = BM * 128;  // one 64-column panel of 128 rows (16 KB)
+constexpr uint32_t TILE = 2 * PANEL;  // 128 rows x 128 bf16 (32 KB)
 constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_STAGE = TILE;           // stage s: K at OFF_STAGE + 2 s TILE, V after it
-constexpr uint32_t OFF_P = OFF_STAGE + kStages * 2 * TILE;
-constexpr uint32_t OFF_BARS = OFF_P + TILE;
+constexpr uint32_t OFF_STAGE = TILE;  // stage s: K at OFF_STAGE + 2 s TILE, V after it
+constexpr uint32_t OFF_RED = OFF_STAGE + kStages * 2 * TILE;  // [2 tiles][2 halves][128] float
+constexpr uint32_t OFF_BARS = OFF_RED + 2 * 2 * BM * 4;
 constexpr uint32_t kSmemBytes = OFF_BARS + 256 + 1024;  // barriers, flags, alignment slack
-
 
 __device__ __forceinline__ float tanh_approx(float x) {
   float y;
@@ -70,15 +77,22 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo_f(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
+// Tensor-memory column of the 8 P columns feeding K step kk (16 keys) of the
+// P V MMA in S buffer sb: keys 0-63 were written by the first half at
+// columns 0-31 of the buffer, keys 64-127 by the second half at 64-95.
+__device__ __forceinline__ uint32_t p_col(int sb, int kk) {
+  return static_cast<uint32_t>(sb * BN + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8));
+}
+
 struct Bars {
   uint64_t* q_full;    // producer -> MMA (tx bytes)
   uint64_t* kv_full;   // [2] producer -> MMA (tx bytes)
   uint64_t* kv_empty;  // [2] MMA commit -> producer
   uint64_t* s_full;    // [2] MMA commit -> softmax
-  uint64_t* s_free;    // [2] softmax (4 warps) -> MMA
-  uint64_t* p_full;    // softmax (4 warps) -> MMA
+  uint64_t* p_full;    // [2] softmax (8 warps) -> MMA
   uint64_t* o_done;    // MMA commit after every P V -> softmax
   uint64_t* done;      // final commit of the MMA warp
+  uint64_t* rv;        // rendezvous of the 8 softmax warps (bounded waits)
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -94,10 +108,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bs.kv_full = bar + 1;
   Bs.kv_empty = bar + 3;
   Bs.s_full = bar + 5;
-  Bs.s_free = bar + 7;
-  Bs.p_full = bar + 9;
-  Bs.o_done = bar + 10;
-  Bs.done = bar + 11;
+  Bs.p_full = bar + 7;
+  Bs.o_done = bar + 9;
+  Bs.done = bar + 10;
+  Bs.rv = bar + 11;
+  float* red = reinterpret_cast<float*>(base + OFF_RED);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_BARS + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + OFF_BARS + 132);
   int* issued = reinterpret_cast<int*>(base + OFF_BARS + 136);  // [2] parity of the last copy per stage, -1 none
@@ -116,12 +131,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(&Bs.kv_full[k], 1);
       dev::mbar_init(&Bs.kv_empty[k], 1);
       dev::mbar_init(&Bs.s_full[k], 1);
-      dev::mbar_init(&Bs.s_free[k], 4);
+      dev::mbar_init(&Bs.p_full[k], kSoftWarps);
       issued[k] = -1;
     }
-    dev::mbar_init(Bs.p_full, 4);
     dev::mbar_init(Bs.o_done, 1);
     dev::mbar_init(Bs.done, 1);
+    dev::mbar_init(Bs.rv, kSoftWarps);
     *abort_flag = 0;
     dev::fence_barrier_init();
   }
@@ -177,22 +192,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Issue order QK(0), QK(1), PV(0), QK(2), PV(1), ...: QK(j + 2) rewrites
+    // S buffer j & 1 only after PV(j) read P_j from it.
     constexpr uint32_t idesc_qk = idesc_bf16(BM, BN, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16(BM, D, 0, 1);
     bool ok = wait_or_abort(Bs.q_full, 0, a.status, abort_flag);
     auto issue_pv = [&](int i) -> bool {
-      if (!wait_or_abort(Bs.p_full, static_cast<uint32_t>(i & 1), a.status, abort_flag)) return false;
+      const int sb = i & 1;
+      if (!wait_or_abort(&Bs.p_full[sb], static_cast<uint32_t>((i >> 1) & 1), a.status, abort_flag)) return false;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t vs = base_u32 + OFF_STAGE + static_cast<uint32_t>(i & 1) * 2 * TILE + TILE;
+        const uint32_t vs = base_u32 + OFF_STAGE + static_cast<uint32_t>(sb) * 2 * TILE + TILE;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t ad = sw128_desc(base_u32 + OFF_P + (kk >> 2) * PANEL + (kk & 3) * 32, 16, 1024);
           const uint64_t bd = sw128_desc(vs + kk * 2048, PANEL, 1024);
-          mma_bf16(tmem + kOCol, ad, bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          mma_bf16_tmem_a(tmem + kOCol, tmem + p_col(sb, kk), bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(Bs.o_done);
-        mma_commit(&Bs.kv_empty[i & 1]);
+        mma_commit(&Bs.kv_empty[sb]);
       }
       __syncwarp();
       return true;
@@ -200,7 +217,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int j = 0; j < nt && ok; ++j) {
       const int st = j & 1;
       if (!wait_or_abort(&Bs.kv_full[st], (j >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
-      if (!wait_or_abort(&Bs.s_free[st], ((j >> 1) & 1) ^ 1, a.status, abort_flag)) { ok = false; break; }
       tc_fence_after();
       if (lane == 0) {
         const uint32_t ks = base_u32 + OFF_STAGE + static_cast<uint32_t>(st) * 2 * TILE;
@@ -227,12 +243,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int qq = warp & 3;  // tensor-memory lane quarter of this warp
+    const int qq = warp & 3;               // tensor-memory lane quarter of this warp
+    const int hf = (warp - 2) >> 2;        // which 64 key columns (and 64 O columns)
     const uint32_t lane_base = static_cast<uint32_t>(32 * qq) << 16;
-    const int r = 32 * qq + lane;  // query row of the tile
+    const int r = 32 * qq + lane;          // query row of the tile
     const int i = q0 + r;
     const bool row_ok = i < a.T;
     const size_t row = static_cast<size_t>(b * a.Hq + h) * a.T + i;
+    const int st_id = t - 64;              // 0..255 among the softmax threads
     float tau = 0.f;
     if (row_ok) {
       if (a.tau_mode == ETA_TAU_LEARNED) {
@@ -258,114 +276,128 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     const float scale = a.scale, beta = a.beta;
-    float m_run = -INFINITY, l_run = 0.f, rsum = 0.f;
+    float m_run = -INFINITY, l_part = 0.f, r_part = 0.f;
     bool ok = true;
-    uint8_t* prow = base + OFF_P + r * 128;
+    // Consecutive rendezvous complete consecutive phases of Bs.rv; a warp can
+    // run at most one phase ahead of the slowest, and every wait is bounded
+    // (an abort anywhere releases all of them).
+    uint32_t rv_phase = 0;
+    auto rendezvous = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) dev::mbar_arrive(Bs.rv);
+      const bool r2 = warp_wait_or_abort(Bs.rv, rv_phase, a.status, abort_flag);
+      rv_phase ^= 1u;
+      return r2;
+    };
     for (int j = 0; j < nt && ok; ++j) {
       const int sb = j & 1;
-      if (!dev::warp_wait_or_abort(&Bs.s_full[sb], (j >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+      if (!warp_wait_or_abort(&Bs.s_full[sb], (j >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) tmem_ld32_nowait(tmem + lane_base + static_cast<uint32_t>(sb) * BN + 32 * k, s[k]);
+      uint32_t s0[32], s1[32];
+      const uint32_t scol = tmem + lane_base + static_cast<uint32_t>(sb * BN + hf * 64);
+      tmem_ld32_nowait(scol, s0);
+      tmem_ld32_nowait(scol + 32, s1);
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(&Bs.s_free[sb]);
 
       // keys j BN + c with c <= lim are seen by this row (causal; rows past
       // the sequence see none)
-      const int lim = row_ok ? min(BN - 1, i - j * BN) : -1;
-      float mt = -INFINITY;
+      const int lim = row_ok ? min(BN - 1, i - j * BN) - hf * 64 : -1;
+      float pm = -INFINITY;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float S = __uint_as_float(s[k][c]) * scale;
-          const float sg = gate(beta * (S - tau));
-          const float x = S * sg * kLog2e;
-          const bool on = 32 * k + c <= lim;
-          rsum += on ? sg : 0.f;
-          mt = fmaxf(mt, on ? x : -INFINITY);
-          s[k][c] = __float_as_uint(on ? x : -INFINITY);
-        }
+      for (int c = 0; c < 64; ++c) {
+        uint32_t& sv = c < 32 ? s0[c] : s1[c - 32];
+        const float S = __uint_as_float(sv) * scale;
+        const float sg = gate(beta * (S - tau));
+        const float x = S * sg * kLog2e;
+        const bool on = c <= lim;
+        r_part += on ? sg : 0.f;
+        pm = fmaxf(pm, on ? x : -INFINITY);
+        sv = __float_as_uint(on ? x : -INFINITY);
       }
-      // P V of the previous tile done: the P buffer is free and O is stable
-      if (j > 0 && !dev::warp_wait_or_abort(Bs.o_done, static_cast<uint32_t>((j - 1) & 1), a.status, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      // A row whose max grew past the margin moves its reference to the new
-      // max; if it had weights already, its O row is rescaled.  Tensor-memory
-      // loads and stores are warp-wide instructions, so the whole warp runs
-      // them when any of its rows needs it (alpha = 1 for the others).
+      // the row's tile max over both halves
+      red[(sb * 2 + hf) * BM + r] = pm;
+      if (!rendezvous()) { ok = false; break; }
+      const float mt = fmaxf(pm, red[(sb * 2 + (hf ^ 1)) * BM + r]);
+
+      // A row whose max grew past the margin moves its reference; if it had
+      // weights already, its O row is rescaled once P V of the previous tile
+      // is done (P_j is not issued yet).  Tensor-memory loads and stores are
+      // warp-wide, so the whole warp runs them (alpha = 1 for other rows).
       const bool grow = mt > m_run + kLazy;
       const bool rescale = grow && m_run != -INFINITY;
       if (__any_sync(0xffffffffu, rescale)) {
+        if (!warp_wait_or_abort(Bs.o_done, static_cast<uint32_t>((j - 1) & 1), a.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         const float alpha = rescale ? dev::fast_exp2(m_run - mt) : 1.f;
+        const uint32_t ocol = tmem + lane_base + kOCol + static_cast<uint32_t>(hf * 64);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 2; ++k) {
           uint32_t o[32];
-          tmem_ld32_nowait(tmem + lane_base + kOCol + 32 * k, o);
+          tmem_ld32_nowait(ocol + 32 * k, o);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-          tmem_st32(tmem + lane_base + kOCol + 32 * k, o);
+          tmem_st32(ocol + 32 * k, o);
         }
         tmem_wait_st();
-        l_run *= alpha;
+        l_part *= alpha;
       }
       if (grow) m_run = mt;
-      // P_j = 2^(x - m_run), bf16, 128-byte swizzle: 16-byte chunk q of row r
-      // sits at chunk q ^ (r & 7) of the row's 128 bytes in its panel
+
+      // P_j = 2^(x - m_run) as bf16 pairs over this half's S columns
+      uint32_t pk[32];
       float lsum = 0.f;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-#pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint32_t w[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float x0 = __uint_as_float(s[k][8 * c8 + 2 * e]);
-            const float x1 = __uint_as_float(s[k][8 * c8 + 2 * e + 1]);
-            const float p0 = x0 == -INFINITY ? 0.f : dev::fast_exp2(x0 - m_run);
-            const float p1 = x1 == -INFINITY ? 0.f : dev::fast_exp2(x1 - m_run);
-            w[e] = pack_bf16(p0, p1);
-            lsum += bf16_lo_f(w[e]) + bf16_hi_f(w[e]);
-          }
-          const int col = 32 * k + 8 * c8;
-          const int panel = col >> 6, chunk = (col & 63) >> 3;
-          *reinterpret_cast<uint4*>(prow + panel * PANEL + ((chunk ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-        }
+      for (int e = 0; e < 32; ++e) {
+        const float x0 = __uint_as_float(e < 16 ? s0[2 * e] : s1[2 * e - 32]);
+        const float x1 = __uint_as_float(e < 16 ? s0[2 * e + 1] : s1[2 * e + 1 - 32]);
+        const float p0 = x0 == -INFINITY ? 0.f : dev::fast_exp2(x0 - m_run);
+        const float p1 = x1 == -INFINITY ? 0.f : dev::fast_exp2(x1 - m_run);
+        pk[e] = pack_bf16(p0, p1);
+        lsum += bf16_lo_f(pk[e]) + bf16_hi_f(pk[e]);
       }
-      l_run += lsum;
+      l_part += lsum;
+      tmem_st32(scol, pk);
+      tmem_wait_st();
       // V rows of this tile past the sequence end hold no key: zeroed so that
       // stale or non-finite bytes there cannot reach O (0 * inf)
       const int kvalid = a.T - j * BN;
       if (kvalid < BN) {
         uint8_t* vt = base + OFF_STAGE + sb * 2 * TILE + TILE;
         const int nz = (BN - kvalid) * 8;  // 16-byte chunks per panel
-        for (int c = t - 64; c < 2 * nz; c += 128) {
+        for (int c = st_id; c < 2 * nz; c += kSoftThreads) {
           const int pnl = c / nz, rem = c - pnl * nz;
           *reinterpret_cast<uint4*>(vt + pnl * PANEL + (kvalid + (rem >> 3)) * 128 + (rem & 7) * 16) =
               make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async();
       }
-      fence_proxy_async();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(Bs.p_full);
+      if (lane == 0) dev::mbar_arrive(&Bs.p_full[sb]);
     }
-    if (ok) ok = dev::warp_wait_or_abort(Bs.o_done, static_cast<uint32_t>((nt - 1) & 1), a.status, abort_flag);
+    if (ok) ok = warp_wait_or_abort(Bs.o_done, static_cast<uint32_t>((nt - 1) & 1), a.status, abort_flag);
     tc_fence_after();
+    // row totals over both halves (every softmax thread reaches this barrier)
+    float* lred = red;            // [2 halves][128]: l
+    float* rred = red + 2 * BM;   // [2 halves][128]: R
+    if (!rendezvous()) ok = false;  // the tile-max exchange slots are free again
+    lred[hf * BM + r] = l_part;
+    rred[hf * BM + r] = r_part;
+    if (!rendezvous()) ok = false;
+    const float l_run = l_part + lred[(hf ^ 1) * BM + r];
+    const float rsum = r_part + rred[(hf ^ 1) * BM + r];
     if (ok) {
       const float inv = (row_ok && l_run > 0.f) ? 1.f / l_run : 0.f;
-      uint4* orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + row * D);
+      uint4* orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + row * D + hf * 64);
+      const uint32_t ocol = tmem + lane_base + kOCol + static_cast<uint32_t>(hf * 64);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
+      for (int k = 0; k < 2; ++k) {
         uint32_t o[32];
-        tmem_ld32_nowait(tmem + lane_base + kOCol + 32 * k, o);
+        tmem_ld32_nowait(ocol + 32 * k, o);
         tmem_wait_ld();
         if (row_ok) {
 #pragma unroll
@@ -378,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (row_ok) {
+      if (row_ok && hf == 0) {
         if (a.lse) a.lse[row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
         if (a.gate_sum) a.gate_sum[row] = rsum;
       }
