@@ -70,8 +70,11 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // sigmoid(x) = (1 + tanh(x / 2)) / 2: one special-function op.
 __device__ __forceinline__ float gate(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
 
+// Two floats to a bf16 pair (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  return static_cast<uint32_t>(dev::f32_to_bf16_rn(lo)) | (static_cast<uint32_t>(dev::f32_to_bf16_rn(hi)) << 16);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ __forceinline__ float bf16_lo_f(uint32_t x) { return __uint_as_float(x << 16); }
@@ -300,19 +303,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_ld();
 
       // keys j BN + c with c <= lim are seen by this row (causal; rows past
-      // the sequence see none)
+      // the sequence see none).  Off the diagonal every key of every row of
+      // the warp is seen: no masking there.
+      // gate(beta (scale S - tau)) = 1/2 + tanh(cb S + ct) / 2, x = cx S gate.
       const int lim = row_ok ? min(BN - 1, i - j * BN) - hf * 64 : -1;
+      const bool full = __all_sync(0xffffffffu, lim >= 63);
+      const float cb = 0.5f * beta * scale, ct = -0.5f * beta * tau, cx = scale * kLog2e;
       float pm = -INFINITY;
+      if (full) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        uint32_t& sv = c < 32 ? s0[c] : s1[c - 32];
-        const float S = __uint_as_float(sv) * scale;
-        const float sg = gate(beta * (S - tau));
-        const float x = S * sg * kLog2e;
-        const bool on = c <= lim;
-        r_part += on ? sg : 0.f;
-        pm = fmaxf(pm, on ? x : -INFINITY);
-        sv = __float_as_uint(on ? x : -INFINITY);
+        for (int c = 0; c < 64; ++c) {
+          uint32_t& sv = c < 32 ? s0[c] : s1[c - 32];
+          const float Sr = __uint_as_float(sv);
+          const float sg = fmaf(0.5f, tanh_approx(fmaf(Sr, cb, ct)), 0.5f);
+          const float x = Sr * cx * sg;
+          r_part += sg;
+          pm = fmaxf(pm, x);
+          sv = __float_as_uint(x);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          uint32_t& sv = c < 32 ? s0[c] : s1[c - 32];
+          const float Sr = __uint_as_float(sv);
+          const float sg = fmaf(0.5f, tanh_approx(fmaf(Sr, cb, ct)), 0.5f);
+          const float x = Sr * cx * sg;
+          const bool on = c <= lim;
+          r_part += on ? sg : 0.f;
+          pm = fmaxf(pm, on ? x : -INFINITY);
+          sv = __float_as_uint(on ? x : -INFINITY);
+        }
       }
       // the row's tile max over both halves
       red[(sb * 2 + hf) * BM + r] = pm;
@@ -347,17 +367,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (grow) m_run = mt;
 
-      // P_j = 2^(x - m_run) as bf16 pairs over this half's S columns
+      // P_j = 2^(x - m_run) as bf16 pairs over this half's S columns; l sums
+      // the fp32 weights (their bf16 rounding is below the output's own)
       uint32_t pk[32];
       float lsum = 0.f;
+      if (full) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const float x0 = __uint_as_float(e < 16 ? s0[2 * e] : s1[2 * e - 32]);
-        const float x1 = __uint_as_float(e < 16 ? s0[2 * e + 1] : s1[2 * e + 1 - 32]);
-        const float p0 = x0 == -INFINITY ? 0.f : dev::fast_exp2(x0 - m_run);
-        const float p1 = x1 == -INFINITY ? 0.f : dev::fast_exp2(x1 - m_run);
-        pk[e] = pack_bf16(p0, p1);
-        lsum += bf16_lo_f(pk[e]) + bf16_hi_f(pk[e]);
+        for (int e = 0; e < 32; ++e) {
+          const float p0 = dev::fast_exp2(__uint_as_float(e < 16 ? s0[2 * e] : s1[2 * e - 32]) - m_run);
+          const float p1 = dev::fast_exp2(__uint_as_float(e < 16 ? s0[2 * e + 1] : s1[2 * e + 1 - 32]) - m_run);
+          pk[e] = pack_bf16(p0, p1);
+          lsum += p0 + p1;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float x0 = __uint_as_float(e < 16 ? s0[2 * e] : s1[2 * e - 32]);
+          const float x1 = __uint_as_float(e < 16 ? s0[2 * e + 1] : s1[2 * e + 1 - 32]);
+          const float p0 = x0 == -INFINITY ? 0.f : dev::fast_exp2(x0 - m_run);
+          const float p1 = x1 == -INFINITY ? 0.f : dev::fast_exp2(x1 - m_run);
+          pk[e] = pack_bf16(p0, p1);
+          lsum += p0 + p1;
+        }
       }
       l_part += lsum;
       tmem_st32(scol, pk);
