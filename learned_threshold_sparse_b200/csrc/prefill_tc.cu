@@ -14,19 +14,22 @@
 // One CTA per (128 query rows, query head, sequence); heavy (late) query tiles
 // are scheduled first.  Per key tile j of 128 keys:
 //   S [128 q x 128 k]  = Q . K_j^T   (M = 128, N = 128; Q, K from shared memory)
-//   O [128 q x 128 d] += P_j . V_j   (A = P from tensor memory, B = V MN-major)
-// Tensor memory: S double-buffered in columns 0-127 / 128-255, O in 256-383.
-// P_j (bf16, two per column) overwrites the S_j columns it was computed from,
-// so tile j + 2's S (issued after P_j . V_j by the same thread, and the MMAs
-// run in issue order) never races it.
+//   O_h [128 q x 128 d] += P_j,h . V_j,h   (h = 0, 1: keys 0-63 / 64-127 of
+//                                          the tile; A = P from tensor
+//                                          memory, B = V MN-major)
+// Tensor memory: S double-buffered in columns 0-127 / 128-255, O_0 in
+// 256-383, O_1 in 384-511.  P_j,h (bf16, two per column) overwrites the S_j
+// columns it was computed from, so tile j + 2's S (issued after P_j . V_j by
+// the same thread, and the MMAs run in issue order) never races it.
 //
 // Roles: warp 0 issues the tensor copies (Q once, K/V tiles into a 2-stage
 // ring); warp 1 owns tensor memory and issues the MMAs; warps 2-9 run the
 // softmax, two warps per query-row quarter (tensor-memory lane quarter),
-// each on 64 of the 128 key columns: gate, causal mask, tile max (exchanged
-// between the two halves of a row through shared memory), exp2 and P.  The
-// running max moves lazily: O is rescaled in tensor memory only when a row's
-// max grows by more than 2^8, so the weights stay <= 2^8.
+// each on one half h of the key columns with its own running max, sum and
+// accumulator O_h (two split-KV partials of the row, merged once at the end
+// by the associative combine), so the halves never wait on each other.  The
+// running max moves lazily: O_h is rescaled in tensor memory only when a
+// row's max grows by more than 2^8, so the weights stay <= 2^8.
 #include <math.h>
 
 #include "attend_common.cuh"
@@ -47,7 +50,7 @@ constexpr int kWarps = 2 + kSoftWarps;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSoftThreads = kSoftWarps * 32;
 constexpr int kStages = 2;
-constexpr uint32_t kTmemCols = 512;  // S0 0..127, S1 128..255, O 256..383
+constexpr uint32_t kTmemCols = 512;  // S0 0..127, S1 128..255, O_0 256..383, O_1 384..511
 constexpr uint32_t kOCol = 256;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -57,8 +60,8 @@ constexpr uint32_t PANEL = BM * 128;  // one 64-column panel of 128 rows (16 KB)
 constexpr uint32_t TILE = 2 * PANEL;  // 128 rows x 128 bf16 (32 KB)
 constexpr uint32_t OFF_Q = 0;
 constexpr uint32_t OFF_STAGE = TILE;  // stage s: K at OFF_STAGE + 2 s TILE, V after it
-constexpr uint32_t OFF_RED = OFF_STAGE + kStages * 2 * TILE;  // [2 tiles][2 halves][128] float
-constexpr uint32_t OFF_BARS = OFF_RED + 2 * 2 * BM * 4;
+constexpr uint32_t OFF_RED = OFF_STAGE + kStages * 2 * TILE;  // [m, l, R][2 halves][128] float
+constexpr uint32_t OFF_BARS = OFF_RED + 3 * 2 * BM * 4;
 constexpr uint32_t kSmemBytes = OFF_BARS + 256 + 1024;  // barriers, flags, alignment slack
 
 __device__ __forceinline__ float tanh_approx(float x) {
@@ -80,11 +83,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo_f(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
-// Tensor-memory column of the 8 P columns feeding K step kk (16 keys) of the
-// P V MMA in S buffer sb: keys 0-63 were written by the first half at
-// columns 0-31 of the buffer, keys 64-127 by the second half at 64-95.
-__device__ __forceinline__ uint32_t p_col(int sb, int kk) {
-  return static_cast<uint32_t>(sb * BN + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8));
+// Tensor-memory column of the 8 P columns feeding K step kk (16 keys) of
+// half h's P V MMA in S buffer sb: half h wrote its 64 keys as 32 columns
+// starting at column 64 h of the buffer.
+__device__ __forceinline__ uint32_t p_col(int sb, int h, int kk) {
+  return static_cast<uint32_t>(sb * BN + h * 64 + kk * 8);
 }
 
 struct Bars {
@@ -92,7 +95,7 @@ struct Bars {
   uint64_t* kv_full;   // [2] producer -> MMA (tx bytes)
   uint64_t* kv_empty;  // [2] MMA commit -> producer
   uint64_t* s_full;    // [2] MMA commit -> softmax
-  uint64_t* p_full;    // [2] softmax (8 warps) -> MMA
+  uint64_t* p_full;    // [2 buffers][2 halves] softmax (4 warps) -> MMA
   uint64_t* o_done;    // MMA commit after every P V -> softmax
   uint64_t* done;      // final commit of the MMA warp
   uint64_t* rv;        // rendezvous of the 8 softmax warps (bounded waits)
@@ -112,9 +115,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   Bs.kv_empty = bar + 3;
   Bs.s_full = bar + 5;
   Bs.p_full = bar + 7;
-  Bs.o_done = bar + 9;
-  Bs.done = bar + 10;
-  Bs.rv = bar + 11;
+  Bs.o_done = bar + 11;
+  Bs.done = bar + 12;
+  Bs.rv = bar + 13;
   float* red = reinterpret_cast<float*>(base + OFF_RED);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_BARS + 128);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + OFF_BARS + 132);
@@ -134,7 +137,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(&Bs.kv_full[k], 1);
       dev::mbar_init(&Bs.kv_empty[k], 1);
       dev::mbar_init(&Bs.s_full[k], 1);
-      dev::mbar_init(&Bs.p_full[k], kSoftWarps);
+      dev::mbar_init(&Bs.p_full[2 * k], kSoftWarps / 2);
+      dev::mbar_init(&Bs.p_full[2 * k + 1], kSoftWarps / 2);
       issued[k] = -1;
     }
     dev::mbar_init(Bs.o_done, 1);
@@ -202,15 +206,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = wait_or_abort(Bs.q_full, 0, a.status, abort_flag);
     auto issue_pv = [&](int i) -> bool {
       const int sb = i & 1;
-      if (!wait_or_abort(&Bs.p_full[sb], static_cast<uint32_t>((i >> 1) & 1), a.status, abort_flag)) return false;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t vs = base_u32 + OFF_STAGE + static_cast<uint32_t>(sb) * 2 * TILE + TILE;
+      const uint32_t vs = base_u32 + OFF_STAGE + static_cast<uint32_t>(sb) * 2 * TILE + TILE;
+      for (int hh = 0; hh < 2; ++hh) {
+        if (!wait_or_abort(&Bs.p_full[2 * sb + hh], static_cast<uint32_t>((i >> 1) & 1), a.status, abort_flag))
+          return false;
+        tc_fence_after();
+        if (lane == 0) {
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sw128_desc(vs + kk * 2048, PANEL, 1024);
-          mma_bf16_tmem_a(tmem + kOCol, tmem + p_col(sb, kk), bd, idesc_pv, (i > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = sw128_desc(vs + (hh * 4 + kk) * 2048, PANEL, 1024);
+            mma_bf16_tmem_a(tmem + kOCol + hh * BN, tmem + p_col(sb, hh, kk), bd, idesc_pv,
+                            (i > 0 || kk > 0) ? 1u : 0u);
+          }
         }
+        __syncwarp();
+      }
+      if (lane == 0) {
         mma_commit(Bs.o_done);
         mma_commit(&Bs.kv_empty[sb]);
       }
@@ -334,10 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           sv = __float_as_uint(on ? x : -INFINITY);
         }
       }
-      // the row's tile max over both halves
-      red[(sb * 2 + hf) * BM + r] = pm;
-      if (!rendezvous()) { ok = false; break; }
-      const float mt = fmaxf(pm, red[(sb * 2 + (hf ^ 1)) * BM + r]);
+      const float mt = pm;
 
       // A row whose max grew past the margin moves its reference; if it had
       // weights already, its O row is rescaled once P V of the previous tile
@@ -352,9 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const float alpha = rescale ? dev::fast_exp2(m_run - mt) : 1.f;
-        const uint32_t ocol = tmem + lane_base + kOCol + static_cast<uint32_t>(hf * 64);
+        const uint32_t ocol = tmem + lane_base + kOCol + static_cast<uint32_t>(hf * BN);
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
+        for (int k = 0; k < 4; ++k) {
           uint32_t o[32];
           tmem_ld32_nowait(ocol + 32 * k, o);
           tmem_wait_ld();
@@ -395,55 +403,66 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_wait_st();
       // V rows of this tile past the sequence end hold no key: zeroed so that
       // stale or non-finite bytes there cannot reach O (0 * inf)
-      const int kvalid = a.T - j * BN;
-      if (kvalid < BN) {
+      // (each half zeroes the rows its own P V reads, before it signals P)
+      const int z0 = max(a.T - j * BN, hf * 64), z1 = hf * 64 + 64;
+      if (z0 < z1) {
         uint8_t* vt = base + OFF_STAGE + sb * 2 * TILE + TILE;
-        const int nz = (BN - kvalid) * 8;  // 16-byte chunks per panel
-        for (int c = st_id; c < 2 * nz; c += kSoftThreads) {
+        const int nz = (z1 - z0) * 8;  // 16-byte chunks per panel
+        for (int c = st_id & 127; c < 2 * nz; c += kSoftThreads / 2) {
           const int pnl = c / nz, rem = c - pnl * nz;
-          *reinterpret_cast<uint4*>(vt + pnl * PANEL + (kvalid + (rem >> 3)) * 128 + (rem & 7) * 16) =
+          *reinterpret_cast<uint4*>(vt + pnl * PANEL + (z0 + (rem >> 3)) * 128 + (rem & 7) * 16) =
               make_uint4(0u, 0u, 0u, 0u);
         }
         fence_proxy_async();
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) dev::mbar_arrive(&Bs.p_full[sb]);
+      if (lane == 0) dev::mbar_arrive(&Bs.p_full[2 * sb + hf]);
     }
     if (ok) ok = warp_wait_or_abort(Bs.o_done, static_cast<uint32_t>((nt - 1) & 1), a.status, abort_flag);
     tc_fence_after();
-    // row totals over both halves (every softmax thread reaches this barrier)
-    float* lred = red;            // [2 halves][128]: l
-    float* rred = red + 2 * BM;   // [2 halves][128]: R
-    if (!rendezvous()) ok = false;  // the tile-max exchange slots are free again
+    // the two halves of a row are merged: m* = max m_h, l = sum 2^(m_h - m*) l_h,
+    // out = sum 2^(m_h - m*) O_h / l (every softmax thread reaches this point)
+    float* mred = red;             // [2 halves][128]
+    float* lred = red + 2 * BM;
+    float* rred = red + 4 * BM;
+    mred[hf * BM + r] = m_run;
     lred[hf * BM + r] = l_part;
     rred[hf * BM + r] = r_part;
     if (!rendezvous()) ok = false;
-    const float l_run = l_part + lred[(hf ^ 1) * BM + r];
-    const float rsum = r_part + rred[(hf ^ 1) * BM + r];
     if (ok) {
+      const float m0 = mred[r], m1 = mred[BM + r];
+      const float ms = fmaxf(m0, m1);
+      const float f0 = m0 == -INFINITY ? 0.f : dev::fast_exp2(m0 - ms);
+      const float f1 = m1 == -INFINITY ? 0.f : dev::fast_exp2(m1 - ms);
+      const float l_run = f0 * lred[r] + f1 * lred[BM + r];
       const float inv = (row_ok && l_run > 0.f) ? 1.f / l_run : 0.f;
+      const float g0 = f0 * inv, g1 = f1 * inv;
       uint4* orow = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + row * D + hf * 64);
       const uint32_t ocol = tmem + lane_base + kOCol + static_cast<uint32_t>(hf * 64);
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        uint32_t o[32];
-        tmem_ld32_nowait(ocol + 32 * k, o);
+        uint32_t o0[32], o1[32];
+        tmem_ld32_nowait(ocol + 32 * k, o0);
+        tmem_ld32_nowait(ocol + BN + 32 * k, o1);
         tmem_wait_ld();
         if (row_ok) {
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
             uint32_t w[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              w[e] = pack_bf16(__uint_as_float(o[8 * c8 + 2 * e]) * inv, __uint_as_float(o[8 * c8 + 2 * e + 1]) * inv);
+            for (int e = 0; e < 4; ++e) {
+              const int c = 8 * c8 + 2 * e;
+              w[e] = pack_bf16(fmaf(__uint_as_float(o0[c]), g0, __uint_as_float(o1[c]) * g1),
+                               fmaf(__uint_as_float(o0[c + 1]), g0, __uint_as_float(o1[c + 1]) * g1));
+            }
             orow[4 * k + c8] = make_uint4(w[0], w[1], w[2], w[3]);
           }
         }
       }
       if (row_ok && hf == 0) {
-        if (a.lse) a.lse[row] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
-        if (a.gate_sum) a.gate_sum[row] = rsum;
+        if (a.lse) a.lse[row] = l_run > 0.f ? (ms + log2f(l_run)) * kLn2 : -INFINITY;
+        if (a.gate_sum) a.gate_sum[row] = rred[r] + rred[BM + r];
       }
     }
   }
