@@ -100,9 +100,15 @@ def union_bytes(wl, union_list, union_count):
     return tot
 
 
-def step_bytes(wl, kv_union):
+def meta_record_bytes(head_dim, meta="fp16"):
+    """Bytes of one block's metadata per KV head: fp16 centroid and spread +
+    fp32 M, or e4m3 codes + two fp32 scales + fp32 M."""
+    return 2 * head_dim + 12 if meta == "fp8" else 4 * head_dim + 4
+
+
+def step_bytes(wl, kv_union, meta="fp16"):
     nb_total = sum(wl.n_blocks(i) for i in range(wl.batch)) * wl.n_kv_heads
-    meta = nb_total * (4 * wl.head_dim + 4)
+    meta = nb_total * meta_record_bytes(wl.head_dim, meta)
     qo = 2 * wl.batch * wl.n_q_heads * wl.head_dim * wl.elt_bytes
     tau = wl.n_q_heads * (wl.head_dim + 1) * 4 if wl.tau_mode == "learned" else wl.n_q_heads * 4
     return kv_union + meta + qo + tau
@@ -213,7 +219,7 @@ def run_eta(args):
     w_tau = None if wl.w_tau is None else torch.from_numpy(wl.w_tau).to(dev)
     b_tau = None if wl.b_tau is None else torch.from_numpy(wl.b_tau).to(dev)
     c_tau = None if wl.c_tau is None else torch.from_numpy(wl.c_tau).to(dev)
-    summ = eta.alloc_summary(wl.batch, wl.n_kv_heads, wl.max_ctx, wl.head_dim, wl.block_size, dev)
+    summ = eta.alloc_summary(wl.batch, wl.n_kv_heads, wl.max_ctx, wl.head_dim, wl.block_size, dev, fmt=args.meta)
     first = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
     eta.eta_block_summary_update(k, v, seq, summ, wl.block_size, first, wl.nb_max, wl.n_q_heads)
 
@@ -227,7 +233,7 @@ def run_eta(args):
     uc = sel["union_count"].cpu().numpy()
     ul = sel["union_list"].cpu().numpy()
     kv_union = union_bytes(wl, ul, uc)
-    nbytes = step_bytes(wl, kv_union)
+    nbytes = step_bytes(wl, kv_union, args.meta)
     nb_total = sum(wl.n_blocks(i) for i in range(wl.batch)) * wl.n_kv_heads
     union_density = float(uc.sum()) / nb_total
     head_density = float(sel["admitted_count"].cpu().numpy().sum()) / (nb_total * wl.group)
@@ -382,6 +388,7 @@ def run_eta(args):
                 "workload": _workload_desc(wl),
                 "seed": args.seed,
                 "screen": "off (dense)" if args.dense else "on",
+                "metadata": args.meta,
                 "attend_impl": {0: "auto", 1: "simt", 2: "tc"}[args.attend_impl],
                 "union_density": round(union_density, 4),
                 "head_density": round(head_density, 4),
@@ -571,6 +578,7 @@ def main():
     ap.add_argument("--attend-impl", type=int, default=0, choices=[0, 1, 2])
     ap.add_argument("--dense", action="store_true", help="screen off: every block loaded")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--meta", default="fp16", choices=["fp16", "fp8"], help="block metadata format")
     ap.add_argument("--prefill", action="store_true", help="time the causal forward pass instead of the decode step")
     ap.add_argument("--prefill-shape", default="1,32,8,8192", help="batch,n_q_heads,n_kv_heads,seq_len")
     args = ap.parse_args()

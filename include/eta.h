@@ -86,14 +86,30 @@ typedef struct {
   const int* seq_lens; /* [batch] device, 0 <= seq_lens[i] <= max_ctx         */
 } eta_cache_desc;
 
+/* Storage of the centroid and spread in eta_summary_desc. */
+typedef enum {
+  ETA_META_FP16 = 0,  /* fp16 values (Appendix F.1)                            */
+  ETA_META_FP8 = 1    /* e4m3 codes with one fp32 scale per block and field:
+                         value = code * scale, the scale mapping the block's
+                         largest magnitude to 448 (FP8 metadata, named as a
+                         systems extension in section 5; format is this
+                         library's choice)                                    */
+} eta_meta_format;
+
 /* Per-block, per-KV-head metadata (Appendix F.1): centroid mu_B, coordinate
- * standard deviation sigma_B (both fp16), maximum norm M_B (fp32) of the
- * block's keys around the stored fp16 centroid, rounded up so that the
- * geometric bound <q, mu_B> + ||q|| M_B never under-estimates a key's logit. */
+ * standard deviation sigma_B, maximum norm M_B (fp32) of the block's keys
+ * around the stored (dequantised) centroid, rounded up so that the geometric
+ * bound <q, mu_B> + ||q|| M_B never under-estimates a key's logit.  A
+ * zero-initialised descriptor with mu, sigma and max_norm set is the fp16
+ * format. */
 typedef struct {
-  void* mu;        /* fp16 [batch, n_kv_heads, nb_max, head_dim]             */
-  void* sigma;     /* fp16 [batch, n_kv_heads, nb_max, head_dim]             */
+  void* mu;        /* [batch, n_kv_heads, nb_max, head_dim]: fp16 values, or
+                      e4m3 codes (one byte each) in the fp8 format           */
+  void* sigma;     /* same layout and type as mu                             */
   float* max_norm; /* fp32 [batch, n_kv_heads, nb_max] (4-byte aligned)      */
+  int format;      /* eta_meta_format                                        */
+  float* mu_scale;    /* fp32 [batch, n_kv_heads, nb_max] (fp8 format only)  */
+  float* sigma_scale; /* fp32 [batch, n_kv_heads, nb_max] (fp8 format only)  */
 } eta_summary_desc;
 
 /*

@@ -59,8 +59,13 @@ class eta_cache_desc(ctypes.Structure):
     ]
 
 
+ETA_META_FP16 = 0
+ETA_META_FP8 = 1
+
+
 class eta_summary_desc(ctypes.Structure):
-    _fields_ = [("mu", ctypes.c_void_p), ("sigma", ctypes.c_void_p), ("max_norm", ctypes.c_void_p)]
+    _fields_ = [("mu", ctypes.c_void_p), ("sigma", ctypes.c_void_p), ("max_norm", ctypes.c_void_p),
+                ("format", ctypes.c_int), ("mu_scale", ctypes.c_void_p), ("sigma_scale", ctypes.c_void_p)]
 
 
 class eta_decode_params(ctypes.Structure):
@@ -167,13 +172,34 @@ def cache_desc(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, n_q_hea
 
 
 def alloc_summary(batch: int, n_kv_heads: int, max_ctx: int, head_dim: int, block_size: int,
-                  device="cuda") -> Dict[str, torch.Tensor]:
+                  device="cuda", fmt: str = "fp16") -> Dict[str, torch.Tensor]:
+    """Metadata buffers: fp16 mu / sigma, or (fmt="fp8") e4m3 codes as uint8
+    plus per-block fp32 mu_scale / sigma_scale; fp32 max_norm either way."""
     nb = (max_ctx + block_size - 1) // block_size
+    if fmt == "fp8":
+        return {
+            "mu": torch.zeros((batch, n_kv_heads, nb, head_dim), dtype=torch.uint8, device=device),
+            "sigma": torch.zeros((batch, n_kv_heads, nb, head_dim), dtype=torch.uint8, device=device),
+            "max_norm": torch.zeros((batch, n_kv_heads, nb), dtype=torch.float32, device=device),
+            "mu_scale": torch.zeros((batch, n_kv_heads, nb), dtype=torch.float32, device=device),
+            "sigma_scale": torch.zeros((batch, n_kv_heads, nb), dtype=torch.float32, device=device),
+        }
+    if fmt != "fp16":
+        raise ValueError(fmt)
     return {
         "mu": torch.zeros((batch, n_kv_heads, nb, head_dim), dtype=torch.float16, device=device),
         "sigma": torch.zeros((batch, n_kv_heads, nb, head_dim), dtype=torch.float16, device=device),
         "max_norm": torch.zeros((batch, n_kv_heads, nb), dtype=torch.float32, device=device),
     }
+
+
+def summary_desc(summary: Dict[str, torch.Tensor]) -> eta_summary_desc:
+    d = eta_summary_desc(summary["mu"].data_ptr(), summary["sigma"].data_ptr(), summary["max_norm"].data_ptr())
+    if "mu_scale" in summary:
+        d.format = ETA_META_FP8
+        d.mu_scale = summary["mu_scale"].data_ptr()
+        d.sigma_scale = summary["sigma_scale"].data_ptr()
+    return d
 
 
 def eta_block_summary_update(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor,
@@ -183,8 +209,7 @@ def eta_block_summary_update(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.T
     """Recompute the metadata of the blocks at or after first_token[i] (at most
     max_blocks per sequence)."""
     cache = cache_desc(k, v, seq_lens, n_q_heads or k.shape[1], block_size)
-    summ = eta_summary_desc(summary["mu"].data_ptr(), summary["sigma"].data_ptr(),
-                            summary["max_norm"].data_ptr())
+    summ = summary_desc(summary)
     rc = _lib.eta_block_summary_update(ctypes.byref(cache), ctypes.byref(summ),
                                        ctypes.c_void_p(first_token.data_ptr()), int(max_blocks),
                                        _stream_handle(stream))
@@ -198,8 +223,7 @@ def eta_append_kv(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, summ
     """Write k_new / v_new [B, Hkv, d] at row pos[i] of each sequence and refresh
     the summary of the block holding it (seq_lens must already count it)."""
     cache = cache_desc(k, v, seq_lens, n_q_heads or k.shape[1], block_size)
-    summ = eta_summary_desc(summary["mu"].data_ptr(), summary["sigma"].data_ptr(),
-                            summary["max_norm"].data_ptr())
+    summ = summary_desc(summary)
     rc = _lib.eta_append_kv(ctypes.byref(cache), ctypes.byref(summ), ctypes.c_void_p(k_new.data_ptr()),
                             ctypes.c_void_p(v_new.data_ptr()), ctypes.c_void_p(pos.data_ptr()), _stream_handle(stream))
     if rc != ETA_OK:
@@ -215,8 +239,7 @@ def make_params(q, k, v, seq_lens, summary, block_size, tau_mode, w_tau=None, b_
     p = eta_decode_params()
     p.cache = cache_desc(k, v, seq_lens, Hq, block_size)
     if summary is not None:
-        p.summary = eta_summary_desc(summary["mu"].data_ptr(), summary["sigma"].data_ptr(),
-                                     summary["max_norm"].data_ptr())
+        p.summary = summary_desc(summary)
     p.q = q.data_ptr()
     p.tau_mode = ETA_TAU_LEARNED if tau_mode in ("learned", ETA_TAU_LEARNED) else ETA_TAU_CALIBRATED
     p.w_tau = None if w_tau is None else w_tau.data_ptr()

@@ -39,7 +39,21 @@ eta_status check_cache(const eta_cache_desc* c) {
 eta_status check_summary(const eta_summary_desc* s) {
   if (!s || !s->mu || !s->sigma || !s->max_norm) return ETA_ERR_INVALID_ARG;
   if (!aligned(s->mu, 16) || !aligned(s->sigma, 16) || !aligned(s->max_norm, 4)) return ETA_ERR_INVALID_ARG;
+  if (s->format != ETA_META_FP16 && s->format != ETA_META_FP8) return ETA_ERR_INVALID_ARG;
+  if (s->format == ETA_META_FP8 &&
+      (!s->mu_scale || !s->sigma_scale || !aligned(s->mu_scale, 4) || !aligned(s->sigma_scale, 4)))
+    return ETA_ERR_INVALID_ARG;
   return ETA_OK;
+}
+
+// The summary descriptor's fields into the kernels' arguments.
+template <class Args>
+void set_summary(Args& a, const eta_summary_desc* s) {
+  a.mu = s->mu;
+  a.sigma = s->sigma;
+  a.max_norm = s->max_norm;
+  a.mu_scale = s->mu_scale;
+  a.sigma_scale = s->sigma_scale;
 }
 
 eta_status make_shape(const eta_decode_params* p, Shape* out) {
@@ -207,9 +221,8 @@ eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summa
   a.k = cache->k_cache;
   a.seq_lens = cache->seq_lens;
   a.first_token = first_token;
-  a.mu = static_cast<uint16_t*>(summary->mu);
-  a.sigma = static_cast<uint16_t*>(summary->sigma);
-  a.max_norm = summary->max_norm;
+  set_summary(a, summary);
+  a.fmt = summary->format;
   a.B = cache->batch;
   a.Hkv = cache->n_kv_heads;
   a.d = cache->head_dim;
@@ -233,9 +246,8 @@ eta_status eta_append_kv(const eta_cache_desc* cache, const eta_summary_desc* su
   a.k = cache->k_cache;
   a.seq_lens = cache->seq_lens;
   a.first_token = nullptr;
-  a.mu = static_cast<uint16_t*>(summary->mu);
-  a.sigma = static_cast<uint16_t*>(summary->sigma);
-  a.max_norm = summary->max_norm;
+  set_summary(a, summary);
+  a.fmt = summary->format;
   a.B = cache->batch;
   a.Hkv = cache->n_kv_heads;
   a.d = cache->head_dim;
@@ -283,9 +295,8 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
   sa.w_tau = p->w_tau;
   sa.b_tau = p->b_tau;
   sa.c_tau = p->c_tau;
-  sa.mu = static_cast<const uint16_t*>(p->summary.mu);
-  sa.sigma = static_cast<const uint16_t*>(p->summary.sigma);
-  sa.max_norm = p->summary.max_norm;
+  set_summary(sa, &p->summary);
+  sa.meta_fmt = p->summary.format;
   sa.seq_lens = p->cache.seq_lens;
   sa.tau_mode = p->tau_mode;
   sa.lwb = p->n_local_blocks;

@@ -51,9 +51,12 @@ struct ScreenArgs {
   const float* w_tau;
   const float* b_tau;
   const float* c_tau;
-  const uint16_t* mu;     // fp16 bits
-  const uint16_t* sigma;  // fp16 bits
+  const void* mu;         // fp16 bits or e4m3 codes (meta_fmt)
+  const void* sigma;
   const float* max_norm;
+  const float* mu_scale;     // fp8 format: per-block scales
+  const float* sigma_scale;
+  int meta_fmt;              // ETA_META_FP16 / ETA_META_FP8
   const int* seq_lens;
   int tau_mode, lwb, screen_enabled;
   float scale, offset_a, z;
@@ -124,9 +127,12 @@ struct SummaryArgs {
   const void* k;
   const int* seq_lens;
   const int* first_token;
-  uint16_t* mu;
-  uint16_t* sigma;
+  void* mu;                // fp16 bits or e4m3 codes (fmt)
+  void* sigma;
   float* max_norm;
+  float* mu_scale;         // fp8 format: per-block scales
+  float* sigma_scale;
+  int fmt;                 // ETA_META_FP16 / ETA_META_FP8
   int B, Hkv, d, b, max_ctx, nbmax, elt, max_blocks;
 };
 

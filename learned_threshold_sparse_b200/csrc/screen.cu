@@ -62,15 +62,27 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[N], int lane) {
 
 constexpr int kRound = 64;  // blocks of metadata staged in shared memory per round
 
-// Staging buffers of mu and sigma rows: the second one is used only when a
-// chunk needs more than one round.
-template <int D>
+// Staging buffers of mu and sigma rows (ESZ bytes per coordinate: 2 for fp16,
+// 1 for e4m3 codes): the second one is used only when a chunk needs more than
+// one round.
+template <int D, int ESZ>
 constexpr size_t screen_smem_bytes(int chunk) {
-  return (chunk > kRound ? 2ull : 1ull) * 2 * kRound * D * sizeof(uint16_t);
+  return (chunk > kRound ? 2ull : 1ull) * 2 * kRound * D * ESZ;
 }
 
-template <int D, int G>
+// Two e4m3 codes (low byte first) as floats.
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint16_t codes) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(codes));
+  return make_float2(dev::fp16_to_f32(static_cast<uint16_t>(h2 & 0xffffu)), dev::fp16_to_f32(static_cast<uint16_t>(h2 >> 16)));
+}
+
+// FMT: ETA_META_FP16 or ETA_META_FP8 (then mu~ = code * mu_scale per block,
+// and <q, mu~> = mu_scale <q, code>, sum q^2 sigma~^2 = sigma_scale^2 sum q^2 code^2:
+// the scales are applied after the reduction over d).
+template <int D, int G, int FMT>
 __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
+  constexpr int ESZ = FMT == ETA_META_FP8 ? 1 : 2;
   constexpr int CPL = D / 32;        // coordinates per lane
   constexpr int NV = 2 * G;          // values per block: <q_h, mu>, sum q_h^2 sigma^2
   constexpr int NB = 32 / NV;        // blocks reduced together (32 values per lane)
@@ -80,11 +92,13 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
   const int t = threadIdx.x, w = t >> 5, lane = t & 31;
 
   extern __shared__ __align__(128) uint8_t dsm[];
-  uint16_t* stage = reinterpret_cast<uint16_t*>(dsm);  // [2 buffers][mu, sigma][kRound][D]
+  uint8_t* stage = dsm;  // [2 buffers][mu, sigma][kRound][D] elements of ESZ bytes
   __shared__ float s_q[G][D];
   __shared__ float s_tau[G];
   __shared__ float s_qn[G];
   __shared__ float s_mn[kMaxChunk];
+  __shared__ float s_ms[FMT == ETA_META_FP8 ? kMaxChunk : 1];
+  __shared__ float s_ss[FMT == ETA_META_FP8 ? kMaxChunk : 1];
   __shared__ uint8_t s_mask[kMaxChunk];
   __shared__ int s_wsum[kWarps];
   __shared__ int s_cnt[G];
@@ -101,22 +115,33 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
   const size_t nbase = static_cast<size_t>(seg) * s.nbmax;
   auto issue_round = [&](int r0, int rows) {
     const int buf = (r0 / kRound) & 1;
-    uint16_t* mu_b = stage + static_cast<size_t>(buf) * 2 * kRound * D;
-    const uint32_t bytes = static_cast<uint32_t>(rows) * D * 2;
+    uint8_t* mu_b = stage + static_cast<size_t>(buf) * 2 * kRound * D * ESZ;
+    const uint32_t bytes = static_cast<uint32_t>(rows) * D * ESZ;
+    const size_t src = (mbase + static_cast<size_t>(blk0 + r0) * D) * ESZ;
     dev::mbar_arrive_expect_tx(&s_bar[buf], 2 * bytes);
-    dev::bulk_g2s(mu_b, a.mu + mbase + static_cast<size_t>(blk0 + r0) * D, bytes, &s_bar[buf]);
-    dev::bulk_g2s(mu_b + kRound * D, a.sigma + mbase + static_cast<size_t>(blk0 + r0) * D, bytes, &s_bar[buf]);
+    dev::bulk_g2s(mu_b, static_cast<const uint8_t*>(a.mu) + src, bytes, &s_bar[buf]);
+    dev::bulk_g2s(mu_b + kRound * D * ESZ, static_cast<const uint8_t*>(a.sigma) + src, bytes, &s_bar[buf]);
   };
   // Stage the first round of metadata before the sequence length is known
   // (rows past it are in bounds and simply not used), together with the
-  // block norms, while the threshold is computed.
+  // block norms (and scales), while the threshold is computed.  With the
+  // screen off no metadata is read at all.
+  const bool meta = a.screen_enabled && avail > 0;
   if (t == 0) {
     dev::mbar_init(&s_bar[0], 1);
     dev::mbar_init(&s_bar[1], 1);
     dev::fence_barrier_init();
-    issue_round(0, min(kRound, avail));
+    if (meta) issue_round(0, min(kRound, avail));
   }
-  for (int x = t; x < avail; x += kThreads) s_mn[x] = a.max_norm[nbase + blk0 + x];
+  if (meta) {
+    for (int x = t; x < avail; x += kThreads) {
+      s_mn[x] = a.max_norm[nbase + blk0 + x];
+      if (FMT == ETA_META_FP8) {
+        s_ms[x] = a.mu_scale[nbase + blk0 + x];
+        s_ss[x] = a.sigma_scale[nbase + blk0 + x];
+      }
+    }
+  }
 
   // Threshold inputs of this warp's head, loaded now so that they share the
   // first round trip with the metadata copies and the query rows.
@@ -197,8 +222,8 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
   for (int r0 = 0; r0 < nscreen && staged_ok; r0 += kRound) {
     const int r = min(kRound, nscreen - r0);
     const int buf = (r0 / kRound) & 1;
-    const uint16_t* mu_s = stage + static_cast<size_t>(buf) * 2 * kRound * D;
-    const uint16_t* sg_s = mu_s + kRound * D;
+    const uint8_t* mu_s = stage + static_cast<size_t>(buf) * 2 * kRound * D * ESZ;
+    const uint8_t* sg_s = mu_s + kRound * D * ESZ;
     if (!dev::mbar_wait(&s_bar[buf], (r0 / (2 * kRound)) & 1, a.status)) { staged_ok = false; break; }
     for (int gb = w * NB; gb < r; gb += kWarps * NB) {
       float v[32];
@@ -208,14 +233,22 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
         float mu[CPL], s2[CPL];
 #pragma unroll
         for (int k = 0; k < CPL / 2; ++k) {
-          const uint32_t m2 = *reinterpret_cast<const uint32_t*>(mu_s + lb * D + lane * CPL + 2 * k);
-          const uint32_t g2 = *reinterpret_cast<const uint32_t*>(sg_s + lb * D + lane * CPL + 2 * k);
-          mu[2 * k] = dev::fp16_to_f32(static_cast<uint16_t>(m2 & 0xffffu));
-          mu[2 * k + 1] = dev::fp16_to_f32(static_cast<uint16_t>(m2 >> 16));
-          const float a0 = dev::fp16_to_f32(static_cast<uint16_t>(g2 & 0xffffu));
-          const float a1 = dev::fp16_to_f32(static_cast<uint16_t>(g2 >> 16));
-          s2[2 * k] = a0 * a0;
-          s2[2 * k + 1] = a1 * a1;
+          float2 m, g2;
+          if (FMT == ETA_META_FP8) {
+            m = e4m3x2_to_f32(*reinterpret_cast<const uint16_t*>(mu_s + lb * D + lane * CPL + 2 * k));
+            g2 = e4m3x2_to_f32(*reinterpret_cast<const uint16_t*>(sg_s + lb * D + lane * CPL + 2 * k));
+          } else {
+            const uint32_t mm = *reinterpret_cast<const uint32_t*>(mu_s + (lb * D + lane * CPL + 2 * k) * 2);
+            const uint32_t gg = *reinterpret_cast<const uint32_t*>(sg_s + (lb * D + lane * CPL + 2 * k) * 2);
+            m = make_float2(dev::fp16_to_f32(static_cast<uint16_t>(mm & 0xffffu)),
+                            dev::fp16_to_f32(static_cast<uint16_t>(mm >> 16)));
+            g2 = make_float2(dev::fp16_to_f32(static_cast<uint16_t>(gg & 0xffffu)),
+                             dev::fp16_to_f32(static_cast<uint16_t>(gg >> 16)));
+          }
+          mu[2 * k] = m.x;
+          mu[2 * k + 1] = m.y;
+          s2[2 * k] = g2.x * g2.x;
+          s2[2 * k + 1] = g2.y * g2.y;
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
@@ -229,13 +262,18 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
           v[u * NV + G + h] = sq;
         }
       }
-      const float red = transpose_reduce32<32>(v, lane);
-      const float sq = __shfl_down_sync(0xffffffffu, red, G);  // sum q^2 sigma^2 of the same (block, head)
+      float red = transpose_reduce32<32>(v, lane);
+      float sq = __shfl_down_sync(0xffffffffu, red, G);  // sum q^2 sigma^2 of the same (block, head)
       const int lb = gb + vb;
       const bool head_lane = vq < G && lb < r;
       float score = 0.f;
       bool pass = false;
       if (head_lane) {
+        if (FMT == ETA_META_FP8) {
+          const float ss = s_ss[r0 + lb];
+          red *= s_ms[r0 + lb];
+          sq *= ss * ss;
+        }
         const float geo = my_qn * s_mn[r0 + lb];
         const float spread = strict ? geo : fminf(geo, z * sqrtf(sq));
         score = scale * (red + spread);
@@ -261,7 +299,7 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
   }
   // The speculative first copy lands before exit even when nothing here
   // was screened.
-  if (t == 0 && nscreen == 0) dev::mbar_wait(&s_bar[0], 0, a.status);
+  if (t == 0 && nscreen == 0 && meta) dev::mbar_wait(&s_bar[0], 0, a.status);
   __syncthreads();
   if (nloc == 0) {
     if (t == 0) a.chunk_count[static_cast<size_t>(seg) * s.nchunks + c] = 0;
@@ -327,24 +365,25 @@ __global__ void rescue_kernel(ScreenArgs a) {
   }
 }
 
-template <int D, int G>
+template <int D, int G, int FMT>
 cudaError_t launch_screen_typed(const ScreenArgs& a, cudaStream_t st) {
-  const size_t smem = screen_smem_bytes<D>(a.s.chunk);
-  auto kern = screen_kernel<D, G>;
+  constexpr int ESZ = FMT == ETA_META_FP8 ? 1 : 2;
+  const size_t smem = screen_smem_bytes<D, ESZ>(a.s.chunk);
+  auto kern = screen_kernel<D, G, FMT>;
   static SmemLimit lim;
-  return launch_with_smem(reinterpret_cast<const void*>(kern), screen_smem_bytes<D>(2 * kRound), lim, [&] {
+  return launch_with_smem(reinterpret_cast<const void*>(kern), screen_smem_bytes<D, ESZ>(2 * kRound), lim, [&] {
     kern<<<dim3(a.s.nchunks, a.s.Hkv, a.s.B), kThreads, smem, st>>>(a);
     return cudaGetLastError();
   });
 }
 
-template <int D>
+template <int D, int FMT>
 cudaError_t launch_screen_d(const ScreenArgs& a, cudaStream_t st) {
   switch (a.s.G) {
-    case 1: return launch_screen_typed<D, 1>(a, st);
-    case 2: return launch_screen_typed<D, 2>(a, st);
-    case 4: return launch_screen_typed<D, 4>(a, st);
-    case 8: return launch_screen_typed<D, 8>(a, st);
+    case 1: return launch_screen_typed<D, 1, FMT>(a, st);
+    case 2: return launch_screen_typed<D, 2, FMT>(a, st);
+    case 4: return launch_screen_typed<D, 4, FMT>(a, st);
+    case 8: return launch_screen_typed<D, 8, FMT>(a, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -353,7 +392,10 @@ cudaError_t launch_screen_d(const ScreenArgs& a, cudaStream_t st) {
 
 cudaError_t launch_screen(const ScreenArgs& a, cudaStream_t st) {
   if (a.s.chunk > kMaxChunk) return cudaErrorInvalidValue;
-  return a.s.d == 64 ? launch_screen_d<64>(a, st) : launch_screen_d<128>(a, st);
+  // with the screen off no metadata is read: the fp16 instance serves
+  if (a.screen_enabled && a.meta_fmt == ETA_META_FP8)
+    return a.s.d == 64 ? launch_screen_d<64, ETA_META_FP8>(a, st) : launch_screen_d<128, ETA_META_FP8>(a, st);
+  return a.s.d == 64 ? launch_screen_d<64, ETA_META_FP16>(a, st) : launch_screen_d<128, ETA_META_FP16>(a, st);
 }
 
 cudaError_t launch_rescue(const ScreenArgs& a, cudaStream_t st) {
