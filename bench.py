@@ -567,6 +567,53 @@ def run_prefill(args):
     }
 
 
+def run_calibrate(args):
+    """Offline calibration histogram (eta_calibration_histogram) over a batch of
+    calibration sequences: causal logits binned per second, and the time of one
+    full pass; the constants solved from it on the host."""
+    import learned_threshold_sparse_b200 as eta
+
+    B, Hq, Hkv, T = (int(x) for x in args.calib_shape.split(","))
+    d = 128
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    case = workloads.prefill_case(args.seed, batch=B, n_q_heads=Hq, n_kv_heads=Hkv, seq_len=T, head_dim=d)
+    q, k = case.q.to(dev), case.k.to(dev)
+    hist = torch.zeros((Hq, 4096 + 2), dtype=torch.float64, device=dev)
+    for _ in range(args.warmup):
+        eta.calibration_histogram(q, k, T, scale=case.scale, hist=hist)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for _ in range(args.steps):
+        hist.zero_()
+        e0.record()
+        eta.calibration_histogram(q, k, T, scale=case.scale, hist=hist)
+        e1.record()
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    c = eta.calibrate_constants(hist, -8.0, 8.0, 0.38)
+    t = statistics.mean(ms)
+    pairs = B * Hq * T * (T + 1) / 2
+    return {
+        "metric": "ETA offline calibration: causal logits binned per second",
+        "value": round(pairs / (t * 1e-3) / 1e9, 3),
+        "unit": "Glogits/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(t, 4),
+        "higher_is_better": True,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": f"calibration: {B} sequences, {Hq} query / {Hkv} KV heads, seq {T}, d {d}, bf16, "
+                               "4096 bins over [-8, 8)",
+                   "tensor_flops_equivalent_per_step": 2.0 * d * pairs,
+                   "constants_at_density_0.38": [round(float(x), 4) for x in c[:4]]},
+        "gpu_launches": args.steps,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -581,11 +628,15 @@ def main():
     ap.add_argument("--meta", default="fp16", choices=["fp16", "fp8"], help="block metadata format")
     ap.add_argument("--prefill", action="store_true", help="time the causal forward pass instead of the decode step")
     ap.add_argument("--prefill-shape", default="1,32,8,8192", help="batch,n_q_heads,n_kv_heads,seq_len")
+    ap.add_argument("--calibrate", action="store_true", help="time the offline calibration histogram")
+    ap.add_argument("--calib-shape", default="16,16,4,4096", help="sequences,n_q_heads,n_kv_heads,seq_len")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.prefill:
         line = run_prefill(args)
+    elif args.calibrate:
+        line = run_calibrate(args)
     else:
         line = run_reference(args) if args.impl == "reference" else run_eta(args)
     if line is not None:

@@ -310,6 +310,51 @@ typedef struct {
 eta_status eta_prefill(const eta_prefill_params* p, void* stream);
 
 /*
+ * ------------------------------------------------------------------------
+ * Offline per-head threshold calibration (section 4.7; Appendix D.2):
+ * frozen constants that replace the threshold projection for a stationary
+ * deployment.  Every causal logit S_tj = scale q_t . k_j (j <= t) of a
+ * query head enters a histogram with weight 1/(t + 1), so each query row
+ * weighs 1; the constant of a head is the logit at which the weighted
+ * fraction of logits at or above it equals the head's target density
+ * (a token-level density; the block screen admits somewhat more).  The value
+ * returned is the effective threshold tau~: use c_tau = value + offset_a.
+ * ------------------------------------------------------------------------
+ */
+typedef struct {
+  int batch, n_q_heads, n_kv_heads, head_dim;
+  int seq_len;                       /* calibration tokens per sequence      */
+  int kv_stride;                     /* rows per KV head in k, >= seq_len    */
+  eta_dtype dtype;                   /* ETA_F32 or ETA_BF16                  */
+  const void* q;                     /* [batch, n_q_heads, seq_len, d]: the
+                                        query of every position              */
+  const void* k;                     /* [batch, n_kv_heads, kv_stride, d]    */
+  float scale;                       /* > 0                                   */
+  float lo, hi;                      /* histogram range of the logits, lo<hi */
+  int nbins;                         /* 1 <= nbins <= 8192                    */
+  double* hist;                      /* device [n_q_heads, nbins + 2],
+                                        8-aligned: slot 0 counts logits < lo,
+                                        slots 1..nbins the equal bins,
+                                        slot nbins+1 logits >= hi.  The call
+                                        ADDS to it (zero it once, then call
+                                        per calibration batch)              */
+} eta_calib_params;
+
+/* eta_calibration_histogram - accumulate the weighted logit histogram of
+ * every query head over the batch (one launch, stream-ordered).
+ * Errors: ETA_ERR_INVALID_ARG, ETA_ERR_UNSUPPORTED (head_dim not 64/128),
+ * ETA_ERR_CUDA. */
+eta_status eta_calibration_histogram(const eta_calib_params* p, void* stream);
+
+/* eta_calibrate_constants - host-only solver: for each head h, the logit at
+ * which the weighted fraction at or above it reaches target[h] (searching
+ * the bins from the top, linear inside the crossing bin; error at most one
+ * bin width).  hist, target and c are HOST arrays ([n_heads][nbins + 2],
+ * [n_heads], [n_heads]).  Errors: ETA_ERR_INVALID_ARG. */
+eta_status eta_calibrate_constants(const double* hist, int n_heads, int nbins, float lo, float hi,
+                                   const float* target, float* c);
+
+/*
  * eta_read_device_status - synchronise `stream`, read and clear the device
  * status word kept in `workspace`.  Returns ETA_OK, ETA_ERR_DEVICE_TIMEOUT
  * or ETA_ERR_DEVICE_RANGE (or ETA_ERR_CUDA if the copy fails).

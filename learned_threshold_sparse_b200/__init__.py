@@ -10,6 +10,8 @@ device memory and the stream.  The functions mirror the C entry points:
     eta_decode(...)                 one decode step (screen, attend, merge)
     eta_read_device_status(...)     read and clear the device status word
     eta_prefill(...) / prefill(...) causal forward pass over whole sequences
+    calibration_histogram(...), calibrate_constants(...)
+                                    offline per-head threshold calibration
     eta_status_string(code), eta_build_info()
 
 There is no fallback: if libeta.so is missing or fails to load, importing
@@ -96,6 +98,15 @@ class eta_prefill_params(ctypes.Structure):
 PREFILL_WORKSPACE_BYTES = 256  # ETA_PREFILL_WORKSPACE_BYTES in include/eta.h
 
 
+class eta_calib_params(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int), ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int), ("seq_len", ctypes.c_int), ("kv_stride", ctypes.c_int),
+        ("dtype", ctypes.c_int), ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("scale", ctypes.c_float),
+        ("lo", ctypes.c_float), ("hi", ctypes.c_float), ("nbins", ctypes.c_int), ("hist", ctypes.c_void_p),
+    ]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is not built; run learned_threshold_sparse_b200.build.build()")
@@ -117,6 +128,11 @@ def _load():
     lib.eta_read_device_status.restype = ctypes.c_int
     lib.eta_prefill.argtypes = [P(eta_prefill_params), ctypes.c_void_p]
     lib.eta_prefill.restype = ctypes.c_int
+    lib.eta_calibration_histogram.argtypes = [P(eta_calib_params), ctypes.c_void_p]
+    lib.eta_calibration_histogram.restype = ctypes.c_int
+    lib.eta_calibrate_constants.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_float,
+                                            ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p]
+    lib.eta_calibrate_constants.restype = ctypes.c_int
     lib.eta_status_string.argtypes = [ctypes.c_int]
     lib.eta_status_string.restype = ctypes.c_char_p
     lib.eta_build_info.argtypes = []
@@ -127,7 +143,8 @@ def _load():
 _lib = _load()
 
 SYMBOLS = ("eta_block_summary_update", "eta_append_kv", "eta_decode_workspace_size", "eta_decode", "eta_decode_noalloc",
-           "eta_read_device_status", "eta_prefill", "eta_status_string", "eta_build_info")
+           "eta_read_device_status", "eta_prefill", "eta_calibration_histogram", "eta_calibrate_constants",
+           "eta_status_string", "eta_build_info")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
 
@@ -384,3 +401,60 @@ def prefill(q, k, v, seq_len: int, tau_mode: str, *, w_tau=None, b_tau=None, c_t
                             beta=beta, offset_a=offset_a, out=out, lse=lse, gate_sum=gate, workspace=ws)
     eta_prefill(p, stream)
     return {"out": out, "lse": lse, "gate_sum": gate, "workspace": ws}
+
+
+# ------------------------------------------------------------ calibration
+
+def calibration_histogram(q: torch.Tensor, k: torch.Tensor, seq_len: int, *, scale: Optional[float] = None,
+                          lo: float = -8.0, hi: float = 8.0, nbins: int = 4096,
+                          hist: Optional[torch.Tensor] = None,
+                          stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Add the 1/(t+1)-weighted causal logit histogram of every query head of
+    q [B, Hq, T, d] against k [B, Hkv, kv_stride, d] to ``hist`` (fp64
+    [Hq, nbins + 2], allocated zeroed when not given) and return it."""
+    B, Hq, T, d = q.shape
+    if hist is None:
+        hist = torch.zeros((Hq, nbins + 2), dtype=torch.float64, device=q.device)
+    p = eta_calib_params()
+    p.batch, p.n_q_heads, p.n_kv_heads, p.head_dim = B, Hq, k.shape[1], d
+    p.seq_len, p.kv_stride = int(seq_len), k.shape[2]
+    p.dtype = _kv_dtype(q)
+    p.q, p.k = q.data_ptr(), k.data_ptr()
+    p.scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    p.lo, p.hi, p.nbins = float(lo), float(hi), int(nbins)
+    p.hist = hist.data_ptr()
+    rc = _lib.eta_calibration_histogram(ctypes.byref(p), _stream_handle(stream))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_calibration_histogram")
+    return hist
+
+
+def calibrate_constants(hist: torch.Tensor, lo: float, hi: float, target) -> "np.ndarray":
+    """Per-head effective thresholds tau~ reaching the target densities (host
+    solver over a histogram from calibration_histogram)."""
+    import numpy as np
+
+    h = np.ascontiguousarray(hist.detach().cpu().numpy(), dtype=np.float64)
+    n, nb2 = h.shape
+    tgt = np.ascontiguousarray(np.broadcast_to(np.asarray(target, dtype=np.float32), (n,)))
+    c = np.zeros(n, np.float32)
+    rc = _lib.eta_calibrate_constants(h.ctypes.data, n, nb2 - 2, float(lo), float(hi), tgt.ctypes.data,
+                                      c.ctypes.data)
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_calibrate_constants")
+    return c
+
+
+def eta_calibration_histogram(params: eta_calib_params, stream: Optional[torch.cuda.Stream] = None) -> None:
+    rc = _lib.eta_calibration_histogram(ctypes.byref(params), _stream_handle(stream))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_calibration_histogram")
+
+
+def eta_calibrate_constants(hist_host, n_heads: int, nbins: int, lo: float, hi: float, target_host, c_host) -> None:
+    """Host arrays (numpy): hist [n_heads, nbins + 2] float64, target and c
+    [n_heads] float32 (c written)."""
+    rc = _lib.eta_calibrate_constants(hist_host.ctypes.data, int(n_heads), int(nbins), float(lo), float(hi),
+                                      target_host.ctypes.data, c_host.ctypes.data)
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_calibrate_constants")

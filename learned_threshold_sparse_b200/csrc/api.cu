@@ -205,7 +205,7 @@ const char* eta_status_string(eta_status s) {
 
 const char* eta_build_info(void) {
   return "eta decode library: sm_100a; kernels: block_summary, screen, rescue, attend_simt, attend_tc, merge, "
-         "export, prefill_tc";
+         "export, prefill_tc, calib_hist";
 }
 
 eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summary_desc* summary,
@@ -414,6 +414,66 @@ eta_status eta_prefill(const eta_prefill_params* p, void* stream) {
   a.beta = p->beta;
   a.offset_a = p->offset_a;
   return launch_prefill_tc(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+eta_status eta_calibration_histogram(const eta_calib_params* p, void* stream) {
+  if (!p) return ETA_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->n_q_heads < 1 || p->n_kv_heads < 1 || p->seq_len < 1 || p->kv_stride < p->seq_len)
+    return ETA_ERR_INVALID_ARG;
+  if (p->n_q_heads % p->n_kv_heads != 0) return ETA_ERR_INVALID_ARG;
+  if (p->dtype != ETA_BF16 && p->dtype != ETA_F32) return ETA_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128) return ETA_ERR_UNSUPPORTED;
+  if (p->batch > 65535 || p->n_q_heads > 65535) return ETA_ERR_UNSUPPORTED;
+  if (!p->q || !p->k || !p->hist || !aligned(p->q, 4) || !aligned(p->k, 4) || !aligned(p->hist, 8))
+    return ETA_ERR_INVALID_ARG;
+  if (!(p->scale > 0.f) || !isfinite(p->scale) || !isfinite(p->lo) || !isfinite(p->hi) || !(p->hi > p->lo))
+    return ETA_ERR_INVALID_ARG;
+  if (p->nbins < 1 || p->nbins > 8192) return ETA_ERR_INVALID_ARG;
+  CalibArgs a;
+  a.q = p->q;
+  a.k = p->k;
+  a.hist = p->hist;
+  a.B = p->batch;
+  a.Hq = p->n_q_heads;
+  a.Hkv = p->n_kv_heads;
+  a.G = p->n_q_heads / p->n_kv_heads;
+  a.T = p->seq_len;
+  a.kv_stride = p->kv_stride;
+  a.d = p->head_dim;
+  a.elt = p->dtype == ETA_F32 ? 4 : 2;
+  a.nbins = p->nbins;
+  a.scale = p->scale;
+  a.lo = p->lo;
+  a.inv_width = static_cast<float>(p->nbins / (static_cast<double>(p->hi) - p->lo));
+  return launch_calib(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
+}
+
+eta_status eta_calibrate_constants(const double* hist, int n_heads, int nbins, float lo, float hi,
+                                   const float* target, float* c) {
+  if (!hist || !target || !c || n_heads < 1 || nbins < 1 || !(hi > lo)) return ETA_ERR_INVALID_ARG;
+  const double width = (static_cast<double>(hi) - lo) / nbins;
+  for (int h = 0; h < n_heads; ++h) {
+    if (!(target[h] >= 0.f && target[h] <= 1.f)) return ETA_ERR_INVALID_ARG;
+    const double* x = hist + static_cast<size_t>(h) * (nbins + 2);
+    double total = 0.0;
+    for (int b = 0; b < nbins + 2; ++b) total += x[b];
+    const double need = target[h] * total;
+    double acc = x[nbins + 1];  // logits >= hi
+    double val = lo;
+    if (acc >= need) {
+      val = hi;
+    } else {
+      for (int b = nbins; b >= 1; --b) {  // slot b: [lo + (b - 1) width, lo + b width)
+        if (acc + x[b] >= need) {
+          val = lo + b * width - (need - acc) / x[b] * width;
+          break;
+        }
+        acc += x[b];
+      }
+    }
+    c[h] = static_cast<float>(val);
+  }
+  return ETA_OK;
 }
 
 eta_status eta_read_device_status(void* workspace, void* stream) {

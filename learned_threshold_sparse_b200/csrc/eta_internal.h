@@ -123,6 +123,15 @@ struct PrefillArgs {
   float scale, beta, offset_a;
 };
 
+// Arguments of the calibration histogram kernel.
+struct CalibArgs {
+  const void* q;           // [B, Hq, T, d] kv dtype
+  const void* k;           // [B, Hkv, kv_stride, d]
+  double* hist;            // [Hq, nbins + 2] (underflow, nbins bins, overflow)
+  int B, Hq, Hkv, G, T, kv_stride, d, elt, nbins;
+  float scale, lo, inv_width;
+};
+
 struct SummaryArgs {
   const void* k;
   const int* seq_lens;
@@ -192,5 +201,7 @@ bool attend_tc_supported(const Shape& s);
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
 cudaError_t launch_export(const ExportArgs& a, cudaStream_t st);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st);
+cudaError_t launch_calib(const CalibArgs& a, cudaStream_t st);
+size_t calib_smem(int d, int nbins);
 
 }  // namespace eta

@@ -118,6 +118,7 @@ def test_struct_layout_matches_header(tmp_path):
         "eta_summary_desc": eta.eta_summary_desc,
         "eta_decode_params": eta.eta_decode_params,
         "eta_prefill_params": eta.eta_prefill_params,
+        "eta_calib_params": eta.eta_calib_params,
     }
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "eta.h"', "int main(void) {"]
     for sname, cls in fields.items():
@@ -187,3 +188,33 @@ def test_prefill_size_limits():
     p.tau_mode = eta.ETA_TAU_CALIBRATED
     p.c_tau = None
     assert eta.library().eta_prefill(ctypes.byref(p), None) == eta.ETA_ERR_INVALID_ARG
+
+
+def test_calibration_host_solver_matches_the_oracle_solver():
+    # host-only entry point: no device involved
+    import numpy as np
+    from oracle import eta_calib_oracle as co
+
+    rng = np.random.default_rng(9)
+    S = rng.standard_normal(20000) * 1.5
+    w = rng.uniform(0.05, 1.0, 20000)
+    lo, hi, nb = -6.0, 6.0, 600
+    hist = np.stack([co.histogram(S, w, lo, hi, nb), co.histogram(S * 0.5, w, lo, hi, nb)])
+    targets = np.array([0.38, 0.1], np.float32)
+    c = np.zeros(2, np.float32)
+    rc = eta.library().eta_calibrate_constants(hist.ctypes.data, 2, nb, lo, hi, targets.ctypes.data, c.ctypes.data)
+    assert rc == eta.ETA_OK
+    for h in range(2):
+        ref = co.histogram_constant(hist[h], lo, hi, float(targets[h]))
+        assert abs(float(c[h]) - ref) <= 1e-5 * max(1.0, abs(ref))
+
+
+def test_calibration_validation():
+    fake = 1 << 20
+    p = eta.eta_calib_params(1, 4, 2, 128, 100, 100, eta.ETA_BF16, fake, fake, 0.088, -8.0, 8.0, 512, fake)
+    lib = eta.library()
+    for field, value, code in [("nbins", 0, 1), ("hi", -9.0, 1), ("head_dim", 96, 2), ("hist", fake + 4, 1),
+                               ("kv_stride", 50, 1), ("n_kv_heads", 3, 1)]:
+        q = eta.eta_calib_params.from_buffer_copy(p)
+        setattr(q, field, value)
+        assert lib.eta_calibration_histogram(ctypes.byref(q), None) == code, field
