@@ -72,7 +72,17 @@ typedef enum {
                             block_size in {64, 128}, group size >= 2)          */
 } eta_attend_impl;
 
-/* The KV cache of one attention layer. */
+/* The KV cache of one attention layer.  Two layouts:
+ *   contiguous (block_table == NULL): k_cache, v_cache are
+ *       [batch, n_kv_heads, max_ctx, head_dim];
+ *   paged (block_table != NULL): k_cache, v_cache are pools of pages
+ *       [num_pages, n_kv_heads, block_size, head_dim], one page per KV block,
+ *       and block_table [batch, nb_max] (int32, device) gives the page of
+ *       logical block j of sequence i (only blocks below ceil(seq_len / b)
+ *       are read; a page id outside [0, num_pages) is replaced by page 0 and
+ *       reported as ETA_ERR_DEVICE_RANGE).  Block metadata stays indexed by
+ *       logical block.
+ * A zero-initialised tail (block_table, num_pages) is the contiguous layout. */
 typedef struct {
   int batch;          /* >= 1                                                */
   int n_q_heads;      /* multiple of n_kv_heads                              */
@@ -84,6 +94,8 @@ typedef struct {
   const void* k_cache;
   const void* v_cache;
   const int* seq_lens; /* [batch] device, 0 <= seq_lens[i] <= max_ctx         */
+  const int* block_table; /* paged layout: [batch, nb_max] device, else NULL */
+  int num_pages;          /* paged layout: pages in k_cache / v_cache, >= 1  */
 } eta_cache_desc;
 
 /* Storage of the centroid and spread in eta_summary_desc. */

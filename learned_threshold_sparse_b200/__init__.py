@@ -57,7 +57,7 @@ class eta_cache_desc(ctypes.Structure):
         ("batch", ctypes.c_int), ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
         ("head_dim", ctypes.c_int), ("block_size", ctypes.c_int), ("max_ctx", ctypes.c_int),
         ("kv_dtype", ctypes.c_int), ("k_cache", ctypes.c_void_p), ("v_cache", ctypes.c_void_p),
-        ("seq_lens", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p), ("block_table", ctypes.c_void_p), ("num_pages", ctypes.c_int),
     ]
 
 
@@ -182,10 +182,23 @@ def _kv_dtype(t: torch.Tensor) -> int:
 
 
 def cache_desc(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, n_q_heads: int,
-               block_size: int) -> eta_cache_desc:
-    B, Hkv, Tmax, d = k.shape
-    return eta_cache_desc(B, n_q_heads, Hkv, d, block_size, Tmax, _kv_dtype(k), k.data_ptr(), v.data_ptr(),
-                          seq_lens.data_ptr())
+               block_size: int, block_table: Optional[torch.Tensor] = None) -> eta_cache_desc:
+    """Contiguous cache: k, v [B, Hkv, max_ctx, d].  Paged cache: k, v are page
+    pools [num_pages, Hkv, block_size, d] and block_table [B, nb_max] int32
+    gives each logical block's page (max_ctx = nb_max * block_size)."""
+    if block_table is None:
+        B, Hkv, Tmax, d = k.shape
+        return eta_cache_desc(B, n_q_heads, Hkv, d, block_size, Tmax, _kv_dtype(k), k.data_ptr(), v.data_ptr(),
+                              seq_lens.data_ptr())
+    P, Hkv, b, d = k.shape
+    if b != block_size:
+        raise ValueError("page rows must equal block_size")
+    B, nbmax = block_table.shape
+    c = eta_cache_desc(B, n_q_heads, Hkv, d, block_size, nbmax * block_size, _kv_dtype(k), k.data_ptr(),
+                       v.data_ptr(), seq_lens.data_ptr())
+    c.block_table = block_table.data_ptr()
+    c.num_pages = P
+    return c
 
 
 def alloc_summary(batch: int, n_kv_heads: int, max_ctx: int, head_dim: int, block_size: int,
@@ -222,10 +235,11 @@ def summary_desc(summary: Dict[str, torch.Tensor]) -> eta_summary_desc:
 def eta_block_summary_update(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor,
                              summary: Dict[str, torch.Tensor], block_size: int,
                              first_token: torch.Tensor, max_blocks: int, n_q_heads: Optional[int] = None,
-                             stream: Optional[torch.cuda.Stream] = None) -> None:
+                             stream: Optional[torch.cuda.Stream] = None,
+                             block_table: Optional[torch.Tensor] = None) -> None:
     """Recompute the metadata of the blocks at or after first_token[i] (at most
     max_blocks per sequence)."""
-    cache = cache_desc(k, v, seq_lens, n_q_heads or k.shape[1], block_size)
+    cache = cache_desc(k, v, seq_lens, n_q_heads or k.shape[1], block_size, block_table)
     summ = summary_desc(summary)
     rc = _lib.eta_block_summary_update(ctypes.byref(cache), ctypes.byref(summ),
                                        ctypes.c_void_p(first_token.data_ptr()), int(max_blocks),
@@ -236,10 +250,11 @@ def eta_block_summary_update(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.T
 
 def eta_append_kv(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, summary: Dict[str, torch.Tensor],
                   block_size: int, k_new: torch.Tensor, v_new: torch.Tensor, pos: torch.Tensor,
-                  n_q_heads: Optional[int] = None, stream: Optional[torch.cuda.Stream] = None) -> None:
+                  n_q_heads: Optional[int] = None, stream: Optional[torch.cuda.Stream] = None,
+                  block_table: Optional[torch.Tensor] = None) -> None:
     """Write k_new / v_new [B, Hkv, d] at row pos[i] of each sequence and refresh
     the summary of the block holding it (seq_lens must already count it)."""
-    cache = cache_desc(k, v, seq_lens, n_q_heads or k.shape[1], block_size)
+    cache = cache_desc(k, v, seq_lens, n_q_heads or k.shape[1], block_size, block_table)
     summ = summary_desc(summary)
     rc = _lib.eta_append_kv(ctypes.byref(cache), ctypes.byref(summ), ctypes.c_void_p(k_new.data_ptr()),
                             ctypes.c_void_p(v_new.data_ptr()), ctypes.c_void_p(pos.data_ptr()), _stream_handle(stream))
@@ -251,10 +266,10 @@ def make_params(q, k, v, seq_lens, summary, block_size, tau_mode, w_tau=None, b_
                 c_tau=None, scale=None, beta=5.0, offset_a=0.0, z=2.0, n_local_blocks=2,
                 screen_enabled=True, attend_impl=ETA_ATTEND_AUTO, out=None, lse=None,
                 admitted_count=None, union_count=None, union_list=None, union_mask=None,
-                workspace=None, events=None) -> eta_decode_params:
+                workspace=None, events=None, block_table=None) -> eta_decode_params:
     B, Hq, d = q.shape
     p = eta_decode_params()
-    p.cache = cache_desc(k, v, seq_lens, Hq, block_size)
+    p.cache = cache_desc(k, v, seq_lens, Hq, block_size, block_table)
     if summary is not None:
         p.summary = summary_desc(summary)
     p.q = q.data_ptr()
@@ -321,13 +336,13 @@ def eta_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.
 def decode(q, k, v, seq_lens, summary, block_size, tau_mode, *, w_tau=None, b_tau=None, c_tau=None,
            scale=None, beta=5.0, offset_a=0.0, z=2.0, n_local_blocks=2, screen_enabled=True,
            attend_impl=ETA_ATTEND_AUTO, selection=False, workspace=None, out=None, lse=None,
-           events=None, stream=None) -> Dict[str, torch.Tensor]:
+           events=None, stream=None, block_table=None) -> Dict[str, torch.Tensor]:
     """Allocate outputs (and the workspace if not given) with torch and run one
     decode step.  Returns {"out", "lse", "workspace"} plus, with selection=True,
     {"admitted_count", "union_count", "union_list", "union_mask"}."""
     B, Hq, d = q.shape
-    Hkv, Tmax = k.shape[1], k.shape[2]
-    nb = (Tmax + block_size - 1) // block_size
+    Hkv = k.shape[1]
+    nb = block_table.shape[1] if block_table is not None else (k.shape[2] + block_size - 1) // block_size
     dev = q.device
     res = {"out": out if out is not None else torch.empty_like(q),
            "lse": lse if lse is not None else torch.empty((B, Hq), dtype=torch.float32, device=dev)}
@@ -340,7 +355,7 @@ def decode(q, k, v, seq_lens, summary, block_size, tau_mode, *, w_tau=None, b_ta
               n_local_blocks=n_local_blocks, screen_enabled=screen_enabled, attend_impl=attend_impl,
               out=res["out"], lse=res["lse"], admitted_count=res.get("admitted_count"),
               union_count=res.get("union_count"), union_list=res.get("union_list"),
-              union_mask=res.get("union_mask"), events=events)
+              union_mask=res.get("union_mask"), events=events, block_table=block_table)
     params = make_params(q, k, v, seq_lens, summary, block_size, tau_mode, **kw)
     if workspace is None:
         workspace = alloc_workspace(eta_decode_workspace_size(params), dev)

@@ -33,6 +33,11 @@ eta_status check_cache(const eta_cache_desc* c) {
   if (!c->k_cache || !c->v_cache || !c->seq_lens) return ETA_ERR_INVALID_ARG;
   if (!aligned(c->k_cache, 16) || !aligned(c->v_cache, 16) || !aligned(c->seq_lens, 4))
     return ETA_ERR_INVALID_ARG;
+  if (c->block_table) {
+    if (!aligned(c->block_table, 4) || c->num_pages < 1) return ETA_ERR_INVALID_ARG;
+    if (static_cast<long long>(c->num_pages) * c->n_kv_heads * c->block_size >= (1ll << 31))
+      return ETA_ERR_UNSUPPORTED;
+  }
   return ETA_OK;
 }
 
@@ -67,6 +72,7 @@ eta_status make_shape(const eta_decode_params* p, Shape* out) {
   s.b = c.block_size;
   s.max_ctx = c.max_ctx;
   s.nbmax = (c.max_ctx + c.block_size - 1) / c.block_size;
+  s.num_pages = c.block_table ? c.num_pages : 0;
   s.elt = c.kv_dtype == ETA_F32 ? 4 : 2;
   s.nseg = s.B * s.Hkv;
   // Screen CTAs cover `chunk` blocks: about two screen CTAs per SM (one
@@ -219,6 +225,8 @@ eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summa
   if (max_blocks < 1 || max_blocks > nbmax) return ETA_ERR_INVALID_ARG;
   SummaryArgs a;
   a.k = cache->k_cache;
+  a.block_table = cache->block_table;
+  a.num_pages = cache->num_pages;
   a.seq_lens = cache->seq_lens;
   a.first_token = first_token;
   set_summary(a, summary);
@@ -244,6 +252,8 @@ eta_status eta_append_kv(const eta_cache_desc* cache, const eta_summary_desc* su
     return ETA_ERR_INVALID_ARG;
   SummaryArgs a;
   a.k = cache->k_cache;
+  a.block_table = cache->block_table;
+  a.num_pages = cache->num_pages;
   a.seq_lens = cache->seq_lens;
   a.first_token = nullptr;
   set_summary(a, summary);
@@ -323,6 +333,7 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
 
   AttendArgs aa;
   aa.k = p->cache.k_cache;
+  aa.block_table = p->cache.block_table;
   aa.v = p->cache.v_cache;
   aa.q = p->q;
   aa.seq_lens = p->cache.seq_lens;

@@ -15,6 +15,7 @@ namespace dev {
 
 struct UnitInfo {
   int seg, blk, mask, nrows;
+  long long row;  // first K/V row of the block in the cache's [rows, d] view
 };
 
 // Exclusive prefix of the chunk counts into prefix[0..n] (prefix[n] = total),
@@ -117,6 +118,7 @@ __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefi
   int idx = u0 - prefix[x];
   int remaining = nunits;
   int cur_seg = -1, T = 0;
+  const KvLayout lay{a.block_table, s.Hkv, s.b, s.max_ctx, s.nbmax, s.num_pages};
   while (remaining > 0) {
     if (x >= nprefix) return false;
     const int cnt = prefix[x + 1] - prefix[x];
@@ -137,13 +139,18 @@ __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefi
     for (int j0 = 0; j0 < take; j0 += 32) {
       const int nn = min(32, take - j0);
       const int e = lane < nn ? list[j0 + lane] : 0;
+      // the rows of the 32 listed blocks (one page-table read per lane)
+      bool bad = false;
+      const long long rw = lane < nn ? lay.row(seg, e & kMaxBlocksPerSeq, &bad) : 0;
+      if (bad) atomicOr(a.status, kStatusRange);
       for (int jj = 0; jj < nn; ++jj) {
         const int ent = __shfl_sync(0xffffffffu, e, jj);
+        const long long er = __shfl_sync(0xffffffffu, rw, jj);
         int ok = 1;
         if (lane == 0) {
           const int blk = ent & kMaxBlocksPerSeq;
           const UnitInfo in{seg, blk, static_cast<int>(static_cast<unsigned>(ent) >> kEntryBlockBits),
-                            min(s.b, T - blk * s.b)};
+                            min(s.b, T - blk * s.b), er};
           ok = issue(in) ? 1 : 0;
         }
         if (__shfl_sync(0xffffffffu, ok, 0) == 0) return false;

@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
       info[stage] = in;
       const uint32_t bytes = static_cast<uint32_t>(in.nrows) * D * ELT;
       dev::mbar_arrive_expect_tx(&full[stage], 2u * bytes);
-      const size_t off = (static_cast<size_t>(in.seg) * s.max_ctx + static_cast<size_t>(in.blk) * s.b) * D * ELT;
+      const size_t off = static_cast<size_t>(in.row) * D * ELT;
       uint8_t* dst = kv + static_cast<size_t>(stage) * 2 * tile_bytes;
       dev::bulk_g2s(dst, static_cast<const uint8_t*>(a.k) + off, bytes, &full[stage]);
       dev::bulk_g2s(dst + tile_bytes, static_cast<const uint8_t*>(a.v) + off, bytes, &full[stage]);

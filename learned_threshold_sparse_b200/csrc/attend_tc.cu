@@ -218,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       TileInfo pend{-1, 0, 0, 0, 0};
-      int pblk[2] = {0, 0};
+      int prow[2] = {0, 0};
       int npend = 0;
       auto emit = [&]() -> bool {
         if (!wait_or_abort(&B.kv_empty[stage], phase ^ 1u, a.status, abort_flag)) return false;
@@ -226,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t st = base_u32 + static_cast<uint32_t>(L.stages + stage * TL::STAGE);
         dev::mbar_arrive_expect_tx(&B.kv_full[stage], static_cast<uint32_t>(npend * 4 * BR * 128 + 4096));
         for (int i = 0; i < npend; ++i) {
-          const int krow = pend.seg * s.max_ctx + pblk[i] * BR;
+          const int krow = prow[i];
           const uint32_t ro = static_cast<uint32_t>(i * BR * 128);
           tma_load_2d(st + TL::K0 + ro, &tk, 0, krow, &B.kv_full[stage]);
           tma_load_2d(st + TL::K1 + ro, &tk, 64, krow, &B.kv_full[stage]);
@@ -245,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 [&](const UnitInfo& in) -> bool {
         if (npend > 0 && in.seg != pend.seg && !emit()) return false;
         if (npend == 0) pend = TileInfo{in.seg, 0, 0, 0, 0};
-        pblk[npend] = in.blk;
+        prow[npend] = static_cast<int>(in.row);
         if (npend == 0) { pend.mask0 = in.mask; pend.nrows0 = in.nrows; }
         else { pend.mask1 = in.mask; pend.nrows1 = in.nrows; }
         ++npend;
@@ -528,8 +528,10 @@ cudaError_t launch_g(const CUtensorMap& tk, const CUtensorMap& tv, const CUtenso
 }  // namespace
 
 bool attend_tc_supported(const Shape& s) {
+  const long long rows = s.num_pages ? static_cast<long long>(s.num_pages) * s.Hkv * s.b
+                                     : static_cast<long long>(s.nseg) * s.max_ctx;
   return s.elt == 2 && s.d == 128 && (s.b == 64 || s.b == 128) && (s.G == 2 || s.G == 4 || s.G == 8) &&
-         static_cast<long long>(s.nseg) * s.max_ctx < (1ll << 31) && static_cast<long long>(s.B) * s.Hq < (1ll << 31);
+         rows < (1ll << 31) && static_cast<long long>(s.B) * s.Hq < (1ll << 31);
 }
 
 size_t attend_tc_smem(const Shape& s) {
@@ -542,7 +544,8 @@ cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st) {
   if (stages == 0) return cudaErrorInvalidConfiguration;
   const size_t smem = tc_layout(stages, a.s.nseg * a.s.nchunks, smem_seqs(a.s.B)).total;
   CUtensorMap tk, tv, tq;
-  const uint64_t rows = static_cast<uint64_t>(a.s.nseg) * a.s.max_ctx;
+  const uint64_t rows = a.s.num_pages ? static_cast<uint64_t>(a.s.num_pages) * a.s.Hkv * a.s.b
+                                      : static_cast<uint64_t>(a.s.nseg) * a.s.max_ctx;
   if (!make_map(&tk, a.k, rows, a.s.b) || !make_map(&tv, a.v, rows, a.s.b) ||
       !make_map(&tq, a.q, static_cast<uint64_t>(a.s.B) * a.s.Hq, NQ))
     return cudaErrorInvalidValue;

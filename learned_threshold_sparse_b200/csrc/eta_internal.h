@@ -36,6 +36,27 @@ struct Shape {
   int attend_ctas;   // persistent attention CTAs
   int attend_kind;   // ETA_ATTEND_SIMT or ETA_ATTEND_TC
   int rescue;        // 1 when n_local_blocks < 0 (top-1 rescue may fire)
+  int num_pages;     // paged cache: pages in the pools (0: contiguous cache)
+};
+
+// Where the K/V rows of logical block blk of segment seg (sequence
+// seg / Hkv, KV head seg % Hkv) start, as a row index of the [rows, d] view
+// of the cache: contiguous  seg max_ctx + blk b;  paged
+// (page Hkv + g) b with page = table[i nb_max + blk].  An out-of-range page
+// id reads page 0 and sets *bad.
+struct KvLayout {
+  const int* table;  // null: contiguous
+  int Hkv, b, max_ctx, nbmax, num_pages;
+  __host__ __device__ long long row(int seg, int blk, bool* bad) const {
+    if (!table) return static_cast<long long>(seg) * max_ctx + static_cast<long long>(blk) * b;
+    const int i = seg / Hkv, g = seg - i * Hkv;
+    int page = table[static_cast<size_t>(i) * nbmax + blk];
+    if (page < 0 || page >= num_pages) {
+      *bad = true;
+      page = 0;
+    }
+    return (static_cast<long long>(page) * Hkv + g) * b;
+  }
 };
 
 // Byte offsets of the workspace regions (all 256-byte aligned).
@@ -74,6 +95,7 @@ struct ScreenArgs {
 struct AttendArgs {
   const void* k;
   const void* v;
+  const int* block_table;  // paged cache (else null), see KvLayout
   const void* q;
   const int* seq_lens;
   const float* tau;
@@ -134,6 +156,8 @@ struct CalibArgs {
 
 struct SummaryArgs {
   const void* k;
+  const int* block_table;  // paged cache (else null), see KvLayout
+  int num_pages;
   const int* seq_lens;
   const int* first_token;
   void* mu;                // fp16 bits or e4m3 codes (fmt)

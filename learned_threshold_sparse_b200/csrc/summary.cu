@@ -57,7 +57,10 @@ __device__ __forceinline__ float cta_max(float v, float* s_w) {
 template <int FMT>
 __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n, uint8_t* stage) {
   const int d = a.d, t = threadIdx.x;
-  const size_t row0 = (static_cast<size_t>(i) * a.Hkv + g) * a.max_ctx + static_cast<size_t>(j) * a.b;
+  const KvLayout lay{a.block_table, a.Hkv, a.b, a.max_ctx, a.nbmax, a.num_pages};
+  bool bad = false;
+  const size_t row0 = static_cast<size_t>(lay.row(i * a.Hkv + g, j, &bad));
+  if (bad) return;  // a page id outside the pool: nothing is read or written (CTA-uniform)
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.k) + row0 * d * a.elt);
   const int nvec = n * d * a.elt / 16;
   for (int x = t; x < nvec; x += kThreads) reinterpret_cast<uint4*>(stage)[x] = src[x];
@@ -168,7 +171,11 @@ __global__ void __launch_bounds__(kThreads) append_kernel(SummaryArgs a, const v
   if (p < 0 || p >= a.max_ctx) return;
   const int d = a.d, t = threadIdx.x;
   const size_t src = (static_cast<size_t>(i) * a.Hkv + g) * d;
-  const size_t dst = ((static_cast<size_t>(i) * a.Hkv + g) * a.max_ctx + p) * d;
+  const KvLayout lay{a.block_table, a.Hkv, a.b, a.max_ctx, a.nbmax, a.num_pages};
+  bool bad = false;
+  const long long brow = lay.row(i * a.Hkv + g, p / a.b, &bad);
+  if (bad) return;  // a page id outside the pool: nothing is written
+  const size_t dst = (static_cast<size_t>(brow) + p % a.b) * d;
   const int nvec = d * a.elt / 16;
   for (int x = t; x < nvec; x += kThreads) {
     reinterpret_cast<uint4*>(static_cast<uint8_t*>(k_cache) + dst * a.elt)[x] =
