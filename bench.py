@@ -103,6 +103,8 @@ def union_bytes(wl, union_list, union_count):
 def meta_record_bytes(head_dim, meta="fp16"):
     """Bytes of one block's metadata per KV head: fp16 centroid and spread +
     fp32 M, or e4m3 codes + two fp32 scales + fp32 M."""
+    if meta == "box":
+        return 4 * head_dim  # fp16 minima and maxima
     return 2 * head_dim + 12 if meta == "fp8" else 4 * head_dim + 4
 
 
@@ -625,7 +627,8 @@ def main():
     ap.add_argument("--attend-impl", type=int, default=0, choices=[0, 1, 2])
     ap.add_argument("--dense", action="store_true", help="screen off: every block loaded")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--meta", default="fp16", choices=["fp16", "fp8"], help="block metadata format")
+    ap.add_argument("--meta", default="fp16", choices=["fp16", "fp8", "box"],
+                    help="block metadata format (box: the comparison coordinate-box screen)")
     ap.add_argument("--prefill", action="store_true", help="time the causal forward pass instead of the decode step")
     ap.add_argument("--prefill-shape", default="1,32,8,8192", help="batch,n_q_heads,n_kv_heads,seq_len")
     ap.add_argument("--calibrate", action="store_true", help="time the offline calibration histogram")

@@ -101,11 +101,16 @@ typedef struct {
 /* Storage of the centroid and spread in eta_summary_desc. */
 typedef enum {
   ETA_META_FP16 = 0,  /* fp16 values (Appendix F.1)                            */
-  ETA_META_FP8 = 1    /* e4m3 codes with one fp32 scale per block and field:
+  ETA_META_FP8 = 1,   /* e4m3 codes with one fp32 scale per block and field:
                          value = code * scale, the scale mapping the block's
                          largest magnitude to 448 (FP8 metadata, named as a
                          systems extension in section 5; format is this
                          library's choice)                                    */
+  ETA_META_BOX = 2    /* the comparison screen of section 4.3 (Quest): mu
+                         holds the per-coordinate minimum and sigma the
+                         maximum of the block's keys (fp16, rounded outward);
+                         Score = scale sum_i max(q_i min_i, q_i max_i), a
+                         strict bound; max_norm is not used                   */
 } eta_meta_format;
 
 /* Per-block, per-KV-head metadata (Appendix F.1): centroid mu_B, coordinate

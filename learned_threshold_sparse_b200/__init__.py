@@ -63,6 +63,7 @@ class eta_cache_desc(ctypes.Structure):
 
 ETA_META_FP16 = 0
 ETA_META_FP8 = 1
+ETA_META_BOX = 2
 
 
 class eta_summary_desc(ctypes.Structure):
@@ -204,8 +205,17 @@ def cache_desc(k: torch.Tensor, v: torch.Tensor, seq_lens: torch.Tensor, n_q_hea
 def alloc_summary(batch: int, n_kv_heads: int, max_ctx: int, head_dim: int, block_size: int,
                   device="cuda", fmt: str = "fp16") -> Dict[str, torch.Tensor]:
     """Metadata buffers: fp16 mu / sigma, or (fmt="fp8") e4m3 codes as uint8
-    plus per-block fp32 mu_scale / sigma_scale; fp32 max_norm either way."""
+    plus per-block fp32 mu_scale / sigma_scale, or (fmt="box") fp16
+    per-coordinate minima / maxima for the comparison box screen (a 0-d "box"
+    marker tensor tells the descriptor); fp32 max_norm either way."""
     nb = (max_ctx + block_size - 1) // block_size
+    if fmt == "box":
+        return {
+            "mu": torch.zeros((batch, n_kv_heads, nb, head_dim), dtype=torch.float16, device=device),
+            "sigma": torch.zeros((batch, n_kv_heads, nb, head_dim), dtype=torch.float16, device=device),
+            "max_norm": torch.zeros((batch, n_kv_heads, nb), dtype=torch.float32, device=device),
+            "box": torch.zeros((), dtype=torch.uint8, device=device),
+        }
     if fmt == "fp8":
         return {
             "mu": torch.zeros((batch, n_kv_heads, nb, head_dim), dtype=torch.uint8, device=device),
@@ -229,6 +239,8 @@ def summary_desc(summary: Dict[str, torch.Tensor]) -> eta_summary_desc:
         d.format = ETA_META_FP8
         d.mu_scale = summary["mu_scale"].data_ptr()
         d.sigma_scale = summary["sigma_scale"].data_ptr()
+    elif "box" in summary:
+        d.format = ETA_META_BOX
     return d
 
 

@@ -44,7 +44,8 @@ eta_status check_cache(const eta_cache_desc* c) {
 eta_status check_summary(const eta_summary_desc* s) {
   if (!s || !s->mu || !s->sigma || !s->max_norm) return ETA_ERR_INVALID_ARG;
   if (!aligned(s->mu, 16) || !aligned(s->sigma, 16) || !aligned(s->max_norm, 4)) return ETA_ERR_INVALID_ARG;
-  if (s->format != ETA_META_FP16 && s->format != ETA_META_FP8) return ETA_ERR_INVALID_ARG;
+  if (s->format != ETA_META_FP16 && s->format != ETA_META_FP8 && s->format != ETA_META_BOX)
+    return ETA_ERR_INVALID_ARG;
   if (s->format == ETA_META_FP8 &&
       (!s->mu_scale || !s->sigma_scale || !aligned(s->mu_scale, 4) || !aligned(s->sigma_scale, 4)))
     return ETA_ERR_INVALID_ARG;

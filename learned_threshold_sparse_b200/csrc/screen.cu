@@ -230,7 +230,7 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
 #pragma unroll
       for (int u = 0; u < NB; ++u) {
         const int lb = min(gb + u, r - 1);  // a short last group repeats a valid row
-        float mu[CPL], s2[CPL];
+        float mu[CPL], s2[CPL], mx[CPL];
 #pragma unroll
         for (int k = 0; k < CPL / 2; ++k) {
           float2 m, g2;
@@ -247,16 +247,24 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
           }
           mu[2 * k] = m.x;
           mu[2 * k + 1] = m.y;
+          mx[2 * k] = g2.x;
+          mx[2 * k + 1] = g2.y;
           s2[2 * k] = g2.x * g2.x;
           s2[2 * k + 1] = g2.y * g2.y;
         }
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           float dot = 0.f, sq = 0.f;
+          if (FMT == ETA_META_BOX) {
+            // mu holds the per-coordinate minima, mx the maxima
 #pragma unroll
-          for (int k = 0; k < CPL; ++k) {
-            dot = fmaf(qr[h][k], mu[k], dot);
-            sq = fmaf(q2[h][k], s2[k], sq);
+            for (int k = 0; k < CPL; ++k) dot += fmaxf(qr[h][k] * mu[k], qr[h][k] * mx[k]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+              dot = fmaf(qr[h][k], mu[k], dot);
+              sq = fmaf(q2[h][k], s2[k], sq);
+            }
           }
           v[u * NV + h] = dot;
           v[u * NV + G + h] = sq;
@@ -274,9 +282,13 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
           red *= s_ms[r0 + lb];
           sq *= ss * ss;
         }
-        const float geo = my_qn * s_mn[r0 + lb];
-        const float spread = strict ? geo : fminf(geo, z * sqrtf(sq));
-        score = scale * (red + spread);
+        if (FMT == ETA_META_BOX) {
+          score = scale * red;
+        } else {
+          const float geo = my_qn * s_mn[r0 + lb];
+          const float spread = strict ? geo : fminf(geo, z * sqrtf(sq));
+          score = scale * (red + spread);
+        }
         pass = score >= my_tau;
       }
       const unsigned bal = __ballot_sync(0xffffffffu, pass);
@@ -367,7 +379,7 @@ __global__ void rescue_kernel(ScreenArgs a) {
 
 template <int D, int G, int FMT>
 cudaError_t launch_screen_typed(const ScreenArgs& a, cudaStream_t st) {
-  constexpr int ESZ = FMT == ETA_META_FP8 ? 1 : 2;
+  constexpr int ESZ = FMT == ETA_META_FP8 ? 1 : 2;  // the box format stores fp16
   const size_t smem = screen_smem_bytes<D, ESZ>(a.s.chunk);
   auto kern = screen_kernel<D, G, FMT>;
   static SmemLimit lim;
@@ -395,6 +407,8 @@ cudaError_t launch_screen(const ScreenArgs& a, cudaStream_t st) {
   // with the screen off no metadata is read: the fp16 instance serves
   if (a.screen_enabled && a.meta_fmt == ETA_META_FP8)
     return a.s.d == 64 ? launch_screen_d<64, ETA_META_FP8>(a, st) : launch_screen_d<128, ETA_META_FP8>(a, st);
+  if (a.screen_enabled && a.meta_fmt == ETA_META_BOX)
+    return a.s.d == 64 ? launch_screen_d<64, ETA_META_BOX>(a, st) : launch_screen_d<128, ETA_META_BOX>(a, st);
   return a.s.d == 64 ? launch_screen_d<64, ETA_META_FP16>(a, st) : launch_screen_d<128, ETA_META_FP16>(a, st);
 }
 

@@ -73,6 +73,24 @@ __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n
     return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(stage)[idx]) << 16);
   };
   const size_t bo = (static_cast<size_t>(i) * a.Hkv + g) * a.nbmax + j;  // block index
+  if (FMT == ETA_META_BOX) {
+    // per-coordinate extrema, fp16 rounded outward (the box bound stays strict)
+    if (t < d) {
+      float lo = at(0, t), hi = lo;
+      for (int r = 1; r < n; ++r) {
+        const float x = at(r, t);
+        lo = fminf(lo, x);
+        hi = fmaxf(hi, x);
+      }
+      uint16_t l16, h16;
+      asm("cvt.rm.f16.f32 %0, %1;" : "=h"(l16) : "f"(lo));
+      asm("cvt.rp.f16.f32 %0, %1;" : "=h"(h16) : "f"(hi));
+      static_cast<uint16_t*>(a.mu)[bo * d + t] = l16;
+      static_cast<uint16_t*>(a.sigma)[bo * d + t] = h16;
+    }
+    if (t == 0) a.max_norm[bo] = 0.f;
+    return;
+  }
   if (FMT == ETA_META_FP16) {
     if (t < d) {
       float sum = 0.f;
@@ -200,7 +218,8 @@ cudaError_t launch_summary(const SummaryArgs& a, cudaStream_t st) {
       return cudaGetLastError();
     });
   };
-  static SmemLimit lim16, lim8;
+  static SmemLimit lim16, lim8, limb;
+  if (a.fmt == ETA_META_BOX) return go(summary_kernel<ETA_META_BOX>, limb);
   return a.fmt == ETA_META_FP8 ? go(summary_kernel<ETA_META_FP8>, lim8) : go(summary_kernel<ETA_META_FP16>, lim16);
 }
 
@@ -213,7 +232,8 @@ cudaError_t launch_append(const SummaryArgs& a, const void* k_new, const void* v
       return cudaGetLastError();
     });
   };
-  static SmemLimit lim16, lim8;
+  static SmemLimit lim16, lim8, limb;
+  if (a.fmt == ETA_META_BOX) return go(append_kernel<ETA_META_BOX>, limb);
   return a.fmt == ETA_META_FP8 ? go(append_kernel<ETA_META_FP8>, lim8) : go(append_kernel<ETA_META_FP16>, lim16);
 }
 
