@@ -2,8 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl eta|reference]
 
-One step = one eta_decode call (threshold + block screen, attention over the
+One step = one decode step (threshold + block screen, attention over the
 admitted GQA-union blocks, split merge) over the whole batch of the workload,
+launched as one replay of the step recorded into a CUDA graph
+(eta_decode_graph_launch; --launch stream: one eta_decode call),
 inputs resident in HBM, L2 flushed before every step outside the step's
 events by reading a 256 MiB buffer (the evicted lines are clean, so the step
 does not pay for writing back a flush buffer).  Prints ONE JSON line (rank 0).
@@ -15,7 +17,8 @@ value  = effective HBM bandwidth of the step: algorithmic bytes (K+V of the
 e2e    = the same bytes / end-to-end step time through the public API: the
          new token's q, k, v copied in one transfer from pinned host memory,
          eta_append_kv (K/V rows written, their block's metadata refreshed),
-         eta_decode, the output copied back to pinned host memory.
+         the decode step (graph replay or eta_decode, as above), the output
+         copied back to pinned host memory.
 roofline = the attention kernel: union K+V bytes per launch / its mean
          launch time (CUDA events on the launch stream, second run of K
          steps) vs the measured HBM copy bandwidth.
@@ -279,6 +282,22 @@ def run_eta(args):
     params_plain.workspace = ws.data_ptr()
     params_plain.workspace_bytes = ws.numel()
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if args.launch == "graph":
+        # the serving-loop launch path: the step recorded once, replayed per step
+        graph = eta.DecodeGraph(params_plain, [q, k, v, seq, summ, out, lse, ws])
+
+        def timed_step():
+            graph.launch(stream)
+    else:
+        graph = None
+
+        def timed_step():
+            eta.eta_decode(params_plain, stream)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        timed_step()
+    torch.cuda.synchronize()
 
     # Timed region: K steps, each bracketed by events on the launch stream;
     # the L2 flush before every step stays outside the events.
@@ -293,7 +312,7 @@ def run_eta(args):
     for _ in range(args.steps):
         flush.fill_(1.0)
         s0.record(stream)
-        eta.eta_decode(params_plain, stream)
+        timed_step()
         s1.record(stream)
         s1.synchronize()
         step_ms.append(s0.elapsed_time(s1))
@@ -340,10 +359,16 @@ def run_eta(args):
     params_e2e.workspace = ws.data_ptr()
     params_e2e.workspace_bytes = ws.numel()
 
+    graph_e2e = eta.DecodeGraph(params_e2e, [packed_d, k, v, seq, summ, out, lse, ws]) \
+        if args.launch == "graph" else None
+
     def e2e_step():
         packed_d.copy_(packed_h, non_blocking=True)
         eta.eta_append_kv(k, v, seq, summ, wl.block_size, k_in, v_in, last, wl.n_q_heads, stream)
-        eta.eta_decode(params_e2e, stream)
+        if graph_e2e is not None:
+            graph_e2e.launch(stream)
+        else:
+            eta.eta_decode(params_e2e, stream)
         out_h.copy_(out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -359,6 +384,9 @@ def run_eta(args):
         e1.synchronize()
         e2e_ms.append(e0.elapsed_time(e1))
     assert torch.equal(out_h, out.cpu())
+    for g in (graph, graph_e2e):
+        if g is not None:
+            g.close()
     e2e = max_over_ranks(statistics.mean(e2e_ms), dev)
     h2d = packed_h.numel() * wl.elt_bytes
     d2h = out_h.numel() * wl.elt_bytes
@@ -397,6 +425,8 @@ def run_eta(args):
                 "bytes_per_step": nbytes,
                 "kv_union_bytes_per_step": kv_union,
                 "l2": "flushed before every step by reading a 256 MiB buffer (outside the step events)",
+                "launch": ("one CUDA graph of the step per launch (eta_decode_graph_launch)"
+                           if args.launch == "graph" else "stream launches (eta_decode)"),
                 "parallelism": f"replicas x{world} (each rank decodes its own batch)",
             },
             "kernels_ms": {"screen": round(statistics.mean(screen_ms), 6), "attend": round(att_ms, 6),
@@ -626,6 +656,8 @@ def main():
     ap.add_argument("--impl", default="eta", choices=["eta", "reference"])
     ap.add_argument("--attend-impl", type=int, default=0, choices=[0, 1, 2])
     ap.add_argument("--dense", action="store_true", help="screen off: every block loaded")
+    ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
+                    help="decode step as one recorded CUDA graph (default) or as stream launches")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--meta", default="fp16", choices=["fp16", "fp8", "box"],
                     help="block metadata format (box: the comparison coordinate-box screen)")

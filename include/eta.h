@@ -267,6 +267,38 @@ eta_status eta_decode(const eta_decode_params* p, void* stream);
 eta_status eta_decode_noalloc(const eta_decode_params* p, void* stream);
 
 /*
+ * eta_decode_graph_* - one decode step captured once into a CUDA graph and
+ * replayed.  No counterpart in the paper: a launch-path variant of eta_decode
+ * for serving loops that run the same step shape every token.
+ *
+ * eta_decode_graph_create validates p exactly as eta_decode does, then
+ * records eta_decode(p) on a private stream under stream capture
+ * (thread-local mode) and instantiates the graph; nothing runs on the GPU.
+ * On success *out receives a handle the caller owns and must release with
+ * eta_decode_graph_destroy; on failure *out is NULL and nothing is kept.
+ * The graph holds the addresses and scalars of p as they were at creation:
+ *   - every buffer p names (q, caches, seq_lens, summary, tau parameters,
+ *     out, lse, selection outputs, workspace) must stay allocated at the
+ *     same address for the graph's lifetime; their CONTENTS may change
+ *     between launches (a new query, appended tokens, new seq_lens within
+ *     [0, max_ctx]): each launch reads them afresh on the device;
+ *   - shapes, tau mode, scale, beta, offset_a, z, n_local_blocks and the
+ *     attention kernel choice are fixed; a new value needs a new graph;
+ *   - timing_events must all be NULL (ETA_ERR_INVALID_ARG otherwise).
+ * eta_decode_graph_launch enqueues one step on `stream` (stream-ordered and
+ * asynchronous like eta_decode).  Launches of one graph must not overlap on
+ * the GPU (they share its workspace).  Device-side problems are reported by
+ * eta_read_device_status on the workspace, as for eta_decode.
+ * Errors: as eta_decode for create (and ETA_ERR_CUDA if capture or
+ * instantiation fails); ETA_ERR_INVALID_ARG for a NULL handle;
+ * ETA_ERR_CUDA if the graph launch fails.
+ */
+typedef struct eta_decode_graph eta_decode_graph;
+eta_status eta_decode_graph_create(const eta_decode_params* p, eta_decode_graph** out);
+eta_status eta_decode_graph_launch(const eta_decode_graph* g, void* stream);
+eta_status eta_decode_graph_destroy(eta_decode_graph* g);
+
+/*
  * ------------------------------------------------------------------------
  * Causal forward pass over whole sequences (prefill / training forward).
  *

@@ -125,6 +125,12 @@ def _load():
     lib.eta_decode.restype = ctypes.c_int
     lib.eta_decode_noalloc.argtypes = [P(eta_decode_params), ctypes.c_void_p]
     lib.eta_decode_noalloc.restype = ctypes.c_int
+    lib.eta_decode_graph_create.argtypes = [P(eta_decode_params), P(ctypes.c_void_p)]
+    lib.eta_decode_graph_create.restype = ctypes.c_int
+    lib.eta_decode_graph_launch.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    lib.eta_decode_graph_launch.restype = ctypes.c_int
+    lib.eta_decode_graph_destroy.argtypes = [ctypes.c_void_p]
+    lib.eta_decode_graph_destroy.restype = ctypes.c_int
     lib.eta_read_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.eta_read_device_status.restype = ctypes.c_int
     lib.eta_prefill.argtypes = [P(eta_prefill_params), ctypes.c_void_p]
@@ -144,7 +150,7 @@ def _load():
 _lib = _load()
 
 SYMBOLS = ("eta_block_summary_update", "eta_append_kv", "eta_decode_workspace_size", "eta_decode", "eta_decode_noalloc",
-           "eta_read_device_status", "eta_prefill", "eta_calibration_histogram", "eta_calibrate_constants",
+           "eta_decode_graph_create", "eta_decode_graph_launch", "eta_decode_graph_destroy", "eta_read_device_status", "eta_prefill", "eta_calibration_histogram", "eta_calibrate_constants",
            "eta_status_string", "eta_build_info")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
@@ -339,6 +345,55 @@ def eta_decode_noalloc(params: eta_decode_params, stream: Optional[torch.cuda.St
     rc = _lib.eta_decode_noalloc(ctypes.byref(params), _stream_handle(stream))
     if rc != ETA_OK:
         raise EtaError(rc, "eta_decode_noalloc")
+
+
+def eta_decode_graph_create(params: eta_decode_params) -> int:
+    """Record one decode step with these parameters into a CUDA graph; returns
+    the graph handle (see include/eta.h: the buffers params points to must
+    stay in place while the graph lives, their contents may change)."""
+    h = ctypes.c_void_p()
+    rc = _lib.eta_decode_graph_create(ctypes.byref(params), ctypes.byref(h))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_decode_graph_create")
+    return int(h.value)
+
+
+def eta_decode_graph_launch(handle: int, stream: Optional[torch.cuda.Stream] = None) -> None:
+    rc = _lib.eta_decode_graph_launch(ctypes.c_void_p(handle), _stream_handle(stream))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_decode_graph_launch")
+
+
+def eta_decode_graph_destroy(handle: int) -> None:
+    rc = _lib.eta_decode_graph_destroy(ctypes.c_void_p(handle))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_decode_graph_destroy")
+
+
+class DecodeGraph:
+    """Owner of a recorded decode step: keeps the parameter block and the
+    tensors it points to alive, launches the graph, releases it on close()."""
+
+    def __init__(self, params: eta_decode_params, tensors=()):
+        self.params = params
+        self._keep = list(tensors)
+        self.handle = eta_decode_graph_create(params)
+
+    def launch(self, stream: Optional[torch.cuda.Stream] = None) -> None:
+        if not self.handle:
+            raise EtaError(ETA_ERR_INVALID_ARG, "eta_decode_graph_launch")
+        eta_decode_graph_launch(self.handle, stream)
+
+    def close(self) -> None:
+        if self.handle:
+            h, self.handle = self.handle, 0
+            eta_decode_graph_destroy(h)
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 def eta_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:

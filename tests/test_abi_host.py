@@ -90,6 +90,28 @@ def test_invalid_arguments_rejected_before_launch(over, code):
     assert eta.library().eta_decode_workspace_size(ctypes.byref(p), ctypes.byref(n)) == code
 
 
+@pytest.mark.parametrize("over", [{"cache.head_dim": 96}, {"cache.batch": 0}, {"q": None}, {"scale": 0.0},
+                                  {"attend_impl": 9}])
+def test_graph_create_validates_like_decode(over):
+    p = _params(**over)
+    h = ctypes.c_void_p(123)
+    code = eta.library().eta_decode(ctypes.byref(p), None)
+    assert code != eta.ETA_OK
+    assert eta.library().eta_decode_graph_create(ctypes.byref(p), ctypes.byref(h)) == code
+    assert h.value is None  # no handle on failure
+
+
+def test_graph_create_rejects_timing_events_and_null():
+    p = _params()
+    p.timing_events[1] = 1 << 12
+    h = ctypes.c_void_p()
+    assert eta.library().eta_decode_graph_create(ctypes.byref(p), ctypes.byref(h)) == eta.ETA_ERR_INVALID_ARG
+    assert eta.library().eta_decode_graph_create(None, ctypes.byref(h)) == eta.ETA_ERR_INVALID_ARG
+    assert eta.library().eta_decode_graph_create(ctypes.byref(_params()), None) == eta.ETA_ERR_INVALID_ARG
+    assert eta.library().eta_decode_graph_launch(None, None) == eta.ETA_ERR_INVALID_ARG
+    assert eta.library().eta_decode_graph_destroy(None) == eta.ETA_ERR_INVALID_ARG
+
+
 def test_null_params():
     assert eta.library().eta_decode(None, None) == eta.ETA_ERR_INVALID_ARG
     assert eta.library().eta_decode_workspace_size(None, None) == eta.ETA_ERR_INVALID_ARG
