@@ -144,3 +144,27 @@ print("first-call graph ok")
     r = subprocess.run([sys.executable, "-c", code, ROOT], capture_output=True, text=True, timeout=240)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "first-call graph ok" in r.stdout
+
+
+@pytest.mark.parametrize("name", ["c2_single", "c3_long", "c4_max", "c5_batched"])
+def test_graph_full_size_equals_decode(name):
+    """The launch the bench times (one graph replay per step) at the workloads'
+    full sizes gives exactly what eta_decode gives; eta_decode itself is held
+    to the oracle at these sizes by the parity suite."""
+    wl = workloads.make(name, 0)
+    t = upload(wl)
+    summ = gpu_summary(wl, t)
+    p, ws, res = _setup(wl, t, summ)
+    eta.eta_decode(p)
+    ref = _host(res, ws)
+    assert ref["status"] == eta.ETA_OK
+    g = eta.DecodeGraph(p, [ws, *res.values()])
+    try:
+        _clear(res)
+        g.launch()
+        got = _host(res, ws)
+    finally:
+        g.close()
+    for k in KEYS:
+        np.testing.assert_array_equal(got[k], ref[k], err_msg=k)
+    assert got["status"] == eta.ETA_OK
