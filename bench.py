@@ -16,9 +16,12 @@ value  = effective HBM bandwidth of the step: algorithmic bytes (K+V of the
          ranks (each rank decodes its own copy of the batch: weak scaling).
 e2e    = the same bytes / end-to-end step time through the public API: the
          new token's q, k, v copied in one transfer from pinned host memory,
-         eta_append_kv (K/V rows written, their block's metadata refreshed),
-         the decode step (graph replay or eta_decode, as above), the output
-         copied back to pinned host memory.
+         the append (K/V rows written, their block's metadata refreshed), the
+         decode step, the output copied back to pinned host memory; by
+         default one recorded graph (eta_step_graph_create) in which the
+         append kernel reads the new rows from pinned host memory and the
+         decode stores its output into pinned host memory directly; with
+         --launch stream, separate calls with copy-engine transfers.
 roofline = the attention kernel: union K+V bytes per launch / its mean
          launch time (CUDA events on the launch stream, second run of K
          steps) vs the measured HBM copy bandwidth.
@@ -359,17 +362,27 @@ def run_eta(args):
     params_e2e.workspace = ws.data_ptr()
     params_e2e.workspace_bytes = ws.numel()
 
-    graph_e2e = eta.DecodeGraph(params_e2e, [packed_d, k, v, seq, summ, out, lse, ws]) \
-        if args.launch == "graph" else None
+    if args.launch == "graph":
+        # the whole token as one recorded graph: the append kernel reads the
+        # new q, k, v rows from page-locked host memory (and puts q where the
+        # decode reads it), the decode stores its output straight into
+        # page-locked host memory
+        params_e2e.out = out_h.data_ptr()
+        graph_e2e = eta.StepGraph(params_e2e, k_new=packed_h[nq:nq + nkv].view(B_, Hkv_, d_),
+                                  v_new=packed_h[nq + nkv:].view(B_, Hkv_, d_), positions=last,
+                                  q_new=packed_h[:nq].view(B_, Hq_, d_),
+                                  tensors=[q_in, k, v, seq, summ, lse, ws, out_h])
 
-    def e2e_step():
-        packed_d.copy_(packed_h, non_blocking=True)
-        eta.eta_append_kv(k, v, seq, summ, wl.block_size, k_in, v_in, last, wl.n_q_heads, stream)
-        if graph_e2e is not None:
+        def e2e_step():
             graph_e2e.launch(stream)
-        else:
+    else:
+        graph_e2e = None
+
+        def e2e_step():
+            packed_d.copy_(packed_h, non_blocking=True)
+            eta.eta_append_kv(k, v, seq, summ, wl.block_size, k_in, v_in, last, wl.n_q_heads, stream)
             eta.eta_decode(params_e2e, stream)
-        out_h.copy_(out, non_blocking=True)
+            out_h.copy_(out, non_blocking=True)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -425,8 +438,10 @@ def run_eta(args):
                 "bytes_per_step": nbytes,
                 "kv_union_bytes_per_step": kv_union,
                 "l2": "flushed before every step by reading a 256 MiB buffer (outside the step events)",
-                "launch": ("one CUDA graph of the step per launch (eta_decode_graph_launch)"
-                           if args.launch == "graph" else "stream launches (eta_decode)"),
+                "launch": ("one CUDA graph replay per step (eta_decode_graph_launch); e2e: one graph per "
+                           "step of append (reading q, k, v from page-locked host memory) and decode (storing "
+                           "out into page-locked host memory) (eta_step_graph_create)"
+                           if args.launch == "graph" else "stream launches (eta_decode; e2e: separate calls)"),
                 "parallelism": f"replicas x{world} (each rank decodes its own batch)",
             },
             "kernels_ms": {"screen": round(statistics.mean(screen_ms), 6), "attend": round(att_ms, 6),

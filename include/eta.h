@@ -299,6 +299,57 @@ eta_status eta_decode_graph_launch(const eta_decode_graph* g, void* stream);
 eta_status eta_decode_graph_destroy(eta_decode_graph* g);
 
 /*
+ * eta_step_graph_create - one token of a serving loop recorded into a CUDA
+ * graph: an optional host-to-device copy of the token's inputs, an optional
+ * KV append (eta_append_kv on the decode step's cache and summary), the
+ * decode step, an optional device-to-host copy of its output, in that order.
+ * No counterpart in the paper: a launch-path variant for serving loops.
+ *   decode      : the decode step, as for eta_decode_graph_create (required)
+ *   k_new, v_new, positions : as eta_append_kv's arguments; all three NULL =
+ *                 no append, all three set = append (anything else is
+ *                 ETA_ERR_INVALID_ARG); k_new and v_new may be page-locked
+ *                 host memory mapped into the device's address space (the
+ *                 append kernel reads them there)
+ *   q_new       : optional, [batch, n_q_heads, head_dim] kv_dtype, 16-byte
+ *                 aligned, device or mapped page-locked host memory: the
+ *                 token's queries, copied into decode->q by the append launch
+ *                 (so decode->q is written; requires the append)
+ *   h2d_src -> h2d_dst, h2d_bytes : copied first; h2d_src must be page-locked
+ *                 host memory (recording fails with ETA_ERR_CUDA otherwise),
+ *                 h2d_dst device memory; h2d_bytes 0 = no copy
+ *   d2h_src -> d2h_dst, d2h_bytes : copied last; d2h_dst page-locked host
+ *                 memory; d2h_bytes 0 = no copy
+ * When the host end of a copy is mapped into the device's address space
+ * (page-locked memory under unified addressing) and the other end is device
+ * memory, the copy is a small kernel that reads or writes the host buffer
+ * directly; otherwise it is a copy-engine transfer.  The cheapest token
+ * needs neither copy: q_new, k_new, v_new in mapped host memory and
+ * decode->out pointing at mapped host memory (the decode kernels store the
+ * output there directly; pass the device view of the buffer, which under
+ * unified addressing is the host pointer of cudaHostAlloc memory).
+ * The handle is launched and released with eta_decode_graph_launch /
+ * eta_decode_graph_destroy, under the same rules (addresses and scalars
+ * fixed at creation, contents read at every launch).
+ * Errors: as eta_decode_graph_create and eta_append_kv; ETA_ERR_INVALID_ARG
+ * for a NULL pointer with a non-zero copy size.
+ */
+typedef struct {
+  const eta_decode_params* decode;
+  const void* k_new;
+  const void* v_new;
+  const int* positions;
+  const void* q_new;
+  const void* h2d_src;
+  void* h2d_dst;
+  size_t h2d_bytes;
+  const void* d2h_src;
+  void* d2h_dst;
+  size_t d2h_bytes;
+} eta_step_desc;
+
+eta_status eta_step_graph_create(const eta_step_desc* d, eta_decode_graph** out);
+
+/*
  * ------------------------------------------------------------------------
  * Causal forward pass over whole sequences (prefill / training forward).
  *

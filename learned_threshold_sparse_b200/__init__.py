@@ -108,6 +108,15 @@ class eta_calib_params(ctypes.Structure):
     ]
 
 
+class eta_step_desc(ctypes.Structure):
+    _fields_ = [
+        ("decode", ctypes.POINTER(eta_decode_params)), ("k_new", ctypes.c_void_p), ("v_new", ctypes.c_void_p),
+        ("positions", ctypes.c_void_p), ("q_new", ctypes.c_void_p), ("h2d_src", ctypes.c_void_p), ("h2d_dst", ctypes.c_void_p),
+        ("h2d_bytes", ctypes.c_size_t), ("d2h_src", ctypes.c_void_p), ("d2h_dst", ctypes.c_void_p),
+        ("d2h_bytes", ctypes.c_size_t),
+    ]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is not built; run learned_threshold_sparse_b200.build.build()")
@@ -127,6 +136,8 @@ def _load():
     lib.eta_decode_noalloc.restype = ctypes.c_int
     lib.eta_decode_graph_create.argtypes = [P(eta_decode_params), P(ctypes.c_void_p)]
     lib.eta_decode_graph_create.restype = ctypes.c_int
+    lib.eta_step_graph_create.argtypes = [P(eta_step_desc), P(ctypes.c_void_p)]
+    lib.eta_step_graph_create.restype = ctypes.c_int
     lib.eta_decode_graph_launch.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.eta_decode_graph_launch.restype = ctypes.c_int
     lib.eta_decode_graph_destroy.argtypes = [ctypes.c_void_p]
@@ -150,7 +161,8 @@ def _load():
 _lib = _load()
 
 SYMBOLS = ("eta_block_summary_update", "eta_append_kv", "eta_decode_workspace_size", "eta_decode", "eta_decode_noalloc",
-           "eta_decode_graph_create", "eta_decode_graph_launch", "eta_decode_graph_destroy", "eta_read_device_status", "eta_prefill", "eta_calibration_histogram", "eta_calibrate_constants",
+           "eta_decode_graph_create", "eta_step_graph_create", "eta_decode_graph_launch", "eta_decode_graph_destroy",
+           "eta_read_device_status", "eta_prefill", "eta_calibration_histogram", "eta_calibrate_constants",
            "eta_status_string", "eta_build_info")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
@@ -358,6 +370,16 @@ def eta_decode_graph_create(params: eta_decode_params) -> int:
     return int(h.value)
 
 
+def eta_step_graph_create(desc: eta_step_desc) -> int:
+    """Record one serving-loop token (input copy, KV append, decode, output
+    copy; see include/eta.h) into a CUDA graph; returns the graph handle."""
+    h = ctypes.c_void_p()
+    rc = _lib.eta_step_graph_create(ctypes.byref(desc), ctypes.byref(h))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_step_graph_create")
+    return int(h.value)
+
+
 def eta_decode_graph_launch(handle: int, stream: Optional[torch.cuda.Stream] = None) -> None:
     rc = _lib.eta_decode_graph_launch(ctypes.c_void_p(handle), _stream_handle(stream))
     if rc != ETA_OK:
@@ -377,6 +399,7 @@ class DecodeGraph:
     def __init__(self, params: eta_decode_params, tensors=()):
         self.params = params
         self._keep = list(tensors)
+        self.handle = 0
         self.handle = eta_decode_graph_create(params)
 
     def launch(self, stream: Optional[torch.cuda.Stream] = None) -> None:
@@ -394,6 +417,33 @@ class DecodeGraph:
             self.close()
         except Exception:
             pass
+
+
+class StepGraph(DecodeGraph):
+    """Owner of a recorded serving-loop token: the host-to-device copy of
+    `h2d` (page-locked host tensor) into `h2d_dst`, the append of k_new / v_new
+    at `positions` with the queries q_new copied into the decode's q
+    (optional; the new rows may be page-locked host tensors), the decode step
+    of `params`, and the copy of `d2h_src` into the page-locked host tensor
+    `d2h`."""
+
+    def __init__(self, params: eta_decode_params, *, k_new=None, v_new=None, positions=None, q_new=None, h2d=None,
+                 h2d_dst=None, d2h_src=None, d2h=None, tensors=()):
+        self.params = params
+        self._keep = [t for t in (k_new, v_new, positions, q_new, h2d, h2d_dst, d2h_src, d2h) if t is not None]
+        self._keep += list(tensors)
+        d = eta_step_desc()
+        d.decode = ctypes.pointer(params)
+        d.k_new, d.v_new, d.positions, d.q_new = _ptr(k_new), _ptr(v_new), _ptr(positions), _ptr(q_new)
+        if h2d is not None:
+            d.h2d_src, d.h2d_dst = _ptr(h2d), _ptr(h2d_dst)
+            d.h2d_bytes = h2d.numel() * h2d.element_size()
+        if d2h is not None:
+            d.d2h_src, d.d2h_dst = _ptr(d2h_src), _ptr(d2h)
+            d.d2h_bytes = d2h.numel() * d2h.element_size()
+        self.desc = d
+        self.handle = 0
+        self.handle = eta_step_graph_create(d)
 
 
 def eta_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:

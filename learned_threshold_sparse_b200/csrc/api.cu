@@ -245,13 +245,27 @@ eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summa
 
 eta_status eta_append_kv(const eta_cache_desc* cache, const eta_summary_desc* summary, const void* k_new,
                          const void* v_new, const int* pos, void* stream) {
+  return eta::append_step(cache, summary, k_new, v_new, pos, nullptr, nullptr, stream);
+}
+
+}  // extern "C"
+
+namespace eta {
+
+eta_status append_step(const eta_cache_desc* cache, const eta_summary_desc* summary, const void* k_new,
+                       const void* v_new, const int* pos, const void* q_src, void* q_dst, void* stream) {
   eta_status st = check_cache(cache);
   if (st != ETA_OK) return st;
   st = check_summary(summary);
   if (st != ETA_OK) return st;
   if (!k_new || !v_new || !pos || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(pos, 4))
     return ETA_ERR_INVALID_ARG;
+  if ((q_src == nullptr) != (q_dst == nullptr)) return ETA_ERR_INVALID_ARG;
+  if (q_src && (!aligned(q_src, 16) || !aligned(q_dst, 16))) return ETA_ERR_INVALID_ARG;
   SummaryArgs a;
+  a.q_src = q_src;
+  a.q_dst = q_dst;
+  a.G = cache->n_q_heads / cache->n_kv_heads;
   a.k = cache->k_cache;
   a.block_table = cache->block_table;
   a.num_pages = cache->num_pages;
@@ -274,6 +288,10 @@ eta_status eta_append_kv(const eta_cache_desc* cache, const eta_summary_desc* su
              ? ETA_OK
              : ETA_ERR_CUDA;
 }
+
+}  // namespace eta
+
+extern "C" {
 
 eta_status eta_decode_workspace_size(const eta_decode_params* p, size_t* bytes) {
   if (!bytes) return ETA_ERR_INVALID_ARG;

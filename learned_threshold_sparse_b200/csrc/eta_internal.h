@@ -167,7 +167,18 @@ struct SummaryArgs {
   float* sigma_scale;
   int fmt;                 // ETA_META_FP16 / ETA_META_FP8
   int B, Hkv, d, b, max_ctx, nbmax, elt, max_blocks;
+  // append only: the token's query rows [B, Hkv * G, d] copied from q_src
+  // (device or mapped page-locked host memory) to q_dst by the same launch
+  const void* q_src = nullptr;
+  void* q_dst = nullptr;
+  int G = 0;
 };
+
+// The append of eta_append_kv, optionally also copying the token's query
+// rows q_src -> q_dst ([batch, n_q_heads, head_dim]) in the same launch
+// (api.cu; used by the recorded serving step).
+eta_status append_step(const eta_cache_desc* cache, const eta_summary_desc* summary, const void* k_new,
+                       const void* v_new, const int* pos, const void* q_src, void* q_dst, void* stream);
 
 // ---------------------------------------------------------------- host helpers
 // Driver attribute queries and settings cost on the order of a microsecond

@@ -106,8 +106,12 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
   __shared__ __align__(8) uint64_t s_bar[2];
 
   // The attention kernel may be scheduled now; it waits for this grid's
-  // completion before reading anything written here.
+  // completion before reading anything written here.  This grid is itself
+  // launched as a dependent of the stream's previous kernel (the token's
+  // append, or the previous step's merge, which reads the chunk counts this
+  // grid rewrites): nothing is read or written before that kernel is done.
   dev::pdl_trigger();
+  dev::pdl_wait();
 
   const int blk0 = c * s.chunk;
   const int avail = min(s.chunk, s.nbmax - blk0);  // rows of this chunk inside the arrays
@@ -383,10 +387,18 @@ cudaError_t launch_screen_typed(const ScreenArgs& a, cudaStream_t st) {
   const size_t smem = screen_smem_bytes<D, ESZ>(a.s.chunk);
   auto kern = screen_kernel<D, G, FMT>;
   static SmemLimit lim;
-  return launch_with_smem(reinterpret_cast<const void*>(kern), screen_smem_bytes<D, ESZ>(2 * kRound), lim, [&] {
-    kern<<<dim3(a.s.nchunks, a.s.Hkv, a.s.B), kThreads, smem, st>>>(a);
-    return cudaGetLastError();
-  });
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.s.nchunks, a.s.Hkv, a.s.B);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return launch_with_smem(reinterpret_cast<const void*>(kern), screen_smem_bytes<D, ESZ>(2 * kRound), lim,
+                          [&] { return cudaLaunchKernelEx(&cfg, kern, a); });
 }
 
 template <int D, int FMT>

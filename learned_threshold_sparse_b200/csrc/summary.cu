@@ -179,27 +179,53 @@ __global__ void __launch_bounds__(kThreads) summary_kernel(SummaryArgs a) {
 // One CTA per (KV head, sequence): write the new token's K and V rows at
 // position pos[i], then refresh the block holding it over the rows present
 // (seq_lens[i] already counts the new token).  A position outside
-// [0, max_ctx) writes nothing.
+// [0, max_ctx) writes nothing.  With q_src set, the CTA also copies the
+// token's G query rows of this KV head to q_dst.  The new rows are loaded
+// with .cv: they may sit in page-locked host memory that the host rewrites
+// between launches.
 template <int FMT>
 __global__ void __launch_bounds__(kThreads) append_kernel(SummaryArgs a, const void* k_new, const void* v_new,
                                                           const int* pos, void* k_cache, void* v_cache) {
   extern __shared__ __align__(16) uint8_t stage[];
   const int g = blockIdx.x, i = blockIdx.y;
-  const int p = pos[i];
-  if (p < 0 || p >= a.max_ctx) return;
   const int d = a.d, t = threadIdx.x;
+  // The decode's screen may be scheduled now: it waits for this grid's
+  // completion before it reads anything.
+  dev::pdl_trigger();
+  // Every load of the new rows is issued before the first use, so rows in
+  // host memory cost one round trip: a K and a V vector per thread
+  // (d * elt / 16 <= 32 vectors per row) and up to kQv query vectors
+  // (G * d * elt / 16 <= 256 = kQv * kThreads).
+  constexpr int kQv = 2;
+  const int nvec = d * a.elt / 16;
   const size_t src = (static_cast<size_t>(i) * a.Hkv + g) * d;
+  uint4 kr = make_uint4(0u, 0u, 0u, 0u), vr = kr, qr[kQv];
+  if (t < nvec) {
+    kr = __ldcv(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_new) + src * a.elt) + t);
+    vr = __ldcv(reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_new) + src * a.elt) + t);
+  }
+  const size_t q0 = (static_cast<size_t>(i) * a.Hkv * a.G + static_cast<size_t>(g) * a.G) * d * a.elt / 16;
+  const int qv = a.q_src ? a.G * d * a.elt / 16 : 0;
+#pragma unroll
+  for (int u = 0; u < kQv; ++u) {
+    const int x = t + u * kThreads;
+    if (x < qv) qr[u] = __ldcv(reinterpret_cast<const uint4*>(a.q_src) + q0 + x);
+  }
+  const int p = pos[i];
+#pragma unroll
+  for (int u = 0; u < kQv; ++u) {
+    const int x = t + u * kThreads;
+    if (x < qv) reinterpret_cast<uint4*>(a.q_dst)[q0 + x] = qr[u];
+  }
+  if (p < 0 || p >= a.max_ctx) return;
   const KvLayout lay{a.block_table, a.Hkv, a.b, a.max_ctx, a.nbmax, a.num_pages};
   bool bad = false;
   const long long brow = lay.row(i * a.Hkv + g, p / a.b, &bad);
   if (bad) return;  // a page id outside the pool: nothing is written
   const size_t dst = (static_cast<size_t>(brow) + p % a.b) * d;
-  const int nvec = d * a.elt / 16;
-  for (int x = t; x < nvec; x += kThreads) {
-    reinterpret_cast<uint4*>(static_cast<uint8_t*>(k_cache) + dst * a.elt)[x] =
-        reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(k_new) + src * a.elt)[x];
-    reinterpret_cast<uint4*>(static_cast<uint8_t*>(v_cache) + dst * a.elt)[x] =
-        reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(v_new) + src * a.elt)[x];
+  if (t < nvec) {
+    reinterpret_cast<uint4*>(static_cast<uint8_t*>(k_cache) + dst * a.elt)[t] = kr;
+    reinterpret_cast<uint4*>(static_cast<uint8_t*>(v_cache) + dst * a.elt)[t] = vr;
   }
   __syncthreads();  // the new row is read back by the block summary below
   const int T = clamp_len(a.seq_lens[i], a.max_ctx);

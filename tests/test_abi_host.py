@@ -112,6 +112,36 @@ def test_graph_create_rejects_timing_events_and_null():
     assert eta.library().eta_decode_graph_destroy(None) == eta.ETA_ERR_INVALID_ARG
 
 
+def test_step_graph_validation():
+    lib = eta.library()
+    h = ctypes.c_void_p()
+    fake = 1 << 20
+    d = eta.eta_step_desc()
+    assert lib.eta_step_graph_create(None, ctypes.byref(h)) == eta.ETA_ERR_INVALID_ARG
+    assert lib.eta_step_graph_create(ctypes.byref(d), ctypes.byref(h)) == eta.ETA_ERR_INVALID_ARG  # no decode
+    bad = _params(**{"cache.head_dim": 96})
+    d.decode = ctypes.pointer(bad)
+    assert lib.eta_step_graph_create(ctypes.byref(d), ctypes.byref(h)) == eta.ETA_ERR_UNSUPPORTED
+    p = _params()
+    p.timing_events[0] = 1 << 12
+    d.decode = ctypes.pointer(p)
+    assert lib.eta_step_graph_create(ctypes.byref(d), ctypes.byref(h)) == eta.ETA_ERR_INVALID_ARG
+    assert h.value is None
+    assert lib.eta_step_graph_create(ctypes.byref(d), None) == eta.ETA_ERR_INVALID_ARG
+    good = _params()
+    d.decode = ctypes.pointer(good)
+    d.k_new = fake  # an append needs all three of k_new, v_new, positions
+    assert lib.eta_step_graph_create(ctypes.byref(d), ctypes.byref(h)) == eta.ETA_ERR_INVALID_ARG
+    d.k_new = None
+    d.h2d_bytes = 64  # a copy needs both ends
+    d.h2d_dst = fake
+    assert lib.eta_step_graph_create(ctypes.byref(d), ctypes.byref(h)) == eta.ETA_ERR_INVALID_ARG
+    d.h2d_bytes = 0
+    d.d2h_bytes = 64
+    d.d2h_src = fake
+    assert lib.eta_step_graph_create(ctypes.byref(d), ctypes.byref(h)) == eta.ETA_ERR_INVALID_ARG
+
+
 def test_null_params():
     assert eta.library().eta_decode(None, None) == eta.ETA_ERR_INVALID_ARG
     assert eta.library().eta_decode_workspace_size(None, None) == eta.ETA_ERR_INVALID_ARG
@@ -141,6 +171,7 @@ def test_struct_layout_matches_header(tmp_path):
         "eta_decode_params": eta.eta_decode_params,
         "eta_prefill_params": eta.eta_prefill_params,
         "eta_calib_params": eta.eta_calib_params,
+        "eta_step_desc": eta.eta_step_desc,
     }
     lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "eta.h"', "int main(void) {"]
     for sname, cls in fields.items():

@@ -168,3 +168,73 @@ def test_graph_full_size_equals_decode(name):
     for k in KEYS:
         np.testing.assert_array_equal(got[k], ref[k], err_msg=k)
     assert got["status"] == eta.ETA_OK
+
+
+@pytest.mark.parametrize("mode", ["copies", "direct"])
+def test_step_graph_equals_separate_calls(mode):
+    """One serving-loop token as one graph leaves the caches, the metadata and
+    the host output exactly as separate calls do, token after token.
+    copies: input copy from page-locked host memory, append, decode, output
+    copy back.  direct: the append reads the new q, k, v rows from
+    page-locked host memory itself and the decode stores its output straight
+    into page-locked host memory (no copies)."""
+    shape = dict(batch=3, n_q_heads=16, n_kv_heads=4, head_dim=128, block_size=64, dtype=BF16, max_ctx=3200)
+    wl = workloads.custom(seed=21, seq_lens=[3000, 1, 777], tau_bias=2.0, tau_std=1.0, **shape)
+    B, Hq, Hkv, d = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
+    nq, nkv = B * Hq * d, B * Hkv * d
+    host = torch.empty(nq + 2 * nkv, dtype=torch.bfloat16).pin_memory()
+    states = []
+    for _ in range(2):  # A: separate calls, B: one recorded step
+        t = upload(wl)
+        summ = gpu_summary(wl, t)
+        packed = torch.empty(host.shape, dtype=host.dtype, device="cuda")
+        q_in = packed[:nq].view(B, Hq, d)
+        k_in, v_in = packed[nq:nq + nkv].view(B, Hkv, d), packed[nq + nkv:].view(B, Hkv, d)
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device="cuda")
+        out_h = torch.zeros((B, Hq, d), dtype=torch.bfloat16).pin_memory()
+        lse = torch.empty((B, Hq), dtype=torch.float32, device="cuda")
+        states.append(dict(t=t, summ=summ, packed=packed, q_in=q_in, k_in=k_in, v_in=v_in, out=out, lse=lse,
+                           out_h=out_h, pos=torch.tensor(wl.seq_lens, dtype=torch.int32, device="cuda")))
+    for n, st in enumerate(states):
+        direct = n == 1 and mode == "direct"
+        st["p"] = eta.make_params(st["q_in"], st["t"]["k"], st["t"]["v"], st["t"]["seq"], st["summ"], wl.block_size,
+                                  wl.tau_mode, w_tau=st["t"]["w_tau"], b_tau=st["t"]["b_tau"], scale=wl.scale,
+                                  beta=wl.beta, z=wl.z, n_local_blocks=wl.n_local_blocks,
+                                  out=st["out_h"] if direct else st["out"], lse=st["lse"])
+        st["ws"] = eta.alloc_workspace(eta.eta_decode_workspace_size(st["p"]))
+        st["p"].workspace, st["p"].workspace_bytes = st["ws"].data_ptr(), st["ws"].numel()
+    a, b = states
+    keep = [b["ws"], b["lse"], b["out"], *b["summ"].values()]
+    if mode == "direct":
+        g = eta.StepGraph(b["p"], k_new=host[nq:nq + nkv].view(B, Hkv, d), v_new=host[nq + nkv:].view(B, Hkv, d),
+                          positions=b["pos"], q_new=host[:nq].view(B, Hq, d), tensors=keep + [b["q_in"]])
+    else:
+        g = eta.StepGraph(b["p"], k_new=b["k_in"], v_new=b["v_in"], positions=b["pos"], h2d=host,
+                          h2d_dst=b["packed"], d2h_src=b["out"], d2h=b["out_h"], tensors=keep)
+    rng = np.random.default_rng(3)
+    try:
+        for _ in range(3):
+            host.copy_(torch.from_numpy(rng.standard_normal(host.numel()).astype(np.float32)).to(torch.bfloat16))
+            for st in (a, b):
+                st["t"]["seq"] += 1  # the new token counts before the append
+            torch.cuda.synchronize()
+            a["packed"].copy_(host, non_blocking=True)
+            eta.eta_append_kv(a["t"]["k"], a["t"]["v"], a["t"]["seq"], a["summ"], wl.block_size, a["k_in"],
+                              a["v_in"], a["pos"], Hq)
+            eta.eta_decode(a["p"])
+            a["out_h"].copy_(a["out"], non_blocking=True)
+            g.launch()
+            torch.cuda.synchronize()
+            for st in (a, b):
+                assert eta.eta_read_device_status(st["ws"]) == eta.ETA_OK
+            assert torch.equal(a["out_h"], b["out_h"])
+            assert torch.equal(a["lse"], b["lse"])
+            if mode == "direct":
+                assert torch.equal(b["q_in"], a["q_in"])  # the queries landed in the decode's q
+            assert torch.equal(a["t"]["k"], b["t"]["k"]) and torch.equal(a["t"]["v"], b["t"]["v"])
+            for name in a["summ"]:
+                assert torch.equal(a["summ"][name], b["summ"][name]), name
+            for st in (a, b):
+                st["pos"] += 1
+    finally:
+        g.close()
