@@ -101,9 +101,8 @@ struct IoCopy {
                                                      bytes, h2d ? 1 : 0);
       return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
     }
-    return cudaMemcpyAsync(dst, src, bytes, h2d ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToHost, cs) == cudaSuccess
-               ? ETA_OK
-               : ETA_ERR_CUDA;
+    // the copy engine, direction taken from the unified address space
+    return cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDefault, cs) == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
   }
 };
 
