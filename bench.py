@@ -453,7 +453,11 @@ def run_eta(args):
                          "algorithmic_bytes_per_launch": kv_union},
             "step_frac_of_peak": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4),
             "e2e": {"value": round(whole_job_gbs(world, nbytes, e2e), 2), "unit": UNIT,
-                    "ms_per_step": round(e2e, 6), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                    "ms_per_step": round(e2e, 6), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "io": ("the append kernel loads the token's q, k, v rows from pinned host memory and the "
+                           "decode stores out into pinned host memory, one graph per token"
+                           if args.launch == "graph" else
+                           "q, k, v copied from pinned host memory and out copied back by the copy engine")},
             "gpu_launches": 3 * args.steps,
             "clocks": clk,
             "wall_s_timed_region": round(wall_s, 3),
