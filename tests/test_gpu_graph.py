@@ -238,3 +238,31 @@ def test_step_graph_equals_separate_calls(mode):
                 st["pos"] += 1
     finally:
         g.close()
+
+
+@pytest.mark.parametrize("nbytes,offset", [(1001, 0), (4096, 3), (16, 0), (70000, 5)])
+def test_step_graph_copies_of_any_size_and_alignment(nbytes, offset):
+    """The step's input and output copies move exactly their bytes, also for
+    sizes that are not a multiple of 16 and for buffers that start off a
+    16-byte boundary (the copy kernel's byte path)."""
+    wl = workloads.custom(seed=8, batch=1, n_q_heads=4, n_kv_heads=1, head_dim=64, block_size=64, seq_lens=[300],
+                          dtype=F32, tau_bias=2.0, tau_std=1.0)
+    t = upload(wl)
+    summ = gpu_summary(wl, t)
+    p, ws, res = _setup(wl, t, summ)
+    rng = np.random.default_rng(nbytes)
+    src_h = torch.from_numpy(rng.integers(0, 256, nbytes + offset, dtype=np.uint8)).pin_memory()
+    dst_d = torch.zeros(nbytes + offset, dtype=torch.uint8, device="cuda")
+    src_d = torch.from_numpy(rng.integers(0, 256, nbytes + offset, dtype=np.uint8)).cuda()
+    dst_h = torch.zeros(nbytes + offset, dtype=torch.uint8).pin_memory()
+    g = eta.StepGraph(p, h2d=src_h[offset:], h2d_dst=dst_d[offset:], d2h_src=src_d[offset:], d2h=dst_h[offset:],
+                      tensors=[ws, *res.values(), src_h, dst_d, src_d, dst_h])
+    try:
+        g.launch()
+        torch.cuda.synchronize()
+    finally:
+        g.close()
+    assert torch.equal(dst_d[offset:].cpu(), src_h[offset:])
+    assert torch.equal(dst_h[offset:], src_d[offset:].cpu())
+    assert not dst_d[:offset].any() and not dst_h[:offset].any()  # nothing written before the buffers
+    assert eta.eta_read_device_status(ws) == eta.ETA_OK
