@@ -75,6 +75,22 @@ def prefill_head(q, K, V, tau_tilde, scale: float, beta: float):
     return O, m + np.log(l), sig.sum(axis=1)
 
 
+def prefill_row(q_i, K_seen, V_seen, tau_i: float, scale: float, beta: float):
+    """One query row of the causal pass: row i sees the keys K_seen = k_0..k_i
+    (all of them, no mask).  Same quantities as prefill_head for that row:
+    (o_i [d], L_i, R_i).  Lets a test check sampled rows of a long sequence
+    without the T x T matrix."""
+    q_i, K, V = _f64(q_i), _f64(K_seen), _f64(V_seen)
+    S = scale * (K @ q_i)
+    with np.errstate(over="ignore"):
+        sig = 1.0 / (1.0 + np.exp(-beta * (S - float(tau_i))))
+    St = S * sig
+    m = St.max()
+    w = np.exp(St - m)
+    l = w.sum()
+    return (w @ V) / l, m + np.log(l), sig.sum()
+
+
 def prefill(q, k, v, seq_len: int, tau_mode: str, w_tau=None, b_tau=None, c_tau=None,
             scale: Optional[float] = None, beta: float = 5.0, offset_a: float = 0.0) -> Dict[str, np.ndarray]:
     """Whole batch: q [B, Hq, T, d], k and v [B, Hkv, >= T, d]; query head h

@@ -97,3 +97,24 @@ def test_prefill_deterministic():
     a, b = _run(case), _run(case)
     for n in ("out", "lse", "gate_sum"):
         np.testing.assert_array_equal(a[n], b[n])
+
+
+def test_prefill_full_size_sampled_rows():
+    """The shape the bench times (batch 1, 32 query / 8 KV heads, 8192 tokens,
+    seed 0): sampled rows (the first and last rows of tiles, the sequence's
+    ends, random interior rows) of sampled heads against the one-row oracle."""
+    case = workloads.prefill_case(0, batch=1, n_q_heads=32, n_kv_heads=8, seq_len=8192)
+    got = _run(case)
+    G = case.n_q_heads // case.n_kv_heads
+    rng = np.random.default_rng(1)
+    rows = sorted({0, 1, 127, 128, 129, 4095, 4096, 8190, 8191, *rng.integers(0, 8192, 8).tolist()})
+    for h in (0, 5, 17, 31):
+        g = h // G
+        q = case.q[0, h].float().double().numpy()
+        tau = po.prefill_thresholds(q, case.tau_mode, case.w_tau[h], case.b_tau[h], None, case.offset_a)
+        for i in rows:
+            o, lse, r = po.prefill_row(q[i], case.k[0, g, :i + 1], case.v[0, g, :i + 1], tau[i], case.scale,
+                                       case.beta)
+            np.testing.assert_allclose(got["out"][0, h, i], o, rtol=OUT_RTOL, atol=OUT_ATOL, err_msg=f"{h} {i}")
+            assert abs(got["lse"][0, h, i] - lse) <= LSE_ATOL, (h, i)
+            assert abs(got["gate_sum"][0, h, i] - r) <= GATE_ATOL + GATE_RTOL * abs(r), (h, i)

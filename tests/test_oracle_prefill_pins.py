@@ -115,3 +115,21 @@ def test_last_row_matches_the_decode_oracle():
 def test_flop_count():
     # 4 d flops per causal (query, key) pair: T (T + 1) / 2 pairs per head
     assert po.prefill_flops(2, 3, 4, 8) == 4 * 8 * 10 * 2 * 3
+
+
+def test_row_form_matches_whole_head_and_decode():
+    # prefill_row(i) over keys 0..i is row i of the whole-head causal pass, and
+    # at every i it is a dense decode step of q_i over a cache of i + 1 keys
+    q, k, v = _inputs(8, Hq=1, Hkv=1, T=33, d=8)
+    scale, beta = 0.4, 5.0
+    tau = po.prefill_thresholds(q[0, 0], "calibrated", c_h=0.3)
+    O, L, R = po.prefill_head(q[0, 0], k[0, 0], v[0, 0], tau, scale, beta)
+    for i in (0, 1, 7, 8, 31, 32):
+        o, lse, r = po.prefill_row(q[0, 0, i], k[0, 0, :i + 1], v[0, 0, :i + 1], tau[i], scale, beta)
+        np.testing.assert_allclose(o, O[i], rtol=1e-12, atol=1e-13)
+        assert math.isclose(lse, L[i], rel_tol=1e-12) and math.isclose(r, R[i], rel_tol=1e-12)
+        nb = (i + 1 + 3) // 4
+        o2, lse2 = oracle.attend_head(q[0, 0, i], k[0, 0], v[0, 0], i + 1, 4, np.ones(nb, dtype=bool), tau[i],
+                                      scale, beta)
+        np.testing.assert_allclose(o, o2, rtol=1e-12, atol=1e-13)
+        assert math.isclose(lse, lse2, rel_tol=1e-12)
