@@ -461,6 +461,20 @@ eta_status eta_calibrate_constants(const double* hist, int n_heads, int nbins, f
  */
 eta_status eta_read_device_status(void* workspace, void* stream);
 
+/*
+ * eta_diag_wait_timeout - diagnostic: one warp waits, with the same bounded
+ * wait the kernels use, on a shared-memory mbarrier that nothing completes;
+ * after the wait's cycle limit (about one second) it gives up and sets the
+ * timeout bit of the status word at the start of `workspace`.  A following
+ * eta_read_device_status(workspace) then returns ETA_ERR_DEVICE_TIMEOUT and
+ * the context stays usable.  It checks the failure-reporting path end to end
+ * without a fault or a hang.  No counterpart in the paper.
+ *   workspace : device memory, 256-byte aligned, at least 4 bytes (a decode
+ *               workspace serves)
+ * Errors: ETA_ERR_INVALID_ARG (NULL or misaligned), ETA_ERR_CUDA (launch).
+ */
+eta_status eta_diag_wait_timeout(void* workspace, void* stream);
+
 /* Static description of a status code. */
 const char* eta_status_string(eta_status s);
 

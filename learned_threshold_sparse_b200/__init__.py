@@ -142,6 +142,8 @@ def _load():
     lib.eta_decode_graph_launch.restype = ctypes.c_int
     lib.eta_decode_graph_destroy.argtypes = [ctypes.c_void_p]
     lib.eta_decode_graph_destroy.restype = ctypes.c_int
+    lib.eta_diag_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
+    lib.eta_diag_wait_timeout.restype = ctypes.c_int
     lib.eta_read_device_status.argtypes = [ctypes.c_void_p, ctypes.c_void_p]
     lib.eta_read_device_status.restype = ctypes.c_int
     lib.eta_prefill.argtypes = [P(eta_prefill_params), ctypes.c_void_p]
@@ -162,7 +164,7 @@ _lib = _load()
 
 SYMBOLS = ("eta_block_summary_update", "eta_append_kv", "eta_decode_workspace_size", "eta_decode", "eta_decode_noalloc",
            "eta_decode_graph_create", "eta_step_graph_create", "eta_decode_graph_launch", "eta_decode_graph_destroy",
-           "eta_read_device_status", "eta_prefill", "eta_calibration_histogram", "eta_calibrate_constants",
+           "eta_read_device_status", "eta_diag_wait_timeout", "eta_prefill", "eta_calibration_histogram", "eta_calibrate_constants",
            "eta_status_string", "eta_build_info")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
@@ -444,6 +446,14 @@ class StepGraph(DecodeGraph):
         self.desc = d
         self.handle = 0
         self.handle = eta_step_graph_create(d)
+
+
+def eta_diag_wait_timeout(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Diagnostic: a bounded device-side wait that nothing completes gives up
+    and sets the workspace's timeout bit (see include/eta.h)."""
+    rc = _lib.eta_diag_wait_timeout(ctypes.c_void_p(workspace.data_ptr()), _stream_handle(stream))
+    if rc != ETA_OK:
+        raise EtaError(rc, "eta_diag_wait_timeout")
 
 
 def eta_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.Stream] = None) -> int:

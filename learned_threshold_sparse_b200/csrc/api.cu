@@ -212,7 +212,7 @@ const char* eta_status_string(eta_status s) {
 
 const char* eta_build_info(void) {
   return "eta decode library: sm_100a; kernels: block_summary, append, screen, rescue, attend_simt, attend_tc, "
-         "merge, export, prefill_tc, calib_hist, io_copy; decode step and serving step as CUDA graphs";
+         "merge, export, prefill_tc, calib_hist, io_copy, diag_wait; decode step and serving step as CUDA graphs";
 }
 
 eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summary_desc* summary,

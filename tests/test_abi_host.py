@@ -142,6 +142,11 @@ def test_step_graph_validation():
     assert lib.eta_step_graph_create(ctypes.byref(d), ctypes.byref(h)) == eta.ETA_ERR_INVALID_ARG
 
 
+def test_diag_wait_timeout_validation():
+    assert eta.library().eta_diag_wait_timeout(None, None) == eta.ETA_ERR_INVALID_ARG
+    assert eta.library().eta_diag_wait_timeout((1 << 20) + 64, None) == eta.ETA_ERR_INVALID_ARG
+
+
 def test_null_params():
     assert eta.library().eta_decode(None, None) == eta.ETA_ERR_INVALID_ARG
     assert eta.library().eta_decode_workspace_size(None, None) == eta.ETA_ERR_INVALID_ARG
