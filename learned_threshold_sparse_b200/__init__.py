@@ -22,7 +22,7 @@ from __future__ import annotations
 import ctypes
 import math
 import os
-from typing import Dict, Optional, Sequence
+from typing import Dict, Optional
 
 import torch
 

@@ -40,7 +40,7 @@ by closed forms), the combination by ``min`` is a reading and is
 from __future__ import annotations
 
 import math
-from typing import Dict, List, Optional, Sequence, Tuple
+from typing import Dict, Optional, Sequence, Tuple
 
 import numpy as np
 

@@ -15,7 +15,6 @@ calibrated mode stores c_tau = tau~ + a.
 Usage:  python tests/golden/make_thresholds.py [name ...]
 """
 import json
-import math
 import os
 import sys
 

@@ -10,7 +10,7 @@ import torch
 
 import learned_threshold_sparse_b200 as eta
 import workloads
-from etatest import compare, gpu_decode, oracle_decode, upload
+from etatest import compare, oracle_decode, upload
 
 pytestmark = pytest.mark.gpu
 
