@@ -70,9 +70,6 @@ __device__ __forceinline__ float tanh_approx(float x) {
   return y;
 }
 
-// sigmoid(x) = (1 + tanh(x / 2)) / 2: one special-function op.
-__device__ __forceinline__ float gate(float x) { return fmaf(0.5f, tanh_approx(0.5f * x), 0.5f); }
-
 // Two floats to a bf16 pair (lo in the low half), round to nearest even.
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   uint32_t r;
