@@ -276,3 +276,18 @@ def test_calibration_validation():
         q = eta.eta_calib_params.from_buffer_copy(p)
         setattr(q, field, value)
         assert lib.eta_calibration_histogram(ctypes.byref(q), None) == code, field
+
+
+def test_c_example_compiles_and_links(tmp_path):
+    # tests/c/decode_example.c drives one decode step through the C ABI from
+    # plain C99 (no Python); here it must compile warning-free and link
+    # against libeta.so (running it needs a GPU)
+    import subprocess
+    cuda = "/usr/local/cuda"
+    exe = tmp_path / "decode_example"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                        "-I", os.path.join(cuda, "include"), os.path.join(ROOT, "tests", "c", "decode_example.c"),
+                        "-L", os.path.join(ROOT, "learned_threshold_sparse_b200"), "-leta",
+                        "-L", os.path.join(cuda, "lib64"), "-lcudart", "-lm", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
