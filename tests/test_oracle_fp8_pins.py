@@ -1,13 +1,17 @@
 """Pins of the FP8 metadata oracle: the e4m3 rounding against a brute-force
-nearest-value search over all codes, closed forms of the scale and of a
-constant block, the strict geometric bound by brute force, and the distance
-of the dequantised statistics from the fp32 ones (at most half an e4m3 step).
+nearest-value search over all codes (fp32 inputs, and float64 points next to
+every rounding boundary), closed forms of the scale and of a constant block,
+codes nearest to numpy's mean and population std, the strict geometric bound
+by brute force, and the distance of the dequantised statistics from the exact
+ones (at most half an e4m3 step).
 A plausible mistake (truncation instead of rounding, a scale off by the max,
 M measured from the fp32 instead of the dequantised centroid, a spread from
 the wrong mean) fails one of them."""
 import math
 
 import numpy as np
+import pytest
+import torch
 
 from oracle import eta_fp8_oracle as fo
 
@@ -40,17 +44,62 @@ def test_e4m3_rounding_is_nearest_even_by_brute_force():
         assert fo.e4m3_decode(np.array([gi], np.uint8))[0] == vals[best[0]], (xi, gi)
 
 
+def _nearest_by_search(x):
+    """Brute force: the e4m3 code whose value is nearest to each float64 x
+    (ties to the even code), saturating at +-448."""
+    codes, vals = _values()
+    out = np.empty(len(x), np.uint8)
+    for n, xi in enumerate(np.asarray(x, np.float64)):
+        xs = min(max(xi, -448.0), 448.0)
+        dist = np.abs(vals - xs)
+        best = np.flatnonzero(dist == dist.min())
+        if len(best) > 1:
+            best = [b for b in best if codes[b] % 2 == 0] or best
+        c = int(codes[best[0]])
+        if vals[best[0]] == 0.0:  # zero takes the value's sign
+            c = 0x80 if np.signbit(xi) else 0x00
+        out[n] = c
+    return out
+
+
+def test_e4m3_rounding_at_float64_points_next_to_every_boundary():
+    # every rounding boundary (midpoint of neighbouring values), the points a
+    # hair above and below it in float64, and the saturation region
+    codes, vals = _values()
+    pos = np.unique(vals[vals >= 0])
+    mids = (pos[:-1] + pos[1:]) / 2
+    eps = 2.0 ** -40
+    x = np.concatenate([mids, mids * (1 + eps), mids * (1 - eps), pos, [448.0 * (1 + eps), 460.0, 470.0, 1e300]])
+    x = np.concatenate([x, -x, [-1e-300, -0.0, 0.0]])
+    np.testing.assert_array_equal(fo.e4m3_encode(x), _nearest_by_search(x))
+
+
 def test_scale_maps_the_largest_coordinate_to_448():
     rng = np.random.default_rng(1)
     k = rng.standard_normal((64, 16)).astype(np.float32)
     s = fo.block_summary_fp8(k)
-    mean = np.float32(0)
-    acc = np.zeros(16, np.float32)
-    for r in range(64):
-        acc = (acc + k[r]).astype(np.float32)
-    mean = (acc / np.float32(64)).astype(np.float32)
-    assert s["mu_scale"] == np.float32(np.abs(mean).max() / np.float32(448))
+    mean = np.mean(k.astype(np.float64), axis=0)
+    assert s["mu_scale"] == np.float32(np.abs(mean).max() / 448.0)
     assert np.abs(fo.e4m3_decode(s["mu_code"])).max() == 448.0
+    std = np.std(k.astype(np.float64), axis=0, ddof=0)
+    assert s["sigma_scale"] == np.float32(std.max() / 448.0)
+
+
+@pytest.mark.parametrize("n,d,dtype", [(64, 128, "bf16"), (7, 32, "f32"), (128, 64, "bf16"), (1, 16, "f32")])
+def test_codes_are_nearest_to_the_exact_statistics(n, d, dtype):
+    # codes of the centroid and the spread are the e4m3 values nearest to
+    # numpy's mean and population std divided by the block's scale
+    rng = np.random.default_rng(n + d)
+    k = torch.from_numpy((rng.standard_normal((n, d)) * 10.0 ** rng.uniform(-2, 1, d)
+                          + rng.uniform(-2, 2, d)).astype(np.float32))
+    if dtype == "bf16":
+        k = k.to(torch.bfloat16)
+    kf = k.float().numpy().astype(np.float64)
+    s = fo.block_summary_fp8(k)
+    for name, val in (("mu", np.mean(kf, axis=0)), ("sigma", np.std(kf, axis=0, ddof=0))):
+        scl = float(s[name + "_scale"])
+        np.testing.assert_array_equal(s[name + "_code"], _nearest_by_search(val / scl), err_msg=name)
+        np.testing.assert_array_equal(s[name], fo.e4m3_decode(s[name + "_code"]).astype(np.float64) * scl)
 
 
 def test_constant_block():
@@ -83,9 +132,9 @@ def test_dequantised_statistics_within_half_a_step():
     s = fo.block_summary_fp8(k)
     mean = k.astype(np.float64).mean(axis=0)
     std = k.astype(np.float64).std(axis=0)
-    # e4m3 keeps 3 fraction bits: half a step is 2^-4 relative, plus the
-    # subnormal step 2^-9 of the scaled range, plus fp32 accumulation error
-    tol_mu = 2.0 ** -4 * np.abs(mean) + 2.0 ** -9 * float(s["mu_scale"]) + 1e-5
-    tol_sd = 2.0 ** -4 * std + 2.0 ** -9 * float(s["sigma_scale"]) + 1e-5
+    # e4m3 keeps 3 fraction bits: half a step is 2^-4 relative, plus half the
+    # subnormal step 2^-10 of the scaled range
+    tol_mu = 2.0 ** -4 * np.abs(mean) + 2.0 ** -10 * float(s["mu_scale"])
+    tol_sd = 2.0 ** -4 * std + 2.0 ** -10 * float(s["sigma_scale"])
     assert np.all(np.abs(s["mu"] - mean) <= tol_mu)
     assert np.all(np.abs(s["sigma"] - std) <= tol_sd)

@@ -80,6 +80,41 @@ def test_sequence_summary_tail_block():
     np.testing.assert_array_equal(mu[1], mu1)
 
 
+@pytest.mark.parametrize("T,b,d,dtype", [(256, 64, 16, "bf16"), (200, 64, 8, "f32"), (130, 16, 32, "f32"),
+                                         (512, 128, 128, "bf16"), (97, 1, 4, "f32"), (64, 64, 8, "f32")])
+def test_sequence_summary_every_full_block(T, b, d, dtype):
+    # Every block of the vectorised path (full blocks) and the tail against
+    # library statistics of that block alone: numpy mean, numpy population
+    # std (ddof = 0) and a brute-force per-row norm loop around the stored
+    # fp16 centroid.  A sample std (ddof = 1), a spread around the rounded
+    # centroid, or M measured from the unrounded mean each fail here.
+    # Coordinates spread from 1e-3 to 4 around offsets up to 3: where the
+    # spread is small next to the offset, the fp16 rounding of the centroid
+    # moves a spread measured around it by more than a half ulp.
+    rng = np.random.default_rng(T * 7 + b * 3 + d)
+    spread = 10.0 ** rng.uniform(-3, 0.6, size=d)
+    k = torch.from_numpy((rng.standard_normal((T, d)) * spread + rng.uniform(-3, 3, size=d)).astype(np.float32))
+    if dtype == "bf16":
+        k = k.to(torch.bfloat16)
+    mu, sg, M = oracle.sequence_summary(k, T, b)
+    kf = k.float().numpy().astype(np.float64)
+    nb = (T + b - 1) // b
+    assert mu.shape == (nb, d) and sg.shape == (nb, d) and M.shape == (nb,)
+    for j in range(nb):
+        rows = kf[j * b:min(T, (j + 1) * b)]
+        np.testing.assert_array_equal(mu[j], np.mean(rows, axis=0).astype(np.float16), err_msg=f"block {j}")
+        np.testing.assert_array_equal(sg[j], np.std(rows, axis=0, ddof=0).astype(np.float16), err_msg=f"block {j}")
+        centre = [float(x) for x in mu[j].astype(np.float64)]
+        brute = 0.0
+        for r in rows:
+            brute = max(brute, math.sqrt(sum((float(r[e]) - centre[e]) ** 2 for e in range(d))))
+        # M is the smallest fp32 value at or above the exact norm
+        assert float(M[j]) >= brute, f"block {j}"
+        assert float(np.nextafter(M[j], np.float32(-np.inf))) < brute, f"block {j}"
+    if T % b == 0 and b > 1:
+        assert sg[-1].any()  # a full last block is not summarised as a 1-row block
+
+
 def test_metadata_overhead_golden():
     g = _golden("metadata_overhead.json")
     rec = oracle.metadata_record_bytes(g["head_dim"])
