@@ -20,11 +20,34 @@ __host__ __device__ inline size_t block_stage_bytes(int b, int d, int elt) {
   return static_cast<size_t>(b) * d * elt;
 }
 
-// One e4m3 code (nearest, ties to even, saturating at +-448).
-__device__ __forceinline__ uint8_t f32_to_e4m3(float x) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.f), "f"(x));
-  return static_cast<uint8_t>(r & 0xffu);
+// Nearest e4m3 code of a float64 value, from the format's definition (sign
+// bit, 4 exponent bits with bias 7, 3 fraction bits, subnormal step 2^-9):
+// ties to the even code, saturating at +-448; a negative value that rounds
+// to zero keeps its sign (code 0x80).
+__device__ __forceinline__ uint8_t f64_to_e4m3(double x) {
+  const double a = fmin(fabs(x), 448.0);
+  int code;
+  if (a < 0.015625) {
+    code = static_cast<int>(rint(a * 512.0));  // multiples of 2^-9; 8 is 2^-6 (code 0x08)
+  } else {
+    // a = m 2^e with m in [1, 2) and -6 <= e <= 8 (a normal double)
+    int e = static_cast<int>((__double_as_longlong(a) >> 52) & 0x7ff) - 1023;
+    const double m8 = a * __longlong_as_double(static_cast<long long>(1023 + 3 - e) << 52);  // m * 8, exact
+    double q = rint(m8);  // 8..16: the mantissa to 3 fraction bits, ties to even
+    if (q == 16.0) {
+      q = 8.0;
+      ++e;
+    }
+    code = (e + 7) * 8 + static_cast<int>(q) - 8;
+  }
+  code = min(code, 0x7E);
+  return static_cast<uint8_t>(signbit(x) ? (code | 0x80) : code);
+}
+
+__device__ __forceinline__ uint16_t f64_to_fp16_rn(double x) {
+  uint16_t h;
+  asm("cvt.rn.f16.f64 %0, %1;" : "=h"(h) : "d"(x));
+  return h;
 }
 
 __device__ __forceinline__ float e4m3_to_f32(uint8_t code) {
@@ -34,26 +57,30 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t code) {
 }
 
 // Largest of v over the CTA's threads (kThreads), in every thread.
-__device__ __forceinline__ float cta_max(float v, float* s_w) {
+__device__ __forceinline__ double cta_max(double v, double* s_w) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
   const int w = threadIdx.x >> 5;
   __syncthreads();  // s_w free from any earlier use
   if ((threadIdx.x & 31) == 0) s_w[w] = v;
   __syncthreads();
-  float m = s_w[0];
-  for (int k = 1; k < kThreads / 32; ++k) m = fmaxf(m, s_w[k]);
+  double m = s_w[0];
+  for (int k = 1; k < kThreads / 32; ++k) m = fmax(m, s_w[k]);
   return m;
 }
 
 // Summary of block j of (sequence i, KV head g) over its n present rows,
-// staged once in shared memory (raw K bytes).  Pass 1: mean per coordinate;
-// pass 2: population variance around the fp32 mean; pass 3: max over rows of
-// ||k - mu~||^2 with mu~ the stored centroid.  All accumulation in fp32
-// (Appendix F.2 promotes squares and dot products to fp32).  In the FP8
-// format every step is one correctly rounded fp32 operation in row order
-// (no contraction), the scale maps the largest magnitude to 448 and the code
-// is the nearest e4m3 value, so the codes are reproducible exactly.
+// staged once in shared memory (raw K bytes).  Every statistic is evaluated
+// in float64 from the exact inputs: pass 1 the mean per coordinate, pass 2
+// the population variance around it, pass 3 the largest distance of a row
+// from the stored (dequantised) centroid.  The stored values are then the
+// correctly rounded statistics: fp16 (nearest) for the centroid and spread;
+// in the FP8 format the fp32 scale nearest to (largest magnitude) / 448 and
+// the e4m3 code nearest to statistic / scale; M rounded up to fp32 after an
+// inflation that covers the float64 rounding of the distance, so that it
+// never falls below the exact distance.  With sums of at most 128 bf16 rows
+// (or fp32 rows of moderate range) the float64 sums are exact, so the stored
+// metadata does not depend on the summation order.
 template <int FMT>
 __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n, uint8_t* stage) {
   const int d = a.d, t = threadIdx.x;
@@ -64,8 +91,8 @@ __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.k) + row0 * d * a.elt);
   const int nvec = n * d * a.elt / 16;
   for (int x = t; x < nvec; x += kThreads) reinterpret_cast<uint4*>(stage)[x] = src[x];
-  __shared__ float s_mu[128];
-  __shared__ float s_wmax[kThreads / 32];
+  __shared__ double s_mu[128];
+  __shared__ double s_wmax[kThreads / 32];
   __syncthreads();
   auto at = [&](int r, int e) -> float {
     const size_t idx = static_cast<size_t>(r) * d + e;
@@ -91,45 +118,50 @@ __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n
     if (t == 0) a.max_norm[bo] = 0.f;
     return;
   }
+  // Passes 1 and 2, one coordinate per thread; four interleaved partial sums
+  // shorten the dependent chains.
+  double mean = 0.0, sd = 0.0;
+  if (t < d) {
+    double s4[4] = {0.0, 0.0, 0.0, 0.0};
+    int r = 0;
+    for (; r + 4 <= n; r += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) s4[u] += static_cast<double>(at(r + u, t));
+    }
+    for (; r < n; ++r) s4[0] += static_cast<double>(at(r, t));
+    mean = ((s4[0] + s4[1]) + (s4[2] + s4[3])) / static_cast<double>(n);
+    double q4[4] = {0.0, 0.0, 0.0, 0.0};
+    for (r = 0; r + 4 <= n; r += 4) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const double x = static_cast<double>(at(r + u, t)) - mean;
+        q4[u] = fma(x, x, q4[u]);
+      }
+    }
+    for (; r < n; ++r) {
+      const double x = static_cast<double>(at(r, t)) - mean;
+      q4[0] = fma(x, x, q4[0]);
+    }
+    sd = sqrt(((q4[0] + q4[1]) + (q4[2] + q4[3])) / static_cast<double>(n));
+  }
   if (FMT == ETA_META_FP16) {
     if (t < d) {
-      float sum = 0.f;
-      for (int r = 0; r < n; ++r) sum += at(r, t);
-      const float mean = sum / static_cast<float>(n);
-      float ss = 0.f;
-      for (int r = 0; r < n; ++r) {
-        const float x = at(r, t) - mean;
-        ss = fmaf(x, x, ss);
-      }
-      const float sd = sqrtf(ss / static_cast<float>(n));
-      const uint16_t mu_h = dev::f32_to_fp16_rn(mean);
+      const uint16_t mu_h = f64_to_fp16_rn(mean);
       static_cast<uint16_t*>(a.mu)[bo * d + t] = mu_h;
-      static_cast<uint16_t*>(a.sigma)[bo * d + t] = dev::f32_to_fp16_rn(sd);
-      s_mu[t] = dev::fp16_to_f32(mu_h);
+      static_cast<uint16_t*>(a.sigma)[bo * d + t] = f64_to_fp16_rn(sd);
+      s_mu[t] = static_cast<double>(dev::fp16_to_f32(mu_h));
     }
   } else {
-    float mean = 0.f, sd = 0.f;
+    const double mmax = cta_max(fabs(mean), s_wmax);
+    const double smax = cta_max(sd, s_wmax);
+    const float mu_scale = mmax > 0.0 ? __double2float_rn(mmax / 448.0) : 1.f;
+    const float sd_scale = smax > 0.0 ? __double2float_rn(smax / 448.0) : 1.f;
     if (t < d) {
-      float sum = 0.f;
-      for (int r = 0; r < n; ++r) sum = __fadd_rn(sum, at(r, t));
-      mean = __fdiv_rn(sum, static_cast<float>(n));
-      float ss = 0.f;
-      for (int r = 0; r < n; ++r) {
-        const float x = __fsub_rn(at(r, t), mean);
-        ss = __fadd_rn(ss, __fmul_rn(x, x));
-      }
-      sd = __fsqrt_rn(__fdiv_rn(ss, static_cast<float>(n)));
-    }
-    const float mmax = cta_max(fabsf(mean), s_wmax);
-    const float smax = cta_max(sd, s_wmax);
-    const float mu_scale = mmax > 0.f ? __fdiv_rn(mmax, 448.f) : 1.f;
-    const float sd_scale = smax > 0.f ? __fdiv_rn(smax, 448.f) : 1.f;
-    if (t < d) {
-      const uint8_t mc = f32_to_e4m3(__fdiv_rn(mean, mu_scale));
-      const uint8_t sc = f32_to_e4m3(__fdiv_rn(sd, sd_scale));
+      const uint8_t mc = f64_to_e4m3(mean / static_cast<double>(mu_scale));
+      const uint8_t sc = f64_to_e4m3(sd / static_cast<double>(sd_scale));
       static_cast<uint8_t*>(a.mu)[bo * d + t] = mc;
       static_cast<uint8_t*>(a.sigma)[bo * d + t] = sc;
-      s_mu[t] = __fmul_rn(e4m3_to_f32(mc), mu_scale);
+      s_mu[t] = static_cast<double>(e4m3_to_f32(mc)) * static_cast<double>(mu_scale);  // exact
     }
     if (t == 0) {
       a.mu_scale[bo] = mu_scale;
@@ -137,26 +169,38 @@ __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n
     }
   }
   __syncthreads();
-  // M_B: warp w takes rows w, w+4, ...; lanes split the coordinates.
+  // Pass 3, M_B: warp w takes rows w, w + 4, ... two at a time; lanes split
+  // the coordinates.  The differences k - mu~ are exact in float64 and the
+  // sum of d squares has a relative error below 2^-48, which the 2^-47
+  // inflation (rounded up) covers before the upward rounding to fp32.
   const int w = t >> 5, lane = t & 31;
-  float best = 0.f;
-  for (int r = w; r < n; r += kThreads / 32) {
-    float ss = 0.f;
+  constexpr int kW = kThreads / 32;
+  double best = 0.0;
+  for (int r = w; r < n; r += 2 * kW) {
+    const int r2 = r + kW < n ? r + kW : r;
+    double s1 = 0.0, s2 = 0.0;
     for (int e = lane; e < d; e += 32) {
-      const float x = at(r, e) - s_mu[e];
-      ss = fmaf(x, x, ss);
+      const double x1 = static_cast<double>(at(r, e)) - s_mu[e];
+      const double x2 = static_cast<double>(at(r2, e)) - s_mu[e];
+      s1 = fma(x1, x1, s1);
+      s2 = fma(x2, x2, s2);
     }
-    best = fmaxf(best, dev::warp_sum(ss));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    best = fmax(best, fmax(s1, s2));
   }
   if (lane == 0) s_wmax[w] = best;
   __syncthreads();
   if (t == 0) {
-    float m2 = s_wmax[0];
-    for (int k = 1; k < kThreads / 32; ++k) m2 = fmaxf(m2, s_wmax[k]);
-    // fp32 rounding of d squares and a 5-level tree is below 16 ulp; the
-    // directed roundings and the 2^-18 inflation keep M_B >= the exact norm.
-    const float m = __fmul_ru(__fsqrt_ru(m2), 1.0f + 3.814697265625e-06f);
-    a.max_norm[bo] = m;
+    double m2 = s_wmax[0];
+    for (int k = 1; k < kW; ++k) m2 = fmax(m2, s_wmax[k]);
+    const double m = __dmul_ru(sqrt(m2), 1.0 + 0x1p-47);
+    float mf;
+    asm("cvt.rp.f32.f64 %0, %1;" : "=f"(mf) : "d"(m));
+    a.max_norm[bo] = mf;
   }
 }
 

@@ -2,15 +2,20 @@
 decode workloads that target a GQA-union admitted density.
 
 Calls only the CPU oracle (block summaries and block scores) and the seeded
-input generator.  For each workload the same score quantile p is used for every
-query head; p is bisected until the union density (always-loaded blocks
-included) reaches the target.  Each head's effective threshold tau~ is then
-placed in the middle of the widest gap between neighbouring block scores near
-its quantile, so that no block score sits close to the threshold (fp32
-evaluation on the device cannot flip a decision).
+input generator.  For the density-targeted workloads the same score quantile p
+is used for every query head; p is bisected until the union density
+(always-loaded blocks included) reaches the target.  Each head's effective
+threshold tau~ is then placed in the middle of the gap between neighbouring
+block scores that is nearest to its quantile among the gaps wide enough that
+every block score stays at least MIN_MARGIN away from tau~ (a guard band: the
+device evaluates the bound in fp32, whose rounding error on these workloads
+is below 2e-5, so no decision can flip).  The batched workload draws its
+per-head constants U[0.5, 2.0]; each is moved to the middle of the nearest
+such gap of that head's scores over all sequences.
 
 Learned mode stores b_tau = tau~ + a - w_tau . q (rounded to fp32);
-calibrated mode stores c_tau = tau~ + a.
+calibrated mode stores c_tau = tau~ + a (rounded to fp32).  The margins are
+measured again after the rounding.
 
 Usage:  python tests/golden/make_thresholds.py [name ...]
 """
@@ -27,7 +32,8 @@ import oracle  # noqa: E402
 import workloads  # noqa: E402
 
 OUT = os.path.join(os.path.dirname(os.path.abspath(__file__)), "thresholds.json")
-TARGETS = {"c2_single": 0.38, "c3_long": 0.38, "c4_max": 0.38}
+TARGETS = {"c2_single": 0.38, "c3_long": 0.38, "c4_max": 0.38, "c5_batched": None}
+MIN_MARGIN = 1e-4
 
 
 def _scores(wl, summary):
@@ -58,6 +64,22 @@ def _tau_for_count(sorted_desc, k):
     return 0.5 * (sorted_desc[k - 1] + sorted_desc[k])
 
 
+def _guarded_tau(sorted_desc, near):
+    """The middle of the gap between neighbouring scores (or beyond the
+    extremes) nearest to `near` whose half-width is at least MIN_MARGIN."""
+    s = sorted_desc
+    cands = []
+    if len(s) == 0:
+        return near
+    cands.append(s[0] + MIN_MARGIN)      # above every score
+    cands.append(s[-1] - MIN_MARGIN)     # below every score
+    gaps = s[:-1] - s[1:]
+    ok = np.flatnonzero(gaps >= 2 * MIN_MARGIN)
+    cands.extend(0.5 * (s[ok] + s[ok + 1]))
+    cands = np.asarray(cands)
+    return float(cands[np.argmin(np.abs(cands - near))])
+
+
 def _union_density(wl, scores, screened_n, taus):
     G = wl.group
     tot = 0.0
@@ -72,15 +94,47 @@ def _union_density(wl, scores, screened_n, taus):
     return tot / (wl.batch * wl.n_kv_heads)
 
 
+def _finish(entry, wl, scores, screened_n, taus):
+    real_margin = min(float(np.min(np.abs(scores[key] - taus[key]))) for key in scores if len(scores[key]))
+    entry["min_margin"] = real_margin
+    assert real_margin >= MIN_MARGIN * 0.999, real_margin
+    entry["union_density"] = _union_density(wl, scores, screened_n, taus)
+    head_dens = []
+    for (i, h), sc in scores.items():
+        ns, nb = screened_n[i]
+        head_dens.append(((sc >= taus[(i, h)]).sum() + nb - ns) / nb)
+    entry["mean_head_density"] = float(np.mean(head_dens))
+    return entry
+
+
+def _place_constants(wl, scores, screened_n):
+    """Calibrated constants drawn per head (the workload's own draw), each
+    moved into the nearest guard-banded gap of that head's scores pooled over
+    the batch (the constant is shared by every sequence)."""
+    pooled = {}
+    for (i, h), sc in scores.items():
+        pooled.setdefault(h, []).append(sc)
+    c32 = np.zeros(wl.n_q_heads, np.float32)
+    for h in range(wl.n_q_heads):
+        sd = np.sort(np.concatenate(pooled[h]))[::-1]
+        tt = _guarded_tau(sd, float(wl.c_tau[h]) - wl.offset_a)
+        c32[h] = np.float32(tt + wl.offset_a)
+    taus = {(i, h): oracle.threshold_calibrated(c32[h], wl.offset_a) for (i, h) in scores}
+    entry = {"drawn_c_tau": [float(x) for x in wl.c_tau], "c_tau": [float(x) for x in c32]}
+    return _finish(entry, wl, scores, screened_n, taus)
+
+
 def calibrate(name, seed=0):
-    wl = workloads.make(name, seed)
+    wl = workloads.make(name, seed, raw_thresholds=True)
     target = TARGETS[name]
     summary = oracle.summarize(wl.k, wl.seq_lens, wl.block_size)
     scores, screened_n = _scores(wl, summary)
+    if target is None:
+        return _place_constants(wl, scores, screened_n)
     srt = {key: np.sort(val)[::-1] for key, val in scores.items()}
 
     def taus_for(p):
-        return {key: _tau_for_count(s, int(round(p * len(s)))) for key, s in srt.items()}
+        return {key: _guarded_tau(s, _tau_for_count(s, int(round(p * len(s))))) for key, s in srt.items()}
 
     lo, hi = 0.0, 1.0
     for _ in range(40):
@@ -90,19 +144,7 @@ def calibrate(name, seed=0):
         else:
             hi = mid
     p = 0.5 * (lo + hi)
-    taus = {}
-    margins = {}
-    for key, s in srt.items():
-        n = len(s)
-        k0 = int(round(p * n))
-        w = max(2, int(0.01 * n))
-        best_k, best_gap = k0, -1.0
-        for k in range(max(1, k0 - w), min(n - 1, k0 + w) + 1):
-            gap = s[k - 1] - s[k]
-            if gap > best_gap:
-                best_k, best_gap = k, gap
-        taus[key] = _tau_for_count(s, best_k)
-        margins[key] = best_gap / 2
+    taus = taus_for(p)
     entry = {"target_union_density": target, "quantile": p}
     if wl.tau_mode == "learned":
         b = np.zeros(wl.n_q_heads, np.float64)
@@ -120,15 +162,7 @@ def calibrate(name, seed=0):
         entry["c_tau"] = [float(x) for x in c32]
         for h in range(wl.n_q_heads):
             taus[(0, h)] = oracle.threshold_calibrated(c32[h], wl.offset_a)
-    real_margin = min(float(np.min(np.abs(scores[key] - taus[key]))) for key in scores)
-    entry["min_margin"] = real_margin
-    entry["union_density"] = _union_density(wl, scores, screened_n, taus)
-    head_dens = []
-    for (i, h), sc in scores.items():
-        ns, nb = screened_n[i]
-        head_dens.append(((sc >= taus[(i, h)]).sum() + nb - ns) / nb)
-    entry["mean_head_density"] = float(np.mean(head_dens))
-    return entry
+    return _finish(entry, wl, scores, screened_n, taus)
 
 
 def main(names):

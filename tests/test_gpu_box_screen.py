@@ -1,8 +1,8 @@
 """The comparison coordinate-box (Quest) screen on the device against the box
 oracle: per-coordinate fp16 extrema rounded outward bit-exact, and decode
 steps screened with the box bound under the same comparison rules as the
-dual bound (identical admitted sets up to fp32-band decisions, outputs within
-tolerance)."""
+dual bound (identical admitted sets up to decisions inside the fp32 error
+bound, outputs within tolerance)."""
 import numpy as np
 import pytest
 import torch
@@ -55,6 +55,7 @@ def _oracle_box_decode(wl):
                                                                   wl.block_size, adm, tt, wl.scale, wl.beta)
     r["admitted_count"] = r["admitted"].sum(axis=2)
     r["union_count"] = r["union"].sum(axis=2)
+    r["kmin"], r["kmax"] = box["kmin"], box["kmax"]  # the metadata this screen read
     return r
 
 

@@ -1,8 +1,11 @@
 """FP8 block metadata on the device against the FP8 oracle: codes and scales
-bit-exact (both sides decide each code in the kernel's fp32 order), M within
-fp32 rounding and a true bound for the device's own dequantised centroid, the
-append path refreshing only the tail block, and whole decode steps screened
-with FP8 metadata under the same comparison rules as the fp16 metadata."""
+bit-exact (the device evaluates the statistics, the scale and each quotient in
+float64 and rounds once, as the oracle's definition does; a code may differ
+only where the exact quotient lies within a float64 hair of an e4m3 rounding
+boundary, counted and printed), M equal or one fp32 step above and a true
+bound for the device's own dequantised centroid, the append path refreshing
+only the tail block, and whole decode steps screened with FP8 metadata under
+the same comparison rules as the fp16 metadata."""
 import numpy as np
 import pytest
 import torch
@@ -10,7 +13,7 @@ import torch
 import learned_threshold_sparse_b200 as eta
 import oracle
 import workloads
-from etatest import compare, gpu_decode, oracle_decode, upload
+from etatest import assert_bits_equal, compare, gpu_decode, oracle_decode, upload
 from oracle import eta_fp8_oracle as fo
 
 pytestmark = pytest.mark.gpu
@@ -28,20 +31,23 @@ def _fp8_summary(wl, t):
 
 def _check_blocks(wl, summ, ref, blocks=None):
     got = {k: v.cpu().numpy() for k, v in summ.items()}
+    n_exc = 0
     for i, T in enumerate(wl.seq_lens):
         nb = wl.n_blocks(i)
         for g in range(wl.n_kv_heads):
             js = range(nb) if blocks is None else blocks(i)
             for j in js:
-                np.testing.assert_array_equal(got["mu"][i, g, j], ref["mu_code"][i, g, j])
-                np.testing.assert_array_equal(got["sigma"][i, g, j], ref["sigma_code"][i, g, j])
-                assert got["mu_scale"][i, g, j] == ref["mu_scale"][i, g, j]
-                assert got["sigma_scale"][i, g, j] == ref["sigma_scale"][i, g, j]
-                m_g, m_r = float(got["max_norm"][i, g, j]), float(ref["max_norm"][i, g, j])
-                assert m_r * (1 - 1e-6) <= m_g <= m_r * (1 + 2e-5)
                 rows = oracle.as_f64(wl.k[i, g, j * wl.block_size:min(T, (j + 1) * wl.block_size)])
+                for name, stat in (("mu", rows.mean(axis=0)), ("sigma", rows.std(axis=0))):
+                    scl = float(ref[name + "_scale"][i, g, j])
+                    assert got[name + "_scale"][i, g, j] == ref[name + "_scale"][i, g, j], (name, i, g, j)
+                    n_exc += assert_bits_equal(got[name][i, g, j], ref[name + "_code"][i, g, j], stat / scl,
+                                               fo.e4m3_encode, f"{name} codes seq {i} kv {g} block {j}")
+                m_g, m_r = got["max_norm"][i, g, j], ref["max_norm"][i, g, j]
+                assert m_g == m_r or m_g == np.nextafter(m_r, np.float32(np.inf)), (i, g, j, m_g, m_r)
                 mu_dev = fo.e4m3_decode(got["mu"][i, g, j]).astype(np.float64) * float(got["mu_scale"][i, g, j])
-                assert np.sqrt(((rows - mu_dev) ** 2).sum(axis=1)).max() <= m_g
+                assert np.sqrt(((rows - mu_dev) ** 2).sum(axis=1)).max() <= float(m_g)
+    print(f"fp8 codes excused next to a rounding boundary: {n_exc}")
 
 
 @pytest.mark.parametrize("case", [

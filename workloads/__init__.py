@@ -226,7 +226,7 @@ def single(seed: int = 0, T: int = 32768) -> Workload:
                   v=_to_kv(v, BF16), w_tau=w_tau, b_tau=None, c_tau=None,
                   scale=1.0 / math.sqrt(d), planted={kk: sorted(vv) for kk, vv in planted.items()},
                   target_union_density=0.38)
-    return _attach_thresholds(wl)
+    return wl
 
 
 def _cluster_keys(rng, T: int, d: int, b: int, n_centres: int = 64, spread: float = 0.3,
@@ -255,7 +255,7 @@ def long(seed: int = 0, T: int = 131072) -> Workload:
                   tau_mode=TAU_CALIBRATED, q=_to_kv(q, BF16), k=_to_kv(k, BF16),
                   v=_to_kv(v, BF16), w_tau=None, b_tau=None, c_tau=None,
                   scale=1.0 / math.sqrt(d), target_union_density=0.38)
-    return _attach_thresholds(wl)
+    return wl
 
 
 def max_context(seed: int = 0, T: int = 524288) -> Workload:
@@ -283,7 +283,7 @@ def max_context(seed: int = 0, T: int = 524288) -> Workload:
                   tau_mode=TAU_LEARNED, q=_to_kv(q, BF16), k=_to_kv(k, BF16),
                   v=_to_kv(v, BF16), w_tau=w_tau, b_tau=None, c_tau=None,
                   scale=1.0 / math.sqrt(d), planted=planted, target_union_density=0.38)
-    return _attach_thresholds(wl)
+    return wl
 
 
 def batched(seed: int = 0, batch: int = 8, t_lo: int = 16384, t_hi: int = 131072) -> Workload:
@@ -301,6 +301,8 @@ def batched(seed: int = 0, batch: int = 8, t_lo: int = 16384, t_hi: int = 131072
         for g in range(Hkv):
             k[i, g, :T] = _to_kv(_cluster_keys(rng, T, d, b, noise_key=[5, seed, 0, i, g]), BF16)
             v[i, g, :T] = _to_kv(_normal_big([5, seed, 1, i, g], (T, d)), BF16)
+    # drawn here; the stored constants move each draw into a guard-banded gap
+    # of that head's block scores (tests/golden/make_thresholds.py)
     c_tau = rng.uniform(0.5, 2.0, size=Hq).astype(np.float32)
     return Workload(name="c5_batched", seed=seed, batch=B, n_q_heads=Hq, n_kv_heads=Hkv,
                     head_dim=d, block_size=b, max_ctx=Tmax, seq_lens=lens, dtype=BF16,
@@ -420,5 +422,9 @@ CONFIGS = {
 }
 
 
-def make(name: str, seed: int = 0, **kw) -> Workload:
-    return CONFIGS[name](seed=seed, **kw)
+def make(name: str, seed: int = 0, raw_thresholds: bool = False, **kw) -> Workload:
+    """Workload `name` with its stored thresholds (tests/golden/thresholds.json)
+    applied; raw_thresholds=True keeps the generator's own draws (the input of
+    the script that writes that file)."""
+    wl = CONFIGS[name](seed=seed, **kw)
+    return wl if raw_thresholds else _attach_thresholds(wl)
