@@ -239,6 +239,11 @@ eta_status eta_decode(const eta_decode_params* p, void* stream);
 /* Size of the fixed device scratch used by eta_decode_noalloc (8 MiB). */
 #define ETA_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
 
+/* Bits of the device status word (eta_decode_noalloc's device_status). */
+#define ETA_DEVICE_STATUS_TIMEOUT 1u  /* a bounded device-side wait ran out  */
+#define ETA_DEVICE_STATUS_RANGE 2u    /* a device-resident length or page id
+                                         was out of range and was clamped    */
+
 /*
  * eta_decode_noalloc - eta_decode for callers that cannot allocate device
  * memory.  No counterpart in the paper: this is a deployment variant.
@@ -251,20 +256,25 @@ eta_status eta_decode(const eta_decode_params* p, void* stream);
  * ETA_NOALLOC_SCRATCH_BYTES that the library declares in device memory
  * (every GPU that loads the library holds it until the process exits).  It
  * calls no cudaMalloc, cudaFree or allocating library routine.
- *   - The first call on a device looks up the array's device address (with
- *     that device current) and caches it; make that first call before any
- *     stream capture.
+ *   - Every call looks up the array's device address in the current
+ *     device's context (with that device current).  The first call on a
+ *     device may load the library's device code; make it before any stream
+ *     capture.
  *   - Every call shares the one array, which keeps the last call's contents.
  *     Calls that overlap on the GPU (different streams, or different host
  *     threads without ordering) race on it and give wrong results.
- *   - The device status word lives in that array: it is cleared at the start
- *     of every call and cannot be read back (eta_read_device_status needs a
- *     caller workspace).
+ *   - The step's device status word lives in that array and is cleared at
+ *     the start of every call.  device_status, when not NULL, is a 4-byte
+ *     aligned word in device memory that receives it after the step (stream-
+ *     ordered): 0, or ETA_DEVICE_STATUS_* bits.  Without it, device-side
+ *     problems (a bounded wait that ran out, a seq_len outside [0, max_ctx]
+ *     that was clamped, a page id outside the pool) go unreported.
  * Errors: as eta_decode, plus ETA_ERR_WORKSPACE when
- * eta_decode_workspace_size(p) exceeds ETA_NOALLOC_SCRATCH_BYTES, and
- * ETA_ERR_CUDA if the array's address cannot be obtained.
+ * eta_decode_workspace_size(p) exceeds ETA_NOALLOC_SCRATCH_BYTES,
+ * ETA_ERR_INVALID_ARG for a misaligned device_status, and ETA_ERR_CUDA if the
+ * array's address cannot be obtained or the status copy fails.
  */
-eta_status eta_decode_noalloc(const eta_decode_params* p, void* stream);
+eta_status eta_decode_noalloc(const eta_decode_params* p, unsigned* device_status, void* stream);
 
 /*
  * eta_decode_graph_* - one decode step captured once into a CUDA graph and

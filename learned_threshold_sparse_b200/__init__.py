@@ -132,7 +132,7 @@ def _load():
     lib.eta_decode_workspace_size.restype = ctypes.c_int
     lib.eta_decode.argtypes = [P(eta_decode_params), ctypes.c_void_p]
     lib.eta_decode.restype = ctypes.c_int
-    lib.eta_decode_noalloc.argtypes = [P(eta_decode_params), ctypes.c_void_p]
+    lib.eta_decode_noalloc.argtypes = [P(eta_decode_params), ctypes.c_void_p, ctypes.c_void_p]
     lib.eta_decode_noalloc.restype = ctypes.c_int
     lib.eta_decode_graph_create.argtypes = [P(eta_decode_params), P(ctypes.c_void_p)]
     lib.eta_decode_graph_create.restype = ctypes.c_int
@@ -167,6 +167,8 @@ SYMBOLS = ("eta_block_summary_update", "eta_append_kv", "eta_decode_workspace_si
            "eta_read_device_status", "eta_diag_wait_timeout", "eta_prefill", "eta_calibration_histogram", "eta_calibrate_constants",
            "eta_status_string", "eta_build_info")
 
+DEVICE_STATUS_TIMEOUT = 1
+DEVICE_STATUS_RANGE = 2
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
 
 
@@ -352,11 +354,15 @@ def eta_decode(params: eta_decode_params, stream: Optional[torch.cuda.Stream] = 
         raise EtaError(rc, "eta_decode")
 
 
-def eta_decode_noalloc(params: eta_decode_params, stream: Optional[torch.cuda.Stream] = None) -> None:
+def eta_decode_noalloc(params: eta_decode_params, device_status: Optional[torch.Tensor] = None,
+                       stream: Optional[torch.cuda.Stream] = None) -> None:
     """eta_decode without a caller workspace, for callers that cannot allocate
     device memory: the library's fixed device scratch is used instead (see
-    include/eta.h).  Calls sharing that scratch must not overlap on the GPU."""
-    rc = _lib.eta_decode_noalloc(ctypes.byref(params), _stream_handle(stream))
+    include/eta.h).  Calls sharing that scratch must not overlap on the GPU.
+    device_status (an int32 device tensor, optional) receives the step's
+    device status bits (DEVICE_STATUS_TIMEOUT, DEVICE_STATUS_RANGE)."""
+    ptr = None if device_status is None else device_status.data_ptr()
+    rc = _lib.eta_decode_noalloc(ctypes.byref(params), ptr, _stream_handle(stream))
     if rc != ETA_OK:
         raise EtaError(rc, "eta_decode_noalloc")
 

@@ -17,8 +17,8 @@ namespace eta {
 __host__ __device__ constexpr int partial_stride(int d) { return d + 4; }
 
 // Device status word bits (first word of the workspace).
-constexpr unsigned kStatusTimeout = 1u;  // a bounded wait ran out
-constexpr unsigned kStatusRange = 2u;    // a device-resident length was clamped
+constexpr unsigned kStatusTimeout = ETA_DEVICE_STATUS_TIMEOUT;  // a bounded wait ran out
+constexpr unsigned kStatusRange = ETA_DEVICE_STATUS_RANGE;      // a device-resident length was clamped
 
 // List entries written by the screen: block id in the low 24 bits, the
 // admitting heads of the group in the high 8 bits.

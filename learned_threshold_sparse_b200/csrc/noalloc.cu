@@ -6,8 +6,6 @@
 // allocation, or a code path where a cudaMalloc would synchronise the whole
 // device.  This variant takes the same parameters but ignores
 // params->workspace / workspace_bytes and uses g_eta_noalloc_scratch instead.
-#include <mutex>
-
 #include "eta_internal.h"
 
 namespace {
@@ -16,30 +14,23 @@ namespace {
 constexpr size_t kNoallocScratchBytes = ETA_NOALLOC_SCRATCH_BYTES;
 __device__ __align__(256) unsigned char g_eta_noalloc_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device.  In host code
-// the array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// Device address of the scratch array in the current device's context.  In
+// host code the array's name is only a host-side stand-in, so the address is
+// looked up with that device current.  It is looked up on every call rather
+// than cached: after a context reset a cached address would point into a
+// context that no longer exists.  The lookup does not touch any stream.
 eta_status scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ETA_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_eta_noalloc_scratch) != cudaSuccess || p == nullptr) return ETA_ERR_CUDA;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_eta_noalloc_scratch) != cudaSuccess || p == nullptr) return ETA_ERR_CUDA;
+  *out = p;
   return ETA_OK;
 }
 
 }  // namespace
 
-extern "C" eta_status eta_decode_noalloc(const eta_decode_params* p, void* stream) {
+extern "C" eta_status eta_decode_noalloc(const eta_decode_params* p, unsigned* device_status, void* stream) {
   if (!p) return ETA_ERR_INVALID_ARG;
+  if (device_status && (reinterpret_cast<uintptr_t>(device_status) % 4) != 0) return ETA_ERR_INVALID_ARG;
   eta_decode_params q = *p;
   q.workspace = nullptr;
   q.workspace_bytes = 0;
@@ -50,11 +41,18 @@ extern "C" eta_status eta_decode_noalloc(const eta_decode_params* p, void* strea
   void* scratch = nullptr;
   st = scratch_address(&scratch);
   if (st != ETA_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
   // The previous call's device status word is cleared; everything else the
   // step reads is rewritten by the step itself (the rescue counters are
   // zeroed inside eta_decode when that mode is on).
-  if (cudaMemsetAsync(scratch, 0, 16, static_cast<cudaStream_t>(stream)) != cudaSuccess) return ETA_ERR_CUDA;
+  if (cudaMemsetAsync(scratch, 0, 16, cs) != cudaSuccess) return ETA_ERR_CUDA;
   q.workspace = scratch;
   q.workspace_bytes = kNoallocScratchBytes;
-  return eta_decode(&q, stream);
+  st = eta_decode(&q, stream);
+  if (st != ETA_OK) return st;
+  // The step's status word, handed to the caller's device word (stream-ordered).
+  if (device_status &&
+      cudaMemcpyAsync(device_status, scratch, sizeof(unsigned), cudaMemcpyDeviceToDevice, cs) != cudaSuccess)
+    return ETA_ERR_CUDA;
+  return ETA_OK;
 }

@@ -1,7 +1,9 @@
 """eta_decode_noalloc: the decode entry point for callers that cannot allocate
 device memory (it uses the library's fixed device scratch instead of a caller
 workspace).  Checked through the C ABI against eta_decode with a workspace on
-two calls in a row with different shapes, and for its size limit."""
+calls in a row with different shapes (a call after one that ran the rescue
+path and left other contents in the shared scratch included), for the status
+word it hands back, and for its size limit."""
 import ctypes
 
 import numpy as np
@@ -26,15 +28,16 @@ def _params(wl, t, summ, out, lse):
 
 
 def test_noalloc_matches_workspace_entry_point_twice():
-    cases = [
-        _case(31, batch=3, n_q_heads=16, n_kv_heads=4, head_dim=128, block_size=64, seq_lens=[3000, 130, 1777],
-              dtype=workloads.BF16, tau_mode="calibrated", key_kind="cluster", tau_bias=1.0),
-        _case(32, batch=2, n_q_heads=8, n_kv_heads=2, head_dim=64, block_size=32, seq_lens=[900, 47],
-              dtype=workloads.F32, tau_bias=1e6).with_params(n_local_blocks=-1),
-    ]
+    first = _case(31, batch=3, n_q_heads=16, n_kv_heads=4, head_dim=128, block_size=64, seq_lens=[3000, 130, 1777],
+                  dtype=workloads.BF16, tau_mode="calibrated", key_kind="cluster", tau_bias=1.0)
+    rescue = _case(32, batch=2, n_q_heads=8, n_kv_heads=2, head_dim=64, block_size=32, seq_lens=[900, 47],
+                   dtype=workloads.F32, tau_bias=1e6).with_params(n_local_blocks=-1)
+    # the third call reuses the first shape after the rescue call, so stale
+    # rescue counters and chunk lists from a different shape sit in the scratch
     lib = eta.library()
     stream = torch.cuda.current_stream()
-    for wl in cases:
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    for wl in (first, rescue, first):
         t = upload(wl)
         summ = gpu_summary(wl, t)
         ref_out = torch.empty_like(t["q"])
@@ -47,12 +50,34 @@ def test_noalloc_matches_workspace_entry_point_twice():
         out = torch.full_like(t["q"], float("nan"))
         lse = torch.full_like(ref_lse, float("nan"))
         p = _params(wl, t, summ, out, lse)  # no workspace: the entry point ignores it anyway
-        rc = lib.eta_decode_noalloc(ctypes.byref(p), ctypes.c_void_p(stream.cuda_stream))
+        status.fill_(-1)
+        rc = lib.eta_decode_noalloc(ctypes.byref(p), ctypes.c_void_p(status.data_ptr()),
+                                    ctypes.c_void_p(stream.cuda_stream))
         assert rc == eta.ETA_OK, eta.eta_status_string(rc)
         torch.cuda.synchronize()
+        assert status.item() == 0
         err = (out.float() - ref_out.float()).abs().max().item()
         assert err <= OUT_TOL[wl.dtype], err
         np.testing.assert_allclose(lse.cpu().numpy(), ref_lse.cpu().numpy(), rtol=1e-5, atol=1e-5)
+
+
+def test_noalloc_hands_back_the_device_status():
+    # a sequence length past the cache capacity is clamped on the device and
+    # reported in the status word; the next clean call reports 0
+    wl = _case(33, batch=1, n_q_heads=4, n_kv_heads=1, head_dim=64, block_size=64, seq_lens=[256],
+               dtype=workloads.BF16, tau_bias=2.0)
+    t = upload(wl)
+    summ = gpu_summary(wl, t)
+    out = torch.empty_like(t["q"])
+    status = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    t["seq"].fill_(257)
+    eta.eta_decode_noalloc(_params(wl, t, summ, out, None), device_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == eta.DEVICE_STATUS_RANGE
+    t["seq"].fill_(256)
+    eta.eta_decode_noalloc(_params(wl, t, summ, out, None), device_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
 
 
 def test_noalloc_rejects_shapes_beyond_the_fixed_scratch():
@@ -67,5 +92,5 @@ def test_noalloc_rejects_shapes_beyond_the_fixed_scratch():
     p.scale, p.beta, p.z, p.n_local_blocks, p.screen_enabled = 0.088, 5.0, 2.0, 2, 1
     need = eta.eta_decode_workspace_size(p)
     assert need > eta.NOALLOC_SCRATCH_BYTES
-    rc = eta.library().eta_decode_noalloc(ctypes.byref(p), None)
+    rc = eta.library().eta_decode_noalloc(ctypes.byref(p), None, None)
     assert rc == eta.ETA_ERR_WORKSPACE
