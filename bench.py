@@ -12,21 +12,28 @@ does not pay for writing back a flush buffer).  Prints ONE JSON line (rank 0).
 
 value  = effective HBM bandwidth of the step: algorithmic bytes (K+V of the
          union-admitted blocks at their real lengths + all block metadata + q,
-         threshold parameters and outputs) / device step time, summed over
-         ranks (each rank decodes its own copy of the batch: weak scaling).
-e2e    = the same bytes / end-to-end step time through the public API: the
-         new token's q, k, v copied in one transfer from pinned host memory,
-         the append (K/V rows written, their block's metadata refreshed), the
-         decode step, the output copied back to pinned host memory; by
-         default one recorded graph (eta_step_graph_create) in which the
-         append kernel reads the new rows from pinned host memory and the
-         decode stores its output into pinned host memory directly; with
-         --launch stream, separate calls with copy-engine transfers.
-roofline = the attention kernel: union K+V bytes per launch / its mean
-         launch time (CUDA events on the launch stream, second run of K
-         steps) vs the measured HBM copy bandwidth.
-cpu_baseline = the CPU oracle (numpy, fp64) on one KV head of the same
-         workload, timed on this host.
+         threshold parameters and outputs) / device step time (mean of the K
+         timed steps), summed over ranks (each rank decodes its own copy of
+         the batch: weak scaling).  latency_us_distribution: a further run of
+         max(100, K) steps (median, p10, p90).
+e2e    = the same bytes / end-to-end step time through the public API with
+         host buffers and a context that grows by one token per step (it
+         crosses a block boundary inside the timed steps): one recorded graph
+         per token (eta_step_graph_create) that copies the new lengths and
+         positions up, appends the new K/V rows read by the append kernel from
+         page-locked host memory (refreshing their block's metadata), decodes,
+         and stores the output into page-locked host memory.
+dense  = the same kernels with the screen off (every block loaded) on the
+         same workload; configs = the other long-context workloads (default
+         c3_long, c5_batched), screened and dense, each with its step time and
+         fraction of the HBM peak.
+roofline = the attention kernel: union K+V bytes per launch / its median
+         isolated launch time (CUDA events on the launch stream between the
+         library's kernels) vs the measured HBM copy bandwidth.
+kernels_us = the isolated per-kernel times and how they add up to the step.
+cpu_baseline = the CPU oracle (numpy, float64) on one KV head of sequence 0
+         of the same workload, timed on this host's cores (median of 3, all
+         cores and one core).
 --impl reference runs that oracle as the reference arm.
 """
 from __future__ import annotations
@@ -204,6 +211,237 @@ def _traffic(workload):
 
 # ------------------------------------------------------------------ eta arm
 
+KERNELS_PER_STEP = 3  # screen, attention, merge (the library's launches per decode step)
+
+
+class Flush:
+    """Evicts L2 before a step: reads a 256 MiB buffer (the evicted lines are
+    clean, so the next step does not pay for writing back a flush buffer)."""
+
+    def __init__(self, dev):
+        self.buf = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        torch.sum(self.buf, dim=0, out=self.sink)
+
+
+class Decode:
+    """One workload resident on the device with its metadata, the decode
+    parameters, a workspace, and (launch=graph) the step recorded as a CUDA
+    graph; `dense` turns the screen off (every block loaded)."""
+
+    def __init__(self, eta, wl, dev, args, dense=False):
+        self.eta, self.wl, self.dense = eta, wl, dense
+        self.q = wl.q.to(dev)
+        self.k = wl.k.to(dev)
+        self.v = wl.v.to(dev)
+        self.seq = torch.tensor(wl.seq_lens, dtype=torch.int32, device=dev)
+        self.w_tau = None if wl.w_tau is None else torch.from_numpy(wl.w_tau).to(dev)
+        self.b_tau = None if wl.b_tau is None else torch.from_numpy(wl.b_tau).to(dev)
+        self.c_tau = None if wl.c_tau is None else torch.from_numpy(wl.c_tau).to(dev)
+        self.summ = eta.alloc_summary(wl.batch, wl.n_kv_heads, wl.max_ctx, wl.head_dim, wl.block_size, dev,
+                                      fmt=args.meta)
+        first = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
+        eta.eta_block_summary_update(self.k, self.v, self.seq, self.summ, wl.block_size, first, wl.nb_max,
+                                     wl.n_q_heads)
+        self.kw = dict(w_tau=self.w_tau, b_tau=self.b_tau, c_tau=self.c_tau, scale=wl.scale, beta=wl.beta,
+                       offset_a=wl.offset_a, z=wl.z, n_local_blocks=wl.n_local_blocks, screen_enabled=not dense,
+                       attend_impl=args.attend_impl)
+        # the admitted selection once, outside any timing, for the byte count
+        sel = eta.decode(self.q, self.k, self.v, self.seq, self.summ, wl.block_size, wl.tau_mode, selection=True,
+                         **self.kw)
+        torch.cuda.synchronize()
+        assert eta.eta_read_device_status(sel["workspace"]) == eta.ETA_OK
+        uc = sel["union_count"].cpu().numpy()
+        self.kv_union = union_bytes(wl, sel["union_list"].cpu().numpy(), uc)
+        self.nbytes = step_bytes(wl, self.kv_union, args.meta)
+        nb_total = sum(wl.n_blocks(i) for i in range(wl.batch)) * wl.n_kv_heads
+        self.union_density = float(uc.sum()) / nb_total
+        self.head_density = float(sel["admitted_count"].cpu().numpy().sum()) / (nb_total * wl.group)
+        del sel
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty((wl.batch, wl.n_q_heads), dtype=torch.float32, device=dev)
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        for e in self.ev:  # materialise the cudaEvent_t handles the library records into
+            e.record()
+        torch.cuda.synchronize()
+        self.params_ev = self.make_params(events=self.ev)
+        self.params = self.make_params()
+        self.ws = eta.alloc_workspace(eta.eta_decode_workspace_size(self.params), dev)
+        for p in (self.params, self.params_ev):
+            p.workspace, p.workspace_bytes = self.ws.data_ptr(), self.ws.numel()
+        self.graph = None
+        if args.launch == "graph":
+            self.graph = eta.DecodeGraph(self.params, [self.q, self.k, self.v, self.seq, self.summ, self.out,
+                                                       self.lse, self.ws])
+
+    def make_params(self, q=None, seq=None, out=None, events=None):
+        return self.eta.make_params(self.q if q is None else q, self.k, self.v, self.seq if seq is None else seq,
+                                    self.summ, self.wl.block_size, self.wl.tau_mode,
+                                    out=self.out if out is None else out, lse=self.lse, events=events, **self.kw)
+
+    def step(self, stream):
+        if self.graph is not None:
+            self.graph.launch(stream)
+        else:
+            self.eta.eta_decode(self.params, stream)
+
+    def close(self):
+        if self.graph is not None:
+            self.graph.close()
+            self.graph = None
+
+
+def time_steps(fn, n, flush, stream):
+    """n steps, each bracketed by events on the launch stream with an L2
+    flush before it (outside the events); per-step milliseconds."""
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for _ in range(n):
+        flush()
+        s0.record(stream)
+        fn()
+        s1.record(stream)
+        s1.synchronize()
+        ms.append(s0.elapsed_time(s1))
+    return ms
+
+
+def kernel_times(d, n, flush, stream):
+    """Per-kernel milliseconds from events the library records between its
+    launches (screen, attention, merge), over n steps."""
+    out = {"screen": [], "attend": [], "merge": []}
+    for _ in range(n):
+        flush()
+        d.eta.eta_decode(d.params_ev, stream)
+        d.ev[3].synchronize()
+        out["screen"].append(d.ev[0].elapsed_time(d.ev[1]))
+        out["attend"].append(d.ev[1].elapsed_time(d.ev[2]))
+        out["merge"].append(d.ev[2].elapsed_time(d.ev[3]))
+    return {k: statistics.median(v) for k, v in out.items()}
+
+
+def _pct(xs, p):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, max(0, int(round(p / 100.0 * (len(xs) - 1)))))]
+
+
+def measure_config(d, args, flush, stream, peak):
+    """Graph-replay step time (W warm-up, then max(100, K) steps) and the
+    attention kernel's own time for one resident workload: the figures of a
+    `configs` / `dense` entry."""
+    for _ in range(args.warmup):
+        flush()
+        d.step(stream)
+    torch.cuda.synchronize()
+    ms = time_steps(lambda: d.step(stream), max(100, args.steps), flush, stream)
+    kt = kernel_times(d, max(20, args.steps), flush, stream)
+    med = statistics.median(ms)
+    return {
+        "workload": _workload_desc(d.wl),
+        "screen": "off (dense)" if d.dense else "on",
+        "steps": len(ms),
+        "step_us_median": round(med * 1e3, 2),
+        "step_us_mean": round(statistics.mean(ms) * 1e3, 2),
+        "step_us_p10_p90": [round(_pct(ms, 10) * 1e3, 2), round(_pct(ms, 90) * 1e3, 2)],
+        "bytes_per_step": d.nbytes,
+        "kv_union_bytes_per_step": d.kv_union,
+        "union_density": round(d.union_density, 4),
+        "head_density": round(d.head_density, 4),
+        "step_gbs": round(d.nbytes / (med * 1e-3) / 1e9, 1),
+        "step_frac_of_peak": round(d.nbytes / (med * 1e-3) / 1e9 / peak, 4),
+        "attend_us_isolated": round(kt["attend"] * 1e3, 2),
+        "attend_frac_of_peak": round(d.kv_union / (kt["attend"] * 1e-3) / 1e9 / peak, 4),
+    }
+
+
+def e2e_append(eta, d, args, flush, stream, dev):
+    """End to end through the public API with host buffers, the sequence
+    growing by one token per step: each step's new query, key and value rows
+    are written into page-locked host memory, the new lengths and positions
+    are copied up (a copy kernel reading the page-locked buffer), the append
+    kernel reads the rows from host memory, writes them into the cache and
+    refreshes their block's metadata, the decode runs and stores its output
+    into page-locked host memory; one recorded graph per step
+    (eta_step_graph_create).  The context starts b + K/2 tokens short of the
+    workload's so that appends cross a block boundary inside the timed
+    steps; the appended rows are the workload's own rows at those positions,
+    so the cache ends as it began.  Returns (per-step ms, h2d bytes, d2h bytes,
+    note)."""
+    wl = d.wl
+    B, Hq, Hkv, hd, b = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim, wl.block_size
+    K = args.steps
+    T0 = [max(1, min(T - b - K // 2, wl.max_ctx - K)) for T in wl.seq_lens]
+    nq, nkv = B * Hq * hd, B * Hkv * hd
+    rows_h = torch.empty(nq + 2 * nkv, dtype=wl.q.dtype).pin_memory()
+    rows_h[:nq].copy_(wl.q.reshape(-1))
+    lens_h = torch.zeros(2 * B, dtype=torch.int32).pin_memory()
+    lens_d = torch.zeros(2 * B, dtype=torch.int32, device=dev)
+    seq_d, pos_d = lens_d[:B], lens_d[B:]
+    q_in = torch.empty_like(d.q)
+    out_h = torch.empty_like(wl.q).pin_memory()
+    p = d.make_params(q=q_in, seq=seq_d, out=out_h)
+    p.workspace, p.workspace_bytes = d.ws.data_ptr(), d.ws.numel()
+    g = eta.StepGraph(p, k_new=rows_h[nq:nq + nkv].view(B, Hkv, hd), v_new=rows_h[nq + nkv:].view(B, Hkv, hd),
+                      positions=pos_d, q_new=rows_h[:nq].view(B, Hq, hd), h2d=lens_h, h2d_dst=lens_d,
+                      tensors=[q_in, d.k, d.v, d.summ, d.lse, d.ws, out_h, lens_d])
+    k_rows = rows_h[nq:nq + nkv].view(B, Hkv, hd)
+    v_rows = rows_h[nq + nkv:].view(B, Hkv, hd)
+
+    def reset():
+        # outside the events: lengths back to T0 and the block holding token
+        # T0 - 1 summarised over its tokens < T0 again
+        seq_d.copy_(torch.tensor(T0, dtype=torch.int32))
+        first = torch.tensor([t - 1 for t in T0], dtype=torch.int32, device=dev)
+        eta.eta_block_summary_update(d.k, d.v, seq_d, d.summ, b, first, 1, Hq)
+        torch.cuda.synchronize()
+
+    def host_token(s):
+        for i in range(B):
+            pos = T0[i] + s
+            k_rows[i].copy_(wl.k[i, :, pos])
+            v_rows[i].copy_(wl.v[i, :, pos])
+            lens_h[i] = pos + 1
+            lens_h[B + i] = pos
+
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    try:
+        for phase, n in (("warmup", args.warmup), ("timed", K)):
+            reset()
+            for s in range(n):
+                host_token(s)
+                flush()
+                e0.record(stream)
+                g.launch(stream)
+                e1.record(stream)
+                e1.synchronize()
+                if phase == "timed":
+                    ms.append(e0.elapsed_time(e1))
+        # the output of the last token equals a fresh decode of the state it left
+        check = torch.empty_like(d.q)
+        pc = d.make_params(q=q_in, seq=seq_d, out=check)
+        pc.workspace, pc.workspace_bytes = d.ws.data_ptr(), d.ws.numel()
+        eta.eta_decode(pc, stream)
+        torch.cuda.synchronize()
+        assert eta.eta_read_device_status(d.ws) == eta.ETA_OK
+        assert torch.equal(check.cpu(), out_h), "e2e output differs from a decode of the final state"
+        crossed = any(T0[i] // b != (T0[i] + K - 1) // b for i in range(B))
+    finally:
+        g.close()
+        # back to the workload's own lengths and tail metadata
+        d.seq.copy_(torch.tensor(wl.seq_lens, dtype=torch.int32))
+        first = torch.tensor([max(0, T - 1) for T in wl.seq_lens], dtype=torch.int32, device=dev)
+        eta.eta_block_summary_update(d.k, d.v, d.seq, d.summ, b, first, 1, Hq)
+        torch.cuda.synchronize()
+    h2d = rows_h.numel() * rows_h.element_size() + lens_h.numel() * 4
+    d2h = out_h.numel() * out_h.element_size()
+    note = (f"context grows one token per step from {min(T0)} (seq 0: {T0[0]} -> {T0[0] + K}); appends cross a "
+            f"block boundary inside the timed steps: {crossed}; bytes per step counted at the full context")
+    return ms, h2d, d2h, note
+
+
 def run_eta(args):
     import learned_threshold_sparse_b200 as eta
 
@@ -217,200 +455,79 @@ def run_eta(args):
                                 device_id=torch.device("cuda", local_rank))
     dev = torch.device("cuda", local_rank if world > 1 else 0)
     torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = Flush(dev)
+    peak, peak_kind = _peaks()
 
     wl = workloads.make(args.workload, args.seed)
-    q = wl.q.to(dev)
-    k = wl.k.to(dev)
-    v = wl.v.to(dev)
-    seq = torch.tensor(wl.seq_lens, dtype=torch.int32, device=dev)
-    w_tau = None if wl.w_tau is None else torch.from_numpy(wl.w_tau).to(dev)
-    b_tau = None if wl.b_tau is None else torch.from_numpy(wl.b_tau).to(dev)
-    c_tau = None if wl.c_tau is None else torch.from_numpy(wl.c_tau).to(dev)
-    summ = eta.alloc_summary(wl.batch, wl.n_kv_heads, wl.max_ctx, wl.head_dim, wl.block_size, dev, fmt=args.meta)
-    first = torch.zeros(wl.batch, dtype=torch.int32, device=dev)
-    eta.eta_block_summary_update(k, v, seq, summ, wl.block_size, first, wl.nb_max, wl.n_q_heads)
-
-    # selection once (outside timing) for the byte count
-    sel = eta.decode(q, k, v, seq, summ, wl.block_size, wl.tau_mode, w_tau=w_tau, b_tau=b_tau, c_tau=c_tau,
-                     scale=wl.scale, beta=wl.beta, offset_a=wl.offset_a, z=wl.z,
-                     n_local_blocks=wl.n_local_blocks, screen_enabled=not args.dense,
-                     attend_impl=args.attend_impl, selection=True)
-    torch.cuda.synchronize()
-    assert eta.eta_read_device_status(sel["workspace"]) == eta.ETA_OK
-    uc = sel["union_count"].cpu().numpy()
-    ul = sel["union_list"].cpu().numpy()
-    kv_union = union_bytes(wl, ul, uc)
-    nbytes = step_bytes(wl, kv_union, args.meta)
-    nb_total = sum(wl.n_blocks(i) for i in range(wl.batch)) * wl.n_kv_heads
-    union_density = float(uc.sum()) / nb_total
-    head_density = float(sel["admitted_count"].cpu().numpy().sum()) / (nb_total * wl.group)
-
-    out = torch.empty_like(q)
-    lse = torch.empty((wl.batch, wl.n_q_heads), dtype=torch.float32, device=dev)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    for e in ev:  # materialise the cudaEvent_t handles the library records into
-        e.record()
-    torch.cuda.synchronize()
-    params = eta.make_params(q, k, v, seq, summ, wl.block_size, wl.tau_mode, w_tau=w_tau, b_tau=b_tau,
-                             c_tau=c_tau, scale=wl.scale, beta=wl.beta, offset_a=wl.offset_a, z=wl.z,
-                             n_local_blocks=wl.n_local_blocks, screen_enabled=not args.dense,
-                             attend_impl=args.attend_impl, out=out, lse=lse, events=ev)
-    ws = eta.alloc_workspace(eta.eta_decode_workspace_size(params), dev)
-    params.workspace = ws.data_ptr()
-    params.workspace_bytes = ws.numel()
-    stream = torch.cuda.current_stream(dev)
-    flush_buf = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
-    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
-
-    class _Flush:
-        @staticmethod
-        def fill_(_):
-            torch.sum(flush_buf, dim=0, out=flush_sink)
-
-    flush = _Flush()
-
-    def one_step():
-        eta.eta_decode(params, stream)
-
+    d = Decode(eta, wl, dev, args, dense=args.dense)
     for _ in range(args.warmup):
-        flush.fill_(1.0)
-        one_step()
+        flush()
+        d.step(stream)
     torch.cuda.synchronize()
 
-    params_plain = eta.make_params(q, k, v, seq, summ, wl.block_size, wl.tau_mode, w_tau=w_tau, b_tau=b_tau,
-                                   c_tau=c_tau, scale=wl.scale, beta=wl.beta, offset_a=wl.offset_a, z=wl.z,
-                                   n_local_blocks=wl.n_local_blocks, screen_enabled=not args.dense,
-                                   attend_impl=args.attend_impl, out=out, lse=lse)
-    params_plain.workspace = ws.data_ptr()
-    params_plain.workspace_bytes = ws.numel()
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if args.launch == "graph":
-        # the serving-loop launch path: the step recorded once, replayed per step
-        graph = eta.DecodeGraph(params_plain, [q, k, v, seq, summ, out, lse, ws])
-
-        def timed_step():
-            graph.launch(stream)
-    else:
-        graph = None
-
-        def timed_step():
-            eta.eta_decode(params_plain, stream)
-
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        timed_step()
-    torch.cuda.synchronize()
-
-    # Timed region: K steps, each bracketed by events on the launch stream;
-    # the L2 flush before every step stays outside the events.
+    # Timed region: exactly K steps, each bracketed by events on the launch
+    # stream; the L2 flush before every step stays outside the events.  The
+    # clock sampler runs over this and every later measurement.
     clocks = ClockSampler(dev.index)
     clocks.start()
     time.sleep(0.3)
-    step_ms = []
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     t_wall = time.perf_counter()
-    for _ in range(args.steps):
-        flush.fill_(1.0)
-        s0.record(stream)
-        timed_step()
-        s1.record(stream)
-        s1.synchronize()
-        step_ms.append(s0.elapsed_time(s1))
+    step_ms = time_steps(lambda: d.step(stream), args.steps, flush, stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     wall_s = time.perf_counter() - t_wall
-    # Per-kernel breakdown over a second run of K steps: the library records
-    # events before the screen, before the attention kernel and after it.
-    screen_ms, attend_ms, merge_ms = [], [], []
-    for _ in range(args.steps):
-        flush.fill_(1.0)
-        one_step()
-        ev[3].synchronize()
-        screen_ms.append(ev[0].elapsed_time(ev[1]))
-        attend_ms.append(ev[1].elapsed_time(ev[2]))
-        merge_ms.append(ev[2].elapsed_time(ev[3]))
-    clk = clocks.stop()
-    assert eta.eta_read_device_status(ws) == eta.ETA_OK
-
     ms = max_over_ranks(statistics.mean(step_ms), dev)
-    value = whole_job_gbs(world, nbytes, ms)
+    value = whole_job_gbs(world, d.nbytes, ms)
+    # A longer run of the same step for the distribution (median of >= 100).
+    dist_ms = time_steps(lambda: d.step(stream), max(100, args.steps), flush, stream)
+    kt = kernel_times(d, max(20, args.steps), flush, stream)
+    assert eta.eta_read_device_status(d.ws) == eta.ETA_OK
+    med = statistics.median(dist_ms)
 
-    # ---- end to end through the public API, host buffers: the step's new
-    # query, key and value rows go up in one copy from pinned memory, the
-    # append writes the K/V rows and refreshes their block, the decode runs,
-    # the output comes back to pinned memory.
-    B_, Hq_, Hkv_, d_ = wl.batch, wl.n_q_heads, wl.n_kv_heads, wl.head_dim
-    nq, nkv = B_ * Hq_ * d_, B_ * Hkv_ * d_
-    knew = torch.stack([wl.k[i, :, wl.seq_lens[i] - 1] for i in range(B_)])
-    vnew = torch.stack([wl.v[i, :, wl.seq_lens[i] - 1] for i in range(B_)])
-    packed_h = torch.cat([wl.q.reshape(-1), knew.reshape(-1), vnew.reshape(-1)]).pin_memory()
-    packed_d = torch.empty(packed_h.shape, dtype=packed_h.dtype, device=dev)
-    q_in = packed_d[:nq].view(B_, Hq_, d_)
-    k_in = packed_d[nq:nq + nkv].view(B_, Hkv_, d_)
-    v_in = packed_d[nq + nkv:].view(B_, Hkv_, d_)
-    out_h = torch.empty_like(wl.q).pin_memory()
-    last = torch.tensor([T - 1 for T in wl.seq_lens], dtype=torch.int32, device=dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    params_e2e = eta.make_params(q_in, k, v, seq, summ, wl.block_size, wl.tau_mode, w_tau=w_tau, b_tau=b_tau,
-                                 c_tau=c_tau, scale=wl.scale, beta=wl.beta, offset_a=wl.offset_a, z=wl.z,
-                                 n_local_blocks=wl.n_local_blocks, screen_enabled=not args.dense,
-                                 attend_impl=args.attend_impl, out=out, lse=lse)
-    params_e2e.workspace = ws.data_ptr()
-    params_e2e.workspace_bytes = ws.numel()
-
-    if args.launch == "graph":
-        # the whole token as one recorded graph: the append kernel reads the
-        # new q, k, v rows from page-locked host memory (and puts q where the
-        # decode reads it), the decode stores its output straight into
-        # page-locked host memory
-        params_e2e.out = out_h.data_ptr()
-        graph_e2e = eta.StepGraph(params_e2e, k_new=packed_h[nq:nq + nkv].view(B_, Hkv_, d_),
-                                  v_new=packed_h[nq + nkv:].view(B_, Hkv_, d_), positions=last,
-                                  q_new=packed_h[:nq].view(B_, Hq_, d_),
-                                  tensors=[q_in, k, v, seq, summ, lse, ws, out_h])
-
-        def e2e_step():
-            graph_e2e.launch(stream)
-    else:
-        graph_e2e = None
-
-        def e2e_step():
-            packed_d.copy_(packed_h, non_blocking=True)
-            eta.eta_append_kv(k, v, seq, summ, wl.block_size, k_in, v_in, last, wl.n_q_heads, stream)
-            eta.eta_decode(params_e2e, stream)
-            out_h.copy_(out, non_blocking=True)
-
-    for _ in range(args.warmup):
-        flush.fill_(1.0)
-        e2e_step()
-    torch.cuda.synchronize()
-    e2e_ms = []
-    for _ in range(args.steps):
-        flush.fill_(1.0)
-        e0.record(stream)
-        e2e_step()
-        e1.record(stream)
-        e1.synchronize()
-        e2e_ms.append(e0.elapsed_time(e1))
-    assert torch.equal(out_h, out.cpu())
-    for g in (graph, graph_e2e):
-        if g is not None:
-            g.close()
+    # ---- end to end through the public API, host buffers, growing context
+    e2e_ms, h2d, d2h, e2e_note = e2e_append(eta, d, args, flush, stream, dev)
     e2e = max_over_ranks(statistics.mean(e2e_ms), dev)
-    h2d = packed_h.numel() * wl.elt_bytes
-    d2h = out_h.numel() * wl.elt_bytes
+    d.close()
+    main = dict(kv_union=d.kv_union, nbytes=d.nbytes, union_density=d.union_density, head_density=d.head_density)
+    del d
+    torch.cuda.empty_cache()
 
-    peak, peak_kind = _peaks()
-    att_ms = statistics.mean(attend_ms)
-    achieved = kv_union / (att_ms * 1e-3) / 1e9
+    # ---- the dense path of the same kernels, and the other long-context configs
+    extra = {}
+    if world == 1 and not args.no_configs:
+        if not args.dense:
+            dd = Decode(eta, wl, dev, args, dense=True)
+            extra["dense"] = measure_config(dd, args, flush, stream, peak)
+            dd.close()
+            del dd
+            torch.cuda.empty_cache()
+        cfgs = {}
+        for name in [c for c in args.configs.split(",") if c and c != args.workload]:
+            w2 = workloads.make(name, args.seed)
+            entry = {}
+            for dense in (False, True):
+                x = Decode(eta, w2, dev, args, dense=dense)
+                entry["dense" if dense else "screened"] = measure_config(x, args, flush, stream, peak)
+                x.close()
+                del x
+                torch.cuda.empty_cache()
+            cfgs[name] = entry
+            del w2
+        extra["configs"] = cfgs
+    clk = clocks.stop()
+
+    att = kt["attend"]
+    achieved = main["kv_union"] / (att * 1e-3) / 1e9
     traffic = _traffic(args.workload + ("_dense" if args.dense else ""))
-
     line = None
     if rank == 0:
         cpu = None if args.no_cpu_baseline or world > 1 else cpu_baseline(wl, args)
+        iso = {k: round(v * 1e3, 2) for k, v in kt.items()}
         line = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -420,6 +537,12 @@ def run_eta(args):
             "warmup": args.warmup,
             "ms_per_step": round(ms, 6),
             "latency_us": round(ms * 1e3, 2),
+            "latency_us_median": round(statistics.median(step_ms) * 1e3, 2),
+            "latency_us_distribution": {"steps": len(dist_ms), "median": round(med * 1e3, 2),
+                                        "mean": round(statistics.mean(dist_ms) * 1e3, 2),
+                                        "p10": round(_pct(dist_ms, 10) * 1e3, 2),
+                                        "p90": round(_pct(dist_ms, 90) * 1e3, 2),
+                                        "note": "a second run of the same step after the K timed steps"},
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
@@ -432,32 +555,39 @@ def run_eta(args):
                 "screen": "off (dense)" if args.dense else "on",
                 "metadata": args.meta,
                 "attend_impl": {0: "auto", 1: "simt", 2: "tc"}[args.attend_impl],
-                "union_density": round(union_density, 4),
-                "head_density": round(head_density, 4),
-                "bytes_per_step": nbytes,
-                "kv_union_bytes_per_step": kv_union,
+                "union_density": round(main["union_density"], 4),
+                "head_density": round(main["head_density"], 4),
+                "bytes_per_step": main["nbytes"],
+                "kv_union_bytes_per_step": main["kv_union"],
                 "l2": "flushed before every step by reading a 256 MiB buffer (outside the step events)",
-                "launch": ("one CUDA graph replay per step (eta_decode_graph_launch); e2e: one graph per "
-                           "step of append (reading q, k, v from page-locked host memory) and decode (storing "
-                           "out into page-locked host memory) (eta_step_graph_create)"
-                           if args.launch == "graph" else "stream launches (eta_decode; e2e: separate calls)"),
+                "launch": ("one CUDA graph replay per step (eta_decode_graph_launch)" if args.launch == "graph"
+                           else "stream launches (eta_decode)"),
                 "parallelism": f"replicas x{world} (each rank decodes its own batch)",
             },
-            "kernels_ms": {"screen": round(statistics.mean(screen_ms), 6), "attend": round(att_ms, 6),
-                           "merge": round(statistics.mean(merge_ms), 6),
-                           "note": "second K-step run with library events between the kernels"},
+            "kernels_us": {
+                "isolated": iso,
+                "sum_isolated": round(sum(iso.values()), 2),
+                "step_median": round(med * 1e3, 2),
+                "overlap_and_gaps": round(med * 1e3 - sum(iso.values()), 2),
+                "note": ("medians of a run with library events recorded between the kernels; those events stop "
+                         "the kernels' programmatic-launch overlap and add a launch gap to each, so the isolated "
+                         "times sum to more than the step: step = sum_isolated + overlap_and_gaps"),
+            },
             "roofline": {"kernel": "attend", "bound": "hbm", "achieved": round(achieved, 2),
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
-                         "algorithmic_bytes_per_launch": kv_union},
-            "step_frac_of_peak": round(nbytes / (ms * 1e-3) / 1e9 / peak, 4),
-            "e2e": {"value": round(whole_job_gbs(world, nbytes, e2e), 2), "unit": UNIT,
-                    "ms_per_step": round(e2e, 6), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "io": ("the append kernel loads the token's q, k, v rows from pinned host memory and the "
-                           "decode stores out into pinned host memory, one graph per token"
-                           if args.launch == "graph" else
-                           "q, k, v copied from pinned host memory and out copied back by the copy engine")},
-            "gpu_launches": 3 * args.steps,
+                         "algorithmic_bytes_per_launch": main["kv_union"],
+                         "time": "isolated attention-kernel time (events on the launch stream; includes its launch gap)"},
+            "step_frac_of_peak": round(main["nbytes"] / (ms * 1e-3) / 1e9 / peak, 4),
+            "e2e": {"value": round(whole_job_gbs(world, main["nbytes"], e2e), 2), "unit": UNIT,
+                    "ms_per_step": round(e2e, 6), "us_median": round(statistics.median(e2e_ms) * 1e3, 2),
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "io": ("one graph per token (eta_step_graph_create): new lengths and positions copied up by a "
+                           "kernel reading page-locked memory, the append kernel reads the new q, k, v rows from "
+                           "page-locked host memory, the decode stores out into page-locked host memory"),
+                    "mode": e2e_note},
+            **extra,
+            "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clk,
             "wall_s_timed_region": round(wall_s, 3),
             "cpu_baseline": cpu,
@@ -493,55 +623,90 @@ def _sample_bytes(s, r):
     return step_bytes(s, union_bytes(s, ul, np.array([[len(ids)]])))
 
 
-def cpu_baseline(wl, args, steps=1, warmup=0):
+def _host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, args, repeats=3):
+    """The CPU oracle (numpy, float64) on a bounded sample of the workload:
+    sequence 0, KV head 0 with its G query heads (1 / (batch x KV heads) of
+    the step), block metadata computed once beforehand.  Median of `repeats`
+    runs with numpy's thread pools limited to all host cores, and again to one
+    core.  value = the sample's algorithmic bytes / median seconds."""
     import oracle
-    from threadpoolctl import threadpool_info, threadpool_limits
+    from threadpoolctl import threadpool_limits
 
     s = _oracle_sample(wl)
     summary = oracle.summarize(s.k, s.seq_lens, s.block_size)
-    cores = os.cpu_count() or 1
-    with threadpool_limits(limits=cores):
-        threads = max([p.get("num_threads", 1) for p in threadpool_info()] or [1])
-        for _ in range(warmup):
-            _oracle_step(oracle, s, summary)
-        ts = []
-        for _ in range(steps):
-            t0 = time.perf_counter()
-            r = _oracle_step(oracle, s, summary)
-            ts.append(time.perf_counter() - t0)
-    sec = statistics.mean(ts)
+    cores = _host_cores()
+    med = {}
+    r = None
+    for label, n in (("all", cores), ("one", 1)):
+        with threadpool_limits(limits=n):
+            ts = []
+            for _ in range(repeats):
+                t0 = time.perf_counter()
+                r = _oracle_step(oracle, s, summary)
+                ts.append(time.perf_counter() - t0)
+        med[label] = statistics.median(ts)
     nbytes = _sample_bytes(s, r)
-    return {"value": round(nbytes / sec / 1e9, 4), "unit": UNIT, "cores": int(threads), "kind": "oracle",
-            "seconds_per_sample": round(sec, 3),
+    per_step = wl.batch * wl.n_kv_heads
+    return {"value": round(nbytes / med["all"] / 1e9, 4), "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "repeats": repeats, "statistic": "median",
+            "seconds_per_sample": round(med["all"], 4),
+            "seconds_per_sample_one_core": round(med["one"], 4),
+            "value_one_core": round(nbytes / med["one"] / 1e9, 4),
+            "samples_per_step": per_step,
+            "seconds_per_step_estimated": round(med["all"] * per_step, 3),
             "sample": (f"{wl.name} seed {wl.seed}: sequence 0, KV head 0 with its {s.n_q_heads} query heads "
-                       f"(1/{wl.batch * wl.n_kv_heads} of the step), block metadata precomputed; numpy fp64"),
-            "ms_per_step": round(sec * 1e3, 3)}
+                       f"(1/{per_step} of the step), block metadata precomputed; numpy float64; 'cores' = the "
+                       "thread limit given to numpy's pools (its matrix products use them, its elementwise work "
+                       "runs on one thread)")}
 
 
 def run_reference(args):
     rank, _, world = _rank_env()
     if rank != 0:
         return None
+    import oracle
+
     wl = workloads.make(args.workload, args.seed)
-    cb = cpu_baseline(wl, args, steps=args.steps, warmup=args.warmup)
+    s = _oracle_sample(wl)
+    summary = oracle.summarize(s.k, s.seq_lens, s.block_size)
+    for _ in range(args.warmup):
+        _oracle_step(oracle, s, summary)
+    ts = []
+    r = None
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        r = _oracle_step(oracle, s, summary)
+        ts.append(time.perf_counter() - t0)
+    sec = statistics.mean(ts)
+    nbytes = _sample_bytes(s, r)
+    value = round(nbytes / sec / 1e9, 4)
+    cores = _host_cores()
+    sample = (f"{wl.name} seed {wl.seed}: each step is sequence 0, KV head 0 with its {s.n_q_heads} query heads "
+              f"(1/{wl.batch * wl.n_kv_heads} of the decode step), block metadata precomputed; numpy float64")
     return {
         "impl": "reference",
         "metric": METRIC,
-        "value": cb["value"],
+        "value": value,
         "unit": UNIT,
         "n_gpus": world,
         "steps": args.steps,
         "warmup": args.warmup,
-        "ms_per_step": cb["ms_per_step"],
+        "ms_per_step": round(sec * 1e3, 3),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": _workload_desc(wl), "seed": args.seed,
-                   "sample": cb["sample"]},
-        "cpu_baseline": cb,
-        "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "config": {"workload": _workload_desc(wl), "seed": args.seed, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
 
@@ -677,6 +842,9 @@ def main():
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="decode step as one recorded CUDA graph (default) or as stream launches")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", default="c3_long,c5_batched",
+                    help="other workloads measured (screened and dense) after the main line")
+    ap.add_argument("--no-configs", action="store_true", help="skip the dense arm and the other workloads")
     ap.add_argument("--meta", default="fp16", choices=["fp16", "fp8", "box"],
                     help="block metadata format (box: the comparison coordinate-box screen)")
     ap.add_argument("--prefill", action="store_true", help="time the causal forward pass instead of the decode step")

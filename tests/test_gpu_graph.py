@@ -266,3 +266,63 @@ def test_step_graph_copies_of_any_size_and_alignment(nbytes, offset):
     assert torch.equal(dst_h[offset:], src_d[offset:].cpu())
     assert not dst_d[:offset].any() and not dst_h[:offset].any()  # nothing written before the buffers
     assert eta.eta_read_device_status(ws) == eta.ETA_OK
+
+
+def test_step_graph_growing_context_across_block_boundaries():
+    """A serving loop whose context grows one token per step, as the bench's
+    end-to-end leg runs it: per token the new lengths and positions are copied
+    up from page-locked memory, the append reads the new q, k, v rows from
+    page-locked host memory, and the decode stores its output into page-locked
+    host memory, all in one recorded graph.  The appends cross block
+    boundaries (and start a fresh block); after every token the outputs, the
+    admitted sets and the refreshed metadata match the oracle for the state
+    reached."""
+    full = workloads.custom(seed=61, batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, block_size=64,
+                            seq_lens=[900, 400], dtype=BF16, tau_bias=2.0, tau_std=1.0, key_kind="cluster")
+    T0 = [700 - 4, 256 - 2]  # the first sequence crosses 704, the second 256
+    B, Hq, Hkv, d, b = full.batch, full.n_q_heads, full.n_kv_heads, full.head_dim, full.block_size
+    wl = full.with_params(seq_lens=list(T0))
+    t = upload(wl)
+    for i in range(B):  # the rows to come are written by the appends
+        t["k"][i, :, T0[i]:] = 0
+        t["v"][i, :, T0[i]:] = 0
+    summ = gpu_summary(wl, t)
+    nq, nkv = B * Hq * d, B * Hkv * d
+    rows_h = torch.empty(nq + 2 * nkv, dtype=torch.bfloat16).pin_memory()
+    rows_h[:nq].copy_(full.q.reshape(-1))
+    lens_h = torch.zeros(2 * B, dtype=torch.int32).pin_memory()
+    lens_d = torch.tensor(T0 + [0] * B, dtype=torch.int32, device="cuda")
+    q_in = torch.empty_like(t["q"])
+    t2 = dict(t, q=q_in, seq=lens_d[:B])
+    p, ws, res = _setup(wl, t2, summ)
+    out_h = torch.zeros((B, Hq, d), dtype=torch.bfloat16).pin_memory()
+    p.out = out_h.data_ptr()
+    g = eta.StepGraph(p, k_new=rows_h[nq:nq + nkv].view(B, Hkv, d), v_new=rows_h[nq + nkv:].view(B, Hkv, d),
+                      positions=lens_d[B:], q_new=rows_h[:nq].view(B, Hq, d), h2d=lens_h, h2d_dst=lens_d,
+                      tensors=[ws, *res.values(), *summ.values(), q_in, t["k"], t["v"], out_h])
+    try:
+        for s in range(8):
+            lens = [T0[i] + s + 1 for i in range(B)]
+            for i in range(B):
+                rows_h[nq + i * Hkv * d:nq + (i + 1) * Hkv * d].copy_(full.k[i, :, lens[i] - 1].reshape(-1))
+                rows_h[nq + nkv + i * Hkv * d:nq + nkv + (i + 1) * Hkv * d].copy_(full.v[i, :, lens[i] - 1].reshape(-1))
+                lens_h[i] = lens[i]
+                lens_h[B + i] = lens[i] - 1
+            g.launch()
+            torch.cuda.synchronize()
+            got = _host(res, ws)
+            got["out"] = out_h.float().numpy()
+            now = full.with_params(seq_lens=lens)
+            ref = oracle_decode(now)
+            compare(now, got, ref)
+            # the refreshed tail metadata is the oracle's
+            for i in range(B):
+                j = (lens[i] - 1) // b
+                np.testing.assert_array_equal(summ["mu"][i, :, j].cpu().numpy(), ref["mu"][i, :, j])
+                np.testing.assert_array_equal(summ["sigma"][i, :, j].cpu().numpy(), ref["sigma"][i, :, j])
+        for i in range(B):
+            n = T0[i] + 8
+            assert torch.equal(t["k"][i, :, :n].cpu(), full.k[i, :, :n])
+            assert torch.equal(t["v"][i, :, :n].cpu(), full.v[i, :, :n])
+    finally:
+        g.close()
