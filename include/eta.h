@@ -68,8 +68,14 @@ typedef enum { ETA_TAU_LEARNED = 0, ETA_TAU_CALIBRATED = 1 } eta_tau_mode;
 typedef enum {
   ETA_ATTEND_AUTO = 0,   /* tensor-core kernel where supported, else CUDA-core */
   ETA_ATTEND_SIMT = 1,   /* CUDA-core FMA kernel (all supported shapes)       */
-  ETA_ATTEND_TC = 2      /* tcgen05 tensor-core kernel (bf16, d = 128,
-                            block_size in {64, 128}, group size >= 2)          */
+  ETA_ATTEND_TC = 2,     /* tcgen05 tensor-core kernel (bf16, d = 128,
+                            block_size in {64, 128}, group size >= 2) between
+                            a separate screen kernel and a merge kernel       */
+  ETA_ATTEND_FUSED = 3   /* one tcgen05 kernel that screens, attends and
+                            merges (the tensor-core shapes above, fp16
+                            metadata or the screen off, n_local_blocks >= 0,
+                            batch <= 256, at most 2048 (sequence, KV head)
+                            segments)                                         */
 } eta_attend_impl;
 
 /* The KV cache of one attention layer.  Two layouts:
@@ -198,7 +204,9 @@ typedef struct {
   unsigned* union_mask;              /* [batch, n_kv_heads, nb_max]: bit j set
                                         if query head g*G + j admitted block
                                         union_list[...]; 0 fill              */
-  void* workspace;                   /* device scratch, 256-byte aligned     */
+  void* workspace;                   /* device scratch, 256-byte aligned; its
+                                        first ETA_WORKSPACE_CONTROL_BYTES must
+                                        be zero before its first use        */
   size_t workspace_bytes;
   void* timing_events[4];            /* optional cudaEvent_t (NULL = none):
                                         recorded before the screen, before
@@ -207,6 +215,17 @@ typedef struct {
                                         (events between the kernels keep
                                         them from overlapping their launch) */
 } eta_decode_params;
+
+/*
+ * Leading control region of a decode workspace: the device status word and
+ * the counters the fused kernel uses to hand out work and to fold partials.
+ * It must be zero before the workspace's first use; every completed step
+ * leaves it at zero again (apart from the status word, which
+ * eta_read_device_status clears), so one workspace serves calls of any shapes
+ * in turn.  After a step that reported ETA_ERR_DEVICE_TIMEOUT, zero it again
+ * before the next call.  The rest of the workspace needs no initialisation.
+ */
+#define ETA_WORKSPACE_CONTROL_BYTES ((size_t)69632)
 
 /*
  * eta_decode_workspace_size - bytes of workspace eta_decode needs for these

@@ -44,6 +44,7 @@ ETA_TAU_CALIBRATED = 1
 ETA_ATTEND_AUTO = 0
 ETA_ATTEND_SIMT = 1
 ETA_ATTEND_TC = 2
+ETA_ATTEND_FUSED = 3
 
 
 class EtaError(RuntimeError):
@@ -167,6 +168,7 @@ SYMBOLS = ("eta_block_summary_update", "eta_append_kv", "eta_decode_workspace_si
            "eta_read_device_status", "eta_diag_wait_timeout", "eta_prefill", "eta_calibration_histogram", "eta_calibrate_constants",
            "eta_status_string", "eta_build_info")
 
+WORKSPACE_CONTROL_BYTES = 69632  # ETA_WORKSPACE_CONTROL_BYTES in include/eta.h
 DEVICE_STATUS_TIMEOUT = 1
 DEVICE_STATUS_RANGE = 2
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h

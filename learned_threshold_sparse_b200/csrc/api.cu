@@ -90,8 +90,10 @@ eta_status make_shape(const eta_decode_params* p, Shape* out) {
   if (static_cast<long long>(s.nseg) * s.nchunks > 16384) return ETA_ERR_UNSUPPORTED;
   s.list_stride = s.nchunks * chunk;
   s.rescue = (p->n_local_blocks < 0 && p->screen_enabled) ? 1 : 0;
+  s.fused = 0;
+  s.nlev = 0;
   const bool tc_ok = attend_tc_supported(s);
-  if (p->attend_impl == ETA_ATTEND_TC && !tc_ok) return ETA_ERR_UNSUPPORTED;
+  if ((p->attend_impl == ETA_ATTEND_TC || p->attend_impl == ETA_ATTEND_FUSED) && !tc_ok) return ETA_ERR_UNSUPPORTED;
   s.attend_kind = (p->attend_impl == ETA_ATTEND_SIMT || !tc_ok) ? ETA_ATTEND_SIMT : ETA_ATTEND_TC;
   if (s.attend_kind == ETA_ATTEND_SIMT) {
     if (attend_simt_smem(s) == 0) return ETA_ERR_UNSUPPORTED;
@@ -100,6 +102,48 @@ eta_status make_shape(const eta_decode_params* p, Shape* out) {
     if (attend_tc_smem(s) == 0) return ETA_ERR_UNSUPPORTED;
     s.attend_ctas = sms;
   }
+  // The fused kernel (screen, attention and merge in one launch) covers the
+  // tensor-core shapes with fp16 metadata (or the screen off), the window on
+  // (no rescue), batches of up to kFusedMaxSeqs sequences and up to 2048
+  // (sequence, KV head) segments.
+  const bool fused_ok = s.attend_kind == ETA_ATTEND_TC && !s.rescue &&
+                        (!p->screen_enabled || p->summary.format == ETA_META_FP16) && s.B <= kFusedMaxSeqs &&
+                        s.nseg <= 2048;
+  if (fused_ok && p->attend_impl == ETA_ATTEND_FUSED) {
+    // chunks of about 256 KB of K+V (8 blocks of 64 rows, 4 of 128): small
+    // enough that the dynamic hand-out balances the SMs to within a chunk;
+    // at most 65536 chunks (one partial slot each) and a fold tree whose
+    // counters fit the control region
+    Shape f = s;
+    int c = s.b == 64 ? 8 : 4;
+    while (c < 32 && static_cast<long long>(s.nseg) * ((s.nbmax + c - 1) / c) > 65536) c *= 2;
+    f.fused = 1;
+    f.chunk = c;
+    f.nchunks = (s.nbmax + c - 1) / c;
+    f.list_stride = f.nchunks * c;
+    f.attend_ctas = sms;
+    f.nlev = 0;
+    f.M[0] = f.nchunks;
+    // counters: chunks handed out per segment, a used-up bit per segment,
+    // then the fold-tree nodes
+    long long ncount = s.nseg + (s.nseg + 31) / 32;
+    while (f.M[f.nlev] > 1 && f.nlev + 1 < kMaxLevels) {
+      f.M[f.nlev + 1] = (f.M[f.nlev] + kFoldFan - 1) / kFoldFan;
+      ++f.nlev;
+      ncount += static_cast<long long>(s.nseg) * f.M[f.nlev];
+    }
+    if (f.nlev == 0) {  // a single chunk per segment still folds once (into the output)
+      f.M[1] = 1;
+      f.nlev = 1;
+      ncount += s.nseg;
+    }
+    if (f.M[f.nlev] == 1 && ncount <= kMaxCounters && static_cast<long long>(s.nseg) * f.nchunks <= 65536 &&
+        fused_tc_smem(f) != 0) {
+      *out = f;
+      return ETA_OK;
+    }
+  }
+  if (p->attend_impl == ETA_ATTEND_FUSED) return ETA_ERR_UNSUPPORTED;
   *out = s;
   return ETA_OK;
 }
@@ -125,7 +169,7 @@ eta_status check_params(const eta_decode_params* p) {
   if (!isfinite(p->offset_a)) return ETA_ERR_INVALID_ARG;
   if (!(p->z > 0.f)) return ETA_ERR_INVALID_ARG;  // +inf allowed, NaN rejected
   if (p->n_local_blocks < -1) return ETA_ERR_INVALID_ARG;
-  if (p->attend_impl < ETA_ATTEND_AUTO || p->attend_impl > ETA_ATTEND_TC) return ETA_ERR_INVALID_ARG;
+  if (p->attend_impl < ETA_ATTEND_AUTO || p->attend_impl > ETA_ATTEND_FUSED) return ETA_ERR_INVALID_ARG;
   if (p->lse && !aligned(p->lse, 4)) return ETA_ERR_INVALID_ARG;
   if ((p->admitted_count && !aligned(p->admitted_count, 4)) || (p->union_count && !aligned(p->union_count, 4)) ||
       (p->union_list && !aligned(p->union_list, 4)) || (p->union_mask && !aligned(p->union_mask, 4)))
@@ -172,9 +216,10 @@ cudaError_t ensure_smem(const void* kern, size_t bytes, SmemLimit& lim, bool* sk
 
 Workspace workspace_layout(const Shape& s) {
   Workspace w;
-  size_t off = 0;
-  w.status = off;
-  off = align256(off + 16);
+  w.status = 0;
+  w.ctrl = kCtrlOffset;
+  w.counters = kCounterOffset;
+  size_t off = kControlBytes;  // the fixed control region comes first
   w.tau = off;
   off = align256(off + static_cast<size_t>(s.B) * s.Hq * sizeof(float));
   w.chunk_count = off;
@@ -185,8 +230,18 @@ Workspace workspace_layout(const Shape& s) {
   off = align256(off + static_cast<size_t>(s.B) * s.Hq * sizeof(int));
   w.head_best = off;
   off = align256(off + static_cast<size_t>(s.B) * s.Hq * sizeof(unsigned long long));
+  const size_t pbytes = static_cast<size_t>(s.G) * partial_stride(s.d) * sizeof(float);
   w.partials = off;
-  off = align256(off + static_cast<size_t>(s.nseg + s.attend_ctas) * s.G * partial_stride(s.d) * sizeof(float));
+  for (int l = 0; l < kMaxLevels; ++l) w.lpart[l] = off;
+  if (s.fused) {
+    const size_t fbytes = static_cast<size_t>(s.G) * fused_partial_stride(s.d) * sizeof(float);
+    for (int l = 0; l < s.nlev; ++l) {
+      w.lpart[l] = off;
+      off = align256(off + static_cast<size_t>(s.nseg) * s.M[l] * fbytes);
+    }
+  } else {
+    off = align256(off + static_cast<size_t>(s.nseg + s.attend_ctas) * pbytes);
+  }
   w.total = off;
   return w;
 }
@@ -211,8 +266,9 @@ const char* eta_status_string(eta_status s) {
 }
 
 const char* eta_build_info(void) {
-  return "eta decode library: sm_100a; kernels: block_summary, append, screen, rescue, attend_simt, attend_tc, "
-         "merge, export, prefill_tc, calib_hist, io_copy, diag_wait; decode step and serving step as CUDA graphs";
+  return "eta decode library: sm_100a; kernels: block_summary, append, fused_tc (screen + attention + merge), "
+         "screen, rescue, attend_simt, attend_tc, merge, export, prefill_tc, calib_hist, io_copy, diag_wait; decode "
+         "step and serving step as CUDA graphs";
 }
 
 eta_status eta_block_summary_update(const eta_cache_desc* cache, const eta_summary_desc* summary,
@@ -342,6 +398,60 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
   sa.lse = p->lse;
   sa.head_count = reinterpret_cast<int*>(ws + w.head_count);
   sa.head_best = reinterpret_cast<unsigned long long*>(ws + w.head_best);
+
+  if (s.fused) {
+    FusedArgs fa;
+    fa.k = p->cache.k_cache;
+    fa.v = p->cache.v_cache;
+    fa.block_table = p->cache.block_table;
+    fa.q = p->q;
+    fa.seq_lens = p->cache.seq_lens;
+    fa.w_tau = p->w_tau;
+    fa.b_tau = p->b_tau;
+    fa.c_tau = p->c_tau;
+    fa.mu = p->summary.mu;
+    fa.sigma = p->summary.sigma;
+    fa.max_norm = p->summary.max_norm;
+    fa.tau_mode = p->tau_mode;
+    fa.lwb = p->n_local_blocks;
+    fa.screen_enabled = p->screen_enabled ? 1 : 0;
+    fa.scale = p->scale;
+    fa.beta = p->beta;
+    fa.offset_a = p->offset_a;
+    fa.z = p->z;
+    fa.s = s;
+    fa.status = reinterpret_cast<unsigned*>(ws + w.status);
+    fa.ctrl = reinterpret_cast<unsigned*>(ws + w.ctrl);
+    fa.counters = reinterpret_cast<unsigned*>(ws + w.counters);
+    fa.chunk_count = reinterpret_cast<int*>(ws + w.chunk_count);
+    fa.chunk_list = reinterpret_cast<int*>(ws + w.chunk_list);
+    int cb = s.nseg + (s.nseg + 31) / 32;  // after the hand-out counters and used-up bits
+    for (int l = 0; l < kMaxLevels; ++l) {
+      fa.lpart[l] = reinterpret_cast<float*>(ws + w.lpart[l]);
+      fa.cbase[l] = cb;
+      if (l >= 1 && l <= s.nlev) cb += s.nseg * s.M[l];
+    }
+    fa.out = p->out;
+    fa.lse = p->lse;
+    ev(0);
+    ev(1);
+    if (launch_fused_tc(fa, cs) != cudaSuccess) return ETA_ERR_CUDA;
+    ev(2);
+    if (p->admitted_count || p->union_count || p->union_list || p->union_mask) {
+      ExportArgs xa;
+      xa.chunk_count = fa.chunk_count;
+      xa.chunk_list = fa.chunk_list;
+      xa.seq_lens = p->cache.seq_lens;
+      xa.s = s;
+      xa.admitted_count = p->admitted_count;
+      xa.union_count = p->union_count;
+      xa.union_list = p->union_list;
+      xa.union_mask = p->union_mask;
+      if (launch_export(xa, cs) != cudaSuccess) return ETA_ERR_CUDA;
+    }
+    ev(3);
+    return ETA_OK;
+  }
 
   ev(0);
   if (s.rescue) {

@@ -15,6 +15,9 @@ namespace eta {
 // Floats per (partial slot, head): d accumulator entries, m, l, 2 pad so
 // every row starts 16-byte aligned.
 __host__ __device__ constexpr int partial_stride(int d) { return d + 4; }
+// Fused path: d accumulator entries, m, the four softmax warps' shares of l
+// (summed in a fixed order when read), 3 pad.
+__host__ __device__ constexpr int fused_partial_stride(int d) { return d + 8; }
 
 // Device status word bits (first word of the workspace).
 constexpr unsigned kStatusTimeout = ETA_DEVICE_STATUS_TIMEOUT;  // a bounded wait ran out
@@ -37,7 +40,17 @@ struct Shape {
   int attend_kind;   // ETA_ATTEND_SIMT or ETA_ATTEND_TC
   int rescue;        // 1 when n_local_blocks < 0 (top-1 rescue may fire)
   int num_pages;     // paged cache: pages in the pools (0: contiguous cache)
+  int fused;         // 1: one fused kernel screens, attends and merges (chunks of `chunk` blocks)
+  int nlev;          // fused: levels of the fold tree above the chunk partials
+  int M[5];          // fused: nodes per segment at fold level l (M[0] = nchunks, M[nlev] = 1)
 };
+
+// Fused path: the partials of a segment's chunks are folded kFoldFan at a
+// time, level by level (a tree of at most kMaxLevels - 1 levels), and
+// sequence tables of up to kFusedMaxSeqs sequences live in shared memory.
+constexpr int kFoldFan = 32;
+constexpr int kMaxLevels = 5;
+constexpr int kFusedMaxSeqs = 256;
 
 // Where the K/V rows of logical block blk of segment seg (sequence
 // seg / Hkv, KV head seg % Hkv) start, as a row index of the [rows, d] view
@@ -61,8 +74,21 @@ struct KvLayout {
 
 // Byte offsets of the workspace regions (all 256-byte aligned).
 struct Workspace {
-  size_t status, tau, chunk_count, chunk_list, head_count, head_best, partials, total;
+  size_t status, ctrl, counters, tau, chunk_count, chunk_list, head_count, head_best, partials, total;
+  size_t lpart[kMaxLevels];  // fused: partials of fold level l (l < nlev)
 };
+
+// Leading control region of every workspace, at fixed offsets whatever the
+// shapes of a call: the status word, the fused path's ticket and
+// finished-CTA counters, and its fold-tree counters.  The counters are back
+// at zero after every completed step (each is reset by the thread that sees
+// it complete), so calls of any shapes may share a workspace; the region
+// must be zero before the first call.
+constexpr size_t kCtrlOffset = 64;
+constexpr size_t kCounterOffset = 4096;
+constexpr int kMaxCounters = 16384;
+constexpr size_t kControlBytes = kCounterOffset + kMaxCounters * sizeof(unsigned);
+static_assert(kControlBytes == ETA_WORKSPACE_CONTROL_BYTES, "control region size in the public header");
 
 Workspace workspace_layout(const Shape& s);
 
@@ -107,6 +133,34 @@ struct AttendArgs {
   float* partials;         // [nseg + attend_ctas][G][partial_stride(d)]
   void* out;               // [B, Hq, d] kv dtype: segments owned by one CTA
   float* lse;              // [B, Hq] or null
+};
+
+// Arguments of the fused decode kernel (screen + attention + merge).
+struct FusedArgs {
+  const void* k;
+  const void* v;
+  const int* block_table;  // paged cache (else null), see KvLayout
+  const void* q;
+  const int* seq_lens;
+  const float* w_tau;
+  const float* b_tau;
+  const float* c_tau;
+  const void* mu;          // fp16 metadata
+  const void* sigma;
+  const float* max_norm;
+  int tau_mode, lwb, screen_enabled;
+  float scale, beta, offset_a, z;
+  Shape s;
+  unsigned* status;
+  unsigned* ctrl;                  // [1] CTAs finished
+  unsigned* counters;              // [nseg] chunks handed out per segment, [ceil(nseg/32)] used-up bits,
+                                   // then the fold-tree node counters (levels 1..nlev, from cbase[1])
+  int* chunk_count;                // [nseg, nchunks]  admitted blocks per chunk (selection export)
+  int* chunk_list;                 // [nseg, list_stride]
+  float* lpart[kMaxLevels];        // level l partials [nseg * M[l]][G][fused_partial_stride(d)], l < nlev
+  int cbase[kMaxLevels];           // first counter of level l (l >= 1)
+  void* out;
+  float* lse;
 };
 
 struct MergeArgs {
@@ -234,6 +288,8 @@ cudaError_t launch_attend_tc(const AttendArgs& a, cudaStream_t st);
 size_t attend_tc_smem(const Shape& s);
 bool attend_tc_supported(const Shape& s);
 cudaError_t launch_merge(const MergeArgs& a, cudaStream_t st);
+cudaError_t launch_fused_tc(const FusedArgs& a, cudaStream_t st);
+size_t fused_tc_smem(const Shape& s);
 cudaError_t launch_export(const ExportArgs& a, cudaStream_t st);
 cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st);
 cudaError_t launch_calib(const CalibArgs& a, cudaStream_t st);

@@ -24,18 +24,25 @@ __global__ void __launch_bounds__(kExportThreads) export_kernel(ExportArgs a) {
   __shared__ int s_head[8];
   if (t < 8) s_head[t] = 0;
   const int* counts = a.chunk_count + static_cast<size_t>(seg) * s.nchunks;
+  // only the chunks that hold blocks of the sequence carry counts of this step
+  int T = a.seq_lens[i];
+  T = T < 0 ? 0 : (T > s.max_ctx ? s.max_ctx : T);
+  const int nch = min(s.nchunks, ((T + s.b - 1) / s.b + s.chunk - 1) / s.chunk);
   if (t == 0) {
+    // a count outside [0, chunk] cannot come from this step's screen: it is
+    // read as 0 rather than trusted (never reads past a chunk's list)
     int run = 0;
-    for (int c = 0; c < s.nchunks; ++c) {
+    for (int c = 0; c < nch; ++c) {
       s_off[c] = run;
-      run += counts[c];
+      const int n = counts[c];
+      run += (n >= 0 && n <= s.chunk) ? n : 0;
     }
-    s_off[s.nchunks] = run;
+    s_off[nch] = run;
   }
   __syncthreads();
-  const int total = s_off[s.nchunks];
+  const int total = s_off[nch];
   int hc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  for (int c = 0; c < s.nchunks; ++c) {
+  for (int c = 0; c < nch; ++c) {
     const int n = s_off[c + 1] - s_off[c];
     const int* list = a.chunk_list + static_cast<size_t>(seg) * s.list_stride + static_cast<size_t>(c) * s.chunk;
     for (int k = t; k < n; k += kExportThreads) {

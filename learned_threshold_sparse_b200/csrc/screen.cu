@@ -33,33 +33,6 @@ constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxChunk = 1024;
 
-// Reduce N values held by every lane across all 32 lanes, exchanging half of
-// the remaining values per butterfly stage.  Afterwards lane l holds the
-// total of value index l / (32 / N) (N a power of two, N <= 32).
-template <int N>
-__device__ __forceinline__ float transpose_reduce32(float (&v)[N], int lane) {
-  int n = N;
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    if (n > 1) {
-      const bool upper = (lane & o) != 0;
-      const int half = n >> 1;
-#pragma unroll
-      for (int j = 0; j < N / 2; ++j) {
-        if (j < half) {
-          const float send = upper ? v[j] : v[j + half];
-          const float keep = upper ? v[j + half] : v[j];
-          v[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
-      }
-      n = half;
-    } else {
-      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
-    }
-  }
-  return v[0];
-}
-
 constexpr int kRound = 64;  // blocks of metadata staged in shared memory per round
 
 // Staging buffers of mu and sigma rows (ESZ bytes per coordinate: 2 for fp16,
@@ -274,7 +247,7 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
           v[u * NV + G + h] = sq;
         }
       }
-      float red = transpose_reduce32<32>(v, lane);
+      float red = dev::transpose_reduce32<32>(v, lane);
       float sq = __shfl_down_sync(0xffffffffu, red, G);  // sum q^2 sigma^2 of the same (block, head)
       const int lb = gb + vb;
       const bool head_lane = vq < G && lb < r;

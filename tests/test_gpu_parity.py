@@ -131,7 +131,8 @@ TC_CASES = [c for c in SMALL if c["dtype"] == BF16 and c["d"] == 128 and c["b"] 
             and c["Hq"] // c["Hkv"] in (2, 4, 8)]
 
 
-@pytest.mark.parametrize("impl", [eta.ETA_ATTEND_SIMT, eta.ETA_ATTEND_TC], ids=["simt", "tc"])
+@pytest.mark.parametrize("impl", [eta.ETA_ATTEND_SIMT, eta.ETA_ATTEND_TC, eta.ETA_ATTEND_FUSED],
+                         ids=["simt", "tc", "fused"])
 @pytest.mark.parametrize("c", TC_CASES, ids=[c["id"] for c in TC_CASES])
 def test_decode_parity_each_attention_kernel(c, impl):
     wl = _small(c)
@@ -220,6 +221,23 @@ def test_workspace_too_small_rejected():
     assert e.value.code == eta.ETA_ERR_WORKSPACE
 
 
+@pytest.mark.parametrize("c", TC_CASES, ids=[c["id"] for c in TC_CASES])
+def test_fused_and_split_kernels_agree(c):
+    # the same admitted sets, outputs within rounding of each other (the
+    # partials are split differently: per chunk vs per attention CTA)
+    wl = _small(c)
+    t = upload(wl)
+    summ = gpu_summary(wl, t)
+    f = gpu_decode(wl, t, summ, attend_impl=eta.ETA_ATTEND_FUSED)
+    sp = gpu_decode(wl, t, summ, attend_impl=eta.ETA_ATTEND_TC)
+    for k in ("union_list", "union_mask", "union_count", "admitted_count"):
+        np.testing.assert_array_equal(f[k], sp[k], err_msg=k)
+    # both are within the oracle tolerances; P is rounded to bf16 over a
+    # different tile packing, so they may differ by up to those
+    assert np.abs(f["out"] - sp["out"]).max() <= 2e-2
+    np.testing.assert_allclose(f["lse"], sp["lse"], rtol=2e-3, atol=2e-3)
+
+
 def test_simt_and_auto_agree():
     wl = _small(SMALL[1])
     t = upload(wl)
@@ -239,14 +257,15 @@ def test_workspace_reuse_across_shapes():
     b = workloads.custom(seed=42, batch=2, n_q_heads=8, n_kv_heads=2, head_dim=64, block_size=32,
                          seq_lens=[900, 47], dtype=F32, tau_bias=1e6).with_params(n_local_blocks=-1)
     ws = eta.alloc_workspace(64 << 20)
-    ws.fill_(0x7f)  # non-zero garbage everywhere except the status word
-    ws[:16].zero_()
-    for wl in (a, b, a, b):
+    ws.fill_(0x7f)  # non-zero garbage everywhere after the control region (zero before first use)
+    ws[:eta.WORKSPACE_CONTROL_BYTES].zero_()
+    for wl, impl in ((a, eta.ETA_ATTEND_AUTO), (b, eta.ETA_ATTEND_AUTO), (a, eta.ETA_ATTEND_FUSED),
+                     (b, eta.ETA_ATTEND_AUTO), (a, eta.ETA_ATTEND_FUSED), (a, eta.ETA_ATTEND_AUTO)):
         t = upload(wl)
         summ = gpu_summary(wl, t)
         res = eta.decode(t["q"], t["k"], t["v"], t["seq"], summ, wl.block_size, wl.tau_mode, w_tau=t["w_tau"],
                          b_tau=t["b_tau"], c_tau=t["c_tau"], n_local_blocks=wl.n_local_blocks, selection=True,
-                         workspace=ws)
+                         workspace=ws, attend_impl=impl)
         torch.cuda.synchronize()
         g = {k: v.float().cpu().numpy() if k == "out" else v.cpu().numpy()
              for k, v in res.items() if k != "workspace"}
@@ -273,7 +292,9 @@ def test_config_parity_full_size(name):
     # be identical with no allowance, both against the oracle's own screen
     # and against the oracle's screen evaluated on the device's metadata.
     wl = workloads.make(name, 0)
-    g = gpu_decode(wl)
+    t = upload(wl)
+    summ = gpu_summary(wl, t)
+    g = gpu_decode(wl, t, summ)
     r = oracle_decode(wl)
     assert_summary_bit_exact(wl, g["summary"], r)
     ratio = min_margin_over_bound(wl, r)
@@ -284,6 +305,10 @@ def test_config_parity_full_size(name):
     n_amb = compare(wl, g, r, strict=strict)
     assert n_amb == 0
     np.testing.assert_array_equal(gpu_admitted(wl, g), oracle_screen_on(wl, g["summary"], r))
+    if wl.dtype == BF16 and wl.head_dim == 128:
+        # the fused screen + attention + merge kernel on the same state
+        gf = gpu_decode(wl, t, summ, attend_impl=eta.ETA_ATTEND_FUSED)
+        assert compare(wl, gf, r, strict=strict) == 0
     if wl.planted:
         adm = r["admitted"]
         for (i, h), blocks in wl.planted.items():
