@@ -58,7 +58,11 @@ typedef enum {
   ETA_ERR_WORKSPACE = 3,       /* workspace NULL or smaller than required   */
   ETA_ERR_CUDA = 4,            /* a CUDA runtime call failed                */
   ETA_ERR_DEVICE_TIMEOUT = 5,  /* a bounded device-side wait ran out        */
-  ETA_ERR_DEVICE_RANGE = 6     /* a device-resident length was out of range */
+  ETA_ERR_DEVICE_RANGE = 6,    /* a device-resident length was out of range */
+  ETA_ERR_DEVICE_LIST = 7      /* the admitted-block tables an attention
+                                  kernel read broke the screen's contract
+                                  (counts, block range, order, head masks);
+                                  the step's output is not valid          */
 } eta_status;
 
 typedef enum { ETA_F32 = 0, ETA_BF16 = 1 } eta_dtype;
@@ -262,6 +266,9 @@ eta_status eta_decode(const eta_decode_params* p, void* stream);
 #define ETA_DEVICE_STATUS_TIMEOUT 1u  /* a bounded device-side wait ran out  */
 #define ETA_DEVICE_STATUS_RANGE 2u    /* a device-resident length or page id
                                          was out of range and was clamped    */
+#define ETA_DEVICE_STATUS_LIST 4u     /* an attention kernel found the chunk
+                                         counts or lists inconsistent and
+                                         stopped (see ETA_ERR_DEVICE_LIST)   */
 
 /*
  * eta_decode_noalloc - eta_decode for callers that cannot allocate device
@@ -485,8 +492,9 @@ eta_status eta_calibrate_constants(const double* hist, int n_heads, int nbins, f
 
 /*
  * eta_read_device_status - synchronise `stream`, read and clear the device
- * status word kept in `workspace`.  Returns ETA_OK, ETA_ERR_DEVICE_TIMEOUT
- * or ETA_ERR_DEVICE_RANGE (or ETA_ERR_CUDA if the copy fails).
+ * status word kept in `workspace`.  Returns ETA_OK, ETA_ERR_DEVICE_TIMEOUT,
+ * ETA_ERR_DEVICE_LIST or ETA_ERR_DEVICE_RANGE, in that order of precedence
+ * when several bits are set (or ETA_ERR_CUDA if the copy fails).
  */
 eta_status eta_read_device_status(void* workspace, void* stream);
 

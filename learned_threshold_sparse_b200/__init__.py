@@ -36,6 +36,7 @@ ETA_ERR_WORKSPACE = 3
 ETA_ERR_CUDA = 4
 ETA_ERR_DEVICE_TIMEOUT = 5
 ETA_ERR_DEVICE_RANGE = 6
+ETA_ERR_DEVICE_LIST = 7
 
 ETA_F32 = 0
 ETA_BF16 = 1
@@ -171,6 +172,7 @@ SYMBOLS = ("eta_block_summary_update", "eta_append_kv", "eta_decode_workspace_si
 WORKSPACE_CONTROL_BYTES = 69632  # ETA_WORKSPACE_CONTROL_BYTES in include/eta.h
 DEVICE_STATUS_TIMEOUT = 1
 DEVICE_STATUS_RANGE = 2
+DEVICE_STATUS_LIST = 4
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
 
 
@@ -362,7 +364,7 @@ def eta_decode_noalloc(params: eta_decode_params, device_status: Optional[torch.
     device memory: the library's fixed device scratch is used instead (see
     include/eta.h).  Calls sharing that scratch must not overlap on the GPU.
     device_status (an int32 device tensor, optional) receives the step's
-    device status bits (DEVICE_STATUS_TIMEOUT, DEVICE_STATUS_RANGE)."""
+    device status bits (DEVICE_STATUS_TIMEOUT, DEVICE_STATUS_RANGE, DEVICE_STATUS_LIST)."""
     ptr = None if device_status is None else device_status.data_ptr()
     rc = _lib.eta_decode_noalloc(ctypes.byref(params), ptr, _stream_handle(stream))
     if rc != ETA_OK:

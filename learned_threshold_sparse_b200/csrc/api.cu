@@ -261,6 +261,7 @@ const char* eta_status_string(eta_status s) {
     case ETA_ERR_CUDA: return "CUDA runtime error";
     case ETA_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait ran out";
     case ETA_ERR_DEVICE_RANGE: return "a device-resident length was out of range (clamped)";
+    case ETA_ERR_DEVICE_LIST: return "inconsistent admitted-block tables (attention stopped; output not valid)";
   }
   return "unknown status";
 }
@@ -626,6 +627,7 @@ eta_status eta_read_device_status(void* workspace, void* stream) {
   if (cudaMemcpyAsync(workspace, &zero, sizeof(zero), cudaMemcpyHostToDevice, cs) != cudaSuccess) return ETA_ERR_CUDA;
   if (cudaStreamSynchronize(cs) != cudaSuccess) return ETA_ERR_CUDA;
   if (word & kStatusTimeout) return ETA_ERR_DEVICE_TIMEOUT;
+  if (word & kStatusList) return ETA_ERR_DEVICE_LIST;
   if (word & kStatusRange) return ETA_ERR_DEVICE_RANGE;
   return ETA_OK;
 }

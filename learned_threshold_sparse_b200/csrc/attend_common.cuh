@@ -100,10 +100,44 @@ struct UnitSplit {
   }
 };
 
+// What the screen (and the top-1 rescue after it) promise about chunk cin of
+// a segment: 0 <= count <= chunk, and `count` entries (head mask << 24 |
+// block) whose blocks ascend strictly inside [cin chunk, min((cin + 1) chunk,
+// nblocks)), nblocks = ceil(T / b), each with a non-zero mask inside the
+// group's G bits.  A walker checks every entry before it reads the page
+// table or streams a row; an entry that breaks the promise stops the CTA and
+// sets kStatusList, so a corrupted or stale table yields an error, never rows
+// the screen did not admit.  Both predicates compile for the host as well.
+// ETA_LIST_CHECK_BEGIN
+constexpr unsigned kFaultCount = 1u;  // count outside [0, chunk]
+constexpr unsigned kFaultBlock = 2u;  // block outside the chunk or past the sequence
+constexpr unsigned kFaultOrder = 4u;  // block not above the entry before it
+constexpr unsigned kFaultMask = 8u;   // empty head mask, or bits beyond G
+
+__host__ __device__ __forceinline__ unsigned chunk_count_faults(int chunk, int count) {
+  return (count < 0 || count > chunk) ? kFaultCount : 0u;
+}
+
+// prev_blk: the block of the entry before this one in the same chunk, or -1.
+__host__ __device__ __forceinline__ unsigned list_entry_faults(int chunk, int G, int nblocks, int cin, int entry,
+                                                               int prev_blk) {
+  const int blk = entry & ((1 << 24) - 1);
+  const unsigned mask = static_cast<unsigned>(entry) >> 24;
+  const int lo = cin * chunk;
+  const int hi = nblocks < lo + chunk ? nblocks : lo + chunk;
+  unsigned f = 0u;
+  if (blk < lo || blk >= hi) f |= kFaultBlock;
+  if (blk <= prev_blk) f |= kFaultOrder;
+  if (mask == 0u || (mask >> G) != 0u) f |= kFaultMask;
+  return f;
+}
+// ETA_LIST_CHECK_END
+
 // Walk the units [u0, u0 + nunits) with one warp.  `issue(info)` runs on lane
 // 0 for every unit, in order, and returns false to stop (abort).  Returns
-// false if the walk was stopped or the counts were inconsistent.  seq_T, when
-// not null, holds the clamped sequence lengths in shared memory.
+// false if the walk was stopped or the tables broke the promise above (then
+// kStatusList is set).  seq_T, when not null, holds the clamped sequence
+// lengths in shared memory.
 template <class Issue>
 __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefix, int nprefix, int u0, int nunits,
                                            const int* seq_T, Issue&& issue) {
@@ -117,11 +151,16 @@ __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefi
   int x = lo;
   int idx = u0 - prefix[x];
   int remaining = nunits;
-  int cur_seg = -1, T = 0;
+  int cur_seg = -1, T = 0, nblk = 0;
   const KvLayout lay{a.block_table, s.Hkv, s.b, s.max_ctx, s.nbmax, s.num_pages};
+  auto fail = [&]() {
+    if (lane == 0) atomicOr(a.status, kStatusList);
+    return false;
+  };
   while (remaining > 0) {
-    if (x >= nprefix) return false;
+    if (x >= nprefix) return fail();
     const int cnt = prefix[x + 1] - prefix[x];
+    if (chunk_count_faults(s.chunk, cnt)) return fail();
     const int take = min(cnt - idx, remaining);
     if (take <= 0) { ++x; idx = 0; continue; }
     const int seg = x / s.nchunks;
@@ -134,11 +173,18 @@ __device__ __forceinline__ bool walk_units(const AttendArgs& a, const int* prefi
         const int tt = a.seq_lens[seg / s.Hkv];
         T = tt < 0 ? 0 : (tt > s.max_ctx ? s.max_ctx : tt);
       }
+      nblk = (T + s.b - 1) / s.b;
     }
     const int* list = a.chunk_list + static_cast<size_t>(seg) * s.list_stride + static_cast<size_t>(cin) * s.chunk + idx;
+    int last = -1;  // block of the entry before the batch (-1: none read in this chunk)
     for (int j0 = 0; j0 < take; j0 += 32) {
       const int nn = min(32, take - j0);
       const int e = lane < nn ? list[j0 + lane] : 0;
+      const int eb = e & kMaxBlocksPerSeq;
+      const int up = __shfl_up_sync(0xffffffffu, eb, 1);
+      const unsigned f = lane < nn ? list_entry_faults(s.chunk, s.G, nblk, cin, e, lane == 0 ? last : up) : 0u;
+      if (__any_sync(0xffffffffu, f != 0u)) return fail();
+      last = __shfl_sync(0xffffffffu, eb, nn - 1);
       // the rows of the 32 listed blocks (one page-table read per lane)
       bool bad = false;
       const long long rw = lane < nn ? lay.row(seg, e & kMaxBlocksPerSeq, &bad) : 0;

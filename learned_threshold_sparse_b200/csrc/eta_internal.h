@@ -22,6 +22,7 @@ __host__ __device__ constexpr int fused_partial_stride(int d) { return d + 8; }
 // Device status word bits (first word of the workspace).
 constexpr unsigned kStatusTimeout = ETA_DEVICE_STATUS_TIMEOUT;  // a bounded wait ran out
 constexpr unsigned kStatusRange = ETA_DEVICE_STATUS_RANGE;      // a device-resident length was clamped
+constexpr unsigned kStatusList = ETA_DEVICE_STATUS_LIST;        // a walker found inconsistent chunk tables
 
 // List entries written by the screen: block id in the low 24 bits, the
 // admitting heads of the group in the high 8 bits.

@@ -506,9 +506,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (u == k) { pq_raw[u] = raw; pq_seg[u] = sg; pq_fixed[u] = is_fixed; }
       ++pq_n;
     };
-    auto take_ahead = [&]() {  // one more counter value in flight, from the current segment
-      if (gseg >= 0 && pq_n < 2) pq_push(grab(), gseg, 0);
-    };
     // the next chunk to process: the oldest queued value, else a value taken
     // now; a value past its segment's end marks the segment used up and moves
     // the warp on to the next open segment
@@ -550,22 +547,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     uint32_t meta_phase[2] = {0u, 0u};
     int meta_pending[2] = {0, 0};
+    // A chunk's metadata: mu and sigma rows by bulk copy (completion on the
+    // buffer's mbarrier), the block norms by 4-byte asynchronous copies (one
+    // commit group per staged chunk, so the scoring waits only for its own).
     auto stage_meta = [&](const Job2& j, int buf) {
-      if (j.nscreen == 0) return;
-      const size_t seg = static_cast<size_t>(j.seq) * s.Hkv + j.kvh;
-      const size_t row = seg * s.nbmax + static_cast<size_t>(j.cidx) * C;
-      float* mn = reinterpret_cast<float*>(base + L.mnorm) + buf * C;
-      if (lane < j.nscreen) mn[lane] = a.max_norm[row + lane];
-      __syncwarp();
-      if (lane == 0) {
-        fence_proxy_async();  // this buffer's previous contents were read through the generic proxy
-        uint8_t* mb = base + L.meta + static_cast<size_t>(buf) * 2 * C * D * 2;
-        const uint32_t bytes = static_cast<uint32_t>(j.nscreen) * D * 2;
-        dev::mbar_arrive_expect_tx(&B.meta[buf], 2 * bytes);
-        dev::bulk_g2s(mb, static_cast<const uint8_t*>(a.mu) + row * D * 2, bytes, &B.meta[buf]);
-        dev::bulk_g2s(mb + C * D * 2, static_cast<const uint8_t*>(a.sigma) + row * D * 2, bytes, &B.meta[buf]);
+      if (j.nscreen > 0) {
+        const size_t seg = static_cast<size_t>(j.seq) * s.Hkv + j.kvh;
+        const size_t row = seg * s.nbmax + static_cast<size_t>(j.cidx) * C;
+        float* mn = reinterpret_cast<float*>(base + L.mnorm) + buf * C;
+        if (lane < j.nscreen) dev::cp_async4(&mn[lane], &a.max_norm[row + lane]);
+        if (lane == 0) {
+          fence_proxy_async();  // this buffer's previous contents were read through the generic proxy
+          uint8_t* mb = base + L.meta + static_cast<size_t>(buf) * 2 * C * D * 2;
+          const uint32_t bytes = static_cast<uint32_t>(j.nscreen) * D * 2;
+          dev::mbar_arrive_expect_tx(&B.meta[buf], 2 * bytes);
+          dev::bulk_g2s(mb, static_cast<const uint8_t*>(a.mu) + row * D * 2, bytes, &B.meta[buf]);
+          dev::bulk_g2s(mb + C * D * 2, static_cast<const uint8_t*>(a.sigma) + row * D * 2, bytes, &B.meta[buf]);
+        }
+        meta_pending[buf] = 1;
       }
-      meta_pending[buf] = 1;
+      dev::cp_async_commit();
     };
     auto push = [&](const FTile& ft) -> bool {
       if (!dev::warp_wait_or_abort(&B.q_empty[qslot], qphase ^ 1u, a.status, abort_flag)) return false;
@@ -580,8 +581,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Two chunks are staged ahead of the one being scored: cur (metadata in
     // buffer buf), nxt (buffer buf ^ 1); the ticket after nxt is taken while
     // cur is scored.
-    // cur and nxt are resolved and their metadata staged; counter values for
-    // later chunks are in flight in the queue.
+    // cur and nxt are resolved and their metadata staged.  Each iteration
+    // takes one more counter value; its atomic's result is first read one
+    // iteration later (queued then), so the warp never waits for it.
     Job2 cur, nxt;
     pq_push(static_cast<unsigned>(rank), home, 1);  // the two fixed chunks of the home segment
     pq_push(static_cast<unsigned>(rank + hsize), home, 1);
@@ -590,12 +592,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     int buf = 0;
     if (have_cur) {
       stage_meta(cur, 0);
-      take_ahead();
       have_nxt = next_job(nxt);
       if (have_nxt) stage_meta(nxt, 1);
     }
     while (have_cur && ok) {
-      take_ahead();
+      int r_seg = -1;
+      const unsigned r_new = (have_nxt && gseg >= 0) ? grab() : 0u;
+      if (have_nxt && gseg >= 0) r_seg = gseg;
       const int seg = cur.seq * s.Hkv + cur.kvh;
       const int T = seqT[cur.seq];
       const int blk0 = cur.cidx * C;
@@ -636,6 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // head masks of the chunk's blocks: lane l <-> block blk0 + l
       unsigned mymask = lane < cur.nloc ? ((1u << G) - 1u) : 0u;  // forced window / screen off
       if (cur.nscreen > 0) {
+        if (have_nxt) dev::cp_async_wait<1>(); else dev::cp_async_wait<0>();  // this chunk's block norms
+        __syncwarp();
         if (!dev::warp_wait_or_abort(&B.meta[buf], meta_phase[buf], a.status, abort_flag)) { ok = false; break; }
         meta_phase[buf] ^= 1u;
         meta_pending[buf] = 0;
@@ -745,6 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       cur = nxt;
       have_cur = have_nxt;
       buf ^= 1;
+      if (r_seg >= 0) pq_push(r_new, r_seg, 0);
       if (have_cur) {
         have_nxt = next_job(nxt);
         if (have_nxt) stage_meta(nxt, buf ^ 1);
@@ -755,6 +761,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       end.flags = kEnd;
       ok = push(end);
     }
+    dev::cp_async_wait<0>();  // no asynchronous copy outlives the warp
     if (!ok && lane == 0) {
       *abort_flag = 1;
       for (int k = 0; k < 2; ++k) {  // staged copies land before the CTA exits

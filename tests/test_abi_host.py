@@ -30,7 +30,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_status_strings():
-    for code in range(7):
+    for code in range(8):
         assert eta.eta_status_string(code)
     assert "sm_100a" in eta.eta_build_info()
 
