@@ -554,7 +554,7 @@ def run_eta(args):
                 "seed": args.seed,
                 "screen": "off (dense)" if args.dense else "on",
                 "metadata": args.meta,
-                "attend_impl": {0: "auto", 1: "simt", 2: "tc"}[args.attend_impl],
+                "attend_impl": {0: "auto", 1: "simt", 2: "tc", 3: "fused"}[args.attend_impl],
                 "union_density": round(main["union_density"], 4),
                 "head_density": round(main["head_density"], 4),
                 "bytes_per_step": main["nbytes"],
@@ -837,7 +837,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(workloads.CONFIGS))
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", default="eta", choices=["eta", "reference"])
-    ap.add_argument("--attend-impl", type=int, default=0, choices=[0, 1, 2])
+    ap.add_argument("--attend-impl", type=int, default=0, choices=[0, 1, 2, 3])
     ap.add_argument("--dense", action="store_true", help="screen off: every block loaded")
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="decode step as one recorded CUDA graph (default) or as stream launches")

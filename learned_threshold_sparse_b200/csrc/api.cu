@@ -91,7 +91,6 @@ eta_status make_shape(const eta_decode_params* p, Shape* out) {
   s.list_stride = s.nchunks * chunk;
   s.rescue = (p->n_local_blocks < 0 && p->screen_enabled) ? 1 : 0;
   s.fused = 0;
-  s.nlev = 0;
   const bool tc_ok = attend_tc_supported(s);
   if ((p->attend_impl == ETA_ATTEND_TC || p->attend_impl == ETA_ATTEND_FUSED) && !tc_ok) return ETA_ERR_UNSUPPORTED;
   s.attend_kind = (p->attend_impl == ETA_ATTEND_SIMT || !tc_ok) ? ETA_ATTEND_SIMT : ETA_ATTEND_TC;
@@ -108,37 +107,20 @@ eta_status make_shape(const eta_decode_params* p, Shape* out) {
   // (sequence, KV head) segments.
   const bool fused_ok = s.attend_kind == ETA_ATTEND_TC && !s.rescue &&
                         (!p->screen_enabled || p->summary.format == ETA_META_FP16) && s.B <= kFusedMaxSeqs &&
-                        s.nseg <= 2048;
+                        s.nseg <= 2048 && sms <= kFusedMaxCtas;
   if (fused_ok && p->attend_impl == ETA_ATTEND_FUSED) {
-    // chunks of about 256 KB of K+V (8 blocks of 64 rows, 4 of 128): small
-    // enough that the dynamic hand-out balances the SMs to within a chunk;
-    // at most 65536 chunks (one partial slot each) and a fold tree whose
-    // counters fit the control region
+    // chunks of about 256 KB of K+V (8 blocks of 64 rows, 4 of 128), larger
+    // when a slice (the chunks one CTA screens) would exceed kFusedMaxSlice
     Shape f = s;
     int c = s.b == 64 ? 8 : 4;
-    while (c < 32 && static_cast<long long>(s.nseg) * ((s.nbmax + c - 1) / c) > 65536) c *= 2;
+    auto chunks = [&](int cc) { return static_cast<long long>(s.nseg) * ((s.nbmax + cc - 1) / cc); };
+    while (c < 32 && chunks(c) > static_cast<long long>(sms) * kFusedMaxSlice) c *= 2;
     f.fused = 1;
     f.chunk = c;
     f.nchunks = (s.nbmax + c - 1) / c;
     f.list_stride = f.nchunks * c;
     f.attend_ctas = sms;
-    f.nlev = 0;
-    f.M[0] = f.nchunks;
-    // counters: chunks handed out per segment, a used-up bit per segment,
-    // then the fold-tree nodes
-    long long ncount = s.nseg + (s.nseg + 31) / 32;
-    while (f.M[f.nlev] > 1 && f.nlev + 1 < kMaxLevels) {
-      f.M[f.nlev + 1] = (f.M[f.nlev] + kFoldFan - 1) / kFoldFan;
-      ++f.nlev;
-      ncount += static_cast<long long>(s.nseg) * f.M[f.nlev];
-    }
-    if (f.nlev == 0) {  // a single chunk per segment still folds once (into the output)
-      f.M[1] = 1;
-      f.nlev = 1;
-      ncount += s.nseg;
-    }
-    if (f.M[f.nlev] == 1 && ncount <= kMaxCounters && static_cast<long long>(s.nseg) * f.nchunks <= 65536 &&
-        fused_tc_smem(f) != 0) {
+    if (chunks(c) <= static_cast<long long>(sms) * kFusedMaxSlice && fused_tc_smem(f) != 0) {
       *out = f;
       return ETA_OK;
     }
@@ -232,13 +214,8 @@ Workspace workspace_layout(const Shape& s) {
   off = align256(off + static_cast<size_t>(s.B) * s.Hq * sizeof(unsigned long long));
   const size_t pbytes = static_cast<size_t>(s.G) * partial_stride(s.d) * sizeof(float);
   w.partials = off;
-  for (int l = 0; l < kMaxLevels; ++l) w.lpart[l] = off;
   if (s.fused) {
-    const size_t fbytes = static_cast<size_t>(s.G) * fused_partial_stride(s.d) * sizeof(float);
-    for (int l = 0; l < s.nlev; ++l) {
-      w.lpart[l] = off;
-      off = align256(off + static_cast<size_t>(s.nseg) * s.M[l] * fbytes);
-    }
+    off = align256(off + 2 * static_cast<size_t>(s.attend_ctas) * pbytes);  // two pieces per CTA
   } else {
     off = align256(off + static_cast<size_t>(s.nseg + s.attend_ctas) * pbytes);
   }
@@ -422,16 +399,14 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
     fa.z = p->z;
     fa.s = s;
     fa.status = reinterpret_cast<unsigned*>(ws + w.status);
-    fa.ctrl = reinterpret_cast<unsigned*>(ws + w.ctrl);
-    fa.counters = reinterpret_cast<unsigned*>(ws + w.counters);
+    fa.done_ctas = reinterpret_cast<unsigned*>(ws + w.ctrl) + 1;
+    fa.arrived = reinterpret_cast<unsigned*>(ws + w.ctrl) + 2;
+    fa.flags = reinterpret_cast<unsigned*>(ws + w.counters);
+    fa.seg_ctr = reinterpret_cast<unsigned long long*>(ws + w.counters + kFusedSegCtrOffset * sizeof(unsigned));
+    fa.tau = reinterpret_cast<float*>(ws + w.tau);
     fa.chunk_count = reinterpret_cast<int*>(ws + w.chunk_count);
     fa.chunk_list = reinterpret_cast<int*>(ws + w.chunk_list);
-    int cb = s.nseg + (s.nseg + 31) / 32;  // after the hand-out counters and used-up bits
-    for (int l = 0; l < kMaxLevels; ++l) {
-      fa.lpart[l] = reinterpret_cast<float*>(ws + w.lpart[l]);
-      fa.cbase[l] = cb;
-      if (l >= 1 && l <= s.nlev) cb += s.nseg * s.M[l];
-    }
+    fa.partials = reinterpret_cast<float*>(ws + w.partials);
     fa.out = p->out;
     fa.lse = p->lse;
     ev(0);

@@ -17,7 +17,6 @@ namespace eta {
 __host__ __device__ constexpr int partial_stride(int d) { return d + 4; }
 // Fused path: d accumulator entries, m, the four softmax warps' shares of l
 // (summed in a fixed order when read), 3 pad.
-__host__ __device__ constexpr int fused_partial_stride(int d) { return d + 8; }
 
 // Device status word bits (first word of the workspace).
 constexpr unsigned kStatusTimeout = ETA_DEVICE_STATUS_TIMEOUT;  // a bounded wait ran out
@@ -42,16 +41,15 @@ struct Shape {
   int rescue;        // 1 when n_local_blocks < 0 (top-1 rescue may fire)
   int num_pages;     // paged cache: pages in the pools (0: contiguous cache)
   int fused;         // 1: one fused kernel screens, attends and merges (chunks of `chunk` blocks)
-  int nlev;          // fused: levels of the fold tree above the chunk partials
-  int M[5];          // fused: nodes per segment at fold level l (M[0] = nchunks, M[nlev] = 1)
 };
 
-// Fused path: the partials of a segment's chunks are folded kFoldFan at a
-// time, level by level (a tree of at most kMaxLevels - 1 levels), and
-// sequence tables of up to kFusedMaxSeqs sequences live in shared memory.
-constexpr int kFoldFan = 32;
-constexpr int kMaxLevels = 5;
+// Fused path: sequence tables of up to kFusedMaxSeqs sequences live in
+// shared memory, a CTA's slice holds at most kFusedMaxSlice chunks, and the
+// grid has at most kFusedMaxCtas CTAs (one slice total each in the control
+// region).
 constexpr int kFusedMaxSeqs = 256;
+constexpr int kFusedMaxSlice = 64;
+constexpr int kFusedMaxCtas = 1024;
 
 // Where the K/V rows of logical block blk of segment seg (sequence
 // seg / Hkv, KV head seg % Hkv) start, as a row index of the [rows, d] view
@@ -76,18 +74,21 @@ struct KvLayout {
 // Byte offsets of the workspace regions (all 256-byte aligned).
 struct Workspace {
   size_t status, ctrl, counters, tau, chunk_count, chunk_list, head_count, head_best, partials, total;
-  size_t lpart[kMaxLevels];  // fused: partials of fold level l (l < nlev)
 };
 
 // Leading control region of every workspace, at fixed offsets whatever the
-// shapes of a call: the status word, the fused path's ticket and
-// finished-CTA counters, and its fold-tree counters.  The counters are back
-// at zero after every completed step (each is reset by the thread that sees
-// it complete), so calls of any shapes may share a workspace; the region
-// must be zero before the first call.
+// shapes of a call: the status word, the fused path's finished-CTA counter,
+// its published slice totals and its per-segment piece counters.  They are
+// back at zero after every completed step (the last CTA to finish clears the
+// totals, the merger of a segment clears its counter), so calls of any
+// shapes may share a workspace; the region must be zero before the first
+// call.
 constexpr size_t kCtrlOffset = 64;
 constexpr size_t kCounterOffset = 4096;
 constexpr int kMaxCounters = 16384;
+// Inside the counter area: [kFusedMaxCtas] slice totals, then the segment
+// counters (64-bit, at most 2048 segments).
+constexpr int kFusedSegCtrOffset = kFusedMaxCtas;
 constexpr size_t kControlBytes = kCounterOffset + kMaxCounters * sizeof(unsigned);
 static_assert(kControlBytes == ETA_WORKSPACE_CONTROL_BYTES, "control region size in the public header");
 
@@ -153,13 +154,14 @@ struct FusedArgs {
   float scale, beta, offset_a, z;
   Shape s;
   unsigned* status;
-  unsigned* ctrl;                  // [1] CTAs finished
-  unsigned* counters;              // [nseg] chunks handed out per segment, [ceil(nseg/32)] used-up bits,
-                                   // then the fold-tree node counters (levels 1..nlev, from cbase[1])
-  int* chunk_count;                // [nseg, nchunks]  admitted blocks per chunk (selection export)
+  unsigned* done_ctas;             // [1] CTAs finished
+  unsigned* arrived;               // [1] slice totals published
+  unsigned* flags;                 // [grid] slice totals + 1 (0: not published yet)
+  unsigned long long* seg_ctr;     // [nseg] pieces announced per segment (fields: see the kernel)
+  float* tau;                      // [B, Hq] tau~ (written by the screen, read by the softmax)
+  int* chunk_count;                // [nseg, nchunks]  admitted blocks per chunk
   int* chunk_list;                 // [nseg, list_stride]
-  float* lpart[kMaxLevels];        // level l partials [nseg * M[l]][G][fused_partial_stride(d)], l < nlev
-  int cbase[kMaxLevels];           // first counter of level l (l >= 1)
+  float* partials;                 // [2 grid][G][partial_stride(d)] pieces of shared segments
   void* out;
   float* lse;
 };

@@ -16,38 +16,48 @@
 //   App. G.1                               S~ = S sigmoid(beta (S - tau~)), weights e^S~,
 //   section 3.2, App. F.3                  split-KV partials merged associatively,
 //   App. F.4                               the tail block's rows >= seq_len masked.
-// The pages screen and attend in one pass over positional chunks (section 3.2);
-// this kernel does the same with chunks handed out dynamically.
 //
-// Work is split into positional chunks of `chunk` consecutive blocks of one
-// (sequence, KV head), numbered in (sequence, KV head, block) order.  Each CTA
-// (one per SM) runs:
-//   warp 6    screen: takes chunk numbers from a global ticket counter (two
-//             ahead), stages a chunk's metadata with bulk copies, scores its
-//             blocks for the G heads, builds the chunk's admitted list (also
-//             written out for the selection export) and queues its tiles (one
-//             or two admitted blocks of the chunk, 128 key rows);
-//   warp 0    producer: tensor copies (TMA, 128-byte swizzle) of each tile's
-//             K and V blocks and the group's query rows into a 3-stage ring;
-//   warp 1    MMA issuer: S^T = K Q^T and O^T = V^T P^T into tensor memory;
-//   warps 2-5 softmax: gate, online softmax, P, folding O^T; at the end of a
-//             chunk its partial (acc, m, l per head) goes to the chunk's own
-//             slot and an event to warp 7; fold jobs from warp 7 are run at
-//             chunk boundaries and, after the last tile, until warp 7 is done;
-//   warp 7    completion: for every finished chunk (or fold) one release /
-//             acquire atomic on the counter of its parent node in the
-//             segment's fold tree (fan-in kFoldFan); the thread that completes
-//             a node resets its counter and hands the node's fold to the
-//             softmax warps.
-// A node's fold combines its children's partials in index order; the root of
-// a segment's tree writes the output rows and lse.  Whichever CTA handles a
-// chunk, every partial and every fold is computed in the same order, so the
-// result is bit-reproducible.  No CTA ever waits for another CTA.
+// Work unit: a positional chunk of C consecutive blocks of one (sequence, KV
+// head) segment; the chunks that exist (blocks below the sequence length) are
+// numbered in (sequence, KV head, block) order and cut into one contiguous
+// slice per CTA (one CTA per SM, all resident together).  Every CTA runs:
+//   1. screen    the slice's block metadata is staged in the (still idle)
+//                K/V ring by asynchronous copies from all threads, then all
+//                six warps screen it, a warp per chunk: the G heads'
+//                thresholds, the bound of every block for each head,
+//                and the chunk's admitted blocks, ascending, with head masks
+//                (list and count written to the workspace, where the
+//                selection export and the other CTAs read them); then the
+//                slice's admitted total is published (then one release
+//                increment of an arrival counter);
+//   2. exchange  the producer warp waits (bounded) for the counter to reach
+//                the grid size and reads all slice totals.  The admitted
+//                units of all lists, in list order, form one sequence of U
+//                units; this CTA takes the equal range [U c / N, U (c + 1) / N);
+//   3. attention as in the split kernel: warp 0 walks the range through the
+//                lists of the slices it covers and copies each tile's K, V
+//                and query rows (TMA, 128-byte swizzle) into a 3-stage ring,
+//                warp 1 issues S^T = K Q^T and O^T = V^T P^T into tensor
+//                memory, warps 2-5 gate, run the online softmax, write P and
+//                fold O^T; an END entry in the ring closes the range;
+//   4. merge     a segment whose units all lie in this range is written out
+//                directly; a segment spread over CTAs c_first..c_last leaves
+//                one partial per CTA, each announced by one atomic on the
+//                segment's counter, and the CTA whose announcement completes
+//                the set (every CTA of the span with a non-empty range) merges
+//                the pieces in CTA order, at its end, with the pieces copied
+//                into the then idle K/V ring.
+// The pages screen and attend in one pass over positional chunks (section
+// 3.2); here the screen of a slice runs before its streaming so that no
+// memory round trip of the screen sits behind the K/V stream.  Ranges, tile
+// order and merge order follow from the admitted sets alone, so results do
+// not depend on timing.  The only cross-CTA wait is the exchange, and it is
+// bounded: if some CTA of the grid is not resident the step ends with the
+// timeout status instead of hanging.
 //
-// Counters (tickets, finished CTAs, fold-tree nodes) live in the workspace's
-// control region and are back at zero when a step completes: the last CTA to
-// finish resets the first two, the completer of a node resets its counter.
-
+// Counters live in the workspace's control region and are back at zero when
+// a step completes: the last CTA to finish clears the slice totals, and the
+// merger of a segment clears that segment's counter.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -62,263 +72,139 @@ using dev::wait_or_abort;
 using namespace tc;
 
 constexpr int D = 128;
-constexpr int NQ = 16;            // N of both MMAs (the G query rows, rest zero)
-constexpr int TR = 128;           // key rows per tile
-constexpr int kWarps = 8;
+constexpr int NQ = 16;              // N of both MMAs
+constexpr int kWarps = 6;
 constexpr int kThreads = kWarps * 32;
-constexpr int kScreenWarp = 6;
-constexpr int kDoneWarp = 7;
-constexpr int kTmemCols = 64;     // S buffers at columns 0, 16; O buffers at 32, 48
+constexpr int kTmemCols = 64;       // S buffers at columns 0, 16; O buffers at 32, 48
 constexpr int kStages = 3;
-constexpr int kQueue = 8;         // tiles queued from the screen warp to the producer
-constexpr int kEvents = 32;       // events from the softmax warps to the completion warp
-constexpr int kJobs = 8;          // fold jobs from the completion warp to the softmax warps
-constexpr int kMaxChunk = 32;     // blocks per chunk (one lane each in the screen warp)
+constexpr int TR = 128;             // key rows per tile
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr int kFirst = 1, kLast = 2, kEnd = 4;
 
 struct Tile {
-  static constexpr int PANEL = TR * 128;  // one 64-column (128-byte) panel of a 128-row tile
+  static constexpr int PANEL = TR * 128;
   static constexpr int K0 = 0, K1 = PANEL, V0 = 2 * PANEL, V1 = 3 * PANEL, Q0 = 4 * PANEL, Q1 = 4 * PANEL + 2048;
   static constexpr int STAGE = 4 * PANEL + 4096;
   static constexpr int P_BYTES = NQ * TR * 2;
 };
 
-// A tile as the screen warp hands it on: up to two admitted blocks of one
-// chunk, their head masks, rows present (0: none) and first K/V rows, the
-// chunk's identity and the thresholds of its heads.
-struct FTile {
-  int seq, kvh, cidx, pad0;
-  int mask0, mask1, nrows0, nrows1;
-  long long row0, row1;
-  int flags, pad1;
-  float tau[8];
+// How the run of units of one segment that just ended leaves this CTA.
+constexpr int kModeShared = 1;  // other CTAs hold units of the segment: write a partial
+constexpr int kModeSlot1 = 2;   // partial slot 1 (the run did not contain the range's first unit)
+constexpr int kModeFirst = 4;   // the run holds the segment's first unit
+constexpr int kModeLast = 8;    // the run holds the segment's last unit
+
+// A ring entry: the tile's segment (-1: END), per block of the tile the
+// admitting heads and the rows present, and the mode of the run this entry
+// closes (a new segment's first tile, or END).
+struct FInfo {
+  int seg, mask0, mask1, nrows0, nrows1, prev_mode;
 };
 
-// Softmax -> completion warp: a partial of fold level `level` (0: a chunk)
-// was written for node `node` of segment (seq, kvh); kind 1 = the last
-// tile's chunk is done and no chunk follows.
-struct Event {
-  int kind, seq, kvh, level, node, pad[3];
-};
-
-// Completion warp -> softmax warps: fold the children of node `node` at
-// level `level` (>= 1) of segment (seq, kvh); kind 1 = nothing more to do.
-struct Job {
-  int kind, seq, kvh, level, node, pad[3];
-};
+constexpr int kEntStage = 256;  // list entries the producer stages per round trip
 
 struct Layout {
-  size_t stages, pbuf, meta, mnorm, bars, info, queue, events, jobs, red, tabs, seen, pend, misc, total;
+  size_t stages, pbuf, bars, info, red, seqs, cseq, prefix, own, ent, spre, sseg, scid, misc, total;
 };
 
-constexpr int kPendNodes = 128;  // completed fold-tree nodes the completion warp holds until the tiles are done
+__host__ __device__ inline size_t align_to(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-constexpr int kMaxSegs = 2048;  // segments (sequence, KV head) the screen warp's used-up mask covers
-
-__host__ __device__ inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
-
-constexpr int kBars = 2 * kStages + 12 + 2 * kQueue + 2 + 2 * kEvents + 2 * kJobs + 1;
-
-__host__ __device__ inline Layout fused_layout(int chunk) {
+// Offsets relative to a 1024-byte aligned base; nctas = grid size.
+__host__ __device__ inline Layout fused_layout(int nctas) {
   Layout L;
   size_t off = 0;
   L.stages = off;
   off += static_cast<size_t>(kStages) * Tile::STAGE;
   L.pbuf = off;
   off += 2 * static_cast<size_t>(Tile::P_BYTES);
-  L.meta = off;  // [2 buffers][mu, sigma][chunk][D] fp16
-  off += 2 * 2 * static_cast<size_t>(chunk) * D * 2;
-  L.mnorm = off;  // [2][chunk] fp32
-  off += 2 * static_cast<size_t>(chunk) * sizeof(float);
-  L.bars = off = align_up(off, 16);
-  off += kBars * sizeof(uint64_t);
-  L.info = off = align_up(off, 16);
-  off += kStages * sizeof(FTile);
-  L.queue = off = align_up(off, 16);
-  off += kQueue * sizeof(FTile);
-  L.events = off = align_up(off, 16);
-  off += kEvents * sizeof(Event);
-  L.jobs = off = align_up(off, 16);
-  off += kJobs * sizeof(Job);
-  L.red = off = align_up(off, 16);
+  L.bars = off = align_to(off, 16);
+  off += (2 * kStages + 12) * sizeof(uint64_t);
+  L.info = off = align_to(off, 16);
+  off += kStages * sizeof(FInfo);
+  L.red = off = align_to(off, 16);
   off += (2 * 4 * 8 + 4 * 8) * sizeof(float);
-  L.tabs = off = align_up(off, 16);  // seqT[S]
+  L.seqs = off = align_to(off, 16);
   off += kFusedMaxSeqs * sizeof(int);
-  L.seen = off = align_up(off, 16);  // segments this CTA found used up, one bit each
-  off += kMaxSegs / 32 * sizeof(unsigned);
-  L.pend = off = align_up(off, 16);
-  off += kPendNodes * sizeof(unsigned);
-  L.misc = off = align_up(off, 16);
-  off += 64;
-  L.total = align_up(off, 128) + 1024;  // + slack to align the dynamic base to 1024
+  L.cseq = off = align_to(off, 16);
+  off += (kFusedMaxSeqs + 1) * sizeof(int);
+  L.prefix = off = align_to(off, 16);
+  off += static_cast<size_t>(nctas + 1) * sizeof(int);
+  L.own = off = align_to(off, 16);
+  off += kFusedMaxSlice * sizeof(int);
+  L.ent = off = align_to(off, 16);
+  off += kEntStage * sizeof(int);
+  L.spre = off = align_to(off, 16);
+  off += (kFusedMaxSlice + 1) * sizeof(int);
+  L.sseg = off = align_to(off, 16);
+  off += kFusedMaxSlice * sizeof(int);
+  L.scid = off = align_to(off, 16);
+  off += kFusedMaxSlice * sizeof(int);
+  L.misc = off = align_to(off, 16);
+  off += 128;
+  L.total = align_to(off, 128) + 1024;  // + slack to align the dynamic base to 1024
   return L;
 }
 
 struct Bars {
-  uint64_t* kv_full;   // [kStages] producer -> MMA, softmax (tx bytes)
-  uint64_t* kv_empty;  // [kStages] MMA commit -> producer
-  uint64_t* s_full;    // [2] MMA commit -> softmax
-  uint64_t* s_free;    // [2] softmax (4 warps) -> MMA
-  uint64_t* p_full;    // [2] softmax (4 warps) -> MMA
-  uint64_t* o_full;    // [2] MMA commit -> softmax
-  uint64_t* o_free;    // [2] softmax (4 warps) -> MMA
-  uint64_t* rv;        // [1] softmax-warp rendezvous (4 warps)
-  uint64_t* done;      // [1] final MMA commit
-  uint64_t* q_full;    // [kQueue] screen -> producer
-  uint64_t* q_empty;   // [kQueue] producer -> screen
-  uint64_t* meta;      // [2] metadata bulk copies landed
-  uint64_t* ev_full;   // [kEvents] softmax -> completion
-  uint64_t* ev_empty;  // [kEvents] completion -> softmax
-  uint64_t* job_full;  // [kJobs] completion -> softmax
-  uint64_t* job_empty; // [kJobs] softmax (4 warps) -> completion
-  uint64_t* fold;      // [1] a fold's children staged in shared memory (bulk copy)
+  uint64_t* kv_full;   // [kStages]  producer -> MMA, softmax   (tx bytes; END: plain arrive)
+  uint64_t* kv_empty;  // [kStages]  MMA commit -> producer
+  uint64_t* s_full;    // [2]        MMA commit -> softmax
+  uint64_t* s_free;    // [2]        softmax (4 warps) -> MMA
+  uint64_t* p_full;    // [2]        softmax (4 warps) -> MMA
+  uint64_t* o_full;    // [2]        MMA commit -> softmax
+  uint64_t* o_free;    // [2]        softmax (4 warps) -> MMA
+  uint64_t* rv;        // [1]        softmax-warp rendezvous (4 warps)
+  uint64_t* done;      // [1]        final MMA commit
 };
 
-// Atomic add with release and acquire semantics at GPU scope: the partials
-// written before it (by this CTA, ordered by a CTA barrier) are visible to
-// whoever reads the counter afterwards, and this thread sees the partials of
-// everyone who incremented it before.
-__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
-  unsigned old;
-  asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_add(unsigned* p, unsigned v) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long atom_add_acq_rel64(unsigned long long* p, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.add.acq_rel.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(p), "l"(v) : "memory");
   return old;
 }
 
-// ---------------------------------------------------------------- sequence tables
+__device__ __forceinline__ unsigned atom_add_acq_rel(unsigned* p, unsigned v) {
+  unsigned old;
+  asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
+}
 
-struct Tables {
-  const int* seqT;  // clamped lengths
-  int b, chunk;
-  __device__ __forceinline__ int nb(int i) const { return (seqT[i] + b - 1) / b; }
-  __device__ __forceinline__ int nch(int i) const { return (nb(i) + chunk - 1) / chunk; }
-  // nodes of sequence i's trees at fold level l
-  __device__ __forceinline__ int nodes(int i, int l) const {
-    int n = nch(i);
-    for (int k = 0; k < l; ++k) n = (n + kFoldFan - 1) / kFoldFan;
-    return n;
+// Chunks that exist, numbered in (sequence, KV head, block) order: sequence
+// i owns Hkv nch(i) consecutive numbers from cseq[i] on.
+struct Chunks {
+  const int* seqT;  // clamped lengths [B]
+  const int* cseq;  // [B + 1]
+  int B, Hkv, b, C;
+  __device__ __forceinline__ int nch(int i) const {
+    const int nb = (seqT[i] + b - 1) / b;
+    return (nb + C - 1) / C;
+  }
+  // chunk number r (< cseq[B]) -> segment and chunk index inside it
+  __device__ __forceinline__ void locate(int r, int& seg, int& cidx) const {
+    int lo = 0, hi = B;  // largest i with cseq[i] <= r; it has chunks since cseq[i + 1] > r
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (cseq[mid] <= r) lo = mid; else hi = mid;
+    }
+    const int n = nch(lo), w = r - cseq[lo];
+    const int g = w / n;
+    seg = lo * Hkv + g;
+    cidx = w - g * n;
+  }
+  __device__ __forceinline__ int first(int seg) const {
+    const int i = seg / Hkv;
+    return cseq[i] + (seg - i * Hkv) * nch(i);
   }
 };
-
-// ---------------------------------------------------------------- folds
-
-// Folds n <= kFoldFan partials (slots first .. first + n - 1 of `src`, each
-// [G][FPS]: acc[D], m, l shares[4]) in slot order for the heads h0,
-// h0 + hstep, ... of the calling warp; lanes own 4 output coordinates.  The
-// result goes to slot `dst` of a partial array (l in the first share), or
-// (dst == nullptr) to the output rows (normalised) and lse.
-template <int G>
-__device__ void fold_partials(const float* src, size_t first, int n, float* dst, const FusedArgs& a, int seq, int kvh,
-                              int h0, int hstep, int lane) {
-  constexpr int FPS = fused_partial_stride(D);
-  constexpr int kB = 8;  // loads in flight per round (registers; a rarely used path)
-  for (int h = h0; h < G; h += hstep) {
-    float mx = -INFINITY, ls = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k0 = 0; k0 < n; k0 += kB) {
-      float4 ml[kB];
-      float l3[kB];
-      float4 x[kB];
-#pragma unroll
-      for (int u = 0; u < kB; ++u) {  // all loads of the round in flight
-        const int k = min(k0 + u, n - 1);
-        const float* p = src + ((first + k) * G + h) * FPS;
-        ml[u] = __ldcg(reinterpret_cast<const float4*>(p + D));
-        l3[u] = __ldcg(p + D + 4);
-        x[u] = __ldcg(reinterpret_cast<const float4*>(p) + lane);
-      }
-#pragma unroll
-      for (int u = 0; u < kB; ++u) {
-        const float l = ((ml[u].y + ml[u].z) + ml[u].w) + l3[u];
-        if (k0 + u >= n || !(l > 0.f)) continue;  // empty partial (l = 0, m = -inf)
-        const float m = ml[u].x;
-        if (m > mx) {
-          const float f = mx == -INFINITY ? 0.f : dev::fast_exp2(mx - m);
-          ls = fmaf(ls, f, l);
-          acc.x = fmaf(acc.x, f, x[u].x);
-          acc.y = fmaf(acc.y, f, x[u].y);
-          acc.z = fmaf(acc.z, f, x[u].z);
-          acc.w = fmaf(acc.w, f, x[u].w);
-          mx = m;
-        } else {
-          const float f = dev::fast_exp2(m - mx);
-          ls = fmaf(l, f, ls);
-          acc.x = fmaf(x[u].x, f, acc.x);
-          acc.y = fmaf(x[u].y, f, acc.y);
-          acc.z = fmaf(x[u].z, f, acc.z);
-          acc.w = fmaf(x[u].w, f, acc.w);
-        }
-      }
-    }
-    if (dst) {
-      float* p = dst + h * FPS;
-      reinterpret_cast<float4*>(p)[lane] = acc;
-      if (lane == 0) {
-        *reinterpret_cast<float4*>(p + D) = make_float4(mx, ls, 0.f, 0.f);
-        p[D + 4] = 0.f;
-      }
-    } else {
-      const size_t orow = static_cast<size_t>(seq) * a.s.Hq + static_cast<size_t>(kvh) * G + h;
-      const float inv = ls > 0.f ? 1.f / ls : 0.f;
-      const float o[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) dev::store_out_slot(a.out, a.s.elt, orow * D + lane * 4 + e, o[e]);
-      if (lane == 0 && a.lse) a.lse[orow] = dev::lse_of(mx, ls);
-    }
-  }
-}
-
-// The same fold with the n children staged in shared memory at `sm`
-// ([n][G][FPS], one bulk copy), for the heads of softmax warp w4.
-template <int G>
-__device__ void fold_staged(const float* sm, int n, float* dst, const FusedArgs& a, int seq, int kvh, int w4, int lane) {
-  constexpr int FPS = fused_partial_stride(D);
-  for (int h = w4; h < G; h += 4) {
-    float mx = -INFINITY, ls = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < n; ++k) {
-      const float* p = sm + (static_cast<size_t>(k) * G + h) * FPS;
-      const float4 ml = *reinterpret_cast<const float4*>(p + D);
-      const float l = ((ml.y + ml.z) + ml.w) + p[D + 4];
-      if (!(l > 0.f)) continue;  // empty partial (l = 0, m = -inf)
-      const float4 x = reinterpret_cast<const float4*>(p)[lane];
-      const float m = ml.x;
-      if (m > mx) {
-        const float f = mx == -INFINITY ? 0.f : dev::fast_exp2(mx - m);
-        ls = fmaf(ls, f, l);
-        acc.x = fmaf(acc.x, f, x.x);
-        acc.y = fmaf(acc.y, f, x.y);
-        acc.z = fmaf(acc.z, f, x.z);
-        acc.w = fmaf(acc.w, f, x.w);
-        mx = m;
-      } else {
-        const float f = dev::fast_exp2(m - mx);
-        ls = fmaf(l, f, ls);
-        acc.x = fmaf(x.x, f, acc.x);
-        acc.y = fmaf(x.y, f, acc.y);
-        acc.z = fmaf(x.z, f, acc.z);
-        acc.w = fmaf(x.w, f, acc.w);
-      }
-    }
-    if (dst) {
-      float* p = dst + h * FPS;
-      reinterpret_cast<float4*>(p)[lane] = acc;
-      if (lane == 0) {
-        *reinterpret_cast<float4*>(p + D) = make_float4(mx, ls, 0.f, 0.f);
-        p[D + 4] = 0.f;
-      }
-    } else {
-      const size_t orow = static_cast<size_t>(seq) * a.s.Hq + static_cast<size_t>(kvh) * G + h;
-      const float inv = ls > 0.f ? 1.f / ls : 0.f;
-      const float o[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) dev::store_out_slot(a.out, a.s.elt, orow * D + lane * 4 + e, o[e]);
-      if (lane == 0 && a.lse) a.lse[orow] = dev::lse_of(mx, ls);
-    }
-  }
-}
-
-// ---------------------------------------------------------------- kernel
 
 template <int BR, int G>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -326,14 +212,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tq, FusedArgs a) {
   using TL = Tile;
   constexpr int BPT = TR / BR;  // blocks per tile
-  constexpr int FPS = fused_partial_stride(D);
+  constexpr int CPL = D / 32;   // coordinates per lane in the screen
+  constexpr int NV = 2 * G;     // values per block: <q_h, mu>, sum q_h^2 sigma^2
+  constexpr int NB = 32 / NV;   // blocks reduced together
+  constexpr unsigned kFullMask = (1u << G) - 1u;
   extern __shared__ uint8_t smem_raw[];
   const Shape& s = a.s;
+  const int N = gridDim.x, cta = blockIdx.x;
   const int C = s.chunk;
   const uint32_t raw = dev::smem_u32(smem_raw);
   const uint32_t base_u32 = (raw + 1023u) & ~1023u;
   uint8_t* base = smem_raw + (base_u32 - raw);
-  const Layout L = fused_layout(C);
+  const Layout L = fused_layout(N);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(base + L.bars);
   Bars B;
@@ -346,23 +236,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   B.o_free = B.o_full + 2;
   B.rv = B.o_free + 2;
   B.done = B.rv + 1;
-  B.q_full = B.done + 1;
-  B.q_empty = B.q_full + kQueue;
-  B.meta = B.q_empty + kQueue;
-  B.ev_full = B.meta + 2;
-  B.ev_empty = B.ev_full + kEvents;
-  B.job_full = B.ev_empty + kEvents;
-  B.job_empty = B.job_full + kJobs;
-  B.fold = B.job_empty + kJobs;
-  FTile* info = reinterpret_cast<FTile*>(base + L.info);
-  FTile* queue = reinterpret_cast<FTile*>(base + L.queue);
-  Event* events = reinterpret_cast<Event*>(base + L.events);
-  Job* jobs = reinterpret_cast<Job*>(base + L.jobs);
-  float* red = reinterpret_cast<float*>(base + L.red);
-  int* seqT = reinterpret_cast<int*>(base + L.tabs);
+  FInfo* info = reinterpret_cast<FInfo*>(base + L.info);
+  float* red = reinterpret_cast<float*>(base + L.red);  // [2][4][8] tile maxima, then [4][8] flush sums
+  int* seqT = reinterpret_cast<int*>(base + L.seqs);
+  int* cseq = reinterpret_cast<int*>(base + L.cseq);
+  int* P = reinterpret_cast<int*>(base + L.prefix);     // [N + 1] admitted units before slice c
+  int* own = reinterpret_cast<int*>(base + L.own);      // admitted units of this slice's chunks
+  int* ent_s = reinterpret_cast<int*>(base + L.ent);    // producer: staged list entries
+  int* spre = reinterpret_cast<int*>(base + L.spre);    // producer: units before chunk k of the current slice
+  int* sseg = reinterpret_cast<int*>(base + L.sseg);    // producer: segment of chunk k of the current slice
+  int* scid = reinterpret_cast<int*>(base + L.scid);    // producer: chunk index (in its segment) of chunk k
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L.misc + 4);
-  int* issued_parity = reinterpret_cast<int*>(base + L.misc + 16);
+  int* pm = reinterpret_cast<int*>(base + L.misc + 64);     // merges to run at the end: [count, (seg, c_first, c_last, slot) x 2]
+  int* mround = reinterpret_cast<int*>(base + L.misc + 100);  // merge round: [pieces, next CTA]
+  int* issued_parity = reinterpret_cast<int*>(base + L.misc + 32);
+  int* units_total = reinterpret_cast<int*>(base + L.misc + 48);  // U, set by the producer before its first tile
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   if (t == 0) {
@@ -377,24 +266,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       dev::mbar_init(&B.p_full[k], 4);
       dev::mbar_init(&B.o_full[k], 1);
       dev::mbar_init(&B.o_free[k], 4);
-      dev::mbar_init(&B.meta[k], 1);
-    }
-    for (int k = 0; k < kQueue; ++k) {
-      dev::mbar_init(&B.q_full[k], 1);
-      dev::mbar_init(&B.q_empty[k], 1);
-    }
-    for (int k = 0; k < kEvents; ++k) {
-      dev::mbar_init(&B.ev_full[k], 4);  // one arrival per softmax warp
-      dev::mbar_init(&B.ev_empty[k], 1);
-    }
-    for (int k = 0; k < kJobs; ++k) {
-      dev::mbar_init(&B.job_full[k], 1);
-      dev::mbar_init(&B.job_empty[k], 4);
     }
     dev::mbar_init(B.rv, 4);
     dev::mbar_init(B.done, 1);
-    dev::mbar_init(B.fold, 1);
     *abort_flag = 0;
+    *reinterpret_cast<int*>(base + L.misc + 64) = 0;
     dev::fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
@@ -407,414 +283,540 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tv)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tq)) : "memory");
   }
-  // Nothing written by the previous kernel of the stream (an append, the
-  // previous step) is read before this point; the next kernel may start its
-  // own prologue now (nothing here waits for another CTA).
+  // Nothing written by the stream's previous kernel is read before this
+  // point.  The next kernel may be scheduled now: its CTAs start only once
+  // every CTA of this grid has passed here, so they never keep one of ours
+  // from becoming resident, and it reads nothing of ours before this grid
+  // has completed.
   dev::pdl_trigger();
   dev::pdl_wait();
 
   for (int x = t; x < s.B; x += kThreads) {
     int tt = a.seq_lens[x];
     if (tt < 0 || tt > s.max_ctx) {
-      if (blockIdx.x == 0) atomicOr(a.status, kStatusRange);
+      if (cta == 0) atomicOr(a.status, kStatusRange);
       tt = tt < 0 ? 0 : s.max_ctx;
     }
     seqT[x] = tt;
   }
+  __syncthreads();
+  if (warp == 0) {  // chunk numbers: cseq[i] = sum over i' < i of Hkv nch(i')
+    const int per = (s.B + 31) / 32;
+    const int lo = min(s.B, lane * per), hi = min(s.B, lo + per);
+    int sum = 0;
+    for (int x = lo; x < hi; ++x) {
+      const int nb = (seqT[x] + s.b - 1) / s.b;
+      sum += s.Hkv * ((nb + C - 1) / C);
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+    for (int x = lo; x < hi; ++x) {
+      cseq[x] = run;
+      const int nb = (seqT[x] + s.b - 1) / s.b;
+      run += s.Hkv * ((nb + C - 1) / C);
+    }
+    if (lane == 31) cseq[s.B] = incl;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const Tables tb{seqT, s.b, C};
   const uint32_t tmem = *tmem_slot;
+  const Chunks ch{seqT, cseq, s.B, s.Hkv, s.b, C};
+  const int NC = cseq[s.B];
+  const dev::UnitSplit slices(static_cast<unsigned>(NC), static_cast<unsigned>(N));
+  const int r_lo = static_cast<int>(slices.start(cta));
+  const int nslice = static_cast<int>(slices.start(cta + 1)) - r_lo;  // <= kFusedMaxSlice (host)
 
-  if (warp == kScreenWarp) {
-    // ============================================================ screen
-    constexpr int CPL = D / 32;  // coordinates per lane
-    constexpr int NV = 2 * G;    // values per block: <q_h, mu>, sum q_h^2 sigma^2
-    constexpr int NB = 32 / NV;  // blocks reduced together
+  // ============================================================ 1. screen
+  {
     // empty sequences have no chunk: their outputs are 0, lse -inf
-    for (int i = blockIdx.x; i < s.B; i += gridDim.x) {
-      if (seqT[i] != 0) continue;
-      for (int x = lane; x < s.Hq * D; x += 32) dev::store_out_slot(a.out, s.elt, static_cast<size_t>(i) * s.Hq * D + x, 0.f);
-      for (int x = lane; x < s.Hq; x += 32)
-        if (a.lse) a.lse[static_cast<size_t>(i) * s.Hq + x] = -INFINITY;
+    if (warp == 0) {
+      for (int i = cta; i < s.B; i += N) {
+        if (seqT[i] != 0) continue;
+        for (int x = lane; x < s.Hq * D; x += 32) dev::store_out_slot(a.out, s.elt, static_cast<size_t>(i) * s.Hq * D + x, 0.f);
+        for (int x = lane; x < s.Hq; x += 32)
+          if (a.lse) a.lse[static_cast<size_t>(i) * s.Hq + x] = -INFINITY;
+      }
     }
-    const KvLayout lay{a.block_table, s.Hkv, s.b, s.max_ctx, s.nbmax, s.num_pages};
     float qr[G][CPL], q2[G][CPL], tau_h[G], qn_h[G];
-    int cur_seg = -1;
-    int qslot = 0;
-    uint32_t qphase = 0;
-    bool ok = true;
-    // Chunks are handed out per (sequence, KV head) segment.  Each CTA has a
-    // home segment (CTAs spread evenly over the segments); the first two
-    // chunks of every home CTA are fixed by its rank in the segment's group
-    // (chunks rank and rank + group size), later ones come from the
-    // segment's counter (offset by the fixed ones), and when a segment is
-    // used up the CTA moves on to the next segments not yet marked used up.
-    // A CTA therefore stays on one segment for most of its chunks, and no
-    // counter is hit by every CTA at once when the kernel starts.
-    struct Job2 { int seq, kvh, cidx, nloc, nscreen; };
-    unsigned* segtk = a.counters;             // [nseg] chunks handed out per segment, beyond the fixed ones
-    unsigned* used_up = a.counters + s.nseg;  // [ceil(nseg / 32)] bit per segment
-    const unsigned grid = gridDim.x;
-    auto group_lo = [&](int sg) -> int {  // first CTA whose home is segment sg
-      return static_cast<int>((static_cast<long long>(sg) * grid + s.nseg - 1) / s.nseg);
+    int cseg = -1;
+    const bool learned = a.tau_mode == ETA_TAU_LEARNED;
+    const float scale = a.scale, z = a.z;
+    const bool strict = isinf(z);
+    const int vb = lane / NV, vq = lane % NV;
+    // The K/V ring is idle until the exchange.  A round of up to R chunks of
+    // the slice has its metadata staged there: mu and sigma rows and the
+    // block norms, by asynchronous copies spread over all threads (16 bytes
+    // per row piece, 4 per norm), all in flight together.
+    uint8_t* scr = base + L.stages;
+    const int mstride = C * D * 2;  // bytes of one chunk's mu (or sigma) rows
+    const int R = static_cast<int>(static_cast<size_t>(kStages) * TL::STAGE / (2 * mstride + C * sizeof(float)));
+    float* mn_s = reinterpret_cast<float*>(scr + static_cast<size_t>(R) * 2 * mstride);
+    const int lc = __ffs(C) - 1;  // C is a power of two
+    // rows of chunk number r: its segment, first block, blocks present and screened ones
+    auto chunk_rows = [&](int r, int& seg, int& cidx, int& nloc, int& nscreen) {
+      ch.locate(r, seg, cidx);
+      const int nb = (seqT[seg / s.Hkv] + s.b - 1) / s.b;
+      const int blk0 = cidx * C;
+      nloc = min(C, nb - blk0);
+      const int first_forced = a.screen_enabled ? max(0, nb - 1 - a.lwb) : 0;
+      nscreen = max(0, min(nloc, first_forced - blk0));
     };
-    // segments this warp itself found used up: its own marks may not be
-    // visible to its next reads of the global bits yet, and must never be
-    // visited again
-    unsigned* seen = reinterpret_cast<unsigned*>(base + L.seen);
-    for (int x = lane; x < kMaxSegs / 32; x += 32) seen[x] = 0u;
-    __syncwarp();
-    const int home = static_cast<int>(static_cast<long long>(blockIdx.x) * s.nseg / grid);
-    const int rank = static_cast<int>(blockIdx.x) - group_lo(home);
-    const int hsize = group_lo(home + 1) - group_lo(home);
-    int gseg = home;
-    auto fixed = [&](int sg) -> int { return 2 * (group_lo(sg + 1) - group_lo(sg)); };
-    auto grab = [&]() -> unsigned {  // the atomic's result is used later, so its latency overlaps work
-      unsigned tk = 0;
-      if (lane == 0) tk = atomicAdd(&segtk[gseg], 1u);
-      return tk;
-    };
-    // the first segment after `from` (circularly, `from` itself excluded) not
-    // marked used up, or -1
-    auto next_open = [&](int from) -> int {
-      for (int k0 = 1; k0 < s.nseg; k0 += 32) {
-        const int k = k0 + lane;
-        const int sg = (from + k) % s.nseg;
-        const bool open = k < s.nseg && (((__ldcg(used_up + (sg >> 5)) | seen[sg >> 5]) >> (sg & 31)) & 1u) == 0u;
-        const unsigned bal = __ballot_sync(0xffffffffu, open);
-        if (bal) return (from + k0 + __ffs(bal) - 1) % s.nseg;
+    // the heads' queries, thresholds and norms of segment seg (all loads
+    // issued first); tau~ also goes to the workspace for the softmax of
+    // whichever CTA streams this segment's units
+    auto compute_tau = [&](int i, int g, int seg) {
+      uint2 qu[G];
+      float wv[G][CPL], bc[G];  // w_tau is only 4-byte aligned: scalar loads
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const int hq = g * G + h;
+        const size_t qo = (static_cast<size_t>(i) * s.Hq + hq) * D + lane * CPL;
+        qu[h] = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(a.q) + qo);
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) wv[h][c] = learned ? __ldg(a.w_tau + static_cast<size_t>(hq) * D + lane * CPL + c) : 0.f;
+        bc[h] = learned ? a.b_tau[hq] : a.c_tau[hq];
       }
-      return -1;
-    };
-    // a counter value taken from segment gs, as a chunk index
-    auto dyn = [&](unsigned raw, int gs) -> int {
-      return static_cast<int>(__shfl_sync(0xffffffffu, raw, 0)) + fixed(gs);
-    };
-    // Counter values taken but not yet looked at wait in a small queue (two
-    // atomics overlap the scoring); every value taken is looked at before the
-    // warp may stop, so no chunk handed out is ever dropped.
-    constexpr int kPend = 4;
-    unsigned pq_raw[kPend];
-    int pq_seg[kPend], pq_fixed[kPend];
-    int pq_head = 0, pq_n = 0;
-    auto pq_push = [&](unsigned raw, int sg, int is_fixed) {
-      const int k = (pq_head + pq_n) % kPend;
 #pragma unroll
-      for (int u = 0; u < kPend; ++u)
-        if (u == k) { pq_raw[u] = raw; pq_seg[u] = sg; pq_fixed[u] = is_fixed; }
-      ++pq_n;
-    };
-    // the next chunk to process: the oldest queued value, else a value taken
-    // now; a value past its segment's end marks the segment used up and moves
-    // the warp on to the next open segment
-    auto next_job = [&](Job2& j) -> bool {
-      for (int iter = 0; iter < 8 + 2 * s.nseg; ++iter) {
-        if (pq_n == 0) {
-          if (gseg < 0) return false;
-          pq_push(grab(), gseg, 0);
-        }
-        unsigned raw = 0;
-        int sg = 0, fx = 0;
+      for (int h = 0; h < G; ++h) {
+        qr[h][0] = dev::bf16_lo(qu[h].x);
+        qr[h][1] = dev::bf16_hi(qu[h].x);
+        qr[h][2] = dev::bf16_lo(qu[h].y);
+        qr[h][3] = dev::bf16_hi(qu[h].y);
+        float tw = 0.f, qq = 0.f;
 #pragma unroll
-        for (int u = 0; u < kPend; ++u)
-          if (u == pq_head) { raw = pq_raw[u]; sg = pq_seg[u]; fx = pq_fixed[u]; }
-        pq_head = (pq_head + 1) % kPend;
-        --pq_n;
-        const int cidx = fx ? static_cast<int>(raw) : dyn(raw, sg);
-        const int i = sg / s.Hkv;
-        if (cidx < tb.nch(i)) {
-          j.seq = i;
-          j.kvh = sg - i * s.Hkv;
-          j.cidx = cidx;
-          const int nb = tb.nb(i);
-          const int blk0 = cidx * C;
-          j.nloc = min(C, nb - blk0);
-          const int first_forced = a.screen_enabled ? max(0, nb - 1 - a.lwb) : 0;
-          j.nscreen = max(0, min(j.nloc, first_forced - blk0));
-          return true;
+        for (int c = 0; c < CPL; ++c) {
+          q2[h][c] = qr[h][c] * qr[h][c];
+          qq = fmaf(qr[h][c], qr[h][c], qq);
+          tw = fmaf(wv[h][c], qr[h][c], tw);
         }
-        if (lane == 0) {
-          atomicOr(&used_up[sg >> 5], 1u << (sg & 31));
-          seen[sg >> 5] |= 1u << (sg & 31);
-        }
-        __syncwarp();
-        if (sg == gseg) gseg = next_open(sg);
+        tw = dev::warp_sum(tw);
+        qq = dev::warp_sum(qq);
+        tau_h[h] = (learned ? tw + bc[h] : bc[h]) - a.offset_a;
+        qn_h[h] = sqrtf(qq);
       }
-      if (lane == 0) atomicOr(a.status, kStatusTimeout);  // cannot happen: counted as a failed wait
-      return false;
-    };
-    uint32_t meta_phase[2] = {0u, 0u};
-    int meta_pending[2] = {0, 0};
-    // A chunk's metadata: mu and sigma rows by bulk copy (completion on the
-    // buffer's mbarrier), the block norms by 4-byte asynchronous copies (one
-    // commit group per staged chunk, so the scoring waits only for its own).
-    auto stage_meta = [&](const Job2& j, int buf) {
-      if (j.nscreen > 0) {
-        const size_t seg = static_cast<size_t>(j.seq) * s.Hkv + j.kvh;
-        const size_t row = seg * s.nbmax + static_cast<size_t>(j.cidx) * C;
-        float* mn = reinterpret_cast<float*>(base + L.mnorm) + buf * C;
-        if (lane < j.nscreen) dev::cp_async4(&mn[lane], &a.max_norm[row + lane]);
-        if (lane == 0) {
-          fence_proxy_async();  // this buffer's previous contents were read through the generic proxy
-          uint8_t* mb = base + L.meta + static_cast<size_t>(buf) * 2 * C * D * 2;
-          const uint32_t bytes = static_cast<uint32_t>(j.nscreen) * D * 2;
-          dev::mbar_arrive_expect_tx(&B.meta[buf], 2 * bytes);
-          dev::bulk_g2s(mb, static_cast<const uint8_t*>(a.mu) + row * D * 2, bytes, &B.meta[buf]);
-          dev::bulk_g2s(mb + C * D * 2, static_cast<const uint8_t*>(a.sigma) + row * D * 2, bytes, &B.meta[buf]);
-        }
-        meta_pending[buf] = 1;
+      if (lane < G) {
+        float tv_ = tau_h[0];
+#pragma unroll
+        for (int h = 1; h < G; ++h)
+          if (lane == h) tv_ = tau_h[h];
+        a.tau[static_cast<size_t>(seg) * G + lane] = tv_;
       }
-      dev::cp_async_commit();
     };
-    auto push = [&](const FTile& ft) -> bool {
-      if (!dev::warp_wait_or_abort(&B.q_empty[qslot], qphase ^ 1u, a.status, abort_flag)) return false;
-      if (lane == 0) {
-        queue[qslot] = ft;
-        dev::mbar_arrive(&B.q_full[qslot]);
-      }
-      __syncwarp();
-      if (++qslot == kQueue) { qslot = 0; qphase ^= 1u; }
-      return true;
-    };
-    // Two chunks are staged ahead of the one being scored: cur (metadata in
-    // buffer buf), nxt (buffer buf ^ 1); the ticket after nxt is taken while
-    // cur is scored.
-    // cur and nxt are resolved and their metadata staged.  Each iteration
-    // takes one more counter value; its atomic's result is first read one
-    // iteration later (queued then), so the warp never waits for it.
-    Job2 cur, nxt;
-    pq_push(static_cast<unsigned>(rank), home, 1);  // the two fixed chunks of the home segment
-    pq_push(static_cast<unsigned>(rank + hsize), home, 1);
-    bool have_cur = next_job(cur);
-    bool have_nxt = false;
-    int buf = 0;
-    if (have_cur) {
-      stage_meta(cur, 0);
-      have_nxt = next_job(nxt);
-      if (have_nxt) stage_meta(nxt, 1);
-    }
-    while (have_cur && ok) {
-      int r_seg = -1;
-      const unsigned r_new = (have_nxt && gseg >= 0) ? grab() : 0u;
-      if (have_nxt && gseg >= 0) r_seg = gseg;
-      const int seg = cur.seq * s.Hkv + cur.kvh;
-      const int T = seqT[cur.seq];
-      const int blk0 = cur.cidx * C;
-      if (seg != cur_seg) {
-        // the heads' queries, thresholds and norms (all loads issued first)
-        cur_seg = seg;
-        uint2 qu[G];
-        float wv[G][CPL], bc[G];
-        const bool learned = a.tau_mode == ETA_TAU_LEARNED;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          const int hq = cur.kvh * G + h;
-          const size_t qo = (static_cast<size_t>(cur.seq) * s.Hq + hq) * D;
-          qu[h] = *reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(a.q) + qo + lane * CPL);
-#pragma unroll
-          for (int k = 0; k < CPL; ++k) wv[h][k] = learned ? a.w_tau[static_cast<size_t>(hq) * D + lane * CPL + k] : 0.f;
-          bc[h] = learned ? a.b_tau[hq] : a.c_tau[hq];
-        }
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-          qr[h][0] = dev::bf16_lo(qu[h].x);
-          qr[h][1] = dev::bf16_hi(qu[h].x);
-          qr[h][2] = dev::bf16_lo(qu[h].y);
-          qr[h][3] = dev::bf16_hi(qu[h].y);
-          float tw = 0.f, qq = 0.f;
-#pragma unroll
-          for (int k = 0; k < CPL; ++k) {
-            q2[h][k] = qr[h][k] * qr[h][k];
-            qq = fmaf(qr[h][k], qr[h][k], qq);
-            tw = fmaf(wv[h][k], qr[h][k], tw);
+    int* r_nsc = sseg;  // per chunk of the round: blocks screened, first metadata row (the
+    int* r_row = scid;  // producer's slice tables are not in use yet)
+    for (int r0 = 0; r0 < nslice; r0 += R) {
+      const int nr = min(R, nslice - r0);
+      if (a.screen_enabled) {
+        if (warp == 0) {
+          for (int k = lane; k < nr; k += 32) {
+            int seg, cidx, nloc, nsc;
+            chunk_rows(r_lo + r0 + k, seg, cidx, nloc, nsc);
+            r_nsc[k] = nsc;
+            r_row[k] = seg * s.nbmax + cidx * C;  // < 2^31: the cache holds fewer rows
           }
-          tw = dev::warp_sum(tw);
-          qq = dev::warp_sum(qq);
-          tau_h[h] = (learned ? tw + bc[h] : bc[h]) - a.offset_a;
-          qn_h[h] = sqrtf(qq);
+        }
+        __syncthreads();
+        const int per_chunk = 32 << lc;  // 16-byte pieces of mu and sigma rows of a full chunk
+        for (int x = t; x < nr * per_chunk; x += kThreads) {
+          const int k = x >> (5 + lc), r = x & (per_chunk - 1);
+          const int arr = r >> (4 + lc), j = (r >> 4) & (C - 1), pc = r & 15;
+          if (j < r_nsc[k]) {
+            const uint8_t* src = static_cast<const uint8_t*>(arr ? a.sigma : a.mu) +
+                                 (static_cast<size_t>(r_row[k]) + j) * D * 2 + pc * 16;
+            dev::cp_async16(scr + static_cast<size_t>(k) * 2 * mstride + arr * mstride + j * D * 2 + pc * 16, src);
+          }
+        }
+        for (int x = t; x < nr * C; x += kThreads) {
+          const int k = x >> lc, j = x & (C - 1);
+          if (j < r_nsc[k]) dev::cp_async4(&mn_s[x], a.max_norm + r_row[k] + j);
+        }
+        dev::cp_async_commit();
+      }
+      // the threshold of each warp's first chunk while the copies fly
+      if (r0 + warp < r0 + nr) {
+        int seg, cidx, nloc, nsc;
+        chunk_rows(r_lo + r0 + warp, seg, cidx, nloc, nsc);
+        if (seg != cseg) {
+          cseg = seg;
+          const int i = seg / s.Hkv, g = seg - i * s.Hkv;
+          compute_tau(i, g, seg);
         }
       }
-      // head masks of the chunk's blocks: lane l <-> block blk0 + l
-      unsigned mymask = lane < cur.nloc ? ((1u << G) - 1u) : 0u;  // forced window / screen off
-      if (cur.nscreen > 0) {
-        if (have_nxt) dev::cp_async_wait<1>(); else dev::cp_async_wait<0>();  // this chunk's block norms
-        __syncwarp();
-        if (!dev::warp_wait_or_abort(&B.meta[buf], meta_phase[buf], a.status, abort_flag)) { ok = false; break; }
-        meta_phase[buf] ^= 1u;
-        meta_pending[buf] = 0;
-        const uint8_t* mu_s = base + L.meta + static_cast<size_t>(buf) * 2 * C * D * 2;
-        const uint8_t* sg_s = mu_s + C * D * 2;
-        const float* mn = reinterpret_cast<const float*>(base + L.mnorm) + buf * C;
-        const float scale = a.scale, z = a.z;
-        const bool strict = isinf(z);
-        const int vb = lane / NV, vq = lane % NV;
-        for (int gb = 0; gb < cur.nscreen; gb += NB) {
-          float v[32];
+      if (a.screen_enabled) dev::cp_async_wait<0>();
+      __syncthreads();  // every thread's copies have landed
+      for (int k = r0 + warp; k < r0 + nr; k += kWarps) {
+        int seg, cidx, nloc, nscreen;
+        chunk_rows(r_lo + k, seg, cidx, nloc, nscreen);
+        const int i = seg / s.Hkv, g = seg - i * s.Hkv;
+        const int blk0 = cidx * C;
+        if (seg != cseg) {
+          cseg = seg;
+          compute_tau(i, g, seg);
+        }
+        // head masks of the chunk's blocks: lane l <-> block blk0 + l
+        unsigned mymask = lane < nloc ? kFullMask : 0u;  // forced window / screen off
+        if (nscreen > 0) {
+          {
+            const uint8_t* mu_s = scr + static_cast<size_t>(k - r0) * 2 * mstride;
+            const uint8_t* sg_s = mu_s + mstride;
+            const float* mn = mn_s + (k - r0) * C;
+            for (int gb = 0; gb < nscreen; gb += NB) {
+              float v[32];
 #pragma unroll
-          for (int u = 0; u < NB; ++u) {
-            const int lb = min(gb + u, cur.nscreen - 1);
-            const uint2 mm = *reinterpret_cast<const uint2*>(mu_s + (lb * D + lane * CPL) * 2);
-            const uint2 gg = *reinterpret_cast<const uint2*>(sg_s + (lb * D + lane * CPL) * 2);
-            float mu[CPL], s2[CPL];
-            mu[0] = dev::fp16_to_f32(static_cast<uint16_t>(mm.x & 0xffffu));
-            mu[1] = dev::fp16_to_f32(static_cast<uint16_t>(mm.x >> 16));
-            mu[2] = dev::fp16_to_f32(static_cast<uint16_t>(mm.y & 0xffffu));
-            mu[3] = dev::fp16_to_f32(static_cast<uint16_t>(mm.y >> 16));
-            const float g0 = dev::fp16_to_f32(static_cast<uint16_t>(gg.x & 0xffffu));
-            const float g1 = dev::fp16_to_f32(static_cast<uint16_t>(gg.x >> 16));
-            const float g2 = dev::fp16_to_f32(static_cast<uint16_t>(gg.y & 0xffffu));
-            const float g3 = dev::fp16_to_f32(static_cast<uint16_t>(gg.y >> 16));
-            s2[0] = g0 * g0;
-            s2[1] = g1 * g1;
-            s2[2] = g2 * g2;
-            s2[3] = g3 * g3;
+              for (int u = 0; u < NB; ++u) {
+                const int lb = min(gb + u, nscreen - 1);
+                const uint2 m2 = *reinterpret_cast<const uint2*>(mu_s + (lb * D + lane * CPL) * 2);
+                const uint2 s2b = *reinterpret_cast<const uint2*>(sg_s + (lb * D + lane * CPL) * 2);
+                float mu[CPL], s2[CPL];
+                mu[0] = dev::fp16_to_f32(static_cast<uint16_t>(m2.x & 0xffffu));
+                mu[1] = dev::fp16_to_f32(static_cast<uint16_t>(m2.x >> 16));
+                mu[2] = dev::fp16_to_f32(static_cast<uint16_t>(m2.y & 0xffffu));
+                mu[3] = dev::fp16_to_f32(static_cast<uint16_t>(m2.y >> 16));
+                const float g0 = dev::fp16_to_f32(static_cast<uint16_t>(s2b.x & 0xffffu));
+                const float g1 = dev::fp16_to_f32(static_cast<uint16_t>(s2b.x >> 16));
+                const float g2 = dev::fp16_to_f32(static_cast<uint16_t>(s2b.y & 0xffffu));
+                const float g3 = dev::fp16_to_f32(static_cast<uint16_t>(s2b.y >> 16));
+                s2[0] = g0 * g0;
+                s2[1] = g1 * g1;
+                s2[2] = g2 * g2;
+                s2[3] = g3 * g3;
 #pragma unroll
-            for (int h = 0; h < G; ++h) {
-              float dot = 0.f, sq = 0.f;
+                for (int h = 0; h < G; ++h) {
+                  float dot = 0.f, sq = 0.f;
 #pragma unroll
-              for (int k = 0; k < CPL; ++k) {
-                dot = fmaf(qr[h][k], mu[k], dot);
-                sq = fmaf(q2[h][k], s2[k], sq);
+                  for (int c = 0; c < CPL; ++c) {
+                    dot = fmaf(qr[h][c], mu[c], dot);
+                    sq = fmaf(q2[h][c], s2[c], sq);
+                  }
+                  v[u * NV + h] = dot;
+                  v[u * NV + G + h] = sq;
+                }
               }
-              v[u * NV + h] = dot;
-              v[u * NV + G + h] = sq;
+              const float redv = dev::transpose_reduce32<32>(v, lane);
+              const float sqv = __shfl_down_sync(0xffffffffu, redv, G);  // sum q^2 sigma^2 of the same (block, head)
+              const int lb = gb + vb;
+              bool pass = false;
+              if (vq < G && lb < nscreen) {
+                float tq = tau_h[0], qn = qn_h[0];
+#pragma unroll
+                for (int h = 1; h < G; ++h)
+                  if (vq == h) { tq = tau_h[h]; qn = qn_h[h]; }
+                const float geo = qn * mn[lb];
+                const float spread = strict ? geo : fminf(geo, z * sqrtf(sqv));
+                pass = scale * (redv + spread) >= tq;
+              }
+              const unsigned bal = __ballot_sync(0xffffffffu, pass);
+              // block gb + u's head bits sit at lanes u NV .. u NV + G - 1
+#pragma unroll
+              for (int u = 0; u < NB; ++u) {
+                const int blk = gb + u;
+                if (lane == blk && blk < nscreen) mymask = (bal >> (u * NV)) & kFullMask;
+              }
             }
           }
-          float redv = dev::transpose_reduce32<32>(v, lane);
-          const float sqv = __shfl_down_sync(0xffffffffu, redv, G);  // sum q^2 sigma^2 of the same (block, head)
-          const int lb = gb + vb;
-          bool pass = false;
-          if (vq < G && lb < cur.nscreen) {
-            float tq = tau_h[0], qn = qn_h[0];
-#pragma unroll
-            for (int h = 1; h < G; ++h)
-              if (vq == h) { tq = tau_h[h]; qn = qn_h[h]; }
-            const float geo = qn * mn[lb];
-            const float spread = strict ? geo : fminf(geo, z * sqrtf(sqv));
-            pass = scale * (redv + spread) >= tq;
-          }
-          const unsigned bal = __ballot_sync(0xffffffffu, pass);
-          // block gb + u's head bits sit at lanes u NV .. u NV + G - 1
-#pragma unroll
-          for (int u = 0; u < NB; ++u) {
-            const unsigned m = (bal >> (u * NV)) & ((1u << G) - 1u);
-            if (lane == gb + u && gb + u < cur.nscreen) mymask = m;
-          }
+        }
+        // ascending admitted list of the chunk and its count
+        const unsigned adm = __ballot_sync(0xffffffffu, mymask != 0u);
+        if (mymask != 0u)
+          a.chunk_list[static_cast<size_t>(seg) * s.list_stride + static_cast<size_t>(cidx) * C +
+                       __popc(adm & ((1u << lane) - 1u))] = (blk0 + lane) | static_cast<int>(mymask << kEntryBlockBits);
+        if (lane == 0) {
+          a.chunk_count[static_cast<size_t>(seg) * s.nchunks + cidx] = __popc(adm);
+          own[k] = __popc(adm);
         }
       }
-      // ascending admitted list of the chunk (selection export) and its tiles
-      const unsigned adm = __ballot_sync(0xffffffffu, mymask != 0u);
-      const int nadm = __popc(adm);
-      if (mymask != 0u) {
-        const int k = __popc(adm & ((1u << lane) - 1u));
-        a.chunk_list[static_cast<size_t>(seg) * s.list_stride + static_cast<size_t>(cur.cidx) * C + k] =
-            (blk0 + lane) | static_cast<int>(mymask << kEntryBlockBits);
-      }
-      if (lane == 0) a.chunk_count[static_cast<size_t>(seg) * s.nchunks + cur.cidx] = nadm;
-      // rows of every block of the chunk (page table lookups in parallel)
-      bool bad = false;
-      const long long myrow = lane < cur.nloc ? lay.row(seg, blk0 + lane, &bad) : 0;
-      if (bad) atomicOr(a.status, kStatusRange);
-      const int ntile = nadm == 0 ? 1 : (nadm + BPT - 1) / BPT;
-      unsigned rest = adm;
-      for (int ti = 0; ti < ntile && ok; ++ti) {
-        FTile ft;
-        ft.seq = cur.seq;
-        ft.kvh = cur.kvh;
-        ft.cidx = cur.cidx;
-        ft.pad0 = 0;
-        ft.flags = (ti == 0 ? kFirst : 0) | (ti == ntile - 1 ? kLast : 0);
-        ft.pad1 = 0;
-#pragma unroll
-        for (int h = 0; h < 8; ++h) ft.tau[h] = h < G ? tau_h[h] : 0.f;
-        int l0 = -1, l1 = -1;
-        if (rest) { l0 = __ffs(rest) - 1; rest &= rest - 1u; }
-        if (BPT == 2 && rest) { l1 = __ffs(rest) - 1; rest &= rest - 1u; }
-        const unsigned m0 = __shfl_sync(0xffffffffu, mymask, l0 < 0 ? 0 : l0);
-        const unsigned m1 = __shfl_sync(0xffffffffu, mymask, l1 < 0 ? 0 : l1);
-        const long long r0 = __shfl_sync(0xffffffffu, myrow, l0 < 0 ? 0 : l0);
-        const long long r1 = __shfl_sync(0xffffffffu, myrow, l1 < 0 ? 0 : l1);
-        ft.mask0 = l0 < 0 ? 0 : static_cast<int>(m0);
-        ft.mask1 = l1 < 0 ? 0 : static_cast<int>(m1);
-        ft.nrows0 = l0 < 0 ? 0 : min(s.b, T - (blk0 + l0) * s.b);
-        ft.nrows1 = l1 < 0 ? 0 : min(s.b, T - (blk0 + l1) * s.b);
-        ft.row0 = l0 < 0 ? 0 : r0;
-        ft.row1 = l1 < 0 ? 0 : r1;
-        if (!push(ft)) ok = false;
-      }
-      if (!ok) break;
-      // advance: nxt becomes cur; the ticket taken above becomes nxt (its
-      // metadata into the buffer cur just released)
-      cur = nxt;
-      have_cur = have_nxt;
-      buf ^= 1;
-      if (r_seg >= 0) pq_push(r_new, r_seg, 0);
-      if (have_cur) {
-        have_nxt = next_job(nxt);
-        if (have_nxt) stage_meta(nxt, buf ^ 1);
-      }
+      fence_proxy_async();  // generic reads of the staging area come before any later copy into it
+      __syncthreads();
     }
-    if (ok) {
-      FTile end{};
-      end.flags = kEnd;
-      ok = push(end);
+    __threadfence();
+    __syncthreads();
+    if (t == 0) {
+      int total = 0;
+      for (int k = 0; k < nslice; ++k) total += own[k];
+      a.flags[cta] = static_cast<unsigned>(total) + 1u;
+      __threadfence();
+      red_release_add(a.arrived, 1u);
     }
-    dev::cp_async_wait<0>();  // no asynchronous copy outlives the warp
-    if (!ok && lane == 0) {
-      *abort_flag = 1;
-      for (int k = 0; k < 2; ++k) {  // staged copies land before the CTA exits
-        if (!meta_pending[k]) continue;
-        const long long t0 = clock64();
-        while (!dev::mbar_try_wait(&B.meta[k], meta_phase[k]) && clock64() - t0 < dev::kWaitCycles) {
-        }
-      }
-    }
-  } else if (warp == 0) {
-    // ============================================================ producer
-    if (lane == 0) {
-      int stage = 0, qslot = 0;
-      uint32_t phase = 0, qphase = 0;
-      bool ok = true;
-      while (ok) {
-        if (!wait_or_abort(&B.q_full[qslot], qphase, a.status, abort_flag)) { ok = false; break; }
-        const FTile ft = queue[qslot];
-        dev::mbar_arrive(&B.q_empty[qslot]);
-        if (++qslot == kQueue) { qslot = 0; qphase ^= 1u; }
-        if (!wait_or_abort(&B.kv_empty[stage], phase ^ 1u, a.status, abort_flag)) { ok = false; break; }
-        info[stage] = ft;
-        if (ft.flags & kEnd) {
-          dev::mbar_arrive(&B.kv_full[stage]);
+  }
+
+  if (warp == 0) {
+    // ============================================================ 2. exchange, 3. producer
+    bool ok = true;
+    {
+      // wait (bounded) until every CTA has published its slice total: the
+      // warp polls one counter, then reads all totals, eight loads in
+      // flight per lane (acquire: the lists published with them are visible)
+      const long long t0 = clock64();
+      for (;;) {
+        const unsigned n = ld_acquire(a.arrived);
+        if (__all_sync(0xffffffffu, n >= static_cast<unsigned>(N))) break;
+        if (clock64() - t0 > dev::kWaitCycles) {
+          ok = false;
           break;
         }
+        __nanosleep(100);
+      }
+      const int per = (N + 31) / 32;
+      const int lo = min(N, lane * per), hi = min(N, lo + per);
+      int sum = 0;
+      for (int x0 = lo; x0 < hi && ok; x0 += 8) {
+        unsigned v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = x0 + u < hi ? __ldcg(a.flags + x0 + u) : 1u;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (x0 + u < hi) {
+            if (v[u] == 0u) ok = false;  // published (the counter says so) yet zero: a stale control region
+            P[x0 + u] = static_cast<int>(v[u]) - 1;
+            sum += static_cast<int>(v[u]) - 1;
+          }
+        }
+      }
+      ok = __all_sync(0xffffffffu, ok ? 1 : 0) != 0;
+      int incl = sum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int run = incl - sum;
+      for (int x = lo; x < hi; ++x) {
+        const int c = P[x];
+        P[x] = run;
+        run += c;
+      }
+      if (lane == 31) P[N] = incl;
+      __syncwarp();
+    }
+    if (!ok) {
+      if (lane == 0) {
+        atomicOr(a.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+    } else {
+      const int U = P[N];
+      if (lane == 0) *units_total = U;  // read by the softmax warps after the ring's first entry
+      const dev::UnitSplit us(static_cast<unsigned>(U), static_cast<unsigned>(N));
+      const int u0 = static_cast<int>(us.start(cta)), u1 = static_cast<int>(us.start(cta + 1));
+      const KvLayout lay{a.block_table, s.Hkv, s.b, s.max_ctx, s.nbmax, s.num_pages};
+      // admitted count of chunk number r, read by one lane
+      auto chunk_count = [&](int r, int sl) -> int {
+        if (sl == cta) return own[r - r_lo];
+        int sg, ci;
+        ch.locate(r, sg, ci);
+        return __ldcg(a.chunk_count + static_cast<size_t>(sg) * s.nchunks + ci);
+      };
+      // units in the chunks numbered below r (warp-wide)
+      auto units_before = [&](int r) -> int {
+        if (r >= NC) return U;
+        const int sl = static_cast<int>(slices.owner(static_cast<unsigned>(r)));
+        const int lo = static_cast<int>(slices.start(sl));
+        int sum = 0;
+        for (int x = lo + lane; x < r; x += 32) sum += chunk_count(x, sl);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        return P[sl] + sum;
+      };
+
+      int stage = 0;
+      uint32_t phase = 0;
+      FInfo pend{-1, 0, 0, 0, 0, 0};
+      int prow[2] = {0, 0};
+      int npend = 0;
+      int carry = 0;  // mode of the run closed by the next ring entry
+      // (lane 0) put the pending tile into the ring
+      auto emit = [&]() -> bool {
+        if (!wait_or_abort(&B.kv_empty[stage], phase ^ 1u, a.status, abort_flag)) return false;
+        pend.prev_mode = carry;
+        carry = 0;
+        info[stage] = pend;
         const uint32_t st = base_u32 + static_cast<uint32_t>(L.stages + stage * TL::STAGE);
-        const int nblk = (ft.nrows0 > 0) + (ft.nrows1 > 0);
-        dev::mbar_arrive_expect_tx(&B.kv_full[stage], static_cast<uint32_t>(nblk * 4 * BR * 128 + 4096));
-        for (int i = 0; i < BPT; ++i) {
-          const int nr = i == 0 ? ft.nrows0 : ft.nrows1;
-          if (nr <= 0) continue;
-          const int krow = static_cast<int>(i == 0 ? ft.row0 : ft.row1);
-          const uint32_t ro = static_cast<uint32_t>(i * BR * 128);
+        dev::mbar_arrive_expect_tx(&B.kv_full[stage], static_cast<uint32_t>(npend * 4 * BR * 128 + 4096));
+        for (int x = 0; x < npend; ++x) {
+          const int krow = prow[x];
+          const uint32_t ro = static_cast<uint32_t>(x * BR * 128);
           tma_load_2d(st + TL::K0 + ro, &tk, 0, krow, &B.kv_full[stage]);
           tma_load_2d(st + TL::K1 + ro, &tk, 64, krow, &B.kv_full[stage]);
           tma_load_2d(st + TL::V0 + ro, &tv, 0, krow, &B.kv_full[stage]);
           tma_load_2d(st + TL::V1 + ro, &tv, 64, krow, &B.kv_full[stage]);
         }
-        const int qrow = (ft.seq * s.Hkv + ft.kvh) * G;
+        const int qrow = pend.seg * s.G;
         tma_load_2d(st + TL::Q0, &tq, 0, qrow, &B.kv_full[stage]);
         tma_load_2d(st + TL::Q1, &tq, 64, qrow, &B.kv_full[stage]);
         issued_parity[stage] = static_cast<int>(phase);
         if (++stage == kStages) { stage = 0; phase ^= 1u; }
-      }
-      if (!ok) {
-        *abort_flag = 1;
-        for (int k = 0; k < kStages; ++k) {  // let issued copies land
-          if (issued_parity[k] < 0) continue;
-          const long long t0 = clock64();
-          while (!dev::mbar_try_wait(&B.kv_full[k], static_cast<uint32_t>(issued_parity[k])) &&
-                 clock64() - t0 < dev::kWaitCycles) {
+        npend = 0;
+        return true;
+      };
+      // (warp) flush the pending tile
+      auto emit_pending = [&]() -> bool {
+        int r = 1;
+        if (lane == 0 && npend > 0) r = emit() ? 1 : 0;
+        return __shfl_sync(0xffffffffu, r, 0) != 0;
+      };
+      // (warp) the mode of the run of segment rseg that ends here
+      auto close_run = [&](int rseg, bool first_run, bool at_u1) -> int {
+        const int f = ch.first(rseg);
+        const bool shared_start = first_run && units_before(f) < u0;
+        const bool shared_end = at_u1 && units_before(f + ch.nch(rseg / s.Hkv)) > u1;
+        int mode = (shared_start ? 0 : kModeFirst) | (shared_end ? 0 : kModeLast);
+        if (shared_start || shared_end) mode |= kModeShared | (first_run ? 0 : kModeSlot1);
+        return mode;
+      };
+
+      int run_seg = -1;
+      bool first_run = true;
+      if (u0 < u1) {
+        int sl = 0, hi = N;  // slice holding unit u0: the last with P[sl] <= u0
+        while (hi - sl > 1) {
+          const int mid = (sl + hi) >> 1;
+          if (P[mid] <= u0) sl = mid; else hi = mid;
+        }
+        int u = u0;
+        for (; ok && u < u1 && sl < N; ++sl) {
+          const int rlo = static_cast<int>(slices.start(sl));
+          const int n = static_cast<int>(slices.start(sl + 1)) - rlo;
+          // the slice's chunk counts (lane l: chunks l and l + 32), their
+          // segments and chunk indices, and the running count before each
+          int cnt0 = 0, cnt1 = 0;
+          if (lane < n) {
+            cnt0 = chunk_count(rlo + lane, sl);
+            ch.locate(rlo + lane, sseg[lane], scid[lane]);
           }
+          if (lane + 32 < n) {
+            cnt1 = chunk_count(rlo + lane + 32, sl);
+            ch.locate(rlo + lane + 32, sseg[lane + 32], scid[lane + 32]);
+          }
+          if (dev::chunk_count_faults(C, cnt0) | dev::chunk_count_faults(C, cnt1)) cnt0 = -1;
+          if (__any_sync(0xffffffffu, cnt0 < 0)) {
+            if (lane == 0) atomicOr(a.status, kStatusList);
+            ok = false;
+            break;
+          }
+          int i0 = cnt0, i1 = cnt1;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y0 = __shfl_up_sync(0xffffffffu, i0, o);
+            const int y1 = __shfl_up_sync(0xffffffffu, i1, o);
+            if (lane >= o) { i0 += y0; i1 += y1; }
+          }
+          const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
+          const int tot = tot0 + __shfl_sync(0xffffffffu, i1, 31);
+          if (lane < n) spre[lane] = i0 - cnt0;
+          if (lane + 32 < n) spre[lane + 32] = tot0 + i1 - cnt1;
+          if (lane == 0) spre[n] = tot;
+          __syncwarp();
+          if (tot != P[sl + 1] - P[sl]) {  // totals and lists disagree
+            if (lane == 0) atomicOr(a.status, kStatusList);
+            ok = false;
+            break;
+          }
+          // chunk k of the slice holding position pos (the last with spre[k] <= pos)
+          auto chunk_of = [&](int pos) -> int {
+            int lo = 0, hi = n;
+            while (hi - lo > 1) {
+              const int mid = (lo + hi) >> 1;
+              if (spre[mid] <= pos) lo = mid; else hi = mid;
+            }
+            return lo;
+          };
+          const int pa = u - P[sl], pb = min(u1, P[sl + 1]) - P[sl];  // this range's positions in the slice
+          for (int bb = pa; bb < pb && ok; bb += kEntStage) {
+            // stage up to kEntStage entries with independent loads (one round trip)
+            const int m = min(kEntStage, pb - bb);
+            for (int x = lane; x < m; x += 32) {
+              const int k = chunk_of(bb + x);
+              ent_s[x] = __ldcg(a.chunk_list + static_cast<size_t>(sseg[k]) * s.list_stride +
+                                static_cast<size_t>(scid[k]) * C + (bb + x - spre[k]));
+            }
+            __syncwarp();
+            for (int k = chunk_of(bb); k < n && spre[k] < bb + m && ok; ++k) {
+              const int xa = max(spre[k], bb) - bb, xb = min(spre[k + 1], bb + m) - bb;
+              if (xb <= xa) continue;
+              const int seg = sseg[k], cidx = scid[k];
+              if (seg != run_seg) {
+                if (run_seg >= 0) {
+                  if (!emit_pending()) { ok = false; break; }
+                  carry = close_run(run_seg, first_run, false);
+                  first_run = false;
+                }
+                run_seg = seg;
+              }
+              const int T = seqT[seg / s.Hkv];
+              const int nblk = (T + s.b - 1) / s.b;
+              const int nn = xb - xa;  // <= C <= 32
+              const int e = lane < nn ? ent_s[xa + lane] : 0;
+              const int eb = e & kMaxBlocksPerSeq;
+              const int up = __shfl_up_sync(0xffffffffu, eb, 1);
+              // the entry before the first one, when it is in the same chunk and staged
+              const int first_prev = (xa > 0 && bb + xa > spre[k]) ? (ent_s[xa - 1] & kMaxBlocksPerSeq) : -1;
+              const unsigned f = lane < nn ? dev::list_entry_faults(C, G, nblk, cidx, e, lane == 0 ? first_prev : up) : 0u;
+              if (__any_sync(0xffffffffu, f != 0u)) {
+                if (lane == 0) atomicOr(a.status, kStatusList);
+                ok = false;
+                break;
+              }
+              bool bad = false;
+              const long long rw = lane < nn ? lay.row(seg, eb, &bad) : 0;
+              if (bad) atomicOr(a.status, kStatusRange);
+              int okl = 1;
+              for (int jj = 0; jj < nn; ++jj) {
+                const int ent = __shfl_sync(0xffffffffu, e, jj);
+                const long long er = __shfl_sync(0xffffffffu, rw, jj);
+                if (lane == 0 && okl) {
+                  const int blk = ent & kMaxBlocksPerSeq;
+                  if (npend > 0 && seg != pend.seg && !emit()) okl = 0;
+                  if (okl) {
+                    if (npend == 0) pend = FInfo{seg, 0, 0, 0, 0, 0};
+                    prow[npend] = static_cast<int>(er);
+                    const int mask = static_cast<int>(static_cast<unsigned>(ent) >> kEntryBlockBits);
+                    const int nrows = min(s.b, T - blk * s.b);
+                    if (npend == 0) { pend.mask0 = mask; pend.nrows0 = nrows; }
+                    else { pend.mask1 = mask; pend.nrows1 = nrows; }
+                    ++npend;
+                    if (npend == BPT && !emit()) okl = 0;
+                  }
+                }
+              }
+              ok = __shfl_sync(0xffffffffu, okl, 0) != 0;
+            }
+            __syncwarp();  // ent_s is restaged next round
+          }
+          u = P[sl] + pb;
+        }
+        if (ok && u != u1) {  // the slices ran out before the range did
+          if (lane == 0) atomicOr(a.status, kStatusList);
+          ok = false;
+        }
+      }
+      if (ok) ok = emit_pending();
+      if (ok) {
+        const int mode = run_seg >= 0 ? close_run(run_seg, first_run, true) : 0;
+        int r = 1;
+        if (lane == 0) {
+          if (wait_or_abort(&B.kv_empty[stage], phase ^ 1u, a.status, abort_flag)) {
+            info[stage] = FInfo{-1, 0, 0, 0, 0, mode};
+            dev::mbar_arrive(&B.kv_full[stage]);
+          } else {
+            r = 0;
+          }
+        }
+        ok = __shfl_sync(0xffffffffu, r, 0) != 0;
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      for (int k = 0; k < kStages; ++k) {  // let issued copies land
+        if (issued_parity[k] < 0) continue;
+        const long long t0 = clock64();
+        while (!dev::mbar_try_wait(&B.kv_full[k], static_cast<uint32_t>(issued_parity[k])) &&
+               clock64() - t0 < dev::kWaitCycles) {
         }
       }
     }
@@ -844,12 +846,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       return true;
     };
-    int j = 0;
-    for (;; ++j) {
+    for (int j = 0; ok; ++j) {
       const int st_j = j % kStages;
       const int sb = j & 1;
       if (!wait_or_abort(&B.kv_full[st_j], (j / kStages) & 1, a.status, abort_flag)) { ok = false; break; }
-      if (info[st_j].flags & kEnd) break;
+      if (info[st_j].seg < 0) {  // END
+        if (j > 0) ok = issue_pv(j - 1);
+        break;
+      }
       if (!wait_or_abort(&B.s_free[sb], ((j >> 1) & 1) ^ 1, a.status, abort_flag)) { ok = false; break; }
       tc_fence_after();
       if (lane == 0) {
@@ -867,7 +871,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
     }
-    if (ok && j > 0) issue_pv(j - 1);
+    // every MMA issued so far has completed once `done` flips
     if (lane == 0) mma_commit(B.done);
     __syncwarp();
     {
@@ -875,127 +879,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (!dev::mbar_try_wait(B.done, 0) && clock64() - t0 < dev::kWaitCycles) {
       }
     }
-  } else if (warp == kDoneWarp) {
-    // ============================================================ completion
-    // Events arrive in the order the softmax warps posted them; each
-    // increments the counter of its parent node, and the thread that
-    // completes a node resets the counter.  While the CTA still streams tiles
-    // the completed nodes only queue up here (counting never waits for a
-    // fold, so a busy CTA does not attract more folds); once the softmax
-    // warps are done (their END event) the nodes go to them as fold jobs,
-    // each staged with one bulk copy into the then idle K/V stage memory.
-    // A node whose fold completes its parent queues the parent in turn.
-    int eslot = 0, jslot = 0, outstanding = 0;
-    uint32_t ephase = 0, jphase = 0;
-    bool got_end = false, ok = true;
-    unsigned* pend_nodes = reinterpret_cast<unsigned*>(base + L.pend);
-    int phead = 0, npend = 0;
-    auto pack = [](int level, int seg, int node) -> unsigned {
-      return (static_cast<unsigned>(level) << 28) | (static_cast<unsigned>(seg) << 14) | static_cast<unsigned>(node);
-    };
-    // node (level, node) of segment seg has its partial (or, at the root,
-    // the output): count it at its parent; a completed parent is queued (or,
-    // with the queue full, folded by this warp alone from global memory)
-    auto complete_up = [&](int seq, int kvh, int level, int node) {
-      const int seg = seq * s.Hkv + kvh;
-      for (;;) {
-        const int nl = tb.nodes(seq, level);
-        if (level > 0 && nl == 1) return;  // the root: the output is written
-        const int lp = level + 1;
-        const int parent = node / kFoldFan;
-        const int nchild = min(kFoldFan, nl - parent * kFoldFan);
-        unsigned* ctr = a.counters + a.cbase[lp] + static_cast<size_t>(seg) * s.M[lp] + parent;
-        int complete = 0;
-        __syncwarp();  // this warp's fold writes precede the release below
-        if (lane == 0) {
-          const unsigned before = atom_add_acq_rel(ctr, 1u);
-          complete = before + 1u == static_cast<unsigned>(nchild);
-          if (complete) *ctr = 0u;  // back to zero for the next step
-        }
-        complete = __shfl_sync(0xffffffffu, complete, 0);
-        if (!complete) return;
-        __syncwarp();  // the other lanes' reads of the children follow lane 0's acquire
-        if (npend < kPendNodes) {
-          if (lane == 0) pend_nodes[(phead + npend) % kPendNodes] = pack(lp, seg, parent);
-          __syncwarp();
-          ++npend;
-          return;
-        }
-        const int nparent = tb.nodes(seq, lp);
-        const size_t first = static_cast<size_t>(seg) * s.M[level] + static_cast<size_t>(parent) * kFoldFan;
-        float* dst = nparent == 1 ? nullptr : a.lpart[lp] + (static_cast<size_t>(seg) * s.M[lp] + parent) * G * FPS;
-        fold_partials<G>(a.lpart[level], first, nchild, dst, a, seq, kvh, 0, 1, lane);
-        level = lp;
-        node = parent;
-      }
-    };
-    long long idle_since = clock64();
-    while (ok) {
-      if (got_end && outstanding == 0 && npend == 0) break;
-      bool progress = false;
-      // a queued node to the softmax warps, if a job slot is free
-      if (got_end && npend > 0 &&
-          __shfl_sync(0xffffffffu, dev::mbar_test_wait(&B.job_empty[jslot], jphase ^ 1u) ? 1 : 0, 0)) {
-        if (lane == 0) {
-          const unsigned pk = pend_nodes[phead];
-          const int seg = static_cast<int>((pk >> 14) & 0x3fffu);
-          jobs[jslot] = Job{0, seg / s.Hkv, seg % s.Hkv, static_cast<int>(pk >> 28), static_cast<int>(pk & 0x3fffu),
-                            {0, 0, 0}};
-          dev::mbar_arrive(&B.job_full[jslot]);
-        }
-        __syncwarp();
-        if (++jslot == kJobs) { jslot = 0; jphase ^= 1u; }
-        phead = (phead + 1) % kPendNodes;
-        --npend;
-        ++outstanding;
-        progress = true;
-      }
-      // the next event, if one is there
-      if (__shfl_sync(0xffffffffu, dev::mbar_test_wait(&B.ev_full[eslot], ephase) ? 1 : 0, 0)) {
-        const Event ev = events[eslot];
-        __syncwarp();
-        if (lane == 0) dev::mbar_arrive(&B.ev_empty[eslot]);
-        if (++eslot == kEvents) { eslot = 0; ephase ^= 1u; }
-        if (ev.kind == 1) {
-          got_end = true;
-        } else {
-          if (ev.level > 0) --outstanding;  // a fold the softmax warps ran
-          complete_up(ev.seq, ev.kvh, ev.level, ev.node);
-        }
-        progress = true;
-      }
-      if (progress) {
-        idle_since = clock64();
-      } else if (*abort_flag) {
-        ok = false;
-      } else if (clock64() - idle_since > dev::kWaitCycles) {
-        if (lane == 0) atomicOr(a.status, kStatusTimeout);
-        ok = false;
-      }
-    }
-    Job fin{1, 0, 0, 0, 0, {0, 0, 0}};
-    if (!ok) *abort_flag = 1;
-    // lets the softmax warps finish (they also stop on an abort)
-    if (dev::warp_wait_or_abort(&B.job_empty[jslot], jphase ^ 1u, a.status, abort_flag)) {
-      if (lane == 0) {
-        jobs[jslot] = fin;
-        dev::mbar_arrive(&B.job_full[jslot]);
-      }
-      __syncwarp();
-    }
   } else {
-    // ============================================================ softmax / correction / folds
-    const int q4 = warp & 3;  // tensor-memory lane quarter of this warp
-    const int w4 = warp - 2;  // 0..3
+    // ============================================================ softmax / correction / merge
+    const int q4 = warp & 3;  // TMEM lane quarter this warp may access
     const uint32_t tlane = static_cast<uint32_t>(32 * q4) << 16;
     const int row = 32 * q4 + lane;  // key row of the tile this thread owns in S^T
     const int rblk = row / BR, rrow = row - rblk * BR;
     const int dcol = 32 * q4 + lane;  // output coordinate of this thread in O^T
     const float scale = a.scale, beta = a.beta;
-    // the current chunk's running state, and the previous chunk's while its
-    // last tile's O^T is folded in (one tile after the chunk ended)
+    constexpr int PS = partial_stride(D);
     float m_run[G], l_thr[G], acc[G], alpha_prev[G], tau_h[G];
-    float m_old[G], l_old[G], acc_old[G], alpha_old[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       m_run[h] = -INFINITY;
@@ -1003,16 +896,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc[h] = 0.f;
       alpha_prev[h] = 1.f;
       tau_h[h] = 0.f;
-      m_old[h] = -INFINITY;
-      l_old[h] = 0.f;
-      acc_old[h] = 0.f;
-      alpha_old[h] = 1.f;
     }
-    int cur_seq = 0, cur_kvh = 0, cur_cidx = 0, old_seq = 0, old_kvh = 0, old_cidx = 0;
-    bool have_old = false;
+    int cur_seg = -1;
     uint32_t rv_phase = 0;
-    int eslot = 0, jslot = 0;
-    uint32_t ephase = 0, jphase = 0;
     bool ok = true;
 
     auto rendezvous = [&]() -> bool {
@@ -1022,49 +908,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       rv_phase ^= 1u;
       return r;
     };
-    // Every softmax warp waits for the slot, (w4 == 0) writes the record,
-    // and arrives once after its own writes: the completion warp sees the
-    // event when all four warps' writes are done.
-    auto post_event = [&](const Event& ev) -> bool {
-      if (!dev::warp_wait_or_abort(&B.ev_empty[eslot], ephase ^ 1u, a.status, abort_flag)) return false;
-      if (w4 == 0 && lane == 0) events[eslot] = ev;
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(&B.ev_full[eslot]);
-      if (++eslot == kEvents) { eslot = 0; ephase ^= 1u; }
-      return true;
-    };
-    // One fold job (all four warps), after the last tile: the children are
-    // staged with one bulk copy into the K/V stage memory (idle by now),
-    // folded from there, and the job's event follows.
-    uint32_t fold_phase = 0;
-    auto run_job = [&](const Job& jb) -> bool {
-      if (!rendezvous()) return false;  // the previous job's reads of the staged children are done
-      const int seg = jb.seq * s.Hkv + jb.kvh;
-      const int nl = tb.nodes(jb.seq, jb.level);
-      const int nprev = tb.nodes(jb.seq, jb.level - 1);
-      const int first = jb.node * kFoldFan;
-      const int n = min(kFoldFan, nprev - first);
-      const float* src = a.lpart[jb.level - 1] + (static_cast<size_t>(seg) * s.M[jb.level - 1] + first) * G * FPS;
-      float* sm = reinterpret_cast<float*>(base + L.stages);
-      if (w4 == 0 && lane == 0) {
-        // the children were written by other CTAs (ordered before the
-        // completion warp's acquire): visible to the bulk copy's proxy too
-        asm volatile("fence.proxy.async.global;" ::: "memory");
-        const uint32_t bytes = static_cast<uint32_t>(n) * G * FPS * sizeof(float);
-        dev::mbar_arrive_expect_tx(B.fold, bytes);
-        dev::bulk_g2s(sm, src, bytes, B.fold);
-      }
-      if (!dev::warp_wait_or_abort(B.fold, fold_phase, a.status, abort_flag)) return false;
-      fold_phase ^= 1u;
-      float* dst = nl == 1 ? nullptr : a.lpart[jb.level] + (static_cast<size_t>(seg) * s.M[jb.level] + jb.node) * G * FPS;
-      fold_staged<G>(sm, n, dst, a, jb.seq, jb.kvh, w4, lane);
-      __syncwarp();
-      if (lane == 0) dev::mbar_arrive(&B.job_empty[jslot]);
-      if (++jslot == kJobs) { jslot = 0; jphase ^= 1u; }
-      Event ev{0, jb.seq, jb.kvh, jb.level, jb.node, {0, 0, 0}};
-      return post_event(ev);
-    };
-    auto correction = [&](int i, float (&accx)[G], const float (&alphax)[G]) -> bool {
+    auto correction = [&](int i) -> bool {
       const int ob = i & 1;
       if (!dev::warp_wait_or_abort(&B.o_full[ob], (i >> 1) & 1, a.status, abort_flag)) return false;
       tc_fence_after();
@@ -1074,57 +918,201 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) dev::mbar_arrive(&B.o_free[ob]);
 #pragma unroll
-      for (int h = 0; h < G; ++h) accx[h] = fmaf(accx[h], alphax[h], o[h]);
+      for (int h = 0; h < G; ++h) acc[h] = fmaf(acc[h], alpha_prev[h], o[h]);
       return true;
     };
-    // A finished chunk's partial into its slot (each warp its columns and
-    // its share of l), then its event.
-    auto flush = [&](const float (&accx)[G], const float (&mx)[G], const float (&lx)[G], int seq, int kvh,
-                     int cidx) -> bool {
-      const int seg = seq * s.Hkv + kvh;
-      float* part = a.lpart[0] + (static_cast<size_t>(seg) * s.M[0] + cidx) * G * FPS;
+    auto write_out = [&](int seg, const float* l_tot, const float* m, const float* o) {
+      const int i = seg / s.Hkv, g = seg - i * s.Hkv;
 #pragma unroll
       for (int h = 0; h < G; ++h) {
-        part[h * FPS + dcol] = accx[h];
-        const float lw = dev::warp_sum(lx[h]);
-        if (lane == 0) {
-          part[h * FPS + D + 1 + q4] = lw;
-          if (q4 == 0) part[h * FPS + D] = mx[h];
+        const size_t orow = static_cast<size_t>(i) * s.Hq + g * G + h;
+        dev::store_out_slot(a.out, s.elt, orow * D + dcol, l_tot[h] > 0.f ? o[h] / l_tot[h] : 0.f);
+        if (dcol == h && a.lse) a.lse[orow] = dev::lse_of(m[h], l_tot[h]);
+      }
+    };
+    // The run of segment seg ends: written out, or left as this CTA's piece
+    // (and merged here if it completes the segment's set of pieces).
+    auto flush = [&](int seg, int mode) -> bool {
+      float* sums = red + 2 * 4 * 8;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float lw = dev::warp_sum(l_thr[h]);
+        if (lane == 0) sums[q4 * 8 + h] = lw;
+      }
+      if (!rendezvous()) return false;
+      float l_tot[G];
+#pragma unroll
+      for (int h = 0; h < G; ++h) l_tot[h] = sums[h] + sums[8 + h] + sums[16 + h] + sums[24 + h];
+      if (!(mode & kModeShared)) {
+        write_out(seg, l_tot, m_run, acc);
+        return true;
+      }
+      const int slot = 2 * cta + ((mode & kModeSlot1) ? 1 : 0);
+      float* part = a.partials + static_cast<size_t>(slot) * G * PS;
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        part[h * PS + dcol] = acc[h];
+        if (dcol == h) {
+          part[h * PS + D] = m_run[h];
+          part[h * PS + D + 1] = l_tot[h];
         }
       }
-      Event ev{0, seq, kvh, 0, cidx, {0, 0, 0}};
-      return post_event(ev);
+      __threadfence();
+      if (!rendezvous()) return false;  // also: every thread has read sums
+      if (warp == 2 && lane == 0) {
+        // one announcement per piece; the first piece also says which slot
+        // holds it (the pieces of later CTAs are always in their slot 0)
+        const unsigned long long c64 = static_cast<unsigned long long>(cta);
+        unsigned long long add = 1ull;
+        if (mode & kModeFirst) add += (1ull << 16) + ((mode & kModeSlot1) ? (1ull << 18) : 0ull) + (c64 << 32);
+        if (mode & kModeLast) add += (1ull << 17) + (c64 << 48);
+        unsigned long long* ctr = a.seg_ctr + seg;
+        const unsigned long long v = atom_add_acq_rel64(ctr, add) + add;
+        const int cf = static_cast<int>((v >> 32) & 0xffffull), cl = static_cast<int>(v >> 48);
+        // once the first and the last piece are in, the set is complete when
+        // every CTA of c_first..c_last with a non-empty range has announced
+        bool complete = (v & (1ull << 16)) && (v & (1ull << 17));
+        if (complete && (cl < cf || cl >= N)) {  // a counter left over from a step that did not finish
+          atomicOr(a.status, kStatusList);
+          complete = false;
+        }
+        if (complete) {
+          const dev::UnitSplit us(static_cast<unsigned>(*units_total), static_cast<unsigned>(N));
+          int expect = 0;
+          for (int c = cf; c <= cl; ++c) expect += us.owns_any(static_cast<unsigned>(c)) ? 1 : 0;
+          complete = static_cast<int>(v & 0xffffull) == expect;
+        }
+        if (complete) {
+          *ctr = 0ull;  // every piece has arrived: nothing else touches it in this step
+          // merged at the end, when the K/V ring is free to receive the pieces
+          const int n = pm[0];
+          pm[1 + 4 * n] = seg;
+          pm[2 + 4 * n] = cf;
+          pm[3 + 4 * n] = cl;
+          pm[4 + 4 * n] = (v >> 18) & 1ull ? 1 : 0;
+          pm[0] = n + 1;
+        }
+      }
+      return true;
+    };
+    // Merge the pieces of segment seg held by CTAs cf..cl (CTA order): the
+    // pieces are copied into the idle K/V ring (bulk copies, rounds of as
+    // many as fit), then each thread combines four output coordinates of one
+    // head over them.
+    auto merge = [&](int seg, int cf, int cl, int slot_cf) -> bool {
+      const dev::UnitSplit us(static_cast<unsigned>(*units_total), static_cast<unsigned>(N));
+      constexpr uint32_t kPiece = G * PS * sizeof(float);
+      constexpr int kMaxPieces = static_cast<int>(static_cast<size_t>(kStages) * TL::STAGE / kPiece);
+      constexpr int kAssign = (G * 32 + 127) / 128;  // (head, quad) pairs per thread
+      uint8_t* ring = base + L.stages;
+      float mx[kAssign], l[kAssign], o4[kAssign][4];
+#pragma unroll
+      for (int w = 0; w < kAssign; ++w) {
+        mx[w] = -INFINITY;
+        l[w] = 0.f;
+        o4[w][0] = o4[w][1] = o4[w][2] = o4[w][3] = 0.f;
+      }
+      int c0 = cf;
+      while (c0 <= cl) {
+        // this round's pieces (the CTAs from c0 on with a non-empty range, as
+        // many as the ring holds): their slots, listed by warp 2
+        if (warp == 2) {
+          int np = 0, c = c0;
+          while (c <= cl && np < kMaxPieces) {
+            const int cc = c + lane;
+            const bool has = cc <= cl && us.owns_any(static_cast<unsigned>(cc));
+            const unsigned bal = __ballot_sync(0xffffffffu, has);
+            const int before = __popc(bal & ((1u << lane) - 1u));
+            if (has && np + before < kMaxPieces) ent_s[np + before] = 2 * cc + (cc == cf ? slot_cf : 0);
+            if (np + __popc(bal) <= kMaxPieces) {
+              np += __popc(bal);
+              c += 32;
+            } else {  // the next round starts at the first piece that does not fit
+              const unsigned first_out = __ballot_sync(0xffffffffu, has && np + before == kMaxPieces);
+              c += __ffs(first_out) - 1;
+              np = kMaxPieces;
+            }
+          }
+          if (lane == 0) {
+            mround[0] = np;
+            mround[1] = min(c, cl + 1);
+          }
+        }
+        if (!rendezvous()) return false;
+        const int np = mround[0];
+        const int next = mround[1];
+        // all pieces in flight at once: 16-byte asynchronous copies through L2
+        fence_proxy_async();  // the ring's earlier tensor copies and reads come first
+        constexpr int kPc = static_cast<int>(kPiece / 16);
+        for (int x = t - 64; x < np * kPc; x += 128) {
+          const int p = x / kPc, o = x - p * kPc;
+          dev::cp_async16(ring + static_cast<size_t>(p) * kPiece + o * 16,
+                          reinterpret_cast<const uint8_t*>(a.partials + static_cast<size_t>(ent_s[p]) * G * PS) + o * 16);
+        }
+        dev::cp_async_commit();
+        dev::cp_async_wait<0>();
+        if (!rendezvous()) return false;  // every thread's copies have landed
+#pragma unroll
+        for (int w = 0; w < kAssign; ++w) {
+          const int hq = (t - 64) + 128 * w;
+          if (hq >= G * 32) continue;
+          const int h = hq >> 5, quad = hq & 31;
+          for (int p = 0; p < np; ++p) {
+            const float* pp = reinterpret_cast<const float*>(ring + static_cast<size_t>(p) * kPiece) + h * PS;
+            const float mc = pp[D], lc = pp[D + 1];
+            const float4 oc = reinterpret_cast<const float4*>(pp)[quad];
+            const float mn = fmaxf(mx[w], mc);
+            const float fo = mx[w] == -INFINITY ? 0.f : dev::fast_exp2(mx[w] - mn);
+            const float fc = mc == -INFINITY ? 0.f : dev::fast_exp2(mc - mn);
+            l[w] = l[w] * fo + lc * fc;
+            o4[w][0] = o4[w][0] * fo + oc.x * fc;
+            o4[w][1] = o4[w][1] * fo + oc.y * fc;
+            o4[w][2] = o4[w][2] * fo + oc.z * fc;
+            o4[w][3] = o4[w][3] * fo + oc.w * fc;
+            mx[w] = mn;
+          }
+        }
+        if (!rendezvous()) return false;  // the ring may be refilled
+        c0 = next;
+      }
+      const int i = seg / s.Hkv, g = seg - i * s.Hkv;
+#pragma unroll
+      for (int w = 0; w < kAssign; ++w) {
+        const int hq = (t - 64) + 128 * w;
+        if (hq >= G * 32) continue;
+        const int h = hq >> 5, quad = hq & 31;
+        const size_t orow = static_cast<size_t>(i) * s.Hq + g * G + h;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          dev::store_out_slot(a.out, s.elt, orow * D + 4 * quad + k, l[w] > 0.f ? o4[w][k] / l[w] : 0.f);
+        if (quad == 0 && a.lse) a.lse[orow] = dev::lse_of(mx[w], l[w]);
+      }
+      return true;
     };
 
     int pending = -1;  // tile whose O^T is not folded in yet
     for (int j = 0; ok; ++j) {
       const int st_j = j % kStages;
       if (!wait_or_abort(&B.kv_full[st_j], (j / kStages) & 1, a.status, abort_flag)) { ok = false; break; }
-      const FTile in = info[st_j];
-      if (in.flags & kEnd) break;
-      if (in.flags & kFirst) {
-        if (pending >= 0) {  // the previous chunk is folded in and flushed after this tile's softmax
-#pragma unroll
-          for (int h = 0; h < G; ++h) {
-            m_old[h] = m_run[h];
-            l_old[h] = l_thr[h];
-            acc_old[h] = acc[h];
-            alpha_old[h] = alpha_prev[h];
-          }
-          old_seq = cur_seq;
-          old_kvh = cur_kvh;
-          old_cidx = cur_cidx;
-          have_old = true;
+      const FInfo in = info[st_j];
+      if (in.seg != cur_seg || in.seg < 0) {  // a new segment, or END (also as the first entry of an empty range)
+        if (pending >= 0) {
+          if (!correction(pending) || !flush(cur_seg, in.prev_mode)) { ok = false; break; }
+          pending = -1;
         }
-        cur_seq = in.seq;
-        cur_kvh = in.kvh;
-        cur_cidx = in.cidx;
+        if (in.seg < 0) {  // END: the ring is free (every tile consumed, every MMA done)
+          if (!rendezvous()) { ok = false; break; }  // the merges recorded by warp 2 are visible
+          const int n = pm[0];
+          for (int x = 0; x < n && ok; ++x) ok = merge(pm[1 + 4 * x], pm[2 + 4 * x], pm[3 + 4 * x], pm[4 + 4 * x]);
+          break;
+        }
+        cur_seg = in.seg;
 #pragma unroll
         for (int h = 0; h < G; ++h) {
           m_run[h] = -INFINITY;
           l_thr[h] = 0.f;
           acc[h] = 0.f;
-          tau_h[h] = in.tau[h];
+          tau_h[h] = __ldcg(a.tau + static_cast<size_t>(in.seg) * G + h);
         }
       }
       const int sb = j & 1;
@@ -1160,24 +1148,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float p = (x[h] == -INFINITY) ? 0.f : dev::fast_exp2(x[h] - m_new);
         const uint16_t pbits = dev::f32_to_bf16_rn(p);
         {
-          const int kp = row >> 6, tc = row & 63;
-          const int off = kp * 2048 + h * 128 + (((tc >> 3) ^ (h & 7)) << 4) + (tc & 7) * 2;
+          const int kp = row >> 6, tcl = row & 63;
+          const int off = kp * 2048 + h * 128 + (((tcl >> 3) ^ (h & 7)) << 4) + (tcl & 7) * 2;
           *reinterpret_cast<uint16_t*>(pbuf + off) = pbits;
         }
         l_thr[h] = fmaf(l_thr[h], alpha[h], __uint_as_float(static_cast<uint32_t>(pbits) << 16));
         m_run[h] = m_new;
       }
       if (in.nrows0 < BR || (BPT == 2 && in.nrows1 < BR)) {
-        // rows of a tile that hold no key (past a sequence end, an absent
-        // second block, or a chunk with nothing admitted) are zeroed in V so
-        // that stale or non-finite bytes there cannot reach the accumulator
-        uint8_t* vb = base + L.stages + st_j * TL::STAGE + TL::V0;
+        // rows of a tile that hold no key (past a sequence end, or an absent
+        // second block) are zeroed in V so that stale or non-finite bytes
+        // there cannot reach the accumulator (0 * inf)
+        uint8_t* vbuf = base + L.stages + st_j * TL::STAGE + TL::V0;
         for (int bi = 0; bi < BPT; ++bi) {
-          const int nr = max(0, bi == 0 ? in.nrows0 : in.nrows1);
+          const int nr = bi == 0 ? in.nrows0 : in.nrows1;
           const int nz = (BR - nr) * 8;  // 16-byte chunks per panel
           for (int c = t - 64; c < 2 * nz; c += 128) {
             const int pnl = c / nz, r = c - pnl * nz;
-            *reinterpret_cast<uint4*>(vb + pnl * TL::PANEL + (bi * BR + nr) * 128 + r * 16) =
+            *reinterpret_cast<uint4*>(vbuf + pnl * TL::PANEL + (bi * BR + nr) * 128 + r * 16) =
                 make_uint4(0u, 0u, 0u, 0u);
           }
         }
@@ -1185,32 +1173,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async();
       __syncwarp();
       if (lane == 0) dev::mbar_arrive(&B.p_full[pb]);
-      if (pending >= 0) {
-        if (have_old) {
-          if (!correction(pending, acc_old, alpha_old) ||
-              !flush(acc_old, m_old, l_old, old_seq, old_kvh, old_cidx)) { ok = false; break; }
-          have_old = false;
-        } else if (!correction(pending, acc, alpha_prev)) {
-          ok = false;
-          break;
-        }
-      }
+      if (pending >= 0 && !correction(pending)) { ok = false; break; }
 #pragma unroll
       for (int h = 0; h < G; ++h) alpha_prev[h] = alpha[h];
       pending = j;
-    }
-    if (ok && pending >= 0) ok = correction(pending, acc, alpha_prev) && flush(acc, m_run, l_thr, cur_seq, cur_kvh, cur_cidx);
-    // no chunk follows: tell the completion warp, then run the folds it
-    // hands over until it reports that nothing is left
-    if (ok) {
-      Event fin{1, 0, 0, 0, 0, {0, 0, 0}};
-      ok = post_event(fin);
-    }
-    while (ok) {
-      if (!dev::warp_wait_or_abort(&B.job_full[jslot], jphase, a.status, abort_flag)) { ok = false; break; }
-      const Job jb = jobs[jslot];
-      if (jb.kind == 1) break;
-      if (!run_job(jb)) ok = false;
     }
     if (!ok) *abort_flag = 1;
   }
@@ -1218,15 +1184,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
-  // The last CTA to finish sets the hand-out counters back to zero for the
-  // next step (the fold-tree counters were reset by their completers).
-  if (t == 0) *reinterpret_cast<volatile int*>(base + L.misc + 32) =
-      atom_add_acq_rel(&a.ctrl[1], 1u) + 1u == gridDim.x ? 1 : 0;
-  __syncthreads();
-  if (*reinterpret_cast<volatile int*>(base + L.misc + 32)) {
-    const int nw = (s.nseg + 31) / 32;
-    for (int x = t; x < s.nseg + nw; x += kThreads) a.counters[x] = 0u;
-    if (t == 0) a.ctrl[1] = 0u;
+  // The last CTA to finish clears the slice totals for the next step (every
+  // CTA read them all before it got here).
+  if (warp == 0) {
+    unsigned last = 0;
+    if (lane == 0) {
+      __threadfence();
+      last = atom_add_acq_rel(a.done_ctas, 1u) + 1u == static_cast<unsigned>(N) ? 1u : 0u;
+    }
+    if (__shfl_sync(0xffffffffu, last, 0)) {
+      for (int x = lane; x < N; x += 32) a.flags[x] = 0u;
+      if (lane == 0) {
+        *a.arrived = 0u;
+        *a.done_ctas = 0u;
+      }
+    }
   }
 }
 
@@ -1267,8 +1239,9 @@ constexpr size_t kSmemBudget = 227 * 1024;
 }  // namespace
 
 size_t fused_tc_smem(const Shape& s) {
-  if (s.chunk < 1 || s.chunk > kMaxChunk || s.B > kFusedMaxSeqs) return 0;
-  const size_t n = fused_layout(s.chunk).total;
+  if (s.chunk < 1 || s.chunk > 32 || s.B > kFusedMaxSeqs || s.attend_ctas < 1 || s.attend_ctas > kFusedMaxCtas)
+    return 0;
+  const size_t n = fused_layout(s.attend_ctas).total;
   return n <= kSmemBudget ? n : 0;
 }
 
