@@ -519,6 +519,21 @@ def run_eta(args):
             cfgs[name] = entry
             del w2
         extra["configs"] = cfgs
+        if args.attend_impl == 0 and not args.dense:
+            # the single-launch alternative (ETA_ATTEND_FUSED: screen, attention
+            # and merge in one persistent kernel) on the same workloads
+            fa = argparse.Namespace(**vars(args))
+            fa.attend_impl = 3
+            fused = {}
+            for name in [args.workload] + [c for c in args.configs.split(",") if c and c != args.workload]:
+                w2 = workloads.make(name, args.seed)
+                x = Decode(eta, w2, dev, fa)
+                fused[name] = measure_config(x, fa, flush, stream, peak)
+                x.close()
+                del x, w2
+                torch.cuda.empty_cache()
+            extra["fused_kernel"] = {"note": ("attend_impl = ETA_ATTEND_FUSED: one launch per step (screen, "
+                                              "attention, merge); attend_us_isolated is that launch"), **fused}
     clk = clocks.stop()
 
     att = kt["attend"]
