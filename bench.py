@@ -268,18 +268,22 @@ class Decode:
         torch.cuda.synchronize()
         self.params_ev = self.make_params(events=self.ev)
         self.params = self.make_params()
+        self.trace = torch.zeros(eta.ETA_TRACE_SLOTS, dtype=torch.int64, device=dev)
+        self.params_tr = self.make_params(trace=self.trace)
         self.ws = eta.alloc_workspace(eta.eta_decode_workspace_size(self.params), dev)
-        for p in (self.params, self.params_ev):
+        for p in (self.params, self.params_ev, self.params_tr):
             p.workspace, p.workspace_bytes = self.ws.data_ptr(), self.ws.numel()
-        self.graph = None
+        self.graph = self.graph_tr = None
         if args.launch == "graph":
-            self.graph = eta.DecodeGraph(self.params, [self.q, self.k, self.v, self.seq, self.summ, self.out,
-                                                       self.lse, self.ws])
+            keep = [self.q, self.k, self.v, self.seq, self.summ, self.out, self.lse, self.ws]
+            self.graph = eta.DecodeGraph(self.params, keep)
+            self.graph_tr = eta.DecodeGraph(self.params_tr, keep + [self.trace])
 
-    def make_params(self, q=None, seq=None, out=None, events=None):
+    def make_params(self, q=None, seq=None, out=None, events=None, trace=None):
         return self.eta.make_params(self.q if q is None else q, self.k, self.v, self.seq if seq is None else seq,
                                     self.summ, self.wl.block_size, self.wl.tau_mode,
-                                    out=self.out if out is None else out, lse=self.lse, events=events, **self.kw)
+                                    out=self.out if out is None else out, lse=self.lse, events=events, trace=trace,
+                                    **self.kw)
 
     def step(self, stream):
         if self.graph is not None:
@@ -287,10 +291,18 @@ class Decode:
         else:
             self.eta.eta_decode(self.params, stream)
 
+    def step_traced(self, stream):
+        if self.graph_tr is not None:
+            self.graph_tr.launch(stream)
+        else:
+            self.eta.eta_decode(self.params_tr, stream)
+
     def close(self):
-        if self.graph is not None:
-            self.graph.close()
-            self.graph = None
+        for gname in ("graph", "graph_tr"):
+            g = getattr(self, gname)
+            if g is not None:
+                g.close()
+                setattr(self, gname, None)
 
 
 def time_steps(fn, n, flush, stream):
@@ -320,6 +332,45 @@ def kernel_times(d, n, flush, stream):
         out["attend"].append(d.ev[1].elapsed_time(d.ev[2]))
         out["merge"].append(d.ev[2].elapsed_time(d.ev[3]))
     return {k: statistics.median(v) for k, v in out.items()}
+
+
+def step_breakdown(d, n, flush, stream):
+    """Where one step's time goes: n steps launched the same way as the timed
+    ones but with the library's step trace on (first-CTA start and last-CTA
+    end of each kernel on the GPU's nanosecond timer, include/eta.h).  Per
+    step, the parts below sum to the step's event time; medians are reported
+    (so the medians need not sum exactly).  `outside` is the time of the step
+    outside the kernels: the first kernel's launch and the last one's
+    completion as the events see them."""
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    parts = {}
+    for _ in range(n):
+        flush()
+        d.trace.zero_()
+        s0.record(stream)
+        d.step_traced(stream)
+        s1.record(stream)
+        s1.synchronize()
+        step = s0.elapsed_time(s1) * 1e3
+        tt = d.eta.trace_times(d.trace)
+        us = lambda a, b: (tt[b] - tt[a]) / 1e3  # noqa: E731
+        if "fused_first" in tt:
+            p = {"start_to_first_tile": us("fused_first", "tile_first") if "tile_first" in tt else 0.0}
+            p["tiles_to_end"] = us("tile_first" if "tile_first" in tt else "fused_first", "fused_last")
+            span = us("fused_first", "fused_last")
+        else:
+            end = "merge_last" if tt.get("merge_last", 0) > tt["attend_last"] else "attend_last"
+            p = {"screen": us("screen_first", "screen_last")}
+            first = "tile_first" if "tile_first" in tt else "attend_first"
+            p["screen_end_to_first_tile"] = us("screen_last", first)
+            p["first_tile_to_attend_end"] = us(first, "attend_last")
+            p["merge_tail"] = us("attend_last", end)
+            span = us("screen_first", end)
+        p["outside_kernels"] = step - span
+        p["step"] = step
+        for k, v in p.items():
+            parts.setdefault(k, []).append(v)
+    return {k: round(statistics.median(v), 2) for k, v in parts.items()}
 
 
 def _pct(xs, p):
@@ -353,6 +404,7 @@ def measure_config(d, args, flush, stream, peak):
         "step_frac_of_peak": round(d.nbytes / (med * 1e-3) / 1e9 / peak, 4),
         "attend_us_isolated": round(kt["attend"] * 1e3, 2),
         "attend_frac_of_peak": round(d.kv_union / (kt["attend"] * 1e-3) / 1e9 / peak, 4),
+        "breakdown_us": step_breakdown(d, 50, flush, stream),
     }
 
 
@@ -486,6 +538,7 @@ def run_eta(args):
     # A longer run of the same step for the distribution (median of >= 100).
     dist_ms = time_steps(lambda: d.step(stream), max(100, args.steps), flush, stream)
     kt = kernel_times(d, max(20, args.steps), flush, stream)
+    bd = step_breakdown(d, 50, flush, stream)
     assert eta.eta_read_device_status(d.ws) == eta.ETA_OK
     med = statistics.median(dist_ms)
 
@@ -586,8 +639,11 @@ def run_eta(args):
                 "overlap_and_gaps": round(med * 1e3 - sum(iso.values()), 2),
                 "note": ("medians of a run with library events recorded between the kernels; those events stop "
                          "the kernels' programmatic-launch overlap and add a launch gap to each, so the isolated "
-                         "times sum to more than the step: step = sum_isolated + overlap_and_gaps"),
+                         "times sum to more than the step: step = sum_isolated + overlap_and_gaps; "
+                         "breakdown_us decomposes the step itself"),
             },
+            "breakdown_us": {**bd, "note": ("medians over 50 graph replays with the library's step trace on: "
+                                            "per step the parts sum to the step's event time")},
             "roofline": {"kernel": "attend", "bound": "hbm", "achieved": round(achieved, 2),
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,
@@ -857,7 +913,7 @@ def main():
     ap.add_argument("--launch", default="graph", choices=["graph", "stream"],
                     help="decode step as one recorded CUDA graph (default) or as stream launches")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--configs", default="c3_long,c5_batched",
+    ap.add_argument("--configs", default="c2_single,c3_long,c5_batched",
                     help="other workloads measured (screened and dense) after the main line")
     ap.add_argument("--no-configs", action="store_true", help="skip the dense arm and the other workloads")
     ap.add_argument("--meta", default="fp16", choices=["fp16", "fp8", "box"],

@@ -218,7 +218,34 @@ typedef struct {
                                         merge and after the last kernel
                                         (events between the kernels keep
                                         them from overlapping their launch) */
+  unsigned long long* trace;         /* optional device array of
+                                        ETA_TRACE_SLOTS words (NULL = off),
+                                        zeroed by the caller before the step:
+                                        see ETA_TRACE_* below               */
 } eta_decode_params;
+
+/*
+ * Step trace.  With eta_decode_params.trace set, the kernels of a step
+ * record device times (the GPU's global nanosecond timer) into the array:
+ * every slot is updated with an atomic maximum, so it must be zero before
+ * the step.  A "first" slot holds the bitwise complement of the earliest
+ * time (first CTA), a "last" slot the latest time (last CTA); a slot no
+ * kernel wrote stays 0.  A kernel starts when its first CTA has passed its
+ * wait for the previous kernel.  Costs two atomics per CTA when on; nothing
+ * when off.  No counterpart in the paper: a measurement aid.
+ */
+#define ETA_TRACE_SLOTS 16
+#define ETA_TRACE_SCREEN_FIRST 0   /* ~ start of the screen kernel          */
+#define ETA_TRACE_SCREEN_LAST 1    /* end of the screen kernel              */
+#define ETA_TRACE_ATTEND_FIRST 2   /* ~ start of the attention kernel       */
+#define ETA_TRACE_ATTEND_LAST 3    /* end of the attention kernel           */
+#define ETA_TRACE_TILE_FIRST 4     /* ~ first K/V tile in shared memory (tensor-core kernels) */
+#define ETA_TRACE_MERGE_FIRST 6    /* ~ start of the merge kernel           */
+#define ETA_TRACE_MERGE_LAST 7     /* end of the merge kernel               */
+#define ETA_TRACE_FUSED_FIRST 8    /* ~ start of the single-launch kernel   */
+#define ETA_TRACE_FUSED_LAST 9     /* end of the single-launch kernel       */
+#define ETA_TRACE_EXPORT_FIRST 10  /* ~ start of the selection export       */
+#define ETA_TRACE_EXPORT_LAST 11   /* end of the selection export           */
 
 /*
  * Leading control region of a decode workspace: the device status word and

@@ -83,6 +83,7 @@ class eta_decode_params(ctypes.Structure):
         ("lse", ctypes.c_void_p), ("admitted_count", ctypes.c_void_p), ("union_count", ctypes.c_void_p),
         ("union_list", ctypes.c_void_p), ("union_mask", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("timing_events", ctypes.c_void_p * 4),
+        ("trace", ctypes.c_void_p),
     ]
 
 
@@ -173,6 +174,12 @@ WORKSPACE_CONTROL_BYTES = 69632  # ETA_WORKSPACE_CONTROL_BYTES in include/eta.h
 DEVICE_STATUS_TIMEOUT = 1
 DEVICE_STATUS_RANGE = 2
 DEVICE_STATUS_LIST = 4
+
+ETA_TRACE_SLOTS = 16
+TRACE_SLOTS = (("screen_first", 0, True), ("screen_last", 1, False), ("attend_first", 2, True),
+               ("attend_last", 3, False), ("tile_first", 4, True), ("merge_first", 6, True),
+               ("merge_last", 7, False), ("fused_first", 8, True), ("fused_last", 9, False),
+               ("export_first", 10, True), ("export_last", 11, False))
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
 
 
@@ -304,7 +311,7 @@ def make_params(q, k, v, seq_lens, summary, block_size, tau_mode, w_tau=None, b_
                 c_tau=None, scale=None, beta=5.0, offset_a=0.0, z=2.0, n_local_blocks=2,
                 screen_enabled=True, attend_impl=ETA_ATTEND_AUTO, out=None, lse=None,
                 admitted_count=None, union_count=None, union_list=None, union_mask=None,
-                workspace=None, events=None, block_table=None) -> eta_decode_params:
+                workspace=None, events=None, block_table=None, trace=None) -> eta_decode_params:
     B, Hq, d = q.shape
     p = eta_decode_params()
     p.cache = cache_desc(k, v, seq_lens, Hq, block_size, block_table)
@@ -336,7 +343,23 @@ def make_params(q, k, v, seq_lens, summary, block_size, tau_mode, w_tau=None, b_
             if e is not None and not e.cuda_event:
                 e.record()  # torch creates the underlying cudaEvent_t lazily
             p.timing_events[j] = None if e is None else e.cuda_event
+    if trace is not None:
+        if trace.dtype != torch.int64 or trace.numel() < ETA_TRACE_SLOTS or not trace.is_cuda:
+            raise ValueError("trace: a CUDA int64 tensor of at least ETA_TRACE_SLOTS elements")
+        p.trace = trace.data_ptr()
     return p
+
+
+def trace_times(trace: torch.Tensor) -> dict:
+    """Decode a step trace (see include/eta.h) into nanosecond times by name;
+    slots no kernel wrote are left out."""
+    raw = [int(x) & 0xFFFFFFFFFFFFFFFF for x in trace[:ETA_TRACE_SLOTS].cpu().tolist()]
+    out = {}
+    for name, slot, first in TRACE_SLOTS:
+        v = raw[slot]
+        if v:
+            out[name] = (~v & 0xFFFFFFFFFFFFFFFF) if first else v
+    return out
 
 
 def eta_decode_workspace_size(params: eta_decode_params) -> int:
@@ -473,10 +496,12 @@ def eta_read_device_status(workspace: torch.Tensor, stream: Optional[torch.cuda.
 def decode(q, k, v, seq_lens, summary, block_size, tau_mode, *, w_tau=None, b_tau=None, c_tau=None,
            scale=None, beta=5.0, offset_a=0.0, z=2.0, n_local_blocks=2, screen_enabled=True,
            attend_impl=ETA_ATTEND_AUTO, selection=False, workspace=None, out=None, lse=None,
-           events=None, stream=None, block_table=None) -> Dict[str, torch.Tensor]:
+           events=None, stream=None, block_table=None, trace=None) -> Dict[str, torch.Tensor]:
     """Allocate outputs (and the workspace if not given) with torch and run one
     decode step.  Returns {"out", "lse", "workspace"} plus, with selection=True,
-    {"admitted_count", "union_count", "union_list", "union_mask"}."""
+    {"admitted_count", "union_count", "union_list", "union_mask"}.  `trace`:
+    an optional zeroed int64 device tensor of ETA_TRACE_SLOTS elements that
+    receives the step trace (read it with trace_times)."""
     B, Hq, d = q.shape
     Hkv = k.shape[1]
     nb = block_table.shape[1] if block_table is not None else (k.shape[2] + block_size - 1) // block_size
@@ -492,7 +517,7 @@ def decode(q, k, v, seq_lens, summary, block_size, tau_mode, *, w_tau=None, b_ta
               n_local_blocks=n_local_blocks, screen_enabled=screen_enabled, attend_impl=attend_impl,
               out=res["out"], lse=res["lse"], admitted_count=res.get("admitted_count"),
               union_count=res.get("union_count"), union_list=res.get("union_list"),
-              union_mask=res.get("union_mask"), events=events, block_table=block_table)
+              union_mask=res.get("union_mask"), events=events, block_table=block_table, trace=trace)
     params = make_params(q, k, v, seq_lens, summary, block_size, tau_mode, **kw)
     if workspace is None:
         workspace = alloc_workspace(eta_decode_workspace_size(params), dev)

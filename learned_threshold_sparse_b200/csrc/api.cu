@@ -354,6 +354,7 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
   };
 
   ScreenArgs sa;
+  sa.trace = p->trace;
   sa.q = p->q;
   sa.w_tau = p->w_tau;
   sa.b_tau = p->b_tau;
@@ -379,6 +380,7 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
 
   if (s.fused) {
     FusedArgs fa;
+    fa.trace = p->trace;
     fa.k = p->cache.k_cache;
     fa.v = p->cache.v_cache;
     fa.block_table = p->cache.block_table;
@@ -415,6 +417,7 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
     ev(2);
     if (p->admitted_count || p->union_count || p->union_list || p->union_mask) {
       ExportArgs xa;
+      xa.trace = p->trace;
       xa.chunk_count = fa.chunk_count;
       xa.chunk_list = fa.chunk_list;
       xa.seq_lens = p->cache.seq_lens;
@@ -437,6 +440,7 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
   if (s.rescue && launch_rescue(sa, cs) != cudaSuccess) return ETA_ERR_CUDA;
 
   AttendArgs aa;
+  aa.trace = p->trace;
   aa.k = p->cache.k_cache;
   aa.block_table = p->cache.block_table;
   aa.v = p->cache.v_cache;
@@ -458,6 +462,7 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
 
   ev(2);
   MergeArgs ma;
+  ma.trace = p->trace;
   ma.chunk_count = sa.chunk_count;
   ma.partials = aa.partials;
   ma.s = s;
@@ -467,6 +472,7 @@ eta_status eta_decode(const eta_decode_params* p, void* stream) {
 
   if (p->admitted_count || p->union_count || p->union_list || p->union_mask) {
     ExportArgs xa;
+    xa.trace = p->trace;
     xa.chunk_count = sa.chunk_count;
     xa.chunk_list = sa.chunk_list;
     xa.seq_lens = p->cache.seq_lens;

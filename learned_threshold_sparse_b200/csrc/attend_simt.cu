@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
   // Everything below reads what the screen wrote.
   dev::pdl_wait();
   dev::pdl_trigger();
+  if (threadIdx.x == 0) dev::trace_first(a.trace, ETA_TRACE_ATTEND_FIRST);
 
   // Exclusive prefix of the per-chunk entry counts, in (segment, chunk) order.
   dev::chunk_prefix<kThreads>(a.chunk_count, nprefix, prefix);
@@ -344,6 +345,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_simt_kernel(AttendArgs a, 
     if (++stage == stages) { stage = 0; phase ^= 1u; }
   }
   if (cur_seg >= 0 && !*abort_flag) flush(cur_seg);
+  if (lane == 0) dev::trace_last(a.trace, ETA_TRACE_ATTEND_LAST);
 }
 
 template <int ELT, int D, int G>

@@ -187,6 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   dev::pdl_wait();  // screen results visible from here on
   dev::pdl_trigger();
+  if (t == 0) dev::trace_first(a.trace, ETA_TRACE_ATTEND_FIRST);
   // The producer scans the chunk counts itself and publishes the table on a
   // named barrier, so its first copies do not wait on CTA-wide barriers; the
   // other warps pick the table up there (large tables: all warps scan).
@@ -400,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st_j = j % nstages;
       if (!wait_or_abort(&B.kv_full[st_j], (j / nstages) & 1, a.status, abort_flag)) { ok = false; break; }
       const TileInfo in = info[st_j];
+      if (j == 0 && warp == 2 && lane == 0) dev::trace_first(a.trace, ETA_TRACE_TILE_FIRST);
       if (in.seg != cur_seg) {
         if (pending >= 0) {
           if (!correction(pending) || !flush(cur_seg)) { ok = false; break; }
@@ -483,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (t == 0) dev::trace_last(a.trace, ETA_TRACE_ATTEND_LAST);
 }
 
 // ------------------------------------------------------------ host side

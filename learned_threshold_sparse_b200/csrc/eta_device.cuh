@@ -106,6 +106,21 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
+// Step trace (eta_decode_params.trace): every slot is updated with an atomic
+// maximum; a "first" slot holds the bitwise complement of the time, so the
+// earliest time wins.  Called by one thread per CTA; nothing when off.
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void trace_first(unsigned long long* tr, int slot) {
+  if (tr) atomicMax(tr + slot, ~global_ns());
+}
+__device__ __forceinline__ void trace_last(unsigned long long* tr, int slot) {
+  if (tr) atomicMax(tr + slot, global_ns());
+}
+
 // Programmatic dependent launch controls (no-ops without the launch attribute).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {

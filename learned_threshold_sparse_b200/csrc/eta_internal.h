@@ -118,6 +118,7 @@ struct ScreenArgs {
   float* lse;
   int* head_count;         // [B, Hq]   (rescue mode)
   unsigned long long* head_best;  // [B, Hq] (rescue mode)
+  unsigned long long* trace = nullptr;  // step trace (include/eta.h) or null
 };
 
 struct AttendArgs {
@@ -135,6 +136,7 @@ struct AttendArgs {
   float* partials;         // [nseg + attend_ctas][G][partial_stride(d)]
   void* out;               // [B, Hq, d] kv dtype: segments owned by one CTA
   float* lse;              // [B, Hq] or null
+  unsigned long long* trace = nullptr;  // step trace (include/eta.h) or null
 };
 
 // Arguments of the fused decode kernel (screen + attention + merge).
@@ -164,6 +166,7 @@ struct FusedArgs {
   float* partials;                 // [2 grid][G][partial_stride(d)] pieces of shared segments
   void* out;
   float* lse;
+  unsigned long long* trace = nullptr;  // step trace (include/eta.h) or null
 };
 
 struct MergeArgs {
@@ -172,6 +175,7 @@ struct MergeArgs {
   Shape s;
   void* out;
   float* lse;
+  unsigned long long* trace = nullptr;  // step trace (include/eta.h) or null
 };
 
 struct ExportArgs {
@@ -183,6 +187,7 @@ struct ExportArgs {
   int* union_count;
   int* union_list;
   unsigned* union_mask;
+  unsigned long long* trace = nullptr;  // step trace (include/eta.h) or null
 };
 
 // Arguments of the causal forward (prefill) kernel; q, k, v also feed the

@@ -20,6 +20,7 @@ __global__ void __launch_bounds__(kExportThreads) export_kernel(ExportArgs a) {
   const int g = blockIdx.x, i = blockIdx.y;
   const int seg = i * s.Hkv + g;
   const int t = threadIdx.x;
+  if (t == 0) dev::trace_first(a.trace, ETA_TRACE_EXPORT_FIRST);
   extern __shared__ int s_off[];  // [nchunks + 1]
   __shared__ int s_head[8];
   if (t < 8) s_head[t] = 0;
@@ -62,6 +63,7 @@ __global__ void __launch_bounds__(kExportThreads) export_kernel(ExportArgs a) {
   __syncthreads();
   if (t == 0 && a.union_count) a.union_count[seg] = total;
   if (t < s.G && a.admitted_count) a.admitted_count[static_cast<size_t>(i) * s.Hq + g * s.G + t] = s_head[t];
+  if (t == 0) dev::trace_last(a.trace, ETA_TRACE_EXPORT_LAST);
 }
 
 }  // namespace

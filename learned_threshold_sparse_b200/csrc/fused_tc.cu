@@ -290,6 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // has completed.
   dev::pdl_trigger();
   dev::pdl_wait();
+  if (t == 0) dev::trace_first(a.trace, ETA_TRACE_FUSED_FIRST);
 
   for (int x = t; x < s.B; x += kThreads) {
     int tt = a.seq_lens[x];
@@ -1095,6 +1096,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st_j = j % kStages;
       if (!wait_or_abort(&B.kv_full[st_j], (j / kStages) & 1, a.status, abort_flag)) { ok = false; break; }
       const FInfo in = info[st_j];
+      if (j == 0 && in.seg >= 0 && warp == 2 && lane == 0) dev::trace_first(a.trace, ETA_TRACE_TILE_FIRST);
       if (in.seg != cur_seg || in.seg < 0) {  // a new segment, or END (also as the first entry of an empty range)
         if (pending >= 0) {
           if (!correction(pending) || !flush(cur_seg, in.prev_mode)) { ok = false; break; }
@@ -1184,6 +1186,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+  if (t == 0) dev::trace_last(a.trace, ETA_TRACE_FUSED_LAST);
   // The last CTA to finish clears the slice totals for the next step (every
   // CTA read them all before it got here).
   if (warp == 0) {

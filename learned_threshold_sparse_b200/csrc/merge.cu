@@ -63,6 +63,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(MergeArgs a) {
   const int c0 = static_cast<int>(split.owner(us)), c1 = static_cast<int>(split.owner(ue - 1));
   if (c0 == c1) return;  // written by its only attention CTA
   dev::pdl_wait();  // the partials are complete from here on
+  if (threadIdx.x == 0) dev::trace_first(a.trace, ETA_TRACE_MERGE_FIRST);
 
   const int PS = partial_stride(s.d);
   const size_t cstride = static_cast<size_t>(s.G) * PS;
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__(kMergeWarps * 32) merge_kernel(MergeArgs a) {
     const size_t orow = static_cast<size_t>(i) * s.Hq + g * s.G + h;
     dev::store_out_slot(a.out, s.elt, orow * s.d + e, lsum > 0.f ? asum / lsum : 0.f);
     if (lane == 0 && slice == 0 && a.lse) a.lse[orow] = dev::lse_of(mstar, lsum);
+    if (lane == 0) dev::trace_last(a.trace, ETA_TRACE_MERGE_LAST);
   }
 }
 

@@ -85,6 +85,7 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
   // grid rewrites): nothing is read or written before that kernel is done.
   dev::pdl_trigger();
   dev::pdl_wait();
+  if (threadIdx.x == 0) dev::trace_first(a.trace, ETA_TRACE_SCREEN_FIRST);
 
   const int blk0 = c * s.chunk;
   const int avail = min(s.chunk, s.nbmax - blk0);  // rows of this chunk inside the arrays
@@ -291,7 +292,10 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
   if (t == 0 && nscreen == 0 && meta) dev::mbar_wait(&s_bar[0], 0, a.status);
   __syncthreads();
   if (nloc == 0) {
-    if (t == 0) a.chunk_count[static_cast<size_t>(seg) * s.nchunks + c] = 0;
+    if (t == 0) {
+      a.chunk_count[static_cast<size_t>(seg) * s.nchunks + c] = 0;
+      dev::trace_last(a.trace, ETA_TRACE_SCREEN_LAST);
+    }
     return;
   }
 
@@ -317,7 +321,10 @@ __global__ void __launch_bounds__(kThreads) screen_kernel(ScreenArgs a) {
     base += tot;
     __syncthreads();
   }
-  if (t == 0) a.chunk_count[static_cast<size_t>(seg) * s.nchunks + c] = base;
+  if (t == 0) {
+    a.chunk_count[static_cast<size_t>(seg) * s.nchunks + c] = base;
+    dev::trace_last(a.trace, ETA_TRACE_SCREEN_LAST);
+  }
   if (s.rescue && t < G) {
     const size_t hq = static_cast<size_t>(i) * s.Hq + g * G + t;
     atomicAdd(&a.head_count[hq], s_cnt[t]);
