@@ -408,6 +408,28 @@ def measure_config(d, args, flush, stream, peak):
     }
 
 
+def append_time(eta, d, flush, stream, n=100):
+    """One-token append timed alone (eta_append_kv: write the token's K/V rows
+    of every (sequence, KV head) and re-summarise the block holding it), the
+    L2 flushed before each; the token re-written is the last one of each
+    sequence with its own values, so the cache is unchanged.  Median us."""
+    wl = d.wl
+    last = [max(0, T - 1) for T in wl.seq_lens]
+    k_new = torch.stack([d.k[i, :, t] for i, t in enumerate(last)]).contiguous()
+    v_new = torch.stack([d.v[i, :, t] for i, t in enumerate(last)]).contiguous()
+    pos = torch.tensor(last, dtype=torch.int32, device=d.q.device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ms = []
+    for _ in range(n):
+        flush()
+        e0.record(stream)
+        eta.eta_append_kv(d.k, d.v, d.seq, d.summ, wl.block_size, k_new, v_new, pos, wl.n_q_heads, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    return round(statistics.median(ms) * 1e3, 2)
+
+
 def e2e_append(eta, d, args, flush, stream, dev):
     """End to end through the public API with host buffers, the sequence
     growing by one token per step: each step's new query, key and value rows
@@ -539,6 +561,7 @@ def run_eta(args):
     dist_ms = time_steps(lambda: d.step(stream), max(100, args.steps), flush, stream)
     kt = kernel_times(d, max(20, args.steps), flush, stream)
     bd = step_breakdown(d, 50, flush, stream)
+    app_us = append_time(eta, d, flush, stream)
     assert eta.eta_read_device_status(d.ws) == eta.ETA_OK
     med = statistics.median(dist_ms)
 
@@ -644,6 +667,9 @@ def run_eta(args):
             },
             "breakdown_us": {**bd, "note": ("medians over 50 graph replays with the library's step trace on: "
                                             "per step the parts sum to the step's event time")},
+            "append_us": {"median": app_us, "steps": 100,
+                          "note": ("eta_append_kv of one token per sequence (K/V rows written, their block "
+                                   "re-summarised), timed alone with the L2 flushed; not part of a decode step")},
             "roofline": {"kernel": "attend", "bound": "hbm", "achieved": round(achieved, 2),
                          "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic,

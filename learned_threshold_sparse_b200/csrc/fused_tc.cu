@@ -87,11 +87,71 @@ struct Tile {
   static constexpr int P_BYTES = NQ * TR * 2;
 };
 
-// How the run of units of one segment that just ended leaves this CTA.
+// Pieces of a segment spread over several CTAs (compiled for the host as
+// well).  A CTA's range [u0, u1) splits into runs of consecutive units of one
+// segment.  A run is shared when the segment has units before u0 (then the
+// run starts at u0) or at or after u1 (then it ends at u1); a shared run
+// leaves a partial in slot 0 of its CTA if it holds u0, else in slot 1, and
+// announces it with one atomic add to the segment's 64-bit counter:
+//   bits 0-15 arrivals, bit 16 the first piece is in, bit 17 the last piece
+//   is in, bit 18 the first piece's slot, bits 32-47 the first piece's CTA,
+//   bits 48-63 the last piece's CTA.
+// Every CTA between the first and the last piece's with a non-empty range
+// holds exactly one piece, in its slot 0 (its range starts inside the
+// segment), so the announcement that completes the set is recognised from
+// the counter alone.
+// ETA_PIECES_BEGIN
 constexpr int kModeShared = 1;  // other CTAs hold units of the segment: write a partial
 constexpr int kModeSlot1 = 2;   // partial slot 1 (the run did not contain the range's first unit)
 constexpr int kModeFirst = 4;   // the run holds the segment's first unit
 constexpr int kModeLast = 8;    // the run holds the segment's last unit
+
+__host__ __device__ inline int run_mode(bool holds_u0, bool shared_start, bool shared_end) {
+  int mode = (shared_start ? 0 : kModeFirst) | (shared_end ? 0 : kModeLast);
+  if (shared_start || shared_end) mode |= kModeShared | (holds_u0 ? 0 : kModeSlot1);
+  return mode;
+}
+
+__host__ __device__ inline unsigned long long piece_announcement(int mode, int cta) {
+  const unsigned long long c64 = static_cast<unsigned long long>(cta);
+  unsigned long long add = 1ull;
+  if (mode & kModeFirst) add += (1ull << 16) + ((mode & kModeSlot1) ? (1ull << 18) : 0ull) + (c64 << 32);
+  if (mode & kModeLast) add += (1ull << 17) + (c64 << 48);
+  return add;
+}
+
+// Fields of a counter value: are both end pieces in, and which CTAs / slot.
+struct PieceSet {
+  bool ends_in;
+  int c_first, c_last, slot_first, arrivals;
+};
+__host__ __device__ inline PieceSet piece_set(unsigned long long v) {
+  PieceSet p;
+  p.ends_in = (v & (1ull << 16)) && (v & (1ull << 17));
+  p.c_first = static_cast<int>((v >> 32) & 0xffffull);
+  p.c_last = static_cast<int>(v >> 48);
+  p.slot_first = static_cast<int>((v >> 18) & 1ull);
+  p.arrivals = static_cast<int>(v & 0xffffull);
+  return p;
+}
+
+// Is the set complete: both end pieces in, and one arrival per CTA of the
+// span with a non-empty range (us: the step's unit split over nctas CTAs).
+// A counter naming CTAs outside the grid (left by a step that did not
+// finish) never completes, and *stale says so.
+template <class Split>
+__host__ __device__ inline bool piece_set_complete(const PieceSet& p, const Split& us, int nctas, bool* stale) {
+  *stale = false;
+  if (!p.ends_in) return false;
+  if (p.c_last < p.c_first || p.c_last >= nctas) {
+    *stale = true;
+    return false;
+  }
+  int expect = 0;
+  for (int c = p.c_first; c <= p.c_last; ++c) expect += us.owns_any(static_cast<unsigned>(c)) ? 1 : 0;
+  return p.arrivals == expect;
+}
+// ETA_PIECES_END
 
 // A ring entry: the tile's segment (-1: END), per block of the tile the
 // admitting heads and the rows present, and the mode of the run this entry
@@ -666,9 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int f = ch.first(rseg);
         const bool shared_start = first_run && units_before(f) < u0;
         const bool shared_end = at_u1 && units_before(f + ch.nch(rseg / s.Hkv)) > u1;
-        int mode = (shared_start ? 0 : kModeFirst) | (shared_end ? 0 : kModeLast);
-        if (shared_start || shared_end) mode |= kModeShared | (first_run ? 0 : kModeSlot1);
-        return mode;
+        return run_mode(first_run, shared_start, shared_end);
       };
 
       int run_seg = -1;
@@ -961,28 +1019,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence();
       if (!rendezvous()) return false;  // also: every thread has read sums
       if (warp == 2 && lane == 0) {
-        // one announcement per piece; the first piece also says which slot
-        // holds it (the pieces of later CTAs are always in their slot 0)
-        const unsigned long long c64 = static_cast<unsigned long long>(cta);
-        unsigned long long add = 1ull;
-        if (mode & kModeFirst) add += (1ull << 16) + ((mode & kModeSlot1) ? (1ull << 18) : 0ull) + (c64 << 32);
-        if (mode & kModeLast) add += (1ull << 17) + (c64 << 48);
+        // one announcement per piece (see piece_announcement)
+        const unsigned long long add = piece_announcement(mode, cta);
         unsigned long long* ctr = a.seg_ctr + seg;
-        const unsigned long long v = atom_add_acq_rel64(ctr, add) + add;
-        const int cf = static_cast<int>((v >> 32) & 0xffffull), cl = static_cast<int>(v >> 48);
-        // once the first and the last piece are in, the set is complete when
-        // every CTA of c_first..c_last with a non-empty range has announced
-        bool complete = (v & (1ull << 16)) && (v & (1ull << 17));
-        if (complete && (cl < cf || cl >= N)) {  // a counter left over from a step that did not finish
-          atomicOr(a.status, kStatusList);
-          complete = false;
-        }
-        if (complete) {
-          const dev::UnitSplit us(static_cast<unsigned>(*units_total), static_cast<unsigned>(N));
-          int expect = 0;
-          for (int c = cf; c <= cl; ++c) expect += us.owns_any(static_cast<unsigned>(c)) ? 1 : 0;
-          complete = static_cast<int>(v & 0xffffull) == expect;
-        }
+        const PieceSet ps = piece_set(atom_add_acq_rel64(ctr, add) + add);
+        const int cf = ps.c_first, cl = ps.c_last;
+        const dev::UnitSplit us(static_cast<unsigned>(*units_total), static_cast<unsigned>(N));
+        bool stale = false;
+        const bool complete = piece_set_complete(ps, us, N, &stale);
+        if (stale) atomicOr(a.status, kStatusList);
         if (complete) {
           *ctr = 0ull;  // every piece has arrived: nothing else touches it in this step
           // merged at the end, when the K/V ring is free to receive the pieces
@@ -990,7 +1035,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           pm[1 + 4 * n] = seg;
           pm[2 + 4 * n] = cf;
           pm[3 + 4 * n] = cl;
-          pm[4 + 4 * n] = (v >> 18) & 1ull ? 1 : 0;
+          pm[4 + 4 * n] = ps.slot_first;
           pm[0] = n + 1;
         }
       }
