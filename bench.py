@@ -502,6 +502,34 @@ def e2e_append(eta, d, args, flush, stream, dev):
         assert eta.eta_read_device_status(d.ws) == eta.ETA_OK
         assert torch.equal(check.cpu(), out_h), "e2e output differs from a decode of the final state"
         crossed = any(T0[i] // b != (T0[i] + K - 1) // b for i in range(B))
+        # the same token path recorded with the step trace on: where its time goes
+        pt = d.make_params(q=q_in, seq=seq_d, out=out_h, trace=d.trace)
+        pt.workspace, pt.workspace_bytes = d.ws.data_ptr(), d.ws.numel()
+        gt = eta.StepGraph(pt, k_new=rows_h[nq:nq + nkv].view(B, Hkv, hd), v_new=rows_h[nq + nkv:].view(B, Hkv, hd),
+                           positions=pos_d, q_new=rows_h[:nq].view(B, Hq, hd), h2d=lens_h, h2d_dst=lens_d,
+                           tensors=[q_in, d.k, d.v, d.summ, d.lse, d.ws, out_h, lens_d, d.trace])
+        try:
+            reset()
+            order = ["in_first", "in_last", "append_first", "append_last", "screen_first", "screen_last",
+                     "tile_first", "attend_last", "merge_last", "out_first", "out_last"]
+            parts = {}
+            for s in range(min(K, 30)):
+                host_token(s)
+                flush()
+                d.trace.zero_()
+                e0.record(stream)
+                gt.launch(stream)
+                e1.record(stream)
+                e1.synchronize()
+                tt = eta.trace_times(d.trace)
+                seq_t = [(n, tt[n]) for n in order if n in tt]
+                for (a, ta), (bn, tb) in zip(seq_t, seq_t[1:]):
+                    parts.setdefault(f"{a}->{bn}", []).append((tb - ta) / 1e3)
+                parts.setdefault("outside_kernels", []).append(e0.elapsed_time(e1) * 1e3 - (seq_t[-1][1] - seq_t[0][1]) / 1e3)
+                parts.setdefault("step", []).append(e0.elapsed_time(e1) * 1e3)
+            e2e_bd = {k: round(statistics.median(v), 2) for k, v in parts.items()}
+        finally:
+            gt.close()
     finally:
         g.close()
         # back to the workload's own lengths and tail metadata
@@ -513,7 +541,7 @@ def e2e_append(eta, d, args, flush, stream, dev):
     d2h = out_h.numel() * out_h.element_size()
     note = (f"context grows one token per step from {min(T0)} (seq 0: {T0[0]} -> {T0[0] + K}); appends cross a "
             f"block boundary inside the timed steps: {crossed}; bytes per step counted at the full context")
-    return ms, h2d, d2h, note
+    return ms, h2d, d2h, note, e2e_bd
 
 
 def run_eta(args):
@@ -566,7 +594,7 @@ def run_eta(args):
     med = statistics.median(dist_ms)
 
     # ---- end to end through the public API, host buffers, growing context
-    e2e_ms, h2d, d2h, e2e_note = e2e_append(eta, d, args, flush, stream, dev)
+    e2e_ms, h2d, d2h, e2e_note, e2e_bd = e2e_append(eta, d, args, flush, stream, dev)
     e2e = max_over_ranks(statistics.mean(e2e_ms), dev)
     d.close()
     main = dict(kv_union=d.kv_union, nbytes=d.nbytes, union_density=d.union_density, head_density=d.head_density)
@@ -682,7 +710,11 @@ def run_eta(args):
                     "io": ("one graph per token (eta_step_graph_create): new lengths and positions copied up by a "
                            "kernel reading page-locked memory, the append kernel reads the new q, k, v rows from "
                            "page-locked host memory, the decode stores out into page-locked host memory"),
-                    "mode": e2e_note},
+                    "mode": e2e_note,
+                    "breakdown_us": {**e2e_bd, "note": ("medians over 30 tokens of the same graph recorded with the "
+                                                        "step trace on: intervals between consecutive kernel "
+                                                        "first-starts / last-ends, in step order, plus the time "
+                                                        "outside the kernels; per token they sum to the step")}},
             **extra,
             "gpu_launches": KERNELS_PER_STEP * args.steps,
             "clocks": clk,

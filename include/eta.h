@@ -234,7 +234,7 @@ typedef struct {
  * wait for the previous kernel.  Costs two atomics per CTA when on; nothing
  * when off.  No counterpart in the paper: a measurement aid.
  */
-#define ETA_TRACE_SLOTS 16
+#define ETA_TRACE_SLOTS 24
 #define ETA_TRACE_SCREEN_FIRST 0   /* ~ start of the screen kernel          */
 #define ETA_TRACE_SCREEN_LAST 1    /* end of the screen kernel              */
 #define ETA_TRACE_ATTEND_FIRST 2   /* ~ start of the attention kernel       */
@@ -246,6 +246,13 @@ typedef struct {
 #define ETA_TRACE_FUSED_LAST 9     /* end of the single-launch kernel       */
 #define ETA_TRACE_EXPORT_FIRST 10  /* ~ start of the selection export       */
 #define ETA_TRACE_EXPORT_LAST 11   /* end of the selection export           */
+/* a recorded serving step (eta_step_graph_create) also records:            */
+#define ETA_TRACE_APPEND_FIRST 12  /* ~ start of the append                 */
+#define ETA_TRACE_APPEND_LAST 13   /* end of the append                     */
+#define ETA_TRACE_IN_FIRST 14      /* ~ start of the input copy (kernel path) */
+#define ETA_TRACE_IN_LAST 15       /* end of the input copy                 */
+#define ETA_TRACE_OUT_FIRST 16     /* ~ start of the output copy (kernel path) */
+#define ETA_TRACE_OUT_LAST 17      /* end of the output copy                */
 
 /*
  * Leading control region of a decode workspace: the device status word and

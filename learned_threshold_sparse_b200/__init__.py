@@ -175,11 +175,13 @@ DEVICE_STATUS_TIMEOUT = 1
 DEVICE_STATUS_RANGE = 2
 DEVICE_STATUS_LIST = 4
 
-ETA_TRACE_SLOTS = 16
+ETA_TRACE_SLOTS = 24
 TRACE_SLOTS = (("screen_first", 0, True), ("screen_last", 1, False), ("attend_first", 2, True),
                ("attend_last", 3, False), ("tile_first", 4, True), ("merge_first", 6, True),
                ("merge_last", 7, False), ("fused_first", 8, True), ("fused_last", 9, False),
-               ("export_first", 10, True), ("export_last", 11, False))
+               ("export_first", 10, True), ("export_last", 11, False), ("append_first", 12, True),
+               ("append_last", 13, False), ("in_first", 14, True), ("in_last", 15, False),
+               ("out_first", 16, True), ("out_last", 17, False))
 NOALLOC_SCRATCH_BYTES = 8 << 20  # ETA_NOALLOC_SCRATCH_BYTES in include/eta.h
 
 

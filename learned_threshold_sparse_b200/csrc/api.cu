@@ -287,7 +287,8 @@ eta_status eta_append_kv(const eta_cache_desc* cache, const eta_summary_desc* su
 namespace eta {
 
 eta_status append_step(const eta_cache_desc* cache, const eta_summary_desc* summary, const void* k_new,
-                       const void* v_new, const int* pos, const void* q_src, void* q_dst, void* stream) {
+                       const void* v_new, const int* pos, const void* q_src, void* q_dst, void* stream,
+                       unsigned long long* trace) {
   eta_status st = check_cache(cache);
   if (st != ETA_OK) return st;
   st = check_summary(summary);
@@ -297,6 +298,7 @@ eta_status append_step(const eta_cache_desc* cache, const eta_summary_desc* summ
   if ((q_src == nullptr) != (q_dst == nullptr)) return ETA_ERR_INVALID_ARG;
   if (q_src && (!aligned(q_src, 16) || !aligned(q_dst, 16))) return ETA_ERR_INVALID_ARG;
   SummaryArgs a;
+  a.trace = trace;
   a.q_src = q_src;
   a.q_dst = q_dst;
   a.G = cache->n_q_heads / cache->n_kv_heads;

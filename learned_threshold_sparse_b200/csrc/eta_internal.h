@@ -234,13 +234,15 @@ struct SummaryArgs {
   const void* q_src = nullptr;
   void* q_dst = nullptr;
   int G = 0;
+  unsigned long long* trace = nullptr;  // step trace (include/eta.h) or null
 };
 
 // The append of eta_append_kv, optionally also copying the token's query
 // rows q_src -> q_dst ([batch, n_q_heads, head_dim]) in the same launch
 // (api.cu; used by the recorded serving step).
 eta_status append_step(const eta_cache_desc* cache, const eta_summary_desc* summary, const void* k_new,
-                       const void* v_new, const int* pos, const void* q_src, void* q_dst, void* stream);
+                       const void* v_new, const int* pos, const void* q_src, void* q_dst, void* stream,
+                       unsigned long long* trace = nullptr);
 
 // ---------------------------------------------------------------- host helpers
 // Driver attribute queries and settings cost on the order of a microsecond

@@ -12,6 +12,7 @@
 // stay in place.
 #include <new>
 
+#include "eta_device.cuh"
 #include "eta_internal.h"
 
 struct eta_decode_graph {
@@ -29,7 +30,9 @@ namespace {
 constexpr int kCopyThreads = 256;
 
 __global__ void __launch_bounds__(kCopyThreads)
-    io_copy_kernel(uint8_t* dst, const uint8_t* src, size_t bytes, int src_host) {
+    io_copy_kernel(uint8_t* dst, const uint8_t* src, size_t bytes, int src_host, unsigned long long* trace,
+                   int slot) {
+  if (threadIdx.x == 0) eta::dev::trace_first(trace, slot);
   const size_t n16 = (reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src)) % 16 == 0 ? bytes / 16 : 0;
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   const size_t t0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -48,6 +51,10 @@ __global__ void __launch_bounds__(kCopyThreads)
     } else {
       __stwt(reinterpret_cast<signed char*>(dst) + x, static_cast<signed char>(src[x]));
     }
+  }
+  if (trace) {
+    __syncthreads();
+    if (threadIdx.x == 0) eta::dev::trace_last(trace, slot + 1);
   }
 }
 
@@ -92,13 +99,14 @@ struct IoCopy {
     }
   }
 
-  eta_status record(cudaStream_t cs) const {
+  // trace / slot: the step trace and this copy's first slot (see include/eta.h)
+  eta_status record(cudaStream_t cs, unsigned long long* trace, int slot) const {
     if (!bytes) return ETA_OK;
     if (kdst) {
       const size_t units = (bytes + 16 * kCopyThreads - 1) / (16 * kCopyThreads);
       const int grid = static_cast<int>(units < 148 ? units : 148);
       io_copy_kernel<<<grid, kCopyThreads, 0, cs>>>(static_cast<uint8_t*>(kdst), static_cast<const uint8_t*>(ksrc),
-                                                     bytes, h2d ? 1 : 0);
+                                                     bytes, h2d ? 1 : 0, trace, slot);
       return cudaGetLastError() == cudaSuccess ? ETA_OK : ETA_ERR_CUDA;
     }
     // the copy engine, direction taken from the unified address space
@@ -117,21 +125,30 @@ eta_status check_decode(const eta_decode_params* p) {
   return ETA_OK;
 }
 
-// Records record(stream) on a private stream under thread-local capture and
-// instantiates the result.  Nothing runs on the GPU.
+// Records record(stream, side) on a private stream under thread-local
+// capture and instantiates the result; `side` is a second private stream
+// that record may fork work onto (an event recorded on `stream` and waited
+// on by `side`) and must join back before it returns.  Nothing runs on the
+// GPU.
 template <typename F>
 eta_status capture(F&& record, eta_decode_graph** out) {
-  cudaStream_t cs = nullptr;
+  cudaStream_t cs = nullptr, side = nullptr;
   if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess) return ETA_ERR_CUDA;
+  if (cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking) != cudaSuccess) {
+    cudaStreamDestroy(cs);
+    return ETA_ERR_CUDA;
+  }
   if (cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
     cudaStreamDestroy(cs);
+    cudaStreamDestroy(side);
     (void)cudaGetLastError();
     return ETA_ERR_CUDA;
   }
-  eta_status st = record(cs);
+  eta_status st = record(cs, side);
   cudaGraph_t graph = nullptr;
   const cudaError_t ec = cudaStreamEndCapture(cs, &graph);
   cudaStreamDestroy(cs);
+  cudaStreamDestroy(side);
   if (st == ETA_OK && (ec != cudaSuccess || !graph)) st = ETA_ERR_CUDA;
   cudaGraphExec_t exec = nullptr;
   if (st == ETA_OK && cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) st = ETA_ERR_CUDA;
@@ -157,7 +174,7 @@ extern "C" eta_status eta_decode_graph_create(const eta_decode_params* p, eta_de
   *out = nullptr;
   const eta_status st = check_decode(p);  // a bad argument records nothing
   if (st != ETA_OK) return st;
-  return capture([&](cudaStream_t cs) { return eta_decode(p, cs); }, out);
+  return capture([&](cudaStream_t cs, cudaStream_t) { return eta_decode(p, cs); }, out);
 }
 
 extern "C" eta_status eta_step_graph_create(const eta_step_desc* d, eta_decode_graph** out) {
@@ -184,17 +201,17 @@ extern "C" eta_status eta_step_graph_create(const eta_step_desc* d, eta_decode_g
   in.plan();
   outc.plan();
   return capture(
-      [&](cudaStream_t cs) -> eta_status {
-        eta_status sc = in.record(cs);
+      [&](cudaStream_t cs, cudaStream_t) -> eta_status {
+        eta_status sc = in.record(cs, p->trace, ETA_TRACE_IN_FIRST);
         if (sc != ETA_OK) return sc;
         if (nappend == 3) {
           const eta_status sa = eta::append_step(&p->cache, &p->summary, d->k_new, d->v_new, d->positions, d->q_new,
-                                                 d->q_new ? const_cast<void*>(p->q) : nullptr, cs);
+                                                 d->q_new ? const_cast<void*>(p->q) : nullptr, cs, p->trace);
           if (sa != ETA_OK) return sa;
         }
         const eta_status sd = eta_decode(p, cs);
         if (sd != ETA_OK) return sd;
-        return outc.record(cs);
+        return outc.record(cs, p->trace, ETA_TRACE_OUT_FIRST);
       },
       out);
 }

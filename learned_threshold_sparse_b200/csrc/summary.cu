@@ -14,7 +14,8 @@
 namespace eta {
 namespace {
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;        // summary_kernel: many blocks, many CTAs
+constexpr int kAppendThreads = 256;   // append_kernel: one block per CTA (1024 measured no faster)
 
 __host__ __device__ inline size_t block_stage_bytes(int b, int d, int elt) {
   return static_cast<size_t>(b) * d * elt;
@@ -56,7 +57,8 @@ __device__ __forceinline__ float e4m3_to_f32(uint8_t code) {
   return dev::fp16_to_f32(static_cast<uint16_t>(h2 & 0xffffu));
 }
 
-// Largest of v over the CTA's threads (kThreads), in every thread.
+// Largest of v over the CTA's NT threads, in every thread.
+template <int NT>
 __device__ __forceinline__ double cta_max(double v, double* s_w) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -65,7 +67,7 @@ __device__ __forceinline__ double cta_max(double v, double* s_w) {
   if ((threadIdx.x & 31) == 0) s_w[w] = v;
   __syncthreads();
   double m = s_w[0];
-  for (int k = 1; k < kThreads / 32; ++k) m = fmax(m, s_w[k]);
+  for (int k = 1; k < NT / 32; ++k) m = fmax(m, s_w[k]);
   return m;
 }
 
@@ -81,7 +83,11 @@ __device__ __forceinline__ double cta_max(double v, double* s_w) {
 // never falls below the exact distance.  With sums of at most 128 bf16 rows
 // (or fp32 rows of moderate range) the float64 sums are exact, so the stored
 // metadata does not depend on the summation order.
-template <int FMT>
+//
+// NT threads per CTA: the more, the shorter every thread's dependent chain
+// (passes 1 and 2 split the rows into NT / d groups, pass 3 gives each row
+// NT / n lanes).
+template <int FMT, int NT>
 __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n, uint8_t* stage) {
   const int d = a.d, t = threadIdx.x;
   const KvLayout lay{a.block_table, a.Hkv, a.b, a.max_ctx, a.nbmax, a.num_pages};
@@ -90,9 +96,19 @@ __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n
   if (bad) return;  // a page id outside the pool: nothing is read or written (CTA-uniform)
   const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.k) + row0 * d * a.elt);
   const int nvec = n * d * a.elt / 16;
-  for (int x = t; x < nvec; x += kThreads) reinterpret_cast<uint4*>(stage)[x] = src[x];
+  // all of a thread's loads in flight before its stores (one round trip)
+  for (int x0 = t; x0 < nvec; x0 += 8 * NT) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (x0 + u * NT < nvec) v[u] = src[x0 + u * NT];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      if (x0 + u * NT < nvec) reinterpret_cast<uint4*>(stage)[x0 + u * NT] = v[u];
+  }
   __shared__ double s_mu[128];
-  __shared__ double s_wmax[kThreads / 32];
+  __shared__ double s_part[NT];
+  __shared__ double s_wmax[NT / 32];
   __syncthreads();
   auto at = [&](int r, int e) -> float {
     const size_t idx = static_cast<size_t>(r) * d + e;
@@ -118,31 +134,57 @@ __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n
     if (t == 0) a.max_norm[bo] = 0.f;
     return;
   }
-  // Passes 1 and 2, one coordinate per thread; four interleaved partial sums
-  // shorten the dependent chains.
-  double mean = 0.0, sd = 0.0;
-  if (t < d) {
-    double s4[4] = {0.0, 0.0, 0.0, 0.0};
-    int r = 0;
-    for (; r + 4 <= n; r += 4) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) s4[u] += static_cast<double>(at(r + u, t));
-    }
-    for (; r < n; ++r) s4[0] += static_cast<double>(at(r, t));
-    mean = ((s4[0] + s4[1]) + (s4[2] + s4[3])) / static_cast<double>(n);
-    double q4[4] = {0.0, 0.0, 0.0, 0.0};
-    for (r = 0; r + 4 <= n; r += 4) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const double x = static_cast<double>(at(r + u, t)) - mean;
-        q4[u] = fma(x, x, q4[u]);
+  // Passes 1 and 2: the threads split into NT / d row groups, each
+  // thread one coordinate over its group's rows (four interleaved partial
+  // sums), the groups' partials added in shared memory.  The pass-1 sums of
+  // bf16 (or moderate fp32) rows are exact in float64, so the mean does not
+  // depend on how the rows are split.
+  const int ngroups = NT / d > 0 ? NT / d : 1;
+  const int e_own = t % d, grp = t / d;
+  const bool active = grp < ngroups && e_own < d;
+  // sum over the thread's rows grp, grp + ngroups, ...: four interleaved
+  // partial sums, the rows past the last full group of four into the first
+  auto group_sum = [&](auto&& term) -> double {  // term(r): row r's term
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+    if (active) {
+      int r = grp;
+      for (; r + 3 * ngroups < n; r += 4 * ngroups) {
+        s0 += term(r);
+        s1 += term(r + ngroups);
+        s2 += term(r + 2 * ngroups);
+        s3 += term(r + 3 * ngroups);
       }
+      for (; r < n; r += ngroups) s0 += term(r);
     }
-    for (; r < n; ++r) {
-      const double x = static_cast<double>(at(r, t)) - mean;
-      q4[0] = fma(x, x, q4[0]);
+    return (s0 + s1) + (s2 + s3);
+  };
+  auto val = [&](int r) -> float { return at(r, e_own); };
+  double mean = 0.0, sd = 0.0;
+  {
+    const double part = group_sum([&](int r) { return static_cast<double>(val(r)); });
+    if (active) s_part[t] = part;
+    __syncthreads();
+    if (t < d) {
+      double tot = 0.0;
+      for (int g2 = 0; g2 < ngroups; ++g2) tot += s_part[g2 * d + t];
+      s_mu[t] = tot / static_cast<double>(n);  // the exact mean, for pass 2
     }
-    sd = sqrt(((q4[0] + q4[1]) + (q4[2] + q4[3])) / static_cast<double>(n));
+    __syncthreads();
+    const double m_own = active ? s_mu[e_own] : 0.0;
+    const double sq = group_sum([&](int r) {
+      const double x = static_cast<double>(val(r)) - m_own;
+      return x * x;
+    });
+    __syncthreads();  // every thread has read s_mu and s_part
+    if (active) s_part[t] = sq;
+    __syncthreads();
+    if (t < d) {
+      double tot = 0.0;
+      for (int g2 = 0; g2 < ngroups; ++g2) tot += s_part[g2 * d + t];
+      mean = s_mu[t];
+      sd = sqrt(tot / static_cast<double>(n));
+    }
+    __syncthreads();  // s_mu is rewritten with the stored centroid below
   }
   if (FMT == ETA_META_FP16) {
     if (t < d) {
@@ -152,8 +194,8 @@ __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n
       s_mu[t] = static_cast<double>(dev::fp16_to_f32(mu_h));
     }
   } else {
-    const double mmax = cta_max(fabs(mean), s_wmax);
-    const double smax = cta_max(sd, s_wmax);
+    const double mmax = cta_max<NT>(fabs(mean), s_wmax);
+    const double smax = cta_max<NT>(sd, s_wmax);
     const float mu_scale = mmax > 0.0 ? __double2float_rn(mmax / 448.0) : 1.f;
     const float sd_scale = smax > 0.0 ? __double2float_rn(smax / 448.0) : 1.f;
     if (t < d) {
@@ -169,29 +211,45 @@ __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n
     }
   }
   __syncthreads();
-  // Pass 3, M_B: warp w takes rows w, w + 4, ... two at a time; lanes split
-  // the coordinates.  The differences k - mu~ are exact in float64 and the
-  // sum of d squares has a relative error below 2^-48, which the 2^-47
-  // inflation (rounded up) covers before the upward rounding to fp32.
+  // Pass 3, M_B: tpr consecutive lanes per row (the most that fit the CTA,
+  // up to a warp), each summing a share of the coordinates, visited in an
+  // order skewed by the row so that the lanes of different rows read
+  // different shared-memory banks; the row's partial sums are added by
+  // shuffles and the largest row is taken over the CTA.  The differences
+  // k - mu~ are exact in float64 and the sum of d squares has a relative
+  // error below 2^-48, which the 2^-47 inflation (rounded up) covers before
+  // the upward rounding to fp32.
   const int w = t >> 5, lane = t & 31;
-  constexpr int kW = kThreads / 32;
+  constexpr int kW = NT / 32;
+  int tpr = 1;
+  while (tpr < 32 && 2 * tpr * n <= NT) tpr *= 2;
+  const int sub = t % tpr, per = d / tpr;
   double best = 0.0;
-  for (int r = w; r < n; r += 2 * kW) {
-    const int r2 = r + kW < n ? r + kW : r;
-    double s1 = 0.0, s2 = 0.0;
-    for (int e = lane; e < d; e += 32) {
-      const double x1 = static_cast<double>(at(r, e)) - s_mu[e];
-      const double x2 = static_cast<double>(at(r2, e)) - s_mu[e];
-      s1 = fma(x1, x1, s1);
-      s2 = fma(x2, x2, s2);
+  for (int r0 = 0; r0 < n; r0 += NT / tpr) {  // the same trip count in every lane
+    const int r = r0 + t / tpr;
+    double rs = 0.0;
+    if (r < n) {
+      auto sq = [&](int k) {
+        const int e = (sub + tpr * k + 2 * r) % d;
+        const double x = static_cast<double>(at(r, e)) - s_mu[e];
+        return x * x;
+      };
+      double q0 = 0.0, q1 = 0.0, q2 = 0.0, q3 = 0.0;
+      int k = 0;
+      for (; k + 4 <= per; k += 4) {
+        q0 += sq(k);
+        q1 += sq(k + 1);
+        q2 += sq(k + 2);
+        q3 += sq(k + 3);
+      }
+      for (; k < per; ++k) q0 += sq(k);
+      rs = (q0 + q1) + (q2 + q3);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-    }
-    best = fmax(best, fmax(s1, s2));
+    for (int o = 1; o < tpr; o <<= 1) rs += __shfl_xor_sync(0xffffffffu, rs, o);
+    if (r < n) best = fmax(best, rs);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) best = fmax(best, __shfl_xor_sync(0xffffffffu, best, o));
   if (lane == 0) s_wmax[w] = best;
   __syncthreads();
   if (t == 0) {
@@ -217,7 +275,7 @@ __global__ void __launch_bounds__(kThreads) summary_kernel(SummaryArgs a) {
   ft = ft < 0 ? 0 : ft;
   const int j = ft / a.b + static_cast<int>(blockIdx.x);
   if (j >= nb) return;
-  summarize_block<FMT>(a, i, g, j, min(a.b, T - j * a.b), stage);
+  summarize_block<FMT, kThreads>(a, i, g, j, min(a.b, T - j * a.b), stage);
 }
 
 // One CTA per (KV head, sequence): write the new token's K and V rows at
@@ -228,7 +286,7 @@ __global__ void __launch_bounds__(kThreads) summary_kernel(SummaryArgs a) {
 // with .cv: they may sit in page-locked host memory that the host rewrites
 // between launches.
 template <int FMT>
-__global__ void __launch_bounds__(kThreads) append_kernel(SummaryArgs a, const void* k_new, const void* v_new,
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(SummaryArgs a, const void* k_new, const void* v_new,
                                                           const int* pos, void* k_cache, void* v_cache) {
   extern __shared__ __align__(16) uint8_t stage[];
   const int g = blockIdx.x, i = blockIdx.y;
@@ -236,11 +294,12 @@ __global__ void __launch_bounds__(kThreads) append_kernel(SummaryArgs a, const v
   // The decode's screen may be scheduled now: it waits for this grid's
   // completion before it reads anything.
   dev::pdl_trigger();
+  if (t == 0) dev::trace_first(a.trace, ETA_TRACE_APPEND_FIRST);
   // Every load of the new rows is issued before the first use, so rows in
   // host memory cost one round trip: a K and a V vector per thread
   // (d * elt / 16 <= 32 vectors per row) and up to kQv query vectors
-  // (G * d * elt / 16 <= 256 = kQv * kThreads).
-  constexpr int kQv = 2;
+  // (G * d * elt / 16 <= 256 <= kQv * kAppendThreads).
+  constexpr int kQv = 1;
   const int nvec = d * a.elt / 16;
   const size_t src = (static_cast<size_t>(i) * a.Hkv + g) * d;
   uint4 kr = make_uint4(0u, 0u, 0u, 0u), vr = kr, qr[kQv];
@@ -252,20 +311,26 @@ __global__ void __launch_bounds__(kThreads) append_kernel(SummaryArgs a, const v
   const int qv = a.q_src ? a.G * d * a.elt / 16 : 0;
 #pragma unroll
   for (int u = 0; u < kQv; ++u) {
-    const int x = t + u * kThreads;
+    const int x = t + u * kAppendThreads;
     if (x < qv) qr[u] = __ldcv(reinterpret_cast<const uint4*>(a.q_src) + q0 + x);
   }
   const int p = pos[i];
 #pragma unroll
   for (int u = 0; u < kQv; ++u) {
-    const int x = t + u * kThreads;
+    const int x = t + u * kAppendThreads;
     if (x < qv) reinterpret_cast<uint4*>(a.q_dst)[q0 + x] = qr[u];
   }
-  if (p < 0 || p >= a.max_ctx) return;
+  if (p < 0 || p >= a.max_ctx) {
+    if (t == 0) dev::trace_last(a.trace, ETA_TRACE_APPEND_LAST);
+    return;
+  }
   const KvLayout lay{a.block_table, a.Hkv, a.b, a.max_ctx, a.nbmax, a.num_pages};
   bool bad = false;
   const long long brow = lay.row(i * a.Hkv + g, p / a.b, &bad);
-  if (bad) return;  // a page id outside the pool: nothing is written
+  if (bad) {  // a page id outside the pool: nothing is written
+    if (t == 0) dev::trace_last(a.trace, ETA_TRACE_APPEND_LAST);
+    return;
+  }
   const size_t dst = (static_cast<size_t>(brow) + p % a.b) * d;
   if (t < nvec) {
     reinterpret_cast<uint4*>(static_cast<uint8_t*>(k_cache) + dst * a.elt)[t] = kr;
@@ -274,8 +339,8 @@ __global__ void __launch_bounds__(kThreads) append_kernel(SummaryArgs a, const v
   __syncthreads();  // the new row is read back by the block summary below
   const int T = clamp_len(a.seq_lens[i], a.max_ctx);
   const int j = p / a.b;
-  if (j * a.b >= T) return;
-  summarize_block<FMT>(a, i, g, j, min(a.b, T - j * a.b), stage);
+  if (j * a.b < T) summarize_block<FMT, kAppendThreads>(a, i, g, j, min(a.b, T - j * a.b), stage);
+  if (t == 0) dev::trace_last(a.trace, ETA_TRACE_APPEND_LAST);
 }
 
 }  // namespace
@@ -298,7 +363,7 @@ cudaError_t launch_append(const SummaryArgs& a, const void* k_new, const void* v
   const size_t smem = block_stage_bytes(a.b, a.d, a.elt);
   auto go = [&](auto kern, SmemLimit& lim) {
     return launch_with_smem(reinterpret_cast<const void*>(kern), smem, lim, [&] {
-      kern<<<dim3(a.Hkv, a.B), kThreads, smem, st>>>(a, k_new, v_new, pos, k_cache, v_cache);
+      kern<<<dim3(a.Hkv, a.B), kAppendThreads, smem, st>>>(a, k_new, v_new, pos, k_cache, v_cache);
       return cudaGetLastError();
     });
   };

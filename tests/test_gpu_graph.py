@@ -268,7 +268,8 @@ def test_step_graph_copies_of_any_size_and_alignment(nbytes, offset):
     assert eta.eta_read_device_status(ws) == eta.ETA_OK
 
 
-def test_step_graph_growing_context_across_block_boundaries():
+@pytest.mark.parametrize("lwb", [2, 0, -1], ids=["window2", "window0", "no_window"])
+def test_step_graph_growing_context_across_block_boundaries(lwb):
     """A serving loop whose context grows one token per step, as the bench's
     end-to-end leg runs it: per token the new lengths and positions are copied
     up from page-locked memory, the append reads the new q, k, v rows from
@@ -276,9 +277,12 @@ def test_step_graph_growing_context_across_block_boundaries():
     host memory, all in one recorded graph.  The appends cross block
     boundaries (and start a fresh block); after every token the outputs, the
     admitted sets and the refreshed metadata match the oracle for the state
-    reached."""
+    reached; with the window of two blocks, of the tail block alone (the block
+    a token completes is screened by the very next token), and without a
+    window (rescue on)."""
     full = workloads.custom(seed=61, batch=2, n_q_heads=8, n_kv_heads=2, head_dim=128, block_size=64,
-                            seq_lens=[900, 400], dtype=BF16, tau_bias=2.0, tau_std=1.0, key_kind="cluster")
+                            seq_lens=[900, 400], dtype=BF16, tau_bias=2.0, tau_std=1.0,
+                            key_kind="cluster").with_params(n_local_blocks=lwb)
     T0 = [700 - 4, 256 - 2]  # the first sequence crosses 704, the second 256
     B, Hq, Hkv, d, b = full.batch, full.n_q_heads, full.n_kv_heads, full.head_dim, full.block_size
     wl = full.with_params(seq_lens=list(T0))
