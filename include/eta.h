@@ -256,7 +256,8 @@ typedef struct {
 
 /*
  * Leading control region of a decode workspace: the device status word and
- * the counters the fused kernel uses to hand out work and to fold partials.
+ * the counters of the fused kernel (finished CTAs, published slice totals
+ * and their arrival count, per-segment piece counters of the merge).
  * It must be zero before the workspace's first use; every completed step
  * leaves it at zero again (apart from the status word, which
  * eta_read_device_status clears), so one workspace serves calls of any shapes

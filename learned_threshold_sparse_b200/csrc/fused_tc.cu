@@ -56,8 +56,9 @@
 // timeout status instead of hanging.
 //
 // Counters live in the workspace's control region and are back at zero when
-// a step completes: the last CTA to finish clears the slice totals, and the
-// merger of a segment clears that segment's counter.
+// a step completes: the last CTA to finish clears the slice totals and the
+// arrival counter, and the merger of a segment clears that segment's
+// counter.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -1042,9 +1043,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
     // Merge the pieces of segment seg held by CTAs cf..cl (CTA order): the
-    // pieces are copied into the idle K/V ring (bulk copies, rounds of as
-    // many as fit), then each thread combines four output coordinates of one
-    // head over them.
+    // pieces are copied into the idle K/V ring (16-byte asynchronous copies
+    // from all softmax threads, rounds of as many as fit), then each thread
+    // combines four output coordinates of one head over them.
     auto merge = [&](int seg, int cf, int cl, int slot_cf) -> bool {
       const dev::UnitSplit us(static_cast<unsigned>(*units_total), static_cast<unsigned>(N));
       constexpr uint32_t kPiece = G * PS * sizeof(float);
