@@ -22,14 +22,17 @@
 // columns it was computed from, so tile j + 2's S (issued after P_j . V_j by
 // the same thread, and the MMAs run in issue order) never races it.
 //
-// Roles: warp 0 issues the tensor copies (Q once, K/V tiles into a 2-stage
-// ring); warp 1 owns tensor memory and issues the MMAs; warps 2-9 run the
+// Roles: warp 0 issues the tensor copies (Q once; K and V tiles into two
+// 2-stage rings with their own barriers, so K_{j+2} is copied as soon as
+// Q K_j^T is done, not after P_j V_j); warp 1 owns tensor memory and issues
+// the MMAs; warps 2-9 run the
 // softmax, two warps per query-row quarter (tensor-memory lane quarter),
 // each on one half h of the key columns with its own running max, sum and
 // accumulator O_h (two split-KV partials of the row, merged once at the end
 // by the associative combine), so the halves never wait on each other.  The
 // running max moves lazily: O_h is rescaled in tensor memory only when a
-// row's max grows by more than 2^8, so the weights stay <= 2^8.
+// row's max grows by more than 2^8, so the weights stay <= 2^8.  Off the
+// diagonal the softmax runs on column pairs with the packed fp32x2 forms.
 #include <math.h>
 
 #include "attend_common.cuh"
@@ -80,6 +83,33 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo_f(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
+// Packed pairs of fp32 operations (one instruction for two columns): a b + c,
+// a b, a + b, each element rounded exactly as its scalar form.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // Tensor-memory column of the 8 P columns feeding K step kk (16 keys) of
 // half h's P V MMA in S buffer sb: half h wrote its 64 keys as 32 columns
 // starting at column 64 h of the buffer.
@@ -89,8 +119,10 @@ __device__ __forceinline__ uint32_t p_col(int sb, int h, int kk) {
 
 struct Bars {
   uint64_t* q_full;    // producer -> MMA (tx bytes)
-  uint64_t* kv_full;   // [2] producer -> MMA (tx bytes)
-  uint64_t* kv_empty;  // [2] MMA commit -> producer
+  uint64_t* k_full;    // [2] producer -> MMA (tx bytes)
+  uint64_t* k_empty;   // [2] Q K^T commit -> producer
+  uint64_t* v_full;    // [2] producer -> MMA, and the softmax before it zeroes rows of V
+  uint64_t* v_empty;   // [2] P V commit -> producer
   uint64_t* s_full;    // [2] MMA commit -> softmax
   uint64_t* p_full;    // [2 buffers][2 halves] softmax (4 warps) -> MMA
   uint64_t* o_done;    // MMA commit after every P V -> softmax
@@ -108,17 +140,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar = reinterpret_cast<uint64_t*>(base + OFF_BARS);
   Bars Bs;
   Bs.q_full = bar;
-  Bs.kv_full = bar + 1;
-  Bs.kv_empty = bar + 3;
-  Bs.s_full = bar + 5;
-  Bs.p_full = bar + 7;
-  Bs.o_done = bar + 11;
-  Bs.done = bar + 12;
-  Bs.rv = bar + 13;
+  Bs.k_full = bar + 1;
+  Bs.k_empty = bar + 3;
+  Bs.v_full = bar + 5;
+  Bs.v_empty = bar + 7;
+  Bs.s_full = bar + 9;
+  Bs.p_full = bar + 11;
+  Bs.o_done = bar + 15;
+  Bs.done = bar + 16;
+  Bs.rv = bar + 17;
   float* red = reinterpret_cast<float*>(base + OFF_RED);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_BARS + 128);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + OFF_BARS + 132);
-  int* issued = reinterpret_cast<int*>(base + OFF_BARS + 136);  // [2] parity of the last copy per stage, -1 none
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_BARS + 160);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + OFF_BARS + 164);
+  int* issued_k = reinterpret_cast<int*>(base + OFF_BARS + 168);  // [2] parity of the last K copy per stage, -1 none
+  int* issued_v = reinterpret_cast<int*>(base + OFF_BARS + 176);  // [2] same for V
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
   const int nqt = (a.T + BM - 1) / BM;
@@ -131,12 +166,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (t == 0) {
     dev::mbar_init(Bs.q_full, 1);
     for (int k = 0; k < kStages; ++k) {
-      dev::mbar_init(&Bs.kv_full[k], 1);
-      dev::mbar_init(&Bs.kv_empty[k], 1);
+      dev::mbar_init(&Bs.k_full[k], 1);
+      dev::mbar_init(&Bs.k_empty[k], 1);
+      dev::mbar_init(&Bs.v_full[k], 1);
+      dev::mbar_init(&Bs.v_empty[k], 1);
       dev::mbar_init(&Bs.s_full[k], 1);
       dev::mbar_init(&Bs.p_full[2 * k], kSoftWarps / 2);
       dev::mbar_init(&Bs.p_full[2 * k + 1], kSoftWarps / 2);
-      issued[k] = -1;
+      issued_k[k] = -1;
+      issued_v[k] = -1;
     }
     dev::mbar_init(Bs.o_done, 1);
     dev::mbar_init(Bs.done, 1);
@@ -166,18 +204,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int krow0 = (b * a.Hkv + g) * a.kv_stride;
       for (int j = 0; j < nt; ++j) {
         const int st = j & 1;
-        if (!wait_or_abort(&Bs.kv_empty[st], ((j >> 1) & 1) ^ 1, a.status, abort_flag)) {
+        const uint32_t par = static_cast<uint32_t>(((j >> 1) & 1) ^ 1);
+        const uint32_t ks = base_u32 + OFF_STAGE + static_cast<uint32_t>(st) * 2 * TILE, vs = ks + TILE;
+        const int krow = krow0 + j * BN;
+        if (!wait_or_abort(&Bs.k_empty[st], par, a.status, abort_flag)) {
           ok = false;
           break;
         }
-        const uint32_t ks = base_u32 + OFF_STAGE + static_cast<uint32_t>(st) * 2 * TILE, vs = ks + TILE;
-        dev::mbar_arrive_expect_tx(&Bs.kv_full[st], 2 * TILE);
-        const int krow = krow0 + j * BN;
-        tma_load_2d(ks, &tk, 0, krow, &Bs.kv_full[st]);
-        tma_load_2d(ks + PANEL, &tk, 64, krow, &Bs.kv_full[st]);
-        tma_load_2d(vs, &tv, 0, krow, &Bs.kv_full[st]);
-        tma_load_2d(vs + PANEL, &tv, 64, krow, &Bs.kv_full[st]);
-        issued[st] = (j >> 1) & 1;
+        dev::mbar_arrive_expect_tx(&Bs.k_full[st], TILE);
+        tma_load_2d(ks, &tk, 0, krow, &Bs.k_full[st]);
+        tma_load_2d(ks + PANEL, &tk, 64, krow, &Bs.k_full[st]);
+        issued_k[st] = (j >> 1) & 1;
+        if (!wait_or_abort(&Bs.v_empty[st], par, a.status, abort_flag)) {
+          ok = false;
+          break;
+        }
+        dev::mbar_arrive_expect_tx(&Bs.v_full[st], TILE);
+        tma_load_2d(vs, &tv, 0, krow, &Bs.v_full[st]);
+        tma_load_2d(vs + PANEL, &tv, 64, krow, &Bs.v_full[st]);
+        issued_v[st] = (j >> 1) & 1;
       }
       if (!ok) {
         *abort_flag = 1;
@@ -186,10 +231,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         while (!dev::mbar_try_wait(Bs.q_full, 0) && clock64() - t0 < dev::kWaitCycles) {
         }
         for (int k = 0; k < kStages; ++k) {
-          if (issued[k] < 0) continue;
-          const long long t1 = clock64();
-          while (!dev::mbar_try_wait(&Bs.kv_full[k], static_cast<uint32_t>(issued[k])) &&
-                 clock64() - t1 < dev::kWaitCycles) {
+          if (issued_k[k] >= 0) {
+            const long long t1 = clock64();
+            while (!dev::mbar_try_wait(&Bs.k_full[k], static_cast<uint32_t>(issued_k[k])) &&
+                   clock64() - t1 < dev::kWaitCycles) {
+            }
+          }
+          if (issued_v[k] >= 0) {
+            const long long t1 = clock64();
+            while (!dev::mbar_try_wait(&Bs.v_full[k], static_cast<uint32_t>(issued_v[k])) &&
+                   clock64() - t1 < dev::kWaitCycles) {
+            }
           }
         }
       }
@@ -204,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto issue_pv = [&](int i) -> bool {
       const int sb = i & 1;
       const uint32_t vs = base_u32 + OFF_STAGE + static_cast<uint32_t>(sb) * 2 * TILE + TILE;
+      if (!wait_or_abort(&Bs.v_full[sb], static_cast<uint32_t>((i >> 1) & 1), a.status, abort_flag)) return false;
       for (int hh = 0; hh < 2; ++hh) {
         if (!wait_or_abort(&Bs.p_full[2 * sb + hh], static_cast<uint32_t>((i >> 1) & 1), a.status, abort_flag))
           return false;
@@ -220,14 +273,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (lane == 0) {
         mma_commit(Bs.o_done);
-        mma_commit(&Bs.kv_empty[sb]);
+        mma_commit(&Bs.v_empty[sb]);
       }
       __syncwarp();
       return true;
     };
     for (int j = 0; j < nt && ok; ++j) {
       const int st = j & 1;
-      if (!wait_or_abort(&Bs.kv_full[st], (j >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
+      if (!wait_or_abort(&Bs.k_full[st], (j >> 1) & 1, a.status, abort_flag)) { ok = false; break; }
       tc_fence_after();
       if (lane == 0) {
         const uint32_t ks = base_u32 + OFF_STAGE + static_cast<uint32_t>(st) * 2 * TILE;
@@ -239,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_bf16(tmem + static_cast<uint32_t>(st) * BN, ad, bd, idesc_qk, kk > 0 ? 1u : 0u);
         }
         mma_commit(&Bs.s_full[st]);
+        mma_commit(&Bs.k_empty[st]);
       }
       __syncwarp();
       if (j > 0 && !issue_pv(j - 1)) { ok = false; break; }
@@ -313,22 +367,34 @@ __global__ void __launch_bounds__(kThreads, 1)
       // keys j BN + c with c <= lim are seen by this row (causal; rows past
       // the sequence see none).  Off the diagonal every key of every row of
       // the warp is seen: no masking there.
-      // gate(beta (scale S - tau)) = 1/2 + tanh(cb S + ct) / 2, x = cx S gate.
+      // gate(beta (scale S - tau)) = 1/2 + t / 2 with t = tanh(cb S + ct),
+      // x = cx S gate = u + u t with u = cx S / 2; the gate sum over a full
+      // half is 32 + (sum t) / 2.
       const int lim = row_ok ? min(BN - 1, i - j * BN) - hf * 64 : -1;
       const bool full = __all_sync(0xffffffffu, lim >= 63);
-      const float cb = 0.5f * beta * scale, ct = -0.5f * beta * tau, cx = scale * kLog2e;
+      const float cb = 0.5f * beta * scale, ct = -0.5f * beta * tau, cx = scale * kLog2e, cu = 0.5f * cx;
       float pm = -INFINITY;
       if (full) {
+        const float2 cb2 = make_float2(cb, cb), ct2 = make_float2(ct, ct), cu2 = make_float2(cu, cu);
+        float2 ts2 = make_float2(0.f, 0.f);
+        float pm1 = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          uint32_t& sv = c < 32 ? s0[c] : s1[c - 32];
-          const float Sr = __uint_as_float(sv);
-          const float sg = fmaf(0.5f, tanh_approx(fmaf(Sr, cb, ct)), 0.5f);
-          const float x = Sr * cx * sg;
-          r_part += sg;
-          pm = fmaxf(pm, x);
-          sv = __float_as_uint(x);
+        for (int e = 0; e < 32; ++e) {
+          uint32_t& sa = e < 16 ? s0[2 * e] : s1[2 * e - 32];
+          uint32_t& sz = e < 16 ? s0[2 * e + 1] : s1[2 * e + 1 - 32];
+          const float2 S2 = make_float2(__uint_as_float(sa), __uint_as_float(sz));
+          const float2 a2 = ffma2(S2, cb2, ct2);
+          const float2 t2 = make_float2(tanh_approx(a2.x), tanh_approx(a2.y));
+          const float2 u2 = fmul2(S2, cu2);
+          const float2 x2 = ffma2(u2, t2, u2);
+          ts2 = fadd2(ts2, t2);
+          pm = fmaxf(pm, x2.x);
+          pm1 = fmaxf(pm1, x2.y);
+          sa = __float_as_uint(x2.x);
+          sz = __float_as_uint(x2.y);
         }
+        pm = fmaxf(pm, pm1);
+        r_part += fmaf(0.5f, ts2.x + ts2.y, 32.f);
       } else {
 #pragma unroll
         for (int c = 0; c < 64; ++c) {
@@ -377,13 +443,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t pk[32];
       float lsum = 0.f;
       if (full) {
+        const float2 nm2 = make_float2(-m_run, -m_run);
+        float2 ls2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
-          const float p0 = dev::fast_exp2(__uint_as_float(e < 16 ? s0[2 * e] : s1[2 * e - 32]) - m_run);
-          const float p1 = dev::fast_exp2(__uint_as_float(e < 16 ? s0[2 * e + 1] : s1[2 * e + 1 - 32]) - m_run);
-          pk[e] = pack_bf16(p0, p1);
-          lsum += p0 + p1;
+          const float2 x2 = make_float2(__uint_as_float(e < 16 ? s0[2 * e] : s1[2 * e - 32]),
+                                        __uint_as_float(e < 16 ? s0[2 * e + 1] : s1[2 * e + 1 - 32]));
+          const float2 y2 = fadd2(x2, nm2);
+          const float2 p2 = make_float2(dev::fast_exp2(y2.x), dev::fast_exp2(y2.y));
+          pk[e] = pack_bf16(p2.x, p2.y);
+          ls2 = fadd2(ls2, p2);
         }
+        lsum = ls2.x + ls2.y;
       } else {
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
@@ -403,6 +474,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // (each half zeroes the rows its own P V reads, before it signals P)
       const int z0 = max(a.T - j * BN, hf * 64), z1 = hf * 64 + 64;
       if (z0 < z1) {
+        // V_j has its own barrier: its copy lands before the zeroing
+        if (!warp_wait_or_abort(&Bs.v_full[sb], static_cast<uint32_t>((j >> 1) & 1), a.status, abort_flag)) {
+          ok = false;
+          break;
+        }
         uint8_t* vt = base + OFF_STAGE + sb * 2 * TILE + TILE;
         const int nz = (z1 - z0) * 8;  // 16-byte chunks per panel
         for (int c = st_id & 127; c < 2 * nz; c += kSoftThreads / 2) {
