@@ -32,8 +32,11 @@
 // by the associative combine), so the halves never wait on each other.  The
 // running max moves lazily: O_h is rescaled in tensor memory only when a
 // row's max grows by more than 2^8, so the weights stay <= 2^8.  Off the
-// diagonal the softmax runs on column pairs with the packed fp32x2 forms.
+// diagonal the softmax runs on column pairs with the packed fp32x2 forms,
+// and 3/8 of the weights' 2^x are computed on the FMA pipes (the gate's tanh
+// and the weight's 2^x otherwise both occupy the special-function unit).
 #include <math.h>
+#include <string.h>
 
 #include "attend_common.cuh"
 #include "tc_common.cuh"
@@ -83,30 +86,90 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo_f(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
 
-// Packed pairs of fp32 operations (one instruction for two columns): a b + c,
-// a b, a + b, each element rounded exactly as its scalar form.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+// ETA_EXP2_BEGIN
+// Packed pairs of fp32 operations (one instruction for two columns on the
+// device): a b + c, a b, a + b, each element rounded exactly as its scalar
+// form (the host forms are those scalar forms).
+__host__ __device__ inline float2 ffma2(float2 a, float2 b, float2 c) {
+#ifdef __CUDA_ARCH__
   float2 d;
   asm("{.reg .b64 ra, rb, rc, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
       "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;}"
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
   return d;
+#else
+  return make_float2(fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y));
+#endif
 }
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+__host__ __device__ inline float2 fmul2(float2 a, float2 b) {
+#ifdef __CUDA_ARCH__
   float2 d;
   asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
       "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
+#else
+  return make_float2(a.x * b.x, a.y * b.y);
+#endif
 }
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+__host__ __device__ inline float2 fadd2(float2 a, float2 b) {
+#ifdef __CUDA_ARCH__
   float2 d;
   asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
       "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+#else
+  return make_float2(a.x + b.x, a.y + b.y);
+#endif
+}
+
+__host__ __device__ inline uint32_t bits_of(float x) {
+#ifdef __CUDA_ARCH__
+  return __float_as_uint(x);
+#else
+  uint32_t u;
+  memcpy(&u, &x, 4);
+  return u;
+#endif
+}
+__host__ __device__ inline float float_of(uint32_t u) {
+#ifdef __CUDA_ARCH__
+  return __uint_as_float(u);
+#else
+  float x;
+  memcpy(&x, &u, 4);
+  return x;
+#endif
+}
+
+// 2^y for a pair on the FMA pipes, to take part of the weights off the
+// special-function unit.  Cody-Waite style reduction: y = n + f with
+// n = rint(y) (adding 1.5 2^23 leaves n in the low mantissa bits) and f in
+// [-1/2, 1/2]; 2^f by the cubic of least maximum relative error on that
+// interval (Remez exchange; 7.5e-5), and n added to its exponent field.  y is
+// clamped at -126 first, so the result stays near 2^-126 or above (where the
+// special-function form flushes its results below 2^-126 to 0).
+__host__ __device__ inline float2 exp2_fma2(float2 y) {
+  constexpr float kRound = 12582912.f;  // 1.5 2^23
+  const float2 yc = make_float2(fmaxf(y.x, -126.f), fmaxf(y.y, -126.f));
+  const float2 t = fadd2(yc, make_float2(kRound, kRound));
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = fadd2(yc, make_float2(-n.x, -n.y));
+  float2 q = ffma2(make_float2(0.05517167f, 0.05517167f), f, make_float2(0.24261113f, 0.24261113f));
+  q = ffma2(q, f, make_float2(0.69326097f, 0.69326097f));
+  q = ffma2(q, f, make_float2(0.99992806f, 0.99992806f));
+  return make_float2(float_of(bits_of(q.x) + (bits_of(t.x) << 23)), float_of(bits_of(q.y) + (bits_of(t.y) << 23)));
+}
+// ETA_EXP2_END
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
 
@@ -388,8 +451,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 u2 = fmul2(S2, cu2);
           const float2 x2 = ffma2(u2, t2, u2);
           ts2 = fadd2(ts2, t2);
-          pm = fmaxf(pm, x2.x);
-          pm1 = fmaxf(pm1, x2.y);
+          if (e & 1) pm1 = max3f(pm1, x2.x, x2.y);
+          else pm = max3f(pm, x2.x, x2.y);
           sa = __float_as_uint(x2.x);
           sz = __float_as_uint(x2.y);
         }
@@ -450,7 +513,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 x2 = make_float2(__uint_as_float(e < 16 ? s0[2 * e] : s1[2 * e - 32]),
                                         __uint_as_float(e < 16 ? s0[2 * e + 1] : s1[2 * e + 1 - 32]));
           const float2 y2 = fadd2(x2, nm2);
-          const float2 p2 = make_float2(dev::fast_exp2(y2.x), dev::fast_exp2(y2.y));
+          // three pairs in eight on the FMA pipes, the rest on the
+          // special-function unit (more shifts the bound to the issue rate)
+          const float2 p2 = (e & 7) < 3 ? exp2_fma2(y2) : make_float2(dev::fast_exp2(y2.x), dev::fast_exp2(y2.y));
           pk[e] = pack_bf16(p2.x, p2.y);
           ls2 = fadd2(ls2, p2);
         }
