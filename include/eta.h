@@ -442,7 +442,8 @@ eta_status eta_step_graph_create(const eta_step_desc* d, eta_decode_graph** out)
  * max_ctx = kv_stride; rows >= seq_len of a head are never used);
  * lse, gate_sum [batch, n_q_heads, seq_len] fp32.
  * Supported: bf16, head_dim = 128, any group size, 1 <= seq_len <= kv_stride,
- * batch * n_q_heads * seq_len and batch * n_kv_heads * kv_stride < 2^31.
+ * seq_len <= 65535 * 128 (8388480), batch * n_q_heads * seq_len and
+ * batch * n_kv_heads * kv_stride < 2^31.
  * ------------------------------------------------------------------------
  */
 typedef struct {

@@ -500,6 +500,9 @@ eta_status eta_prefill(const eta_prefill_params* p, void* stream) {
   if (static_cast<long long>(p->batch) * p->n_q_heads * p->seq_len >= (1ll << 31) ||
       static_cast<long long>(p->batch) * p->n_kv_heads * p->kv_stride >= (1ll << 31))
     return ETA_ERR_UNSUPPORTED;
+  // one grid row per 128-query tile (the grid's y extent is at most 65535)
+  constexpr int kPrefillMaxSeq = 65535 * 128;
+  if (p->seq_len > kPrefillMaxSeq) return ETA_ERR_UNSUPPORTED;
   if (!p->q || !p->k || !p->v || !p->out) return ETA_ERR_INVALID_ARG;
   if (!aligned(p->q, 16) || !aligned(p->k, 16) || !aligned(p->v, 16) || !aligned(p->out, 16))
     return ETA_ERR_INVALID_ARG;

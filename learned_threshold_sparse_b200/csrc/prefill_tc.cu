@@ -12,7 +12,7 @@
 //   Appendix G.1         tau~ = tau - a, tau = w_tau . q + b_tau or a constant.
 //
 // One CTA per (128 query rows, query head, sequence); heavy (late) query tiles
-// are scheduled first.  Per key tile j of 128 keys:
+// of all heads and sequences are dispatched first.  Per key tile j of 128 keys:
 //   S [128 q x 128 k]  = Q . K_j^T   (M = 128, N = 128; Q, K from shared memory)
 //   O_h [128 q x 128 d] += P_j,h . V_j,h   (h = 0, 1: keys 0-63 / 64-127 of
 //                                          the tile; A = P from tensor
@@ -219,9 +219,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* issued_v = reinterpret_cast<int*>(base + OFF_BARS + 176);  // [2] same for V
 
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  // blockIdx.x runs over (head, sequence) and blockIdx.y over query tiles,
+  // last tile first: CTAs are dispatched in linear order, so the whole grid
+  // goes heaviest first and the light tiles fill the end
   const int nqt = (a.T + BM - 1) / BM;
-  const int qt = nqt - 1 - static_cast<int>(blockIdx.x);  // heavy tiles first
-  const int h = blockIdx.y, b = blockIdx.z;
+  const int qt = nqt - 1 - static_cast<int>(blockIdx.y);
+  const int h = static_cast<int>(blockIdx.x) % a.Hq, b = static_cast<int>(blockIdx.x) / a.Hq;
   const int g = h / a.G;
   const int q0 = qt * BM;
   const int nt = qt + 1;  // key tiles 0..qt (causal)
@@ -619,7 +622,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs& a, cudaStream_t st) {
   if (!make_map(&tq, a.q, qrows, BM) || !make_map(&tk, a.k, kvrows, BN) || !make_map(&tv, a.v, kvrows, BN))
     return cudaErrorInvalidValue;
   static SmemLimit lim;
-  const dim3 grid((a.T + BM - 1) / BM, a.Hq, a.B);
+  const dim3 grid(a.Hq * a.B, (a.T + BM - 1) / BM);
   return launch_with_smem(reinterpret_cast<const void*>(prefill_tc_kernel), kSmemBytes, lim, [&] {
     prefill_tc_kernel<<<grid, kThreads, kSmemBytes, st>>>(tq, tk, tv, a);
     return cudaGetLastError();

@@ -242,6 +242,11 @@ def test_prefill_size_limits():
     p = _prefill_ok()
     p.batch, p.n_q_heads, p.n_kv_heads, p.seq_len, p.kv_stride = 64, 64, 64, 1 << 20, 1 << 20
     assert eta.library().eta_prefill(ctypes.byref(p), None) == eta.ETA_ERR_UNSUPPORTED
+    # one grid row per 128-query tile: at most 65535 tiles
+    p = _prefill_ok()
+    p.n_q_heads = p.n_kv_heads = 1
+    p.seq_len = p.kv_stride = 65535 * 128 + 1
+    assert eta.library().eta_prefill(ctypes.byref(p), None) == eta.ETA_ERR_UNSUPPORTED
     p = _prefill_ok()
     p.tau_mode = eta.ETA_TAU_CALIBRATED
     p.c_tau = None
