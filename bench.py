@@ -843,7 +843,8 @@ def run_reference(args):
 def run_prefill(args):
     """Causal forward pass (eta_prefill) over a whole sequence: tensor flops of
     the two contractions over the causal triangle per second, against the
-    measured dense bf16 peak.  Not the decode metric; printed on its own line."""
+    measured dense bf16 peak (median step; the mean beside it).  Not the
+    decode metric; printed on its own line."""
     import learned_threshold_sparse_b200 as eta
 
     B, Hq, Hkv, T = (int(x) for x in args.prefill_shape.split(","))
@@ -872,7 +873,8 @@ def run_prefill(args):
     clocks.start()
     time.sleep(0.3)
     ms = []
-    for _ in range(args.steps):
+    steps = max(args.steps, 20)
+    for _ in range(steps):
         torch.sum(flush_buf, dim=0, out=flush_sink)
         e0.record(stream)
         eta.eta_prefill(params, stream)
@@ -882,8 +884,9 @@ def run_prefill(args):
     clk = clocks.stop()
     assert eta.eta_read_device_status(ws) == eta.ETA_OK
     flops = 4.0 * d * (T * (T + 1) / 2) * B * Hq
-    t = statistics.mean(ms)
+    t = statistics.median(ms)
     tflops = flops / (t * 1e-3) / 1e12
+    t_mean = statistics.mean(ms)
     peak_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     peak, kind = 1590.0, "fallback"
     if os.path.exists(peak_path):
@@ -894,9 +897,13 @@ def run_prefill(args):
         "value": round(tflops, 2),
         "unit": "TFLOP/s",
         "n_gpus": 1,
-        "steps": args.steps,
+        "steps": steps,
         "warmup": args.warmup,
         "ms_per_step": round(t, 4),
+        "statistic": "median of the timed steps",
+        "ms_mean": round(t_mean, 4),
+        "tflops_mean": round(flops / (t_mean * 1e-3) / 1e12, 2),
+        "ms_p10_p90": [round(_pct(ms, 10), 4), round(_pct(ms, 90), 4)],
         "higher_is_better": True,
         "dtype": "bf16",
         "accum": "f32",
@@ -906,7 +913,7 @@ def run_prefill(args):
                    "l2": "flushed before every step by reading a 256 MiB buffer (outside the events)"},
         "roofline": {"kernel": "prefill_tc", "bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
                      "peak_kind": kind + " dense bf16 (burst)", "unit": "TFLOP/s", "frac": round(tflops / peak, 4)},
-        "gpu_launches": args.steps,
+        "gpu_launches": steps,
         "clocks": clk,
     }
 
