@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + L.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + L.misc + 4);
   int* pm = reinterpret_cast<int*>(base + L.misc + 64);     // merges to run at the end: [count, (seg, c_first, c_last, slot) x 2]
-  int* mround = reinterpret_cast<int*>(base + L.misc + 100);  // merge round: [pieces, next CTA]
+  int* mbatch = reinterpret_cast<int*>(base + L.misc + 100);  // merge batch: [pieces, next CTA]
   int* issued_parity = reinterpret_cast<int*>(base + L.misc + 32);
   int* units_total = reinterpret_cast<int*>(base + L.misc + 48);  // U, set by the producer before its first tile
 
@@ -1044,7 +1044,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     // Merge the pieces of segment seg held by CTAs cf..cl (CTA order): the
     // pieces are copied into the idle K/V ring (16-byte asynchronous copies
-    // from all softmax threads, rounds of as many as fit), then each thread
+    // from all softmax threads, batches of as many as fit), then each thread
     // combines four output coordinates of one head over them.
     auto merge = [&](int seg, int cf, int cl, int slot_cf) -> bool {
       const dev::UnitSplit us(static_cast<unsigned>(*units_total), static_cast<unsigned>(N));
@@ -1061,7 +1061,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int c0 = cf;
       while (c0 <= cl) {
-        // this round's pieces (the CTAs from c0 on with a non-empty range, as
+        // this batch's pieces (the CTAs from c0 on with a non-empty range, as
         // many as the ring holds): their slots, listed by warp 2
         if (warp == 2) {
           int np = 0, c = c0;
@@ -1074,20 +1074,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (np + __popc(bal) <= kMaxPieces) {
               np += __popc(bal);
               c += 32;
-            } else {  // the next round starts at the first piece that does not fit
+            } else {  // the next batch starts at the first piece that does not fit
               const unsigned first_out = __ballot_sync(0xffffffffu, has && np + before == kMaxPieces);
               c += __ffs(first_out) - 1;
               np = kMaxPieces;
             }
           }
           if (lane == 0) {
-            mround[0] = np;
-            mround[1] = min(c, cl + 1);
+            mbatch[0] = np;
+            mbatch[1] = min(c, cl + 1);
           }
         }
         if (!rendezvous()) return false;
-        const int np = mround[0];
-        const int next = mround[1];
+        const int np = mbatch[0];
+        const int next = mbatch[1];
         // all pieces in flight at once: 16-byte asynchronous copies through L2
         fence_proxy_async();  // the ring's earlier tensor copies and reads come first
         constexpr int kPc = static_cast<int>(kPiece / 16);
