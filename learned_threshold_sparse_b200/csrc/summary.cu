@@ -86,16 +86,18 @@ __device__ __forceinline__ double cta_max(double v, double* s_w) {
 //
 // NT threads per CTA: the more, the shorter every thread's dependent chain
 // (passes 1 and 2 split the rows into NT / d groups, pass 3 gives each row
-// NT / n lanes).
-template <int FMT, int NT>
+// NT / n lanes).  DC, EC: the head dimension and element size when known at
+// compile time (0: taken from the arguments), so that the index arithmetic
+// of the common case folds to shifts and masks.
+template <int FMT, int NT, int DC = 0, int EC = 0>
 __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n, uint8_t* stage) {
-  const int d = a.d, t = threadIdx.x;
+  const int d = DC > 0 ? DC : a.d, elt = EC > 0 ? EC : a.elt, t = threadIdx.x;
   const KvLayout lay{a.block_table, a.Hkv, a.b, a.max_ctx, a.nbmax, a.num_pages};
   bool bad = false;
   const size_t row0 = static_cast<size_t>(lay.row(i * a.Hkv + g, j, &bad));
   if (bad) return;  // a page id outside the pool: nothing is read or written (CTA-uniform)
-  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.k) + row0 * d * a.elt);
-  const int nvec = n * d * a.elt / 16;
+  const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint8_t*>(a.k) + row0 * d * elt);
+  const int nvec = n * d * elt / 16;
   // all of a thread's loads in flight before its stores (one round trip)
   for (int x0 = t; x0 < nvec; x0 += 8 * NT) {
     uint4 v[8];
@@ -112,7 +114,7 @@ __device__ void summarize_block(const SummaryArgs& a, int i, int g, int j, int n
   __syncthreads();
   auto at = [&](int r, int e) -> float {
     const size_t idx = static_cast<size_t>(r) * d + e;
-    if (a.elt == 4) return reinterpret_cast<const float*>(stage)[idx];
+    if (elt == 4) return reinterpret_cast<const float*>(stage)[idx];
     return __uint_as_float(static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(stage)[idx]) << 16);
   };
   const size_t bo = (static_cast<size_t>(i) * a.Hkv + g) * a.nbmax + j;  // block index
@@ -275,7 +277,9 @@ __global__ void __launch_bounds__(kThreads) summary_kernel(SummaryArgs a) {
   ft = ft < 0 ? 0 : ft;
   const int j = ft / a.b + static_cast<int>(blockIdx.x);
   if (j >= nb) return;
-  summarize_block<FMT, kThreads>(a, i, g, j, min(a.b, T - j * a.b), stage);
+  const int n = min(a.b, T - j * a.b);
+  if (a.d == 128 && a.elt == 2) summarize_block<FMT, kThreads, 128, 2>(a, i, g, j, n, stage);
+  else summarize_block<FMT, kThreads>(a, i, g, j, n, stage);
 }
 
 // One CTA per (KV head, sequence): write the new token's K and V rows at
@@ -339,7 +343,11 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(SummaryArgs a, c
   __syncthreads();  // the new row is read back by the block summary below
   const int T = clamp_len(a.seq_lens[i], a.max_ctx);
   const int j = p / a.b;
-  if (j * a.b < T) summarize_block<FMT, kAppendThreads>(a, i, g, j, min(a.b, T - j * a.b), stage);
+  if (j * a.b < T) {
+    const int n = min(a.b, T - j * a.b);
+    if (a.d == 128 && a.elt == 2) summarize_block<FMT, kAppendThreads, 128, 2>(a, i, g, j, n, stage);
+    else summarize_block<FMT, kAppendThreads>(a, i, g, j, n, stage);
+  }
   if (t == 0) dev::trace_last(a.trace, ETA_TRACE_APPEND_LAST);
 }
 
