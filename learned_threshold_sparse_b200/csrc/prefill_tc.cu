@@ -152,7 +152,9 @@ __host__ __device__ inline float float_of(uint32_t u) {
 // [-1/2, 1/2]; 2^f by the cubic of least maximum relative error on that
 // interval (Remez exchange; 7.5e-5), and n added to its exponent field.  y is
 // clamped at -126 first, so the result stays near 2^-126 or above (where the
-// special-function form flushes its results below 2^-126 to 0).
+// special-function form flushes its results below 2^-126 to 0); the clamp
+// also maps a NaN y (a NaN key inside the sequence) to 2^-126, where the
+// special-function form gives NaN.
 __host__ __device__ inline float2 exp2_fma2(float2 y) {
   constexpr float kRound = 12582912.f;  // 1.5 2^23
   const float2 yc = make_float2(fmaxf(y.x, -126.f), fmaxf(y.y, -126.f));
