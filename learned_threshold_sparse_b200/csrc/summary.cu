@@ -295,9 +295,6 @@ __global__ void __launch_bounds__(kAppendThreads) append_kernel(SummaryArgs a, c
   extern __shared__ __align__(16) uint8_t stage[];
   const int g = blockIdx.x, i = blockIdx.y;
   const int d = a.d, t = threadIdx.x;
-  // The decode's screen may be scheduled now: it waits for this grid's
-  // completion before it reads anything.
-  dev::pdl_trigger();
   if (t == 0) dev::trace_first(a.trace, ETA_TRACE_APPEND_FIRST);
   // Every load of the new rows is issued before the first use, so rows in
   // host memory cost one round trip: a K and a V vector per thread
