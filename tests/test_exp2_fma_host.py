@@ -116,3 +116,43 @@ def test_a_planted_mistake_fails(tmp_path, old, new):
     run = _build(tmp_path, "bad", _block(src.replace(old, new)))
     y, got = run(np.linspace(-20.0, 8.0, 2001).astype(np.float32))
     assert _rel_err(y, got).max() > 8e-5
+
+
+def _remez_cubic_for_exp2():
+    """Cubic of least maximum relative error for 2^f on [-1/2, 1/2], by the
+    Remez exchange: solve p(x_i) - 2^x_i = (-1)^i E 2^x_i on n + 2 points,
+    move the points to the extrema of the relative error, repeat."""
+    a, b, n = -0.5, 0.5, 3
+    x = 0.5 * (a + b) + 0.5 * (b - a) * np.cos(np.pi * np.arange(n + 2)[::-1] / (n + 1))
+    grid = np.linspace(a, b, 200001)
+    for _ in range(30):
+        y = 2.0 ** x
+        A = np.zeros((n + 2, n + 2))
+        for i in range(n + 2):
+            A[i, :n + 1] = x[i] ** np.arange(n + 1)
+            A[i, n + 1] = -((-1) ** i) * y[i]
+        c = np.linalg.solve(A, y)[:n + 1]
+        r = (np.polyval(c[::-1], grid) - 2.0 ** grid) / 2.0 ** grid
+        idx = [0] + [i for i in range(1, len(grid) - 1) if (r[i] - r[i - 1]) * (r[i + 1] - r[i]) <= 0] + [len(grid) - 1]
+        sel = []
+        for xi, ri in zip(grid[idx], r[idx]):
+            if sel and np.sign(ri) == np.sign(sel[-1][1]):
+                if abs(ri) > abs(sel[-1][1]):
+                    sel[-1] = (xi, ri)
+            else:
+                sel.append((xi, ri))
+        while len(sel) > n + 2:
+            sel.pop(0 if abs(sel[0][1]) < abs(sel[-1][1]) else -1)
+        x = np.array([s[0] for s in sel])
+    return c, float(np.abs(r).max())
+
+
+def test_coefficients_are_the_minimax_cubic():
+    # the constants in the kernel are this fit rounded to fp32
+    c, err = _remez_cubic_for_exp2()
+    assert 7.4e-5 < err < 7.6e-5
+    block = _block()
+    m = re.findall(r"make_float2\(([0-9.]+)f, \1f\)", block)
+    coeffs = sorted(float(v) for v in m if float(v) < 2.0)  # the four polynomial constants
+    assert len(coeffs) == 4, coeffs
+    np.testing.assert_allclose(sorted(c), coeffs, rtol=2e-7, atol=0)
