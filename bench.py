@@ -639,6 +639,16 @@ def run_eta(args):
             extra["fused_kernel"] = {"note": ("attend_impl = ETA_ATTEND_FUSED: one launch per step (screen, "
                                               "attention, merge); attend_us_isolated is that launch"), **fused}
     clk = clocks.stop()
+    if world == 1 and not args.no_configs and not args.dense:
+        # the causal forward pass (prefill) at its default shape on the same
+        # GPU, after the decode's clock record: its own line's figures
+        pa = argparse.Namespace(**vars(args))
+        pa.steps = 20
+        pl = run_prefill(pa)
+        extra["prefill"] = {"workload": pl["config"]["workload"], "metric": pl["metric"],
+                            **{k: pl[k] for k in ("value", "unit", "statistic", "ms_per_step", "ms_mean", "tflops_mean",
+                                                  "ms_p10_p90", "roofline", "clocks")}}
+        torch.cuda.empty_cache()
 
     att = kt["attend"]
     achieved = main["kv_union"] / (att * 1e-3) / 1e9
@@ -980,7 +990,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--configs", default="c2_single,c3_long,c5_batched",
                     help="other workloads measured (screened and dense) after the main line")
-    ap.add_argument("--no-configs", action="store_true", help="skip the dense arm and the other workloads")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the dense arm, the other workloads, the single-launch kernel and the prefill")
     ap.add_argument("--meta", default="fp16", choices=["fp16", "fp8", "box"],
                     help="block metadata format (box: the comparison coordinate-box screen)")
     ap.add_argument("--prefill", action="store_true", help="time the causal forward pass instead of the decode step")
